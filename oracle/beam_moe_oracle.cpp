@@ -1,0 +1,282 @@
+// Beam sparse-MoE layer: plain CPU oracle.
+//
+// TEST INFRASTRUCTURE, not part of the product.  Only the tests, the smoke
+// check and the benchmark's CPU-baseline leg may load this library.  It shares
+// no code, header, table or helper with the CUDA path.
+//
+// What it computes, and where each step comes from:
+//   * router logits in FP32 from FP32 router weights; sigmoid scores; a
+//     learned per-expert bias added for selection only; the best topk_group of
+//     n_group expert groups; top_k experts inside them; weights normalised to
+//     sum 1 and scaled by routed_scaling_factor  -- Transformers "Beam" model
+//     doc, Overview ("Sparse MoE" bullet and the FP32-numerics paragraph) and
+//     BeamConfig (n_group, topk_group, norm_topk_prob, routed_scaling_factor).
+//   * group score = sum of the top-2 biased scores of the group -- archdb
+//     "Beam-1.0-501B-A23B" fact sheet, expert-groups entry.
+//   * contiguous groups of E/n_group experts ("8 groups of 32") and SwiGLU
+//     experts with intermediate size 2560, no shared expert -- news article
+//     "Reflection lança o Beam", section "Onde o Beam economiza ...".
+//   * SwiGLU activation in FP32, RMSNorm scaling in FP32 -- "Beam" model doc,
+//     Overview, FP32-numerics paragraph.
+//   * sandwich RMSNorm (eps 1e-6) and the depth-scaled residual
+//     r*sqrt((k-1)/k) + f/sqrt(k) -- "Beam" model doc, Overview ("Sandwich
+//     norms" bullet); archdb fact sheet, residual-design entry.
+//
+// Numerics: every dot product accumulates in double and is rounded once to
+// FP32 (the exactly rounded FP32 result up to one rounding); transcendental
+// functions run in double and are rounded once.  Ties in selection go to the
+// lower group / expert index.  Selected experts are reported in ascending id
+// order with their weights permuted alongside; the combine sums in that order.
+//
+// Plain loops, no BLAS, no intrinsics; std::thread over tokens.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <thread>
+#include <vector>
+
+namespace {
+
+float bf16_bits_to_float(uint16_t b) {
+  uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+// Round-to-nearest-even of an FP32 value to BF16 (keep the top 16 bits).
+uint16_t float_to_bf16_bits(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, sizeof u);
+  if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu) != 0u)
+    return static_cast<uint16_t>((u >> 16) | 0x0040u);  // quiet NaN
+  const uint32_t lower = u & 0xffffu;
+  uint32_t upper = u >> 16;
+  if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;
+  return static_cast<uint16_t>(upper);
+}
+
+int resolve_threads(int nthreads) {
+  if (nthreads > 0) return nthreads;
+  unsigned hc = std::thread::hardware_concurrency();
+  return hc ? static_cast<int>(hc) : 1;
+}
+
+template <class F>
+void parallel_for(int64_t n, int nthreads, F body) {
+  nthreads = resolve_threads(nthreads);
+  if (nthreads <= 1 || n <= 1) {
+    for (int64_t i = 0; i < n; ++i) body(i);
+    return;
+  }
+  if (nthreads > n) nthreads = static_cast<int>(n);
+  std::vector<std::thread> pool;
+  pool.reserve(nthreads);
+  for (int w = 0; w < nthreads; ++w) {
+    pool.emplace_back([=, &body] {
+      for (int64_t i = w; i < n; i += nthreads) body(i);
+    });
+  }
+  for (auto& th : pool) th.join();
+}
+
+double sigmoid(double x) { return 1.0 / (1.0 + std::exp(-x)); }
+
+}  // namespace
+
+extern "C" {
+
+int oracle_hardware_threads(void) { return resolve_threads(0); }
+
+void oracle_f32_to_bf16(int64_t n, const float* in, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = float_to_bf16_bits(in[i]);
+}
+
+void oracle_bf16_to_f32(int64_t n, const uint16_t* in, float* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = bf16_bits_to_float(in[i]);
+}
+
+// logits[t, e] = fl32( sum_j h[t, j] * Wr[e, j] ), h BF16 widened exactly.
+void oracle_router_logits(int64_t T, int64_t d, int64_t E, const uint16_t* h,
+                          const float* Wr, float* logits, int nthreads) {
+  parallel_for(T, nthreads, [&](int64_t t) {
+    const uint16_t* ht = h + t * d;
+    for (int64_t e = 0; e < E; ++e) {
+      const float* we = Wr + e * d;
+      double acc = 0.0;
+      for (int64_t j = 0; j < d; ++j)
+        acc += static_cast<double>(bf16_bits_to_float(ht[j])) * static_cast<double>(we[j]);
+      logits[t * E + e] = static_cast<float>(acc);
+    }
+  });
+}
+
+// Selection and weights for T tokens from their router logits.
+//   s  = sigmoid(logit)                  (FP32)
+//   sb = s + bias                        (FP32; used only to choose)
+//   group score gs_g = sum of the top-2 sb in group g (top-1 if a group has one expert)
+//   keep the topk_group groups with the largest gs (lower g wins ties)
+//   choose the top_k experts with the largest sb among kept groups (lower e wins ties)
+//   w = S * s / sum(s over the chosen)   (or S * s without normalisation)
+// idx[t, :] lists the chosen experts in ascending id; w[t, :] follows it.
+// margin_expert[t] = sb of the k-th chosen minus sb of the best unchosen expert in a
+// kept group (+inf if none); margin_group[t] = gs of the last kept group minus gs of
+// the best dropped group (+inf if none).  Either margin array may be NULL.
+// Returns 0, or -1 on an invalid shape.
+int oracle_route(int64_t T, int E, int G, int Gk, int k, float S, int norm_topk_prob,
+                 const float* logits, const float* bias, int32_t* idx, float* w,
+                 float* margin_expert, float* margin_group, int nthreads) {
+  if (E <= 0 || G <= 0 || E % G != 0 || Gk <= 0 || Gk > G || k <= 0 ||
+      k > Gk * (E / G))
+    return -1;
+  const int per = E / G;
+  parallel_for(T, nthreads, [&](int64_t t) {
+    const float* lt = logits + t * E;
+    std::vector<float> s(E), sb(E);
+    for (int e = 0; e < E; ++e) {
+      s[e] = static_cast<float>(sigmoid(static_cast<double>(lt[e])));
+      sb[e] = s[e] + bias[e];
+    }
+    // group scores
+    std::vector<float> gs(G);
+    for (int g = 0; g < G; ++g) {
+      std::vector<float> v(sb.begin() + g * per, sb.begin() + (g + 1) * per);
+      std::sort(v.begin(), v.end(), [](float a, float b) { return a > b; });
+      gs[g] = per >= 2 ? v[0] + v[1] : v[0];
+    }
+    std::vector<int> gorder(G);
+    for (int g = 0; g < G; ++g) gorder[g] = g;
+    std::sort(gorder.begin(), gorder.end(), [&](int a, int b) {
+      if (gs[a] != gs[b]) return gs[a] > gs[b];
+      return a < b;
+    });
+    std::vector<char> kept(G, 0);
+    for (int i = 0; i < Gk; ++i) kept[gorder[i]] = 1;
+    // candidate experts in kept groups, best first
+    std::vector<int> cand;
+    for (int e = 0; e < E; ++e)
+      if (kept[e / per]) cand.push_back(e);
+    std::sort(cand.begin(), cand.end(), [&](int a, int b) {
+      if (sb[a] != sb[b]) return sb[a] > sb[b];
+      return a < b;
+    });
+    std::vector<int> chosen(cand.begin(), cand.begin() + k);
+    std::sort(chosen.begin(), chosen.end());
+    double denom = 0.0;
+    for (int e : chosen) denom += static_cast<double>(s[e]);
+    for (int j = 0; j < k; ++j) {
+      const int e = chosen[j];
+      idx[t * k + j] = e;
+      const double num = static_cast<double>(S) * static_cast<double>(s[e]);
+      w[t * k + j] = static_cast<float>(norm_topk_prob ? num / denom : num);
+    }
+    const float inf = std::numeric_limits<float>::infinity();
+    if (margin_expert)
+      margin_expert[t] = static_cast<int>(cand.size()) > k ? sb[cand[k - 1]] - sb[cand[k]] : inf;
+    if (margin_group)
+      margin_group[t] = G > Gk ? gs[gorder[Gk - 1]] - gs[gorder[Gk]] : inf;
+  });
+  return 0;
+}
+
+// One SwiGLU expert on one input row x [d] (BF16):
+//   g_i = fl32(sum_j x_j Wg[i, j]),  u_i = fl32(sum_j x_j Wu[i, j])
+//   a_i = bf16( fl32(silu(g_i)) * u_i ),  silu(g) = g / (1 + exp(-g))
+//   y_c = fl32(sum_i a_i Wd[c, i])
+// Wg, Wu are [I, d]; Wd is [d, I] (nn.Linear out x in).  a_out [I] (BF16 bits) may be NULL.
+void oracle_expert_mlp(int64_t d, int64_t I, const uint16_t* x, const uint16_t* Wg,
+                       const uint16_t* Wu, const uint16_t* Wd, float* y, uint16_t* a_out) {
+  std::vector<double> xd(d);
+  for (int64_t j = 0; j < d; ++j) xd[j] = bf16_bits_to_float(x[j]);
+  std::vector<double> a(I);
+  for (int64_t i = 0; i < I; ++i) {
+    double gacc = 0.0, uacc = 0.0;
+    const uint16_t* wg = Wg + i * d;
+    const uint16_t* wu = Wu + i * d;
+    for (int64_t j = 0; j < d; ++j) {
+      gacc += xd[j] * static_cast<double>(bf16_bits_to_float(wg[j]));
+      uacc += xd[j] * static_cast<double>(bf16_bits_to_float(wu[j]));
+    }
+    const float g = static_cast<float>(gacc);
+    const float u = static_cast<float>(uacc);
+    const float act = static_cast<float>(static_cast<double>(g) * sigmoid(static_cast<double>(g)));
+    const uint16_t ab = float_to_bf16_bits(act * u);
+    if (a_out) a_out[i] = ab;
+    a[i] = bf16_bits_to_float(ab);
+  }
+  for (int64_t c = 0; c < d; ++c) {
+    const uint16_t* wd = Wd + c * I;
+    double acc = 0.0;
+    for (int64_t i = 0; i < I; ++i) acc += a[i] * static_cast<double>(bf16_bits_to_float(wd[i]));
+    y[c] = static_cast<float>(acc);
+  }
+}
+
+// MoE output for a list of tokens: out[n, c] = fl32( sum_j w[t, j] * y_{idx[t, j]}[c] )
+// summed in the order of idx (ascending expert id), t = tokens[n].  Expert weights
+// are passed as per-expert pointer arrays so that callers may supply only the
+// experts these tokens use; a NULL entry that is needed makes the call return -1.
+int oracle_moe_tokens(int64_t ntok, const int64_t* tokens, int64_t d, int64_t I, int k,
+                      const uint16_t* h, const int32_t* idx, const float* w,
+                      const uint16_t* const* Wg, const uint16_t* const* Wu,
+                      const uint16_t* const* Wd, float* out, int nthreads) {
+  for (int64_t n = 0; n < ntok; ++n)
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[tokens[n] * k + j];
+      if (!Wg[e] || !Wu[e] || !Wd[e]) return -1;
+    }
+  // one work item per (token, slot); the reduction over slots runs afterwards in order
+  std::vector<float> ys(static_cast<size_t>(ntok) * k * d);
+  parallel_for(ntok * k, nthreads, [&](int64_t item) {
+    const int64_t n = item / k;
+    const int j = static_cast<int>(item % k);
+    const int64_t t = tokens[n];
+    const int e = idx[t * k + j];
+    oracle_expert_mlp(d, I, h + t * d, Wg[e], Wu[e], Wd[e], ys.data() + item * d, nullptr);
+  });
+  for (int64_t n = 0; n < ntok; ++n) {
+    const int64_t t = tokens[n];
+    for (int64_t c = 0; c < d; ++c) {
+      double acc = 0.0;
+      for (int j = 0; j < k; ++j)
+        acc += static_cast<double>(w[t * k + j]) *
+               static_cast<double>(ys[(static_cast<size_t>(n) * k + j) * d + c]);
+      out[n * d + c] = static_cast<float>(acc);
+    }
+  }
+  return 0;
+}
+
+// RMSNorm in FP32 semantics: y = fl32( x / sqrt(mean(x^2) + eps) * g ), row-wise over [T, d].
+void oracle_rmsnorm(int64_t T, int64_t d, const float* x, const float* g, float eps, float* y,
+                    int nthreads) {
+  parallel_for(T, nthreads, [&](int64_t t) {
+    const float* xt = x + t * d;
+    double ss = 0.0;
+    for (int64_t j = 0; j < d; ++j) ss += static_cast<double>(xt[j]) * static_cast<double>(xt[j]);
+    const double rms = std::sqrt(ss / static_cast<double>(d) + static_cast<double>(eps));
+    for (int64_t j = 0; j < d; ++j)
+      y[t * d + j] = static_cast<float>(static_cast<double>(xt[j]) / rms * static_cast<double>(g[j]));
+  });
+}
+
+// Depth-scaled residual after the k-th contribution:
+//   out = fl32( x * sqrt((k-1)/k) + f * (1/sqrt(k)) ).
+void oracle_residual(int64_t n, const float* x, const float* f, int k, float* out) {
+  const double kk = static_cast<double>(k);
+  const double cx = std::sqrt((kk - 1.0) / kk);
+  const double cf = 1.0 / std::sqrt(kk);
+  for (int64_t i = 0; i < n; ++i)
+    out[i] = static_cast<float>(static_cast<double>(x[i]) * cx + static_cast<double>(f[i]) * cf);
+}
+
+void oracle_residual_coefficients(int k, double* cx, double* cf) {
+  const double kk = static_cast<double>(k);
+  *cx = std::sqrt((kk - 1.0) / kk);
+  *cf = 1.0 / std::sqrt(kk);
+}
+
+}  // extern "C"

@@ -1,0 +1,96 @@
+"""Planted mistakes: each mutant copy of the oracle must fail at least one pin.
+
+A mutant is the oracle's C++ source with one plausible error written into it
+(a dropped term, a wrong index, a swapped operand, a wrong convention).  It is
+compiled into a temporary library on the CPU, swapped in for the real one, and
+the pins in test_oracle_pins are run against it.  Every mutant must be caught.
+"""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "beam_moe_oracle.cpp")
+
+MUTANTS = {
+    "group_score_is_max": ("gs[g] = per >= 2 ? v[0] + v[1] : v[0];", "gs[g] = v[0];"),
+    "group_score_sums_all": ("gs[g] = per >= 2 ? v[0] + v[1] : v[0];",
+                             "gs[g] = 0; for (float q : v) gs[g] += q;"),
+    "bias_in_weights": ("static_cast<double>(S) * static_cast<double>(s[e]);",
+                        "static_cast<double>(S) * static_cast<double>(sb[e]);"),
+    "group_tie_upper_wins": ("      if (gs[a] != gs[b]) return gs[a] > gs[b];\n      return a < b;",
+                             "      if (gs[a] != gs[b]) return gs[a] > gs[b];\n      return a > b;"),
+    "expert_tie_upper_wins": ("      if (sb[a] != sb[b]) return sb[a] > sb[b];\n      return a < b;",
+                              "      if (sb[a] != sb[b]) return sb[a] > sb[b];\n      return a > b;"),
+    "select_by_unbiased_score": ("      if (sb[a] != sb[b]) return sb[a] > sb[b];",
+                                 "      if (s[a] != s[b]) return s[a] > s[b];"),
+    "down_proj_transposed": ("const uint16_t* wd = Wd + c * I;", "const uint16_t* wd = Wd + c;"),
+    "no_silu": ("static_cast<double>(g) * sigmoid(static_cast<double>(g))",
+                "static_cast<double>(g)"),
+    "gate_up_swapped": ("static_cast<double>(g) * sigmoid(static_cast<double>(g))",
+                        "static_cast<double>(u) * sigmoid(static_cast<double>(u))"),
+    "no_normalisation": ("w[t * k + j] = static_cast<float>(norm_topk_prob ? num / denom : num);",
+                         "w[t * k + j] = static_cast<float>(num);"),
+    "residual_coefficient": ("const double cf = 1.0 / std::sqrt(kk);", "const double cf = 1.0 / kk;"),
+    "rmsnorm_no_mean": ("std::sqrt(ss / static_cast<double>(d) + static_cast<double>(eps))",
+                        "std::sqrt(ss + static_cast<double>(eps))"),
+    "router_drops_last_term": ("      for (int64_t j = 0; j < d; ++j)\n        acc += static_cast<double>(bf16_bits_to_float(ht[j]))",
+                               "      for (int64_t j = 0; j < d - 1; ++j)\n        acc += static_cast<double>(bf16_bits_to_float(ht[j]))"),
+    "combine_drops_slot": ("      for (int j = 0; j < k; ++j)\n        acc += static_cast<double>(w[t * k + j])",
+                           "      for (int j = 1; j < k; ++j)\n        acc += static_cast<double>(w[t * k + j])"),
+    "bf16_truncates": ("if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;", ""),
+}
+
+PIN_TESTS = [
+    (pins.test_route_matches_brute_force, [(8, 2, 1, 2), (16, 4, 2, 4)]),
+    (pins.test_group_score_hand_examples, [()]),
+    (pins.test_bias_is_selection_only, [()]),
+    (pins.test_weights_sum_to_scaling_factor, [("tiny",)]),
+    (pins.test_unnormalised_weights_are_scaled_scores, [()]),
+    (pins.test_router_logits_match_float64_matmul, [()]),
+    (pins.test_expert_mlp_matches_torch_float64, [()]),
+    (pins.test_identical_experts_equal_scaled_dense_swiglu, [()]),
+    (pins.test_combine_is_weighted_sum_of_expert_outputs, [()]),
+    (pins.test_residual_coefficients_square_sum_is_one, [()]),
+    (pins.test_residual_after_104_contributions_weighs_each_equally, [()]),
+    (pins.test_rmsnorm_matches_torch_and_closed_form, [()]),
+    (pins.test_bf16_rounding_matches_torch, [()]),
+]
+
+
+def _build_mutant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation {name} does not apply uniquely"
+    path = tmp_path / f"{name}.cpp"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / f"lib{name}.so"
+    subprocess.run(["g++", "-O1", "-std=c++17", "-ffp-contract=off", "-shared", "-fPIC",
+                    "-pthread", "-o", str(so), str(path)], check=True)
+    return str(so)
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(tmp_path, monkeypatch, name):
+    old, new = MUTANTS[name]
+    so = _build_mutant(tmp_path, name, old, new)
+    real = oracle.lib()
+    mut = ctypes.CDLL(so)
+    for fn in ("oracle_hardware_threads", "oracle_f32_to_bf16", "oracle_bf16_to_f32",
+               "oracle_router_logits", "oracle_route", "oracle_expert_mlp", "oracle_moe_tokens",
+               "oracle_rmsnorm", "oracle_residual", "oracle_residual_coefficients"):
+        f, g = getattr(real, fn), getattr(mut, fn)
+        g.argtypes, g.restype = f.argtypes, f.restype
+    monkeypatch.setattr(oracle, "_lib", mut)
+    caught = []
+    for test, params in PIN_TESTS:
+        for p in params:
+            try:
+                test(*p)
+            except (AssertionError, ValueError):
+                caught.append(test.__name__)
+                break
+    assert caught, f"mutant {name} passed every pin"
