@@ -1,0 +1,557 @@
+#!/usr/bin/env python
+"""Throughput of the Beam sparse-MoE layer forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill] [--impl cuda|reference]
+
+One step is one whole layer forward (router, dispatch, gate/up GEMM + SwiGLU, down GEMM,
+combine; the block workload adds the two RMSNorms and the residual) over one batch of
+synthetic tokens, through the C ABI.  With N > 1 (launched by torch.distributed.run) every
+rank runs an independent replica of the layer on its own GPU and its own tokens: the layer is
+data parallel over tokens and has no exchange step, so there is no collective on the data
+path; the barrier and the max-over-ranks of the timed region are the only cross-rank calls.
+
+``--impl reference`` times the CPU oracle (the plain C++ reference of the same layer) on the
+host cores on a bounded sample of the same workload, and prints the same JSON line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import contextlib
+import dataclasses
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from sparse_moe_transformer_fp32_b200 import workloads as W  # noqa: E402
+
+METRIC = "MoE-layer tokens/s at Beam shape T=4096 BF16; % BF16 tensor peak / % HBM BW"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0, "source": "fallback"}
+N_SMS = 148
+FFMA_PER_SM_PER_CLK = 128
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--workload", default="prefill", choices=sorted(W.WORKLOADS))
+    p.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    p.add_argument("--cpu-sample-tokens", type=int, default=32,
+                   help="tokens in the oracle's bounded sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--dry-run", action="store_true",
+                   help="exercise the launch/aggregation logic on CPU (gloo); measures nothing")
+    args = p.parse_args(argv)
+    if args.warmup < 3 and not args.dry_run:
+        p.error("--warmup must be >= 3")
+    return args
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+@contextlib.contextmanager
+def process_group(world, backend):
+    if world <= 1:
+        yield None
+        return
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    try:
+        yield dist
+    finally:
+        dist.destroy_process_group()
+
+
+def barrier(dist, device=None):
+    if dist is None:
+        return
+    if device is not None and device.type == "cuda":
+        dist.barrier(device_ids=[device.index])
+    else:
+        dist.barrier()
+
+
+def max_over_ranks(dist, value: float, device) -> float:
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(dist, value: float, device) -> float:
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ peaks and clocks
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS)
+
+
+def _gpu_selector(device_index: int):
+    try:
+        bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+        if bus:
+            return bus
+    except Exception:
+        pass
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if device_index < len(ids):
+            return ids[device_index]
+    return str(device_index)
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs."""
+
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int, period_ms: int = 50):
+        self.sel = _gpu_selector(device_index)
+        self.period_ms = period_ms
+        self.samples = []
+        self.proc = None
+        self.window = None
+
+    def start(self):
+        cmd = ["nvidia-smi", "-i", self.sel, "--query-gpu=" + ",".join(self.FIELDS),
+               "--format=csv,noheader,nounits", "-lms", str(self.period_ms)]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True, bufsize=1)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._reader, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.samples and time.time() - t0 < 5.0:
+            time.sleep(0.01)
+
+    def _reader(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == len(self.FIELDS):
+                self.samples.append((time.time(), parts))
+
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "nvidia-smi unavailable"}
+        rows = self.samples
+        if self.window:
+            inside = [r for r in rows if self.window[0] <= r[0] <= self.window[1]]
+            rows = inside or rows
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = sorted(v for v in (num(r[1][1]) for r in rows) if v is not None)
+        mx = [v for v in (num(r[1][2]) for r in rows) if v is not None]
+        pw = [v for v in (num(r[1][3]) for r in rows) if v is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[1][5 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ algorithmic work
+
+def kernel_work(wl, touched: int):
+    """Algorithmic bytes and FLOPs per launch of each kernel (the minimum each must move)."""
+    T, d, E, k, I = wl.T, wl.d, wl.E, wl.top_k, wl.I
+    R = T * k
+    bf, f4 = 2, 4
+    w_gu = touched * 2 * I * d * bf
+    w_dn = touched * d * I * bf
+    return {
+        "router_gemm": {"flops": 2 * T * d * E, "bytes": T * d * bf + E * d * f4 + T * E * f4},
+        "router_select": {"flops": 0, "bytes": T * E * f4 + 2 * R * f4},
+        "permute": {"flops": 0, "bytes": T * d * bf + R * d * bf},
+        "expert_gemm_gate_up": {"flops": 4 * R * d * I, "bytes": w_gu + R * d * bf + R * I * bf},
+        "expert_gemm_down": {"flops": 2 * R * d * I, "bytes": w_dn + R * I * bf + R * d * bf},
+        "combine": {"flops": 2 * R * d, "bytes": R * d * bf + T * d * bf},
+        "combine_block": {"flops": 2 * R * d, "bytes": R * d * bf + 3 * T * d * f4},
+        "prenorm": {"flops": 3 * T * d, "bytes": T * d * f4 + T * d * bf},
+    }
+
+
+def layer_min_bytes(wl, touched: int):
+    T, d, I = wl.T, wl.d, wl.I
+    b = touched * 3 * d * I * 2 + T * d * 2 * 2
+    if wl.block:
+        b += 2 * T * d * 4
+    return b
+
+
+def traffic_from_profile(kernel: str, workload: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"source_sha256:\s*([0-9a-f]{16,64})", text)
+    if not m or not h:
+        return None
+    src = os.path.join(ROOT, "sparse_moe_transformer_fp32_b200", "csrc")
+    cur = hashlib.sha256()
+    for name in ("expert_gemm.cu", "beam_moe_internal.cuh"):
+        with open(os.path.join(src, name), "rb") as f:
+            cur.update(f.read())
+    if not cur.hexdigest().startswith(h.group(1)):
+        return None
+    return float(m.group(1))
+
+
+# ------------------------------------------------------------------ oracle (CPU) timing
+
+def oracle_sample_rate(wl, router_w, bias, hidden_cpu, weights_dev, n_tokens: int, repeats=1):
+    """Tokens/s of the CPU oracle on the first n tokens (full layer: logits, routing, experts,
+    combine), expert weights copied from the device (not timed)."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    h = hidden_cpu[:n_tokens]
+    sample = wl.with_tokens(n_tokens)
+    _, idx, w, _, _ = oracle.layer_routing(h, router_w, bias, sample)
+    ex = sorted({int(e) for e in idx.reshape(-1)})
+    experts = {e: tuple(m[e].cpu() for m in weights_dev) for e in ex}
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        _, idx, w, _, _ = oracle.layer_routing(h, router_w, bias, sample)
+        oracle.moe_tokens(np.arange(n_tokens), h, idx, w, experts)
+    dt = time.perf_counter() - t0
+    return n_tokens * repeats / dt, dt, oracle.hardware_threads()
+
+
+# ------------------------------------------------------------------ the CUDA arm
+
+def replica_workload(wl, rank):
+    # every replica holds the same layer weights and processes its own tokens
+    return dataclasses.replace(wl, seed=W.seed_for(wl.seed, 1000 + rank)) if rank else wl
+
+
+def run_cuda(args, rank, world, local):
+    from sparse_moe_transformer_fp32_b200 import beam_moe as bm
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device; the CUDA path has no CPU fallback")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    bm.lib()  # fails loudly if the extension is missing
+    wl = W.WORKLOADS[args.workload]
+    peaks = load_peaks()
+    with process_group(world, "nccl") as dist:
+        s = bm.shape_of(wl)
+        router_w = W.router_weight(wl).to(dev)
+        bias = W.router_bias(wl).to(dev)
+        weights = W.expert_weights(wl, dev)
+        mine = replica_workload(wl, rank)
+        if wl.block:
+            x_cpu = W.residual_x(mine)
+            g_pre, g_post = (g.to(dev) for g in W.norm_gains(wl))
+            x = x_cpu.to(dev)
+            x_out = torch.empty_like(x)
+            inp_cpu, inp, res = x_cpu, x, x_out
+        else:
+            h_cpu = W.hidden(mine)
+            h = h_cpu.to(dev)
+            out = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
+            inp_cpu, inp, res = h_cpu, h, out
+        ws = bm.workspace(s, dev)
+        stream = torch.cuda.current_stream(dev)
+
+        def step(src=None, dst=None):
+            src = inp if src is None else src
+            dst = res if dst is None else dst
+            if wl.block:
+                bm.beam_moe_block(s, src, g_pre, g_post, wl.eps, wl.k_resid, router_w, bias,
+                                  *weights, dst, ws=ws)
+            else:
+                bm.beam_moe_forward(s, src, router_w, bias, *weights, dst, ws=ws)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        st = bm.beam_moe_sync_status(ws)
+        if st != bm.BEAM_OK:
+            raise SystemExit(f"bench.py: device status {bm.status_string(st)}")
+        counts = bm.beam_moe_expert_counts(s, ws)
+        touched = int((counts > 0).sum())
+
+        # ---- timed region (device time, max over ranks)
+        clocks = ClockSampler(dev.index)
+        clocks.start()
+        bm.beam_moe_profile_reset()
+        bm.beam_moe_profile_enable(True)
+        launches0 = bm.beam_moe_launch_count()
+        barrier(dist, dev)
+        torch.cuda.synchronize(dev)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0 = time.time()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        w1 = time.time()
+        barrier(dist, dev)
+        bm.beam_moe_profile_enable(False)
+        clocks.mark(w0, w1)
+        clocks.stop()
+        gpu_launches = bm.beam_moe_launch_count() - launches0
+        ms_local = ev0.elapsed_time(ev1)
+        ms_total = max_over_ranks(dist, ms_local, dev)
+        prof = bm.beam_moe_profile_read()
+        st = bm.beam_moe_sync_status(ws)
+        if st != bm.BEAM_OK:
+            raise SystemExit(f"bench.py: device status {bm.status_string(st)}")
+        tokens_all = sum_over_ranks(dist, float(wl.T * args.steps), dev)
+        value = tokens_all / (ms_total / 1e3)
+        ms_per_step = ms_total / args.steps
+
+        # ---- end to end: pinned host input -> device -> layer -> host result, every step
+        e2e = None
+        if not args.no_e2e:
+            host_in = inp_cpu.pin_memory()
+            host_out = torch.empty(res.shape, dtype=res.dtype).pin_memory()
+            dev_in = torch.empty_like(inp)
+            for _ in range(3):
+                dev_in.copy_(host_in, non_blocking=True)
+                step(dev_in, res)
+                host_out.copy_(res, non_blocking=True)
+            barrier(dist, dev)
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                dev_in.copy_(host_in, non_blocking=True)
+                step(dev_in, res)
+                host_out.copy_(res, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier(dist, dev)
+            e_ms = max_over_ranks(dist, e0.elapsed_time(e1), dev)
+            e2e = {"value": tokens_all / (e_ms / 1e3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": host_in.numel() * host_in.element_size(),
+                   "d2h_bytes_per_step": host_out.numel() * host_out.element_size()}
+
+        result = None
+        if rank == 0:
+            work = kernel_work(wl, touched)
+            per_kernel = {k: {"launches": n, "ms_per_launch": (ms / n if n else None)}
+                          for k, (n, ms) in prof.items() if n}
+            dom = max((k for k in per_kernel), key=lambda k: prof[k][1])
+            n_dom, ms_dom = prof[dom]
+            avg_s = ms_dom / n_dom / 1e3
+            wk = work[dom]
+            hbm_t = wk["bytes"] / (peaks["hbm_gbs"] * 1e9)
+            ten_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+            if dom == "router_gemm":
+                clk = float(peaks.get("sm_max_mhz", 1965.0))
+                alu_peak = N_SMS * FFMA_PER_SM_PER_CLK * 2 * clk * 1e6 / 1e12
+                roof = {"bound": "alu", "achieved": wk["flops"] / avg_s / 1e12, "peak": alu_peak,
+                        "unit": "TFLOP/s"}
+            elif wk["flops"] / (ten_peak * 1e12) > hbm_t:
+                roof = {"bound": "tensor", "achieved": wk["flops"] / avg_s / 1e12,
+                        "peak": ten_peak, "unit": "TFLOP/s"}
+            else:
+                roof = {"bound": "hbm", "achieved": wk["bytes"] / avg_s / 1e9,
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+            roof["frac"] = roof["achieved"] / roof["peak"]
+            roof["kernel"] = dom
+            roof["peak_source"] = peaks.get("source", "measured")
+            roof["traffic"] = traffic_from_profile(dom, args.workload)
+            roof["algorithmic_per_launch"] = wk["bytes"] if roof["bound"] == "hbm" else wk["flops"]
+            roof["tensor_frac_of_sustained"] = (wk["flops"] / avg_s / 1e12) / ten_peak
+            roof["hbm_frac"] = (wk["bytes"] / avg_s / 1e9) / peaks["hbm_gbs"]
+
+            step_s = ms_per_step / 1e3
+            flops_step = 6 * wl.T * wl.top_k * wl.d * wl.I
+            bytes_step = layer_min_bytes(wl, touched)
+            cpu = None
+            if not args.no_cpu_baseline and world == 1:
+                rate, secs, cores = oracle_sample_rate(
+                    wl, W.router_weight(wl), W.router_bias(wl),
+                    inp_cpu if not wl.block else _block_h(wl, mine, g_pre), weights,
+                    args.cpu_sample_tokens)
+                cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                       "sample": f"first {args.cpu_sample_tokens} tokens of the {wl.name} workload, "
+                                 f"full layer (router logits, routing, {wl.top_k} SwiGLU experts "
+                                 f"each, combine) in double-accumulating C++; {secs:.2f} s"}
+            result = {
+                "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": f"{wl.name}: T={wl.T} d={wl.d} E={wl.E} n_group={wl.n_group} "
+                                       f"topk_group={wl.topk_group} top_k={wl.top_k} I={wl.I}"
+                                       + (" block" if wl.block else ""),
+                           "tokens_per_gpu": wl.T, "global_tokens": wl.T * world,
+                           "parallelism": f"replicas x{world} (data parallel over tokens)",
+                           "l2": "inputs larger than L2: every step streams the touched experts' "
+                                 f"weights ({touched} of {wl.E} experts, "
+                                 f"{touched * 3 * wl.d * wl.I * 2 / 1e9:.2f} GB) from HBM",
+                           "touched_experts": touched,
+                           "max_expert_load": int(counts.max()),
+                           "top16_share": float(counts.sort(descending=True).values[:16].sum()
+                                                / counts.sum())},
+                "tflops": flops_step / step_s / 1e12,
+                "hbm_gbs_layer_min_bytes": bytes_step / step_s / 1e9,
+                "roofline": roof,
+                "kernels": per_kernel,
+                "gpu_launches": gpu_launches,
+                "clocks": clocks.summary(),
+                "e2e": e2e,
+                "cpu_baseline": cpu,
+            }
+        barrier(dist, dev)
+        del weights
+    return result
+
+
+def _block_h(wl, mine, g_pre):
+    import numpy as np
+    import oracle
+    x = W.residual_x(mine)
+    bits = oracle.block_prenorm(x, g_pre.cpu(), wl.eps)
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+
+
+# ------------------------------------------------------------------ the reference arm (oracle)
+
+def run_reference(args, rank, world, local):
+    if rank != 0:
+        return None
+    wl = W.WORKLOADS[args.workload]
+    n = max(1, min(args.cpu_sample_tokens, wl.T))
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    router_w, bias = W.router_weight(wl), W.router_bias(wl)
+    if wl.block:
+        g_pre, _ = W.norm_gains(wl)
+        h = _block_h(wl, wl, g_pre)
+    else:
+        h = W.hidden(wl)
+    import numpy as np
+    import oracle
+    oracle.build()
+    sample = wl.with_tokens(n)
+    _, idx, w, _, _ = oracle.layer_routing(h[:n], router_w, bias, sample)
+    ex = sorted({int(e) for e in idx.reshape(-1)})
+    experts = {e: tuple(W.expert_weight(wl, m, e, dev).cpu() for m in ("gate", "up", "down"))
+                for e in ex}
+
+    def one_step():
+        _, ix, ww, _, _ = oracle.layer_routing(h[:n], router_w, bias, sample)
+        oracle.moe_tokens(np.arange(n), h[:n], ix, ww, experts)
+
+    for _ in range(args.warmup):
+        one_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one_step()
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    cores = oracle.hardware_threads()
+    desc = (f"first {n} tokens of the {wl.name} workload per step, full layer in "
+            f"double-accumulating C++ on {cores} host threads")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: T={wl.T} d={wl.d} E={wl.E} top_k={wl.top_k} "
+                                   f"I={wl.I} (sample of {n} tokens per step)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------ dry run (host logic only)
+
+def run_dry(args, rank, world, local):
+    """Exercises rank setup, barriers and the max/sum aggregation on CPU ranks (gloo)."""
+    with process_group(world, "gloo") as dist:
+        dev = torch.device("cpu")
+        barrier(dist)
+        local_ms = 10.0 * (rank + 1)
+        ms = max_over_ranks(dist, local_ms, dev)
+        tokens = sum_over_ranks(dist, float(W.WORKLOADS[args.workload].T * args.steps), dev)
+        barrier(dist)
+    if rank != 0:
+        return None
+    return {"dry_run": True, "n_gpus": world, "steps": args.steps, "max_ms": ms,
+            "tokens_all_ranks": tokens, "value_if_measured": tokens / (ms / 1e3)}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if world != args.gpus and not args.dry_run:
+        if world == 1 and args.gpus > 1:
+            raise SystemExit("bench.py: --gpus N > 1 must be launched with torch.distributed.run")
+    if args.dry_run:
+        res = run_dry(args, rank, world, local)
+    elif args.impl == "reference":
+        res = run_reference(args, rank, world, local)
+    else:
+        res = run_cuda(args, rank, world, local)
+    if res is not None and rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

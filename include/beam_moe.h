@@ -1,0 +1,174 @@
+/*
+ * beam_moe.h -- C ABI of the B200 (sm_100a) forward pass of one Beam sparse-MoE layer.
+ *
+ * The layer (Transformers model doc "Beam", Overview, "Sparse MoE" bullet, and
+ * BeamConfig; archdb fact sheet "Beam-1.0-501B-A23B", expert-groups entry; news
+ * article "Reflection lança o Beam", section "Onde o Beam economiza ..."):
+ *
+ *   logits  = h . W_r^T                      FP32 router weights, FP32 logits
+ *   s       = sigmoid(logits)                FP32
+ *   sb      = s + bias                       bias chooses experts, never weighs them
+ *   gs_g    = top1(sb in g) + top2(sb in g)  groups are contiguous runs of E/n_group experts
+ *   keep the topk_group groups of largest gs, then the top_k experts of largest sb
+ *   among them (ties: lower group / expert index wins)
+ *   w       = routed_scaling_factor * s / sum(s over chosen)   (norm_topk_prob)
+ *   y_e     = W_down,e . ( silu(W_gate,e . h) * (W_up,e . h) )  SwiGLU in FP32, BF16 weights
+ *   out     = sum_j w_j y_{e_j}                no shared expert
+ *
+ * and its block form (Overview, "Sandwich norms with depth-scaled residuals"; archdb
+ * residual-design entry): h = RMSNorm(x) * g_pre (FP32, then BF16), the layer above,
+ * o = RMSNorm(out) * g_post, x' = x * sqrt((k-1)/k) + o / sqrt(k).
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device, owned by the
+ *    caller, row-major and dense.  The library allocates no device memory: scratch space
+ *    is the caller's workspace `ws` of at least beam_moe_workspace_size() bytes, aligned
+ *    to 256 bytes.  Tensor pointers must be 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (NULL = legacy default stream).  Argument errors
+ *    are returned before anything is launched; a failed launch returns BEAM_ERR_CUDA.
+ *    Errors found on the device (a bounded wait that ran out, a failed index check)
+ *    are recorded in a status word inside `ws` and read by beam_moe_sync_status().
+ *  - One workspace serves one call at a time: calls that share a workspace must be
+ *    ordered on one stream.
+ *  - Outputs topk_idx [T, top_k] list the chosen experts in ascending id order; topk_w
+ *    [T, top_k] holds their weights in the same order; the combine sums in that order,
+ *    so results are deterministic run to run.
+ *  - Supported shapes: d % 256 == 0, d <= 8192, I % 128 == 0, 1 <= E <= 256,
+ *    E % n_group == 0, n_group <= 32, 1 <= topk_group <= n_group, 1 <= top_k <= 8,
+ *    top_k <= topk_group * E / n_group, T >= 0, T * top_k < 2^31.  Others return
+ *    BEAM_ERR_UNSUPPORTED.  T == 0 is a no-op.
+ */
+#ifndef BEAM_MOE_H_
+#define BEAM_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BEAM_API __attribute__((visibility("default")))
+#else
+#define BEAM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BEAM_OK = 0,
+  BEAM_ERR_INVALID_ARG = 1,    /* NULL / misaligned pointer, bad scalar */
+  BEAM_ERR_UNSUPPORTED = 2,    /* shape outside the supported set */
+  BEAM_ERR_WORKSPACE = 3,      /* ws NULL, misaligned or smaller than required */
+  BEAM_ERR_CUDA = 4,           /* a CUDA runtime / driver call failed */
+  BEAM_ERR_TIMEOUT = 5,        /* a device-side bounded wait ran out (read by sync_status) */
+  BEAM_ERR_DEVICE_ASSERT = 6   /* a device-side index check failed (read by sync_status) */
+} beam_status;
+
+/* Layer configuration; field names follow BeamConfig. */
+typedef struct {
+  int32_t T;                    /* tokens in this call */
+  int32_t d;                    /* hidden_size (5120 for Beam) */
+  int32_t E;                    /* num_experts (256) */
+  int32_t n_group;              /* n_group (8) */
+  int32_t topk_group;           /* topk_group (4) */
+  int32_t top_k;                /* num_experts_per_tok (8) */
+  int32_t I;                    /* moe_intermediate_size (2560) */
+  float routed_scaling_factor;  /* 2.5 */
+  int32_t norm_topk_prob;       /* nonzero: weights normalised to sum 1 before scaling */
+} beam_moe_shape;
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* beam_stream;
+
+/* Bytes of workspace the given shape needs for route, forward or block (the maximum of
+ * the three); 0 if the shape is unsupported or NULL. */
+BEAM_API size_t beam_moe_workspace_size(const beam_moe_shape* shape);
+
+/* Router only: logits, sigmoid, bias, group-limited top-k, weights.
+ *   hidden     BF16 [T, d]
+ *   router_w   FP32 [E, d]
+ *   bias       FP32 [E]
+ *   topk_idx   INT32 [T, top_k] out, ascending expert id per token
+ *   topk_w     FP32 [T, top_k] out, weights aligned with topk_idx (sum = scale if normalised)
+ *   logits_out FP32 [T, E] out (the raw router logits), or NULL
+ * Cites: "Beam" model doc, Overview ("Sparse MoE" bullet, FP32 routing) and Notes
+ * ("output_router_logits=True still returns the router logits"). */
+BEAM_API beam_status beam_moe_route(const beam_moe_shape* shape, const void* hidden, const float* router_w,
+                           const float* bias, int32_t* topk_idx, float* topk_w, float* logits_out,
+                           void* ws, size_t ws_bytes, beam_stream stream);
+
+/* Whole MoE layer forward.
+ *   hidden           BF16 [T, d]
+ *   router_w, bias   as for beam_moe_route
+ *   w_gate, w_up     BF16 [E, I, d]  (per expert nn.Linear weight: out x in)
+ *   w_down           BF16 [E, d, I]
+ *   out              BF16 [T, d] out
+ *   topk_idx, topk_w optional outputs (NULL: kept inside ws)
+ * Cites: "Beam" model doc, Overview ("Sparse MoE" bullet; SwiGLU in FP32) and BeamConfig
+ * (moe_intermediate_size, num_experts_per_tok, routed_scaling_factor). */
+BEAM_API beam_status beam_moe_forward(const beam_moe_shape* shape, const void* hidden, const float* router_w,
+                             const float* bias, const void* w_gate, const void* w_up,
+                             const void* w_down, void* out, int32_t* topk_idx, float* topk_w,
+                             void* ws, size_t ws_bytes, beam_stream stream);
+
+/* MoE block: x' = x * sqrt((k_resid-1)/k_resid) + RMSNorm(MoE(bf16(RMSNorm(x) g_pre))) g_post
+ *                 / sqrt(k_resid), RMSNorm(v) = v / sqrt(mean(v^2) + eps), all FP32.
+ *   x       FP32 [T, d] residual stream in
+ *   g_pre, g_post FP32 [d]
+ *   eps     > 0 (rms_norm_eps, 1e-6 for Beam)
+ *   k_resid >= 1: index of this contribution in the residual stream (embedding = 1)
+ *   x_out   FP32 [T, d] out; may equal x (in place), must not otherwise overlap it
+ * Cites: "Beam" model doc, Overview ("Sandwich norms with depth-scaled residuals");
+ * archdb "Beam-1.0-501B-A23B", residual-design entry (FP32 residual accumulation). */
+BEAM_API beam_status beam_moe_block(const beam_moe_shape* shape, const float* x, const float* g_pre,
+                           const float* g_post, float eps, int32_t k_resid, const float* router_w,
+                           const float* bias, const void* w_gate, const void* w_up,
+                           const void* w_down, float* x_out, int32_t* topk_idx, float* topk_w,
+                           void* ws, size_t ws_bytes, beam_stream stream);
+
+/* Synchronises `stream`, reads and clears the device status word kept in `ws`, and
+ * returns BEAM_OK, BEAM_ERR_TIMEOUT or BEAM_ERR_DEVICE_ASSERT (or BEAM_ERR_CUDA if the
+ * stream itself reports an error).  `ws` must have been used with a call of this shape
+ * family (the status word sits at offset 0 of every workspace). */
+BEAM_API beam_status beam_moe_sync_status(void* ws, beam_stream stream);
+
+/* Human-readable name of a status code (static storage). */
+BEAM_API const char* beam_status_string(beam_status status);
+
+/* Text of the last CUDA error seen by this library on the calling thread, or "". */
+BEAM_API const char* beam_moe_last_cuda_error(void);
+
+/* Per-expert token counts of the last forward/block call that used `ws` (synchronises
+ * `stream` and copies E int32 values to the HOST buffer counts_host). */
+BEAM_API beam_status beam_moe_expert_counts(const beam_moe_shape* shape, const void* ws,
+                                   int32_t* counts_host, beam_stream stream);
+
+/* ---- diagnostics (process-wide settings) ---- */
+
+/* Limit, in nanoseconds, of every device-side wait in the expert GEMM kernels; after it
+ * the kernel records BEAM_ERR_TIMEOUT, drains its own copies, frees its tensor memory and
+ * returns.  Default 4e9 (4 s).  Applies to launches made after the call. */
+BEAM_API void beam_moe_set_wait_limit_ns(uint64_t ns);
+BEAM_API uint64_t beam_moe_get_wait_limit_ns(void);
+
+/* Total kernels this library has launched in this process. */
+BEAM_API uint64_t beam_moe_launch_count(void);
+
+/* Kernel timing: when enabled, every launch is bracketed by CUDA events on its stream.
+ * beam_moe_profile_read() synchronises those events and returns, for kernel `id`
+ * (0 <= id < beam_moe_kernel_count()), its launches and total milliseconds since the last
+ * reset; beam_moe_profile_reset() clears the counters. */
+BEAM_API void beam_moe_profile_enable(int on);
+BEAM_API void beam_moe_profile_reset(void);
+BEAM_API int beam_moe_kernel_count(void);
+BEAM_API const char* beam_moe_kernel_name(int id);
+BEAM_API beam_status beam_moe_profile_read(int id, int64_t* launches, double* total_ms);
+
+/* ABI version of this header (bumped on any incompatible change). */
+BEAM_API int beam_moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BEAM_MOE_H_ */

@@ -1,0 +1,268 @@
+"""Python binding of libbeam_moe.so (include/beam_moe.h): argument marshalling only.
+
+Every function here checks tensor devices, dtypes, shapes and contiguity, turns tensors
+into raw device pointers and the current torch stream into a cudaStream_t, and calls the C
+function of the same name.  All arithmetic runs in the library's CUDA kernels; if the
+library is missing this module raises instead of computing anything itself.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbeam_moe.so")
+
+BEAM_OK = 0
+BEAM_ERR_INVALID_ARG = 1
+BEAM_ERR_UNSUPPORTED = 2
+BEAM_ERR_WORKSPACE = 3
+BEAM_ERR_CUDA = 4
+BEAM_ERR_TIMEOUT = 5
+BEAM_ERR_DEVICE_ASSERT = 6
+
+EXPORTED = [
+    "beam_moe_workspace_size", "beam_moe_route", "beam_moe_forward", "beam_moe_block",
+    "beam_moe_sync_status", "beam_status_string", "beam_moe_last_cuda_error",
+    "beam_moe_expert_counts", "beam_moe_set_wait_limit_ns", "beam_moe_get_wait_limit_ns",
+    "beam_moe_launch_count", "beam_moe_profile_enable", "beam_moe_profile_reset",
+    "beam_moe_kernel_count", "beam_moe_kernel_name", "beam_moe_profile_read",
+    "beam_moe_abi_version",
+]
+
+
+class BeamError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: {status_string(status)}"
+        detail = last_cuda_error()
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+class beam_moe_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("routed_scaling_factor", ctypes.c_float), ("norm_topk_prob", ctypes.c_int32)]
+
+    def __repr__(self):
+        return "beam_moe_shape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def make_shape(T, d, E, n_group, topk_group, top_k, I, routed_scaling_factor=2.5,
+               norm_topk_prob=True) -> beam_moe_shape:
+    return beam_moe_shape(T, d, E, n_group, topk_group, top_k, I, routed_scaling_factor,
+                          1 if norm_topk_prob else 0)
+
+
+def shape_of(w, T: int | None = None) -> beam_moe_shape:
+    """Shape of a workloads.Workload (optionally with another token count)."""
+    return make_shape(w.T if T is None else T, w.d, w.E, w.n_group, w.topk_group, w.top_k, w.I,
+                      w.scale, w.norm_topk_prob)
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is not built: run "
+                           "`python -m sparse_moe_transformer_fp32_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, sz, i32, u64, f32 = (ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_uint64,
+                             ctypes.c_float)
+    shp = ctypes.POINTER(beam_moe_shape)
+    L.beam_moe_workspace_size.argtypes = [shp]
+    L.beam_moe_workspace_size.restype = sz
+    L.beam_moe_route.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.beam_moe_forward.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.beam_moe_block.argtypes = [shp, vp, vp, vp, f32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                 sz, vp]
+    L.beam_moe_sync_status.argtypes = [vp, vp]
+    L.beam_status_string.argtypes = [ctypes.c_int]
+    L.beam_status_string.restype = ctypes.c_char_p
+    L.beam_moe_last_cuda_error.restype = ctypes.c_char_p
+    L.beam_moe_expert_counts.argtypes = [shp, vp, vp, vp]
+    L.beam_moe_set_wait_limit_ns.argtypes = [u64]
+    L.beam_moe_get_wait_limit_ns.restype = u64
+    L.beam_moe_launch_count.restype = u64
+    L.beam_moe_profile_enable.argtypes = [ctypes.c_int]
+    L.beam_moe_kernel_name.argtypes = [ctypes.c_int]
+    L.beam_moe_kernel_name.restype = ctypes.c_char_p
+    L.beam_moe_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int64),
+                                        ctypes.POINTER(ctypes.c_double)]
+    for name in ("beam_moe_route", "beam_moe_forward", "beam_moe_block", "beam_moe_sync_status",
+                 "beam_moe_expert_counts", "beam_moe_profile_read"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().beam_status_string(int(status)).decode()
+
+
+def last_cuda_error() -> str:
+    return lib().beam_moe_last_cuda_error().decode()
+
+
+# ------------------------------------------------------------------ marshalling helpers
+
+def _ptr(t, dtype, name, shape=None, optional=False):
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} (got {t.dtype})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def beam_moe_workspace_size(shape: beam_moe_shape) -> int:
+    return int(lib().beam_moe_workspace_size(ctypes.byref(shape)))
+
+
+def workspace(shape: beam_moe_shape, device="cuda") -> torch.Tensor:
+    n = beam_moe_workspace_size(shape)
+    if n == 0:
+        raise BeamError(BEAM_ERR_UNSUPPORTED, "beam_moe_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _ws(shape, ws, device):
+    if ws is None:
+        ws = workspace(shape, device)
+    _ptr(ws, torch.uint8, "ws")
+    return ws
+
+
+def _check(status, where):
+    if status != BEAM_OK:
+        raise BeamError(status, where)
+
+
+# ------------------------------------------------------------------ entry points
+
+def beam_moe_route(shape, hidden, router_w, bias, topk_idx, topk_w, logits_out=None, ws=None,
+                   stream=None):
+    T, d, E, k = shape.T, shape.d, shape.E, shape.top_k
+    args = [_ptr(hidden, torch.bfloat16, "hidden", (T, d)),
+            _ptr(router_w, torch.float32, "router_w", (E, d)),
+            _ptr(bias, torch.float32, "bias", (E,)),
+            _ptr(topk_idx, torch.int32, "topk_idx", (T, k)),
+            _ptr(topk_w, torch.float32, "topk_w", (T, k)),
+            _ptr(logits_out, torch.float32, "logits_out", (T, E), optional=True)]
+    ws = _ws(shape, ws, hidden.device)
+    _check(lib().beam_moe_route(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
+                                _stream(stream)), "beam_moe_route")
+    return ws
+
+
+def beam_moe_forward(shape, hidden, router_w, bias, w_gate, w_up, w_down, out, topk_idx=None,
+                     topk_w=None, ws=None, stream=None):
+    T, d, E, k, I = shape.T, shape.d, shape.E, shape.top_k, shape.I
+    args = [_ptr(hidden, torch.bfloat16, "hidden", (T, d)),
+            _ptr(router_w, torch.float32, "router_w", (E, d)),
+            _ptr(bias, torch.float32, "bias", (E,)),
+            _ptr(w_gate, torch.bfloat16, "w_gate", (E, I, d)),
+            _ptr(w_up, torch.bfloat16, "w_up", (E, I, d)),
+            _ptr(w_down, torch.bfloat16, "w_down", (E, d, I)),
+            _ptr(out, torch.bfloat16, "out", (T, d)),
+            _ptr(topk_idx, torch.int32, "topk_idx", (T, k), optional=True),
+            _ptr(topk_w, torch.float32, "topk_w", (T, k), optional=True)]
+    ws = _ws(shape, ws, hidden.device)
+    _check(lib().beam_moe_forward(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
+                                  _stream(stream)), "beam_moe_forward")
+    return ws
+
+
+def beam_moe_block(shape, x, g_pre, g_post, eps, k_resid, router_w, bias, w_gate, w_up, w_down,
+                   x_out, topk_idx=None, topk_w=None, ws=None, stream=None):
+    T, d, E, k, I = shape.T, shape.d, shape.E, shape.top_k, shape.I
+    args = [_ptr(x, torch.float32, "x", (T, d)),
+            _ptr(g_pre, torch.float32, "g_pre", (d,)),
+            _ptr(g_post, torch.float32, "g_post", (d,)),
+            ctypes.c_float(eps), ctypes.c_int32(k_resid),
+            _ptr(router_w, torch.float32, "router_w", (E, d)),
+            _ptr(bias, torch.float32, "bias", (E,)),
+            _ptr(w_gate, torch.bfloat16, "w_gate", (E, I, d)),
+            _ptr(w_up, torch.bfloat16, "w_up", (E, I, d)),
+            _ptr(w_down, torch.bfloat16, "w_down", (E, d, I)),
+            _ptr(x_out, torch.float32, "x_out", (T, d)),
+            _ptr(topk_idx, torch.int32, "topk_idx", (T, k), optional=True),
+            _ptr(topk_w, torch.float32, "topk_w", (T, k), optional=True)]
+    ws = _ws(shape, ws, x.device)
+    _check(lib().beam_moe_block(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
+                                _stream(stream)), "beam_moe_block")
+    return ws
+
+
+def beam_moe_sync_status(ws, stream=None) -> int:
+    """Synchronises and returns the device status code of the latest call on ``ws``."""
+    return int(lib().beam_moe_sync_status(_ptr(ws, torch.uint8, "ws"), _stream(stream)))
+
+
+def beam_moe_expert_counts(shape, ws, stream=None) -> torch.Tensor:
+    out = torch.empty(shape.E, dtype=torch.int32)
+    _check(lib().beam_moe_expert_counts(ctypes.byref(shape), _ptr(ws, torch.uint8, "ws"),
+                                        out.data_ptr(), _stream(stream)), "beam_moe_expert_counts")
+    return out
+
+
+def beam_moe_set_wait_limit_ns(ns: int) -> None:
+    lib().beam_moe_set_wait_limit_ns(int(ns))
+
+
+def beam_moe_get_wait_limit_ns() -> int:
+    return int(lib().beam_moe_get_wait_limit_ns())
+
+
+def beam_moe_launch_count() -> int:
+    return int(lib().beam_moe_launch_count())
+
+
+def beam_moe_profile_enable(on: bool) -> None:
+    lib().beam_moe_profile_enable(1 if on else 0)
+
+
+def beam_moe_profile_reset() -> None:
+    lib().beam_moe_profile_reset()
+
+
+def kernel_names():
+    L = lib()
+    return [L.beam_moe_kernel_name(i).decode() for i in range(L.beam_moe_kernel_count())]
+
+
+def beam_moe_profile_read():
+    """{kernel name: (launches, total ms)} since the last reset."""
+    L = lib()
+    out = {}
+    for i, name in enumerate(kernel_names()):
+        n, ms = ctypes.c_int64(), ctypes.c_double()
+        _check(L.beam_moe_profile_read(i, ctypes.byref(n), ctypes.byref(ms)), "beam_moe_profile_read")
+        out[name] = (n.value, ms.value)
+    return out

@@ -1,0 +1,577 @@
+// C ABI of the Beam MoE layer (declared in include/beam_moe.h): argument checks, workspace
+// layout, TMA tensor maps, kernel launch sequence, device status, launch counting and timing.
+#include "beam_moe.h"
+#include "beam_moe_internal.cuh"
+
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+namespace {
+
+using namespace beam;
+
+std::atomic<uint64_t> g_wait_limit_ns{4000000000ull};
+std::atomic<uint64_t> g_launches{0};
+thread_local char g_last_cuda_error[256] = "";
+
+// ------------------------------------------------------------------ kernel ids and timing
+
+enum KernelId {
+  kKRouterGemm = 0,
+  kKRouterSelect,
+  kKDispatchScan,
+  kKPermute,
+  kKGemmGateUp,
+  kKGemmDown,
+  kKCombine,
+  kKCombineBlock,
+  kKPreNorm,
+  kNumKernels
+};
+const char* const kKernelNames[kNumKernels] = {
+    "router_gemm", "router_select", "dispatch_scan", "permute", "expert_gemm_gate_up",
+    "expert_gemm_down", "combine", "combine_block", "prenorm"};
+
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  struct Rec {
+    int id;
+    cudaEvent_t a, b;
+  };
+  std::vector<Rec> pending;
+  std::vector<cudaEvent_t> pool;
+  int64_t launches[kNumKernels] = {};
+  double ms[kNumKernels] = {};
+
+  cudaEvent_t take() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+Profiler g_prof;
+
+struct ProfScope {
+  int id;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  ProfScope(int id_, cudaStream_t s_) : id(id_), s(s_) {
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    if (!g_prof.on) return;
+    a = g_prof.take();
+    cudaEventRecord(a, s);
+  }
+  ~ProfScope() {
+    if (!a) return;
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    cudaEvent_t b = g_prof.take();
+    cudaEventRecord(b, s);
+    g_prof.pending.push_back({id, a, b});
+  }
+};
+
+beam_status cuda_fail(cudaError_t e) {
+  std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return BEAM_ERR_CUDA;
+}
+
+#define BEAM_LAUNCH(id, stream, call)                 \
+  do {                                                \
+    cudaError_t err_;                                 \
+    {                                                 \
+      ProfScope ps_(id, stream);                      \
+      err_ = (call);                                  \
+    }                                                 \
+    if (err_ != cudaSuccess) return cuda_fail(err_);  \
+    g_launches.fetch_add(1, std::memory_order_relaxed); \
+  } while (0)
+
+// ------------------------------------------------------------------ shapes and workspace
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+beam_status check_shape(const beam_moe_shape* s) {
+  if (!s) return BEAM_ERR_INVALID_ARG;
+  if (s->T < 0 || s->d <= 0 || s->E <= 0 || s->n_group <= 0 || s->topk_group <= 0 ||
+      s->top_k <= 0 || s->I <= 0)
+    return BEAM_ERR_INVALID_ARG;
+  if (!std::isfinite(s->routed_scaling_factor)) return BEAM_ERR_INVALID_ARG;
+  if (s->d % 256 != 0 || s->d > kMaxD) return BEAM_ERR_UNSUPPORTED;
+  if (s->I % 128 != 0 || s->I > 65536) return BEAM_ERR_UNSUPPORTED;
+  if (s->E > kMaxE || s->E % s->n_group != 0 || s->n_group > kMaxGroups)
+    return BEAM_ERR_UNSUPPORTED;
+  if (s->topk_group > s->n_group || s->top_k > kMaxTopK) return BEAM_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(s->top_k) > static_cast<int64_t>(s->topk_group) * (s->E / s->n_group))
+    return BEAM_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(s->T) * s->top_k >= (int64_t(1) << 31)) return BEAM_ERR_UNSUPPORTED;
+  return BEAM_OK;
+}
+
+struct Layout {
+  size_t status, cnt, off, mt_count, mtiles, rank, rowmap, idx, w, part, h, xp, act, y, total;
+  int S, kchunk;
+  int64_t R, mt_cap;
+};
+
+// Router split-K: enough (token tile, expert tile, K chunk) blocks to cover two waves of the
+// 148 SMs, K chunks a multiple of the router's K step.
+Layout plan(const beam_moe_shape& s) {
+  Layout L{};
+  const int64_t T = s.T, R = T * s.top_k;
+  L.R = R;
+  const int64_t tiles = ceil_div(T, kRM) * ceil_div(s.E, kRN);
+  const int64_t want = ceil_div(2 * 148, tiles > 0 ? tiles : 1);
+  const int64_t kblocks = s.d / kRK;
+  const int64_t S0 = want < 1 ? 1 : (want > s.d / 256 ? s.d / 256 : want);
+  const int64_t per = ceil_div(kblocks, S0);
+  L.kchunk = static_cast<int>(per * kRK);
+  L.S = static_cast<int>(ceil_div(s.d, L.kchunk));
+  L.mt_cap = ceil_div(R, kBM) + s.E;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o = align_up(o + (bytes ? bytes : 1), 1024);
+    return r;
+  };
+  L.status = take(256);
+  L.cnt = take(sizeof(int32_t) * s.E);
+  L.off = take(sizeof(int32_t) * (s.E + 1));
+  L.mt_count = take(16);
+  L.mtiles = take(sizeof(MTile) * L.mt_cap);
+  L.rank = take(sizeof(int32_t) * R);
+  L.rowmap = take(sizeof(int32_t) * R);
+  L.idx = take(sizeof(int32_t) * R);
+  L.w = take(sizeof(float) * R);
+  L.part = take(sizeof(float) * static_cast<size_t>(L.S) * T * s.E);
+  L.h = take(sizeof(__nv_bfloat16) * T * s.d);
+  L.xp = take(sizeof(__nv_bfloat16) * R * s.d);
+  L.act = take(sizeof(__nv_bfloat16) * R * s.I);
+  L.y = take(sizeof(__nv_bfloat16) * R * s.d);
+  L.total = o;
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+beam_status check_ws(const Layout& L, void* ws, size_t ws_bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < L.total)
+    return BEAM_ERR_WORKSPACE;
+  return BEAM_OK;
+}
+
+// ------------------------------------------------------------------ TMA tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D BF16 view [outer, inner] (inner contiguous), box [box_outer, 64] with 128-byte swizzle;
+// rows past `outer` read as zeros.
+beam_status make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                     uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return cuda_fail(cudaErrorNotSupported);
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_outer};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled: %d",
+                  static_cast<int>(r));
+    return BEAM_ERR_CUDA;
+  }
+  return BEAM_OK;
+}
+
+// ------------------------------------------------------------------ per-device state
+
+struct DeviceInfo {
+  int sms = 0;
+  bool prepared = false;
+};
+
+beam_status device_info(DeviceInfo** out) {
+  static DeviceInfo info[64];
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= 64) return BEAM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  DeviceInfo& d = info[dev];
+  if (!d.prepared) {
+    e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = prepare_gemm_kernels();
+    if (e != cudaSuccess) return cuda_fail(e);
+    d.prepared = true;
+  }
+  *out = &d;
+  return BEAM_OK;
+}
+
+// ------------------------------------------------------------------ launch sequences
+
+// Router: logits partials, then selection (+ counts and ranks when dispatching).
+beam_status run_router(const beam_moe_shape& s, const Layout& L, const __nv_bfloat16* h,
+                       const float* router_w, const float* bias, int32_t* idx, float* w,
+                       float* logits_out, bool dispatch, void* ws, cudaStream_t st) {
+  RouterGemmArgs ga{};
+  ga.h = h;
+  ga.W = router_w;
+  ga.part = at<float>(ws, L.part);
+  ga.zero_counts = at<int32_t>(ws, L.cnt);
+  ga.T = s.T;
+  ga.d = s.d;
+  ga.E = s.E;
+  ga.kchunk = L.kchunk;
+  // the status words reflect the latest call: cleared before the first kernel runs
+  cudaError_t e = cudaMemsetAsync(at<uint32_t>(ws, L.status), 0, 16, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  BEAM_LAUNCH(kKRouterGemm, st, launch_router_gemm(ga, L.S, st));
+
+  SelectArgs sa{};
+  sa.part = ga.part;
+  sa.bias = bias;
+  sa.logits_out = logits_out;
+  sa.idx = idx;
+  sa.w = w;
+  sa.cnt = dispatch ? at<int32_t>(ws, L.cnt) : nullptr;
+  sa.rank = dispatch ? at<int32_t>(ws, L.rank) : nullptr;
+  sa.status = at<uint32_t>(ws, L.status);
+  sa.S = L.S;
+  sa.T = s.T;
+  sa.E = s.E;
+  sa.G = s.n_group;
+  sa.Gk = s.topk_group;
+  sa.k = s.top_k;
+  sa.scale = s.routed_scaling_factor;
+  sa.norm = s.norm_topk_prob ? 1 : 0;
+  BEAM_LAUNCH(kKRouterSelect, st, launch_router_select(sa, st));
+  return BEAM_OK;
+}
+
+// Dispatch, the two expert GEMMs; leaves Y and rowmap in the workspace.
+beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceInfo& dev,
+                        const __nv_bfloat16* h, const int32_t* idx, const void* w_gate,
+                        const void* w_up, const void* w_down, void* ws, cudaStream_t st) {
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  DispatchArgs da{};
+  da.cnt = at<int32_t>(ws, L.cnt);
+  da.off = at<int32_t>(ws, L.off);
+  da.mt_count = at<int32_t>(ws, L.mt_count);
+  da.mtiles = at<MTile>(ws, L.mtiles);
+  da.E = s.E;
+  BEAM_LAUNCH(kKDispatchScan, st, launch_dispatch_scan(da, st));
+
+  PermuteArgs pa{};
+  pa.h = h;
+  pa.idx = idx;
+  pa.rank = at<int32_t>(ws, L.rank);
+  pa.off = da.off;
+  pa.rowmap = at<int32_t>(ws, L.rowmap);
+  pa.xp = at<__nv_bfloat16>(ws, L.xp);
+  pa.status = status;
+  pa.T = s.T;
+  pa.d = s.d;
+  pa.k = s.top_k;
+  pa.E = s.E;
+  BEAM_LAUNCH(kKPermute, st, launch_permute(pa, st));
+
+  const uint64_t R = static_cast<uint64_t>(L.R);
+  CUtensorMap tm_xp, tm_g, tm_u, tm_act, tm_d;
+  beam_status b;
+  if ((b = make_map(&tm_xp, pa.xp, s.d, R, kBM)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_g, w_gate, s.d, static_cast<uint64_t>(s.E) * s.I, kN1Half)) != BEAM_OK)
+    return b;
+  if ((b = make_map(&tm_u, w_up, s.d, static_cast<uint64_t>(s.E) * s.I, kN1Half)) != BEAM_OK)
+    return b;
+  if ((b = make_map(&tm_act, at<void>(ws, L.act), s.I, R, kBM)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_d, w_down, s.I, static_cast<uint64_t>(s.E) * s.d, kN2)) != BEAM_OK)
+    return b;
+
+  const uint64_t limit = g_wait_limit_ns.load(std::memory_order_relaxed);
+  GemmArgs g1{};
+  g1.mtiles = da.mtiles;
+  g1.mt_count = da.mt_count;
+  g1.out = at<__nv_bfloat16>(ws, L.act);
+  g1.status = status;
+  g1.wait_limit_ns = limit;
+  g1.out_ld = s.I;
+  g1.n_tiles_n = s.I / kN1Half;
+  g1.k_blocks = s.d / kBK;
+  g1.b_rows_per_expert = s.I;
+  const int64_t max_tiles1 = L.mt_cap * g1.n_tiles_n;
+  const int grid1 = static_cast<int>(max_tiles1 < dev.sms ? max_tiles1 : dev.sms);
+  BEAM_LAUNCH(kKGemmGateUp, st, launch_gemm_gate_up(tm_xp, tm_g, tm_u, g1, grid1, st));
+
+  GemmArgs g2 = g1;
+  g2.out = at<__nv_bfloat16>(ws, L.y);
+  g2.out_ld = s.d;
+  g2.n_tiles_n = s.d / kN2;
+  g2.k_blocks = s.I / kBK;
+  g2.b_rows_per_expert = s.d;
+  const int64_t max_tiles2 = L.mt_cap * g2.n_tiles_n;
+  const int grid2 = static_cast<int>(max_tiles2 < dev.sms ? max_tiles2 : dev.sms);
+  BEAM_LAUNCH(kKGemmDown, st, launch_gemm_down(tm_act, tm_d, g2, grid2, st));
+  return BEAM_OK;
+}
+
+bool any_misaligned(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (!p || !aligned16(p)) return true;
+  return false;
+}
+
+}  // namespace
+
+extern "C" {
+
+int beam_moe_abi_version(void) { return 1; }
+
+size_t beam_moe_workspace_size(const beam_moe_shape* shape) {
+  if (check_shape(shape) != BEAM_OK) return 0;
+  return plan(*shape).total;
+}
+
+const char* beam_status_string(beam_status s) {
+  switch (s) {
+    case BEAM_OK: return "BEAM_OK";
+    case BEAM_ERR_INVALID_ARG: return "BEAM_ERR_INVALID_ARG";
+    case BEAM_ERR_UNSUPPORTED: return "BEAM_ERR_UNSUPPORTED";
+    case BEAM_ERR_WORKSPACE: return "BEAM_ERR_WORKSPACE";
+    case BEAM_ERR_CUDA: return "BEAM_ERR_CUDA";
+    case BEAM_ERR_TIMEOUT: return "BEAM_ERR_TIMEOUT";
+    case BEAM_ERR_DEVICE_ASSERT: return "BEAM_ERR_DEVICE_ASSERT";
+  }
+  return "BEAM_ERR_UNKNOWN";
+}
+
+const char* beam_moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+void beam_moe_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+uint64_t beam_moe_get_wait_limit_ns(void) { return g_wait_limit_ns.load(); }
+uint64_t beam_moe_launch_count(void) { return g_launches.load(); }
+
+beam_status beam_moe_route(const beam_moe_shape* shape, const void* hidden, const float* router_w,
+                           const float* bias, int32_t* topk_idx, float* topk_w, float* logits_out,
+                           void* ws, size_t ws_bytes, beam_stream stream) {
+  beam_status b = check_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (any_misaligned({hidden, router_w, topk_idx, topk_w}) || !bias ||
+      (logits_out && !aligned16(logits_out)))
+    return BEAM_ERR_INVALID_ARG;
+  const Layout L = plan(*shape);
+  if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;
+  DeviceInfo* dev;
+  if ((b = device_info(&dev)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return run_router(*shape, L, static_cast<const __nv_bfloat16*>(hidden), router_w, bias, topk_idx,
+                    topk_w, logits_out, false, ws, st);
+}
+
+beam_status beam_moe_forward(const beam_moe_shape* shape, const void* hidden, const float* router_w,
+                             const float* bias, const void* w_gate, const void* w_up,
+                             const void* w_down, void* out, int32_t* topk_idx, float* topk_w,
+                             void* ws, size_t ws_bytes, beam_stream stream) {
+  beam_status b = check_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (any_misaligned({hidden, router_w, w_gate, w_up, w_down, out}) || !bias ||
+      (topk_idx && !aligned16(topk_idx)) || (topk_w && !aligned16(topk_w)))
+    return BEAM_ERR_INVALID_ARG;
+  const Layout L = plan(*shape);
+  if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;
+  DeviceInfo* dev;
+  if ((b = device_info(&dev)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
+  float* w = topk_w ? topk_w : at<float>(ws, L.w);
+  const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(hidden);
+  if ((b = run_router(*shape, L, h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
+    return b;
+  if ((b = run_experts(*shape, L, *dev, h, idx, w_gate, w_up, w_down, ws, st)) != BEAM_OK)
+    return b;
+  CombineArgs ca{};
+  ca.y = at<__nv_bfloat16>(ws, L.y);
+  ca.rowmap = at<int32_t>(ws, L.rowmap);
+  ca.w = w;
+  ca.out = static_cast<__nv_bfloat16*>(out);
+  ca.status = at<uint32_t>(ws, L.status);
+  ca.T = shape->T;
+  ca.d = shape->d;
+  ca.k = shape->top_k;
+  ca.R = static_cast<int>(L.R);
+  BEAM_LAUNCH(kKCombine, st, launch_combine(ca, st));
+  return BEAM_OK;
+}
+
+beam_status beam_moe_block(const beam_moe_shape* shape, const float* x, const float* g_pre,
+                           const float* g_post, float eps, int32_t k_resid, const float* router_w,
+                           const float* bias, const void* w_gate, const void* w_up,
+                           const void* w_down, float* x_out, int32_t* topk_idx, float* topk_w,
+                           void* ws, size_t ws_bytes, beam_stream stream) {
+  beam_status b = check_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (any_misaligned({x, g_pre, g_post, router_w, w_gate, w_up, w_down, x_out}) || !bias ||
+      (topk_idx && !aligned16(topk_idx)) || (topk_w && !aligned16(topk_w)))
+    return BEAM_ERR_INVALID_ARG;
+  if (!(eps > 0.f) || !std::isfinite(eps) || k_resid < 1) return BEAM_ERR_INVALID_ARG;
+  if (x_out != x) {  // in place or disjoint
+    const char* a0 = reinterpret_cast<const char*>(x);
+    const char* b0 = reinterpret_cast<const char*>(x_out);
+    const size_t n = sizeof(float) * static_cast<size_t>(shape->T) * shape->d;
+    if (a0 < b0 + n && b0 < a0 + n) return BEAM_ERR_INVALID_ARG;
+  }
+  const Layout L = plan(*shape);
+  if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;
+  DeviceInfo* dev;
+  if ((b = device_info(&dev)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  PreNormArgs pn{};
+  pn.x = x;
+  pn.g_pre = g_pre;
+  pn.h = at<__nv_bfloat16>(ws, L.h);
+  pn.eps = eps;
+  pn.T = shape->T;
+  pn.d = shape->d;
+  BEAM_LAUNCH(kKPreNorm, st, launch_prenorm(pn, st));
+
+  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
+  float* w = topk_w ? topk_w : at<float>(ws, L.w);
+  if ((b = run_router(*shape, L, pn.h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
+    return b;
+  if ((b = run_experts(*shape, L, *dev, pn.h, idx, w_gate, w_up, w_down, ws, st)) != BEAM_OK)
+    return b;
+  const double kk = static_cast<double>(k_resid);
+  CombineArgs ca{};
+  ca.y = at<__nv_bfloat16>(ws, L.y);
+  ca.rowmap = at<int32_t>(ws, L.rowmap);
+  ca.w = w;
+  ca.x = x;
+  ca.g_post = g_post;
+  ca.x_out = x_out;
+  ca.eps = eps;
+  ca.coef_x = static_cast<float>(std::sqrt((kk - 1.0) / kk));
+  ca.coef_f = static_cast<float>(1.0 / std::sqrt(kk));
+  ca.status = at<uint32_t>(ws, L.status);
+  ca.T = shape->T;
+  ca.d = shape->d;
+  ca.k = shape->top_k;
+  ca.R = static_cast<int>(L.R);
+  BEAM_LAUNCH(kKCombineBlock, st, launch_combine_block(ca, st));
+  return BEAM_OK;
+}
+
+beam_status beam_moe_sync_status(void* ws, beam_stream stream) {
+  if (!ws) return BEAM_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  uint32_t words[4] = {0, 0, 0, 0};
+  e = cudaMemcpy(words, ws, sizeof words, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (words[0] == kDevOk) return BEAM_OK;
+  std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,
+                "device status %u at site %u, block %u", words[0], words[1], words[2]);
+  e = cudaMemset(ws, 0, sizeof words);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return words[0] == kDevTimeout ? BEAM_ERR_TIMEOUT : BEAM_ERR_DEVICE_ASSERT;
+}
+
+beam_status beam_moe_expert_counts(const beam_moe_shape* shape, const void* ws,
+                                   int32_t* counts_host, beam_stream stream) {
+  beam_status b = check_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (!ws || !counts_host) return BEAM_ERR_INVALID_ARG;
+  const Layout L = plan(*shape);
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaMemcpy(counts_host, static_cast<const char*>(ws) + L.cnt, sizeof(int32_t) * shape->E,
+                 cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return BEAM_OK;
+}
+
+void beam_moe_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  g_prof.on = on != 0;
+}
+
+void beam_moe_profile_reset(void) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  for (auto& r : g_prof.pending) {
+    cudaEventSynchronize(r.b);
+    g_prof.pool.push_back(r.a);
+    g_prof.pool.push_back(r.b);
+  }
+  g_prof.pending.clear();
+  for (int i = 0; i < kNumKernels; ++i) {
+    g_prof.launches[i] = 0;
+    g_prof.ms[i] = 0.0;
+  }
+}
+
+int beam_moe_kernel_count(void) { return kNumKernels; }
+
+const char* beam_moe_kernel_name(int id) {
+  return id >= 0 && id < kNumKernels ? kKernelNames[id] : "";
+}
+
+beam_status beam_moe_profile_read(int id, int64_t* launches, double* total_ms) {
+  if (id < 0 || id >= kNumKernels || !launches || !total_ms) return BEAM_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  for (auto& r : g_prof.pending) {
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e != cudaSuccess) return cuda_fail(e);
+    float ms = 0.f;
+    e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_prof.launches[r.id] += 1;
+    g_prof.ms[r.id] += ms;
+    g_prof.pool.push_back(r.a);
+    g_prof.pool.push_back(r.b);
+  }
+  g_prof.pending.clear();
+  *launches = g_prof.launches[id];
+  *total_ms = g_prof.ms[id];
+  return BEAM_OK;
+}
+
+}  // extern "C"

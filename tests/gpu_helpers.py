@@ -1,0 +1,164 @@
+"""Shared pieces of the GPU parity tests: inputs with near ties removed (decided by the
+oracle), runs of the CUDA path through the C ABI, and oracle references for sampled tokens.
+
+Nothing here feeds a value computed by the CUDA path into the oracle: inputs come from
+sparse_moe_transformer_fp32_b200.workloads (weights drawn on the GPU and copied to the host
+byte for byte), and every expected value is computed by the oracle from those inputs.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+import oracle
+from sparse_moe_transformer_fp32_b200 import beam_moe as bm
+from sparse_moe_transformer_fp32_b200 import workloads as W
+
+# Near-tie margin in biased-score units.  The CUDA router sums FP32 products in another order
+# than the oracle's double sum (|difference| ~1e-6 in a logit for d = 5120); a selection whose
+# margin is below DELTA is re-drawn so that the chosen set is unique at FP32 accuracy.
+DELTA = 1e-4
+DELTA_BLOCK = 1e-3  # the block's BF16 rounding of the normed input may differ by one ulp
+
+
+def rel_l2(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def assert_close_out(got, ref, what=""):
+    """Output tolerance: relative L2 <= 1e-2 and max |err| <= 5e-2 * RMS(ref)."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    r = rel_l2(got, ref)
+    m = float(np.max(np.abs(got - ref)))
+    assert r <= 1e-2, f"{what}: relative L2 {r:.3e} > 1e-2"
+    assert m <= 5e-2 * rms, f"{what}: max abs {m:.3e} > 5e-2 * RMS {rms:.3e}"
+    return r, m / rms
+
+
+@dataclasses.dataclass
+class Case:
+    wl: W.Workload
+    h: torch.Tensor          # BF16 [T, d] CPU (layer) -- oracle's normed input for the block
+    router_w: torch.Tensor   # FP32 [E, d] CPU
+    bias: torch.Tensor       # FP32 [E] CPU
+    idx: np.ndarray          # oracle routing
+    w: np.ndarray
+    logits: np.ndarray
+    resampled: int
+    x: torch.Tensor | None = None       # FP32 [T, d] CPU (block)
+    g_pre: torch.Tensor | None = None
+    g_post: torch.Tensor | None = None
+
+
+def make_case(wl: W.Workload, max_attempts: int = 64) -> Case:
+    """Inputs of workload ``wl`` with every near-tie token re-drawn (counter attempt+1)."""
+    router_w = W.router_weight(wl)
+    bias = W.router_bias(wl)
+    x = g_pre = g_post = None
+    if wl.block:
+        x = W.residual_x(wl)
+        g_pre, g_post = W.norm_gains(wl)
+        h = torch.from_numpy(oracle.block_prenorm(x, g_pre, wl.eps).view(np.int16)).view(torch.bfloat16)
+        delta = DELTA_BLOCK
+    else:
+        h = W.hidden(wl)
+        delta = DELTA
+    resampled = 0
+    rows = np.arange(wl.T)
+    logits = np.empty((wl.T, wl.E), np.float32)
+    idx = np.empty((wl.T, wl.top_k), np.int32)
+    w = np.empty((wl.T, wl.top_k), np.float32)
+    attempt = np.zeros(wl.T, np.int64)
+    for _ in range(max_attempts + 1):
+        L, ix, ww, me, mg = oracle.layer_routing(h[rows], router_w, bias, wl)
+        logits[rows], idx[rows], w[rows] = L, ix, ww
+        bad = rows[(me < delta) | (mg < delta)]
+        if len(bad) == 0:
+            break
+        resampled += len(bad)
+        for t in bad:
+            attempt[t] += 1
+            if wl.block:
+                x[t] = W.residual_row(wl, int(t), int(attempt[t]))
+                nb = oracle.block_prenorm(x[t:t + 1], g_pre, wl.eps).view(np.int16)
+                h[t] = torch.from_numpy(nb[0]).view(torch.bfloat16)
+            else:
+                h[t] = W.hidden_row(wl, int(t), int(attempt[t]))
+        rows = bad
+    else:
+        raise RuntimeError("could not remove near ties")
+    return Case(wl, h, router_w, bias, idx, w, logits, resampled, x, g_pre, g_post)
+
+
+def device_weights(wl: W.Workload, identical: bool = False):
+    """Expert weights drawn on the GPU (bytes shared with the oracle by copying to host)."""
+    if identical:
+        g = W.expert_weight(wl, "gate", 0, "cuda")
+        u = W.expert_weight(wl, "up", 0, "cuda")
+        d = W.expert_weight(wl, "down", 0, "cuda")
+        return (g.expand(wl.E, -1, -1).contiguous(), u.expand(wl.E, -1, -1).contiguous(),
+                d.expand(wl.E, -1, -1).contiguous())
+    return W.expert_weights(wl, "cuda")
+
+
+def run_forward(case: Case, weights, ws=None):
+    wl = case.wl
+    s = bm.shape_of(wl)
+    dev = "cuda"
+    out = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(wl.T, wl.top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(wl.T, wl.top_k, dtype=torch.float32, device=dev)
+    ws = bm.beam_moe_forward(s, case.h.to(dev), case.router_w.to(dev), case.bias.to(dev),
+                             *weights, out, idx, w, ws=ws)
+    st = bm.beam_moe_sync_status(ws)
+    assert st == bm.BEAM_OK, bm.status_string(st)
+    return out, idx, w, ws
+
+
+def run_block(case: Case, weights, in_place=False):
+    wl = case.wl
+    s = bm.shape_of(wl)
+    dev = "cuda"
+    x = case.x.to(dev)
+    x_out = x if in_place else torch.empty_like(x)
+    idx = torch.empty(wl.T, wl.top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(wl.T, wl.top_k, dtype=torch.float32, device=dev)
+    ws = bm.beam_moe_block(s, x, case.g_pre.to(dev), case.g_post.to(dev), wl.eps, wl.k_resid,
+                           case.router_w.to(dev), case.bias.to(dev), *weights, x_out, idx, w)
+    st = bm.beam_moe_sync_status(ws)
+    assert st == bm.BEAM_OK, bm.status_string(st)
+    return x_out, idx, w, ws
+
+
+def oracle_out(case: Case, weights, tokens, batch: int = 4):
+    """Oracle MoE output (FP32) for ``tokens``, copying only the experts each batch uses."""
+    tokens = list(tokens)
+    out = np.empty((len(tokens), case.wl.d), np.float32)
+    for b0 in range(0, len(tokens), batch):
+        tb = tokens[b0:b0 + batch]
+        ex = sorted({int(e) for t in tb for e in case.idx[t]})
+        experts = {e: tuple(m[e].cpu() for m in weights) for e in ex}
+        out[b0:b0 + len(tb)] = oracle.moe_tokens(tb, case.h, case.idx, case.w, experts)
+    return out
+
+
+def sample_tokens(case: Case, n: int, seed: int = 0):
+    """First, last and random tokens, plus tokens of the most loaded expert."""
+    T = case.wl.T
+    rng = np.random.default_rng(seed)
+    picks = {0, T - 1}
+    counts = np.bincount(case.idx.reshape(-1), minlength=case.wl.E)
+    hot = int(np.argmax(counts))
+    hot_tokens = np.nonzero((case.idx == hot).any(axis=1))[0]
+    if len(hot_tokens):
+        picks.update(rng.choice(hot_tokens, size=min(2, len(hot_tokens)), replace=False).tolist())
+    while len(picks) < min(n, T):
+        picks.add(int(rng.integers(0, T)))
+    return sorted(picks)

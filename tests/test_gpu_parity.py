@@ -1,0 +1,187 @@
+"""Parity of the CUDA path (called through the C ABI) with the CPU oracle.
+
+Routing indices must match bit-exactly (inputs have near ties removed); outputs must be within
+relative L2 1e-2 and max |err| 5e-2 * RMS of the oracle's.  Small cases are compared on every
+token; the full-size workloads are compared on every token's routing and on sampled tokens'
+outputs, in the same launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_moe_transformer_fp32_b200 import beam_moe as bm
+from sparse_moe_transformer_fp32_b200 import workloads as W
+from tests import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    from sparse_moe_transformer_fp32_b200 import build
+    build.build()
+    bm.lib()
+    yield
+    torch.cuda.empty_cache()
+
+
+def _check_routing(case, idx, w):
+    idx = idx.cpu().numpy()
+    assert np.array_equal(idx, case.idx), np.argwhere(idx != case.idx)[:5]
+    np.testing.assert_allclose(w.cpu().numpy(), case.w, rtol=2e-6, atol=1e-7)
+
+
+# ------------------------------------------------------------------ small cases, every token
+
+def test_route_tiny_with_logits():
+    case = H.make_case(W.WORKLOADS["tiny"])
+    wl = case.wl
+    s = bm.shape_of(wl)
+    idx = torch.empty(wl.T, wl.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(wl.T, wl.top_k, dtype=torch.float32, device="cuda")
+    logits = torch.empty(wl.T, wl.E, dtype=torch.float32, device="cuda")
+    ws = bm.beam_moe_route(s, case.h.cuda(), case.router_w.cuda(), case.bias.cuda(), idx, w, logits)
+    assert bm.beam_moe_sync_status(ws) == bm.BEAM_OK
+    _check_routing(case, idx, w)
+    np.testing.assert_allclose(logits.cpu().numpy(), case.logits, rtol=1e-5, atol=2e-6)
+
+
+def test_forward_tiny_every_token():
+    case = H.make_case(W.WORKLOADS["tiny"])
+    weights = H.device_weights(case.wl)
+    out, idx, w, _ = H.run_forward(case, weights)
+    _check_routing(case, idx, w)
+    ref = H.oracle_out(case, weights, range(case.wl.T), batch=64)
+    H.assert_close_out(out.float().cpu().numpy(), ref, "tiny")
+
+
+@pytest.mark.parametrize("T", [1, 2, 7, 33, 129, 300])
+def test_forward_ragged_token_counts(T):
+    case = H.make_case(W.WORKLOADS["tiny"].with_tokens(T))
+    weights = H.device_weights(case.wl)
+    out, idx, w, _ = H.run_forward(case, weights)
+    _check_routing(case, idx, w)
+    ref = H.oracle_out(case, weights, range(T), batch=64)
+    H.assert_close_out(out.float().cpu().numpy(), ref, f"tiny T={T}")
+
+
+def test_forward_unnormalised_weights():
+    wl = W.WORKLOADS["tiny"]
+    import dataclasses
+    wl = dataclasses.replace(wl, norm_topk_prob=False)
+    case = H.make_case(wl)
+    weights = H.device_weights(wl)
+    out, idx, w, _ = H.run_forward(case, weights)
+    _check_routing(case, idx, w)
+    ref = H.oracle_out(case, weights, range(wl.T), batch=64)
+    H.assert_close_out(out.float().cpu().numpy(), ref, "unnormalised")
+
+
+def test_forward_deterministic_and_workspace_reuse():
+    case = H.make_case(W.WORKLOADS["tiny"].with_tokens(200))
+    weights = H.device_weights(case.wl)
+    big = bm.workspace(bm.shape_of(case.wl.with_tokens(1000)))
+    out1, _, _, _ = H.run_forward(case, weights, ws=big)
+    out2, _, _, _ = H.run_forward(case, weights, ws=big)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_identical_experts_equal_scaled_dense_swiglu():
+    wl = W.WORKLOADS["tiny"]
+    case = H.make_case(wl)
+    weights = H.device_weights(wl, identical=True)
+    out, _, _, _ = H.run_forward(case, weights)
+    g, u, d = (m[0].cpu() for m in weights)
+    dense = (torch.nn.functional.silu((case.h.double() @ g.double().T).float().double()).float()
+             * (case.h.double() @ u.double().T).float()).to(torch.bfloat16)
+    ref = 2.5 * (dense.double() @ d.double().T)
+    H.assert_close_out(out.float().cpu().numpy(), ref.numpy(), "identical experts")
+
+
+# ------------------------------------------------------------------ Beam shapes
+
+@pytest.fixture(scope="module")
+def beam_weights():
+    """One set of Beam-shape expert weights (20 GB) shared by the Beam-shape tests; each
+    workload keeps its own router, bias and hidden rows."""
+    wl = W.WORKLOADS["prefill"]
+    ws = H.device_weights(wl)
+    yield ws
+    del ws
+    torch.cuda.empty_cache()
+
+
+def test_decode_every_token(beam_weights):
+    case = H.make_case(W.WORKLOADS["decode"])
+    out, idx, w, _ = H.run_forward(case, beam_weights)
+    _check_routing(case, idx, w)
+    ref = H.oracle_out(case, beam_weights, range(case.wl.T))
+    H.assert_close_out(out.float().cpu().numpy(), ref, "decode")
+
+
+@pytest.mark.parametrize("name,n_sample", [("prefill", 12), ("skewed", 12)])
+def test_full_size_routing_all_tokens_output_sampled(beam_weights, name, n_sample):
+    case = H.make_case(W.WORKLOADS[name])
+    out, idx, w, ws = H.run_forward(case, beam_weights)
+    _check_routing(case, idx, w)
+    counts = bm.beam_moe_expert_counts(bm.shape_of(case.wl), ws).numpy()
+    assert np.array_equal(counts, np.bincount(case.idx.reshape(-1), minlength=case.wl.E))
+    toks = H.sample_tokens(case, n_sample)
+    ref = H.oracle_out(case, beam_weights, toks)
+    H.assert_close_out(out[toks].float().cpu().numpy(), ref, name)
+
+
+def test_block_routing_all_tokens_output_sampled(beam_weights):
+    case = H.make_case(W.WORKLOADS["block"])
+    x_out, idx, w, _ = H.run_block(case, beam_weights)
+    _check_routing(case, idx, w)
+    toks = H.sample_tokens(case, 10)
+    moe = H.oracle_out(case, beam_weights, toks)
+    ref = oracle.block_tail(case.x[toks], moe, case.g_post, case.wl.eps, case.wl.k_resid)
+    got = x_out[toks].cpu().numpy()
+    H.assert_close_out(got, ref, "block")
+    # the residual term alone is far larger than the MoE term; check the MoE part too
+    cx, cf = oracle.residual_coefficients(case.wl.k_resid)
+    H.assert_close_out((got - cx * case.x[toks].numpy()) / cf,
+                       (ref - cx * case.x[toks].numpy()) / cf, "block moe term")
+
+
+def test_block_in_place_small():
+    import dataclasses
+    wl = dataclasses.replace(W.WORKLOADS["tiny"], block=True, T=96)
+    case = H.make_case(wl)
+    weights = H.device_weights(wl)
+    x_out, idx, w, _ = H.run_block(case, weights, in_place=True)
+    _check_routing(case, idx, w)
+    moe = H.oracle_out(case, weights, range(wl.T), batch=96)
+    ref = oracle.block_tail(case.x, moe, case.g_post, wl.eps, wl.k_resid)
+    cx, cf = oracle.residual_coefficients(wl.k_resid)
+    got = x_out.cpu().numpy()
+    H.assert_close_out((got - cx * case.x.numpy()) / cf, (ref - cx * case.x.numpy()) / cf,
+                       "block in place")
+
+
+# ------------------------------------------------------------------ failure path
+
+def test_wait_timeout_is_reported_and_context_survives():
+    case = H.make_case(W.WORKLOADS["tiny"].with_tokens(512))
+    weights = H.device_weights(case.wl)
+    s = bm.shape_of(case.wl)
+    out = torch.empty(case.wl.T, case.wl.d, dtype=torch.bfloat16, device="cuda")
+    old = bm.beam_moe_get_wait_limit_ns()
+    bm.beam_moe_set_wait_limit_ns(0)
+    try:
+        ws = bm.beam_moe_forward(s, case.h.cuda(), case.router_w.cuda(), case.bias.cuda(),
+                                 *weights, out)
+        st = bm.beam_moe_sync_status(ws)
+    finally:
+        bm.beam_moe_set_wait_limit_ns(old)
+    assert st == bm.BEAM_ERR_TIMEOUT, bm.status_string(st)
+    # the context is still usable and the next call is correct
+    out2, idx, w, _ = H.run_forward(case, weights)
+    _check_routing(case, idx, w)
+    ref = H.oracle_out(case, weights, range(0, case.wl.T, 37), batch=64)
+    H.assert_close_out(out2[::37].float().cpu().numpy(), ref, "after timeout")
