@@ -49,17 +49,38 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", default="prefill", choices=sorted(W.WORKLOADS))
+    p.add_argument("--tokens", type=int, default=None,
+                   help="override T (profiling-size runs; the JSON names the reduced workload)")
+    p.add_argument("--experts", type=int, default=None,
+                   help="override E, keeping n_group and topk_group (profiling-size runs)")
     p.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    p.add_argument("--cpu-sample-tokens", type=int, default=32,
+    p.add_argument("--cpu-sample-tokens", type=int, default=128,
                    help="tokens in the oracle's bounded sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--route-only", action="store_true",
+                   help="time beam_moe_route alone (router profiling; not the layer metric)")
     p.add_argument("--dry-run", action="store_true",
                    help="exercise the launch/aggregation logic on CPU (gloo); measures nothing")
     args = p.parse_args(argv)
     if args.warmup < 3 and not args.dry_run:
         p.error("--warmup must be >= 3")
     return args
+
+
+def selected_workload(args):
+    wl = W.WORKLOADS[args.workload]
+    changes = {}
+    if args.tokens is not None:
+        changes["T"] = args.tokens
+    if args.experts is not None:
+        changes["E"] = args.experts
+    if changes:
+        wl = dataclasses.replace(wl, name=wl.name + "-reduced", **changes)
+        if wl.E % wl.n_group or wl.top_k > wl.topk_group * (wl.E // wl.n_group):
+            raise SystemExit("bench.py: --experts must keep E % n_group == 0 and "
+                             "top_k <= topk_group * E / n_group")
+    return wl
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -123,18 +144,18 @@ def load_peaks():
         return dict(FALLBACK_PEAKS)
 
 
-def _gpu_selector(device_index: int):
+def _gpu_selector(device_index: int) -> str:
+    """nvidia-smi -i selector of torch's device: its PCI bus id, else its visible index."""
     try:
-        bus = torch.cuda.get_device_properties(device_index).pci_bus_id
-        if bus:
-            return bus
+        p = torch.cuda.get_device_properties(device_index)
+        return "%08X:%02X:%02X.0" % (int(p.pci_domain_id), int(p.pci_bus_id), int(p.pci_device_id))
     except Exception:
         pass
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
         ids = [v.strip() for v in vis.split(",") if v.strip()]
         if device_index < len(ids):
-            return ids[device_index]
+            return str(ids[device_index])
     return str(device_index)
 
 
@@ -158,7 +179,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True, bufsize=1)
-        except OSError:
+        except (OSError, TypeError, ValueError):
             self.proc = None
             return
         self.thread = threading.Thread(target=self._reader, daemon=True)
@@ -292,7 +313,7 @@ def run_cuda(args, rank, world, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     bm.lib()  # fails loudly if the extension is missing
-    wl = W.WORKLOADS[args.workload]
+    wl = selected_workload(args)
     peaks = load_peaks()
     with process_group(world, "nccl") as dist:
         s = bm.shape_of(wl)
@@ -414,7 +435,7 @@ def run_cuda(args, rank, world, local):
             roof["frac"] = roof["achieved"] / roof["peak"]
             roof["kernel"] = dom
             roof["peak_source"] = peaks.get("source", "measured")
-            roof["traffic"] = traffic_from_profile(dom, args.workload)
+            roof["traffic"] = traffic_from_profile(dom, wl.name)
             roof["algorithmic_per_launch"] = wk["bytes"] if roof["bound"] == "hbm" else wk["flops"]
             roof["tensor_frac_of_sustained"] = (wk["flops"] / avg_s / 1e12) / ten_peak
             roof["hbm_frac"] = (wk["bytes"] / avg_s / 1e9) / peaks["hbm_gbs"]
@@ -474,10 +495,15 @@ def _block_h(wl, mine, g_pre):
 # ------------------------------------------------------------------ the reference arm (oracle)
 
 def run_reference(args, rank, world, local):
+    """The oracle on the host cores, one bounded sample of the workload per step.  The sample
+    size is chosen from a one-token calibration so that warm-up plus timed steps take about
+    two minutes."""
     if rank != 0:
         return None
-    wl = W.WORKLOADS[args.workload]
-    n = max(1, min(args.cpu_sample_tokens, wl.T))
+    import numpy as np
+    import oracle
+    oracle.build()
+    wl = selected_workload(args)
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     router_w, bias = W.router_weight(wl), W.router_bias(wl)
     if wl.block:
@@ -485,29 +511,38 @@ def run_reference(args, rank, world, local):
         h = _block_h(wl, wl, g_pre)
     else:
         h = W.hidden(wl)
-    import numpy as np
-    import oracle
-    oracle.build()
-    sample = wl.with_tokens(n)
-    _, idx, w, _, _ = oracle.layer_routing(h[:n], router_w, bias, sample)
-    ex = sorted({int(e) for e in idx.reshape(-1)})
-    experts = {e: tuple(W.expert_weight(wl, m, e, dev).cpu() for m in ("gate", "up", "down"))
-                for e in ex}
 
-    def one_step():
+    def prepare(n):
+        sample = wl.with_tokens(n)
+        _, idx, _, _, _ = oracle.layer_routing(h[:n], router_w, bias, sample)
+        ex = sorted({int(e) for e in idx.reshape(-1)})
+        experts = {e: tuple(W.expert_weight(wl, m, e, dev).cpu() for m in ("gate", "up", "down"))
+                   for e in ex}
+        return sample, experts
+
+    def one_step(n, sample, experts):
         _, ix, ww, _, _ = oracle.layer_routing(h[:n], router_w, bias, sample)
         oracle.moe_tokens(np.arange(n), h[:n], ix, ww, experts)
 
+    sample1, experts1 = prepare(1)
+    t0 = time.perf_counter()
+    one_step(1, sample1, experts1)
+    t_tok = time.perf_counter() - t0
+    budget_s = 120.0
+    n = int(budget_s / max(1e-6, (args.steps + args.warmup) * t_tok))
+    n = max(1, min(n, args.cpu_sample_tokens, wl.T))
+    sample, experts = prepare(n)
     for _ in range(args.warmup):
-        one_step()
+        one_step(n, sample, experts)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        one_step()
+        one_step(n, sample, experts)
     dt = time.perf_counter() - t0
     value = n * args.steps / dt
     cores = oracle.hardware_threads()
-    desc = (f"first {n} tokens of the {wl.name} workload per step, full layer in "
-            f"double-accumulating C++ on {cores} host threads")
+    desc = (f"first {n} tokens of the {wl.name} workload per step, full layer (router logits, "
+            f"routing, {wl.top_k} SwiGLU experts per token, combine) in double-accumulating C++ "
+            f"on {cores} host threads")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -518,6 +553,46 @@ def run_reference(args, rank, world, local):
                              "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------ router alone (profiling)
+
+def run_route_only(args, rank, world, local):
+    from sparse_moe_transformer_fp32_b200 import beam_moe as bm
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = selected_workload(args)
+    s = bm.shape_of(wl)
+    h = W.hidden(wl).to(dev)
+    router_w, bias = W.router_weight(wl).to(dev), W.router_bias(wl).to(dev)
+    idx = torch.empty(wl.T, wl.top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(wl.T, wl.top_k, dtype=torch.float32, device=dev)
+    ws = bm.workspace(s, dev)
+    for _ in range(args.warmup):
+        bm.beam_moe_route(s, h, router_w, bias, idx, w, ws=ws)
+    torch.cuda.synchronize(dev)
+    bm.beam_moe_profile_reset()
+    bm.beam_moe_profile_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(args.steps):
+        bm.beam_moe_route(s, h, router_w, bias, idx, w, ws=ws)
+    ev1.record()
+    torch.cuda.synchronize(dev)
+    bm.beam_moe_profile_enable(False)
+    ms = ev0.elapsed_time(ev1) / args.steps
+    prof = bm.beam_moe_profile_read()
+    st = bm.beam_moe_sync_status(ws)
+    if st != bm.BEAM_OK:
+        raise SystemExit(f"bench.py: device status {bm.status_string(st)}")
+    flops = 2.0 * wl.T * wl.d * wl.E
+    return {"metric": "router tokens/s (beam_moe_route alone)", "value": wl.T / (ms / 1e3),
+            "unit": "tokens/s", "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
+            "router_fp32_tflops": flops / (ms / 1e3) / 1e12,
+            "config": {"workload": f"{wl.name}: T={wl.T} d={wl.d} E={wl.E}"},
+            "kernels": {k: {"launches": n, "ms_per_launch": ms_ / n} for k, (n, ms_) in prof.items() if n}}
 
 
 # ------------------------------------------------------------------ dry run (host logic only)
@@ -545,6 +620,8 @@ def main(argv=None):
             raise SystemExit("bench.py: --gpus N > 1 must be launched with torch.distributed.run")
     if args.dry_run:
         res = run_dry(args, rank, world, local)
+    elif args.route_only:
+        res = run_route_only(args, rank, world, local)
     elif args.impl == "reference":
         res = run_reference(args, rank, world, local)
     else:

@@ -34,7 +34,7 @@
  *    [T, top_k] holds their weights in the same order; the combine sums in that order,
  *    so results are deterministic run to run.
  *  - Supported shapes: d % 256 == 0, d <= 8192, I % 128 == 0, 1 <= E <= 256,
- *    E % n_group == 0, n_group <= 32, 1 <= topk_group <= n_group, 1 <= top_k <= 8,
+ *    E % 4 == 0, E % n_group == 0, n_group <= 32, 1 <= topk_group <= n_group, 1 <= top_k <= 8,
  *    top_k <= topk_group * E / n_group, T >= 0, T * top_k < 2^31.  Others return
  *    BEAM_ERR_UNSUPPORTED.  T == 0 is a no-op.
  */

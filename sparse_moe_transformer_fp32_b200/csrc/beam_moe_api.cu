@@ -32,11 +32,12 @@ enum KernelId {
   kKCombine,
   kKCombineBlock,
   kKPreNorm,
+  kKRouterTranspose,
   kNumKernels
 };
 const char* const kKernelNames[kNumKernels] = {
     "router_gemm", "router_select", "dispatch_scan", "permute", "expert_gemm_gate_up",
-    "expert_gemm_down", "combine", "combine_block", "prenorm"};
+    "expert_gemm_down", "combine", "combine_block", "prenorm", "router_transpose"};
 
 struct Profiler {
   std::mutex mu;
@@ -112,7 +113,7 @@ beam_status check_shape(const beam_moe_shape* s) {
   if (!std::isfinite(s->routed_scaling_factor)) return BEAM_ERR_INVALID_ARG;
   if (s->d % 256 != 0 || s->d > kMaxD) return BEAM_ERR_UNSUPPORTED;
   if (s->I % 128 != 0 || s->I > 65536) return BEAM_ERR_UNSUPPORTED;
-  if (s->E > kMaxE || s->E % s->n_group != 0 || s->n_group > kMaxGroups)
+  if (s->E > kMaxE || s->E % 4 != 0 || s->E % s->n_group != 0 || s->n_group > kMaxGroups)
     return BEAM_ERR_UNSUPPORTED;
   if (s->topk_group > s->n_group || s->top_k > kMaxTopK) return BEAM_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(s->top_k) > static_cast<int64_t>(s->topk_group) * (s->E / s->n_group))
@@ -122,23 +123,45 @@ beam_status check_shape(const beam_moe_shape* s) {
 }
 
 struct Layout {
-  size_t status, cnt, off, mt_count, mtiles, rank, rowmap, idx, w, part, h, xp, act, y, total;
+  size_t status, cnt, off, mt_count, mtiles, rank, rowmap, idx, w, wt, part, h, xp, act, y, total;
   int S, kchunk;
   int64_t R, mt_cap;
 };
 
-// Router split-K: enough (token tile, expert tile, K chunk) blocks to cover two waves of the
-// 148 SMs, K chunks a multiple of the router's K step.
+// Router split-K factor S from a simple cost model: the FFMA time of the waves of
+// (token tile, expert tile, K chunk) blocks over the resident router blocks of a 148-SM B200,
+// plus the traffic of writing and re-reading S partial logit arrays.  K chunks are a multiple
+// of the router's K step.
+int router_split(const beam_moe_shape& s) {
+  const int64_t tiles = ceil_div(s.T, kRM) * ceil_div(s.E, kRN);
+  const int64_t kblocks = s.d / kRK;
+  const double block_flops_per_k = 2.0 * kRM * kRN;
+  const double slot_rate = 70e12 / kRouterSlots;  // FP32 FLOP/s per resident block
+  const double hbm = 6.5e12;
+  int best = 1;
+  double best_t = 1e30;
+  for (int S = 1; S <= 16 && S <= kblocks; ++S) {
+    const int64_t per = ceil_div(kblocks, S);
+    const int64_t Sx = ceil_div(kblocks, per);
+    if (Sx != S) continue;
+    const double waves = static_cast<double>(ceil_div(tiles * S, kRouterSlots));
+    const double t = waves * per * kRK * block_flops_per_k / slot_rate +
+                     static_cast<double>(S) * s.T * s.E * 8.0 / hbm;
+    if (t < best_t * 0.97) {  // a larger split must win clearly
+      best_t = t;
+      best = S;
+    }
+  }
+  return best;
+}
+
 Layout plan(const beam_moe_shape& s) {
   Layout L{};
   const int64_t T = s.T, R = T * s.top_k;
   L.R = R;
-  const int64_t tiles = ceil_div(T, kRM) * ceil_div(s.E, kRN);
-  const int64_t want = ceil_div(2 * 148, tiles > 0 ? tiles : 1);
   const int64_t kblocks = s.d / kRK;
-  const int64_t S0 = want < 1 ? 1 : (want > s.d / 256 ? s.d / 256 : want);
-  const int64_t per = ceil_div(kblocks, S0);
-  L.kchunk = static_cast<int>(per * kRK);
+  const int S = router_split(s);
+  L.kchunk = static_cast<int>(ceil_div(kblocks, S) * kRK);
   L.S = static_cast<int>(ceil_div(s.d, L.kchunk));
   L.mt_cap = ceil_div(R, kBM) + s.E;
   size_t o = 0;
@@ -156,6 +179,7 @@ Layout plan(const beam_moe_shape& s) {
   L.rowmap = take(sizeof(int32_t) * R);
   L.idx = take(sizeof(int32_t) * R);
   L.w = take(sizeof(float) * R);
+  L.wt = take(sizeof(float) * static_cast<size_t>(s.E) * s.d);
   L.part = take(sizeof(float) * static_cast<size_t>(L.S) * T * s.E);
   L.h = take(sizeof(__nv_bfloat16) * T * s.d);
   L.xp = take(sizeof(__nv_bfloat16) * R * s.d);
@@ -251,7 +275,7 @@ beam_status run_router(const beam_moe_shape& s, const Layout& L, const __nv_bflo
                        float* logits_out, bool dispatch, void* ws, cudaStream_t st) {
   RouterGemmArgs ga{};
   ga.h = h;
-  ga.W = router_w;
+  ga.WT = at<float>(ws, L.wt);
   ga.part = at<float>(ws, L.part);
   ga.zero_counts = at<int32_t>(ws, L.cnt);
   ga.T = s.T;
@@ -261,6 +285,8 @@ beam_status run_router(const beam_moe_shape& s, const Layout& L, const __nv_bflo
   // the status words reflect the latest call: cleared before the first kernel runs
   cudaError_t e = cudaMemsetAsync(at<uint32_t>(ws, L.status), 0, 16, st);
   if (e != cudaSuccess) return cuda_fail(e);
+  BEAM_LAUNCH(kKRouterTranspose, st,
+              launch_router_transpose(router_w, at<float>(ws, L.wt), s.E, s.d, st));
   BEAM_LAUNCH(kKRouterGemm, st, launch_router_gemm(ga, L.S, st));
 
   SelectArgs sa{};

@@ -29,7 +29,8 @@ constexpr int kStageBytes = kStageABytes + kStageBBytes;
 constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*align*/;
 
 // router GEMM tiling (FP32 FFMA)
-constexpr int kRM = 64, kRN = 128, kRK = 32, kRThreads = 128;
+constexpr int kRM = 128, kRN = 128, kRK = 16, kRThreads = 256, kRBStages = 3;
+constexpr int kRouterSlots = 2 * 148;  // resident router blocks on a 148-SM B200
 
 constexpr int kMaxTopK = 8;
 constexpr int kMaxE = 256;
@@ -65,7 +66,7 @@ struct MTile {
 
 struct RouterGemmArgs {
   const __nv_bfloat16* h;  // [T, d]
-  const float* W;          // [E, d]
+  const float* WT;         // [d, E] (transposed router weight)
   float* part;             // [S, T, E]
   int32_t* zero_counts;    // [E] zeroed by block (0,0,0), or null
   int T, d, E, kchunk;
@@ -140,6 +141,7 @@ struct PreNormArgs {
 
 // ------------------------------------------------------------------ launchers (one per kernel)
 
+cudaError_t launch_router_transpose(const float* W, float* WT, int E, int d, cudaStream_t s);
 cudaError_t launch_router_gemm(const RouterGemmArgs& a, int S, cudaStream_t s);
 cudaError_t launch_router_select(const SelectArgs& a, cudaStream_t s);
 cudaError_t launch_dispatch_scan(const DispatchArgs& a, cudaStream_t s);

@@ -29,9 +29,15 @@ def _lib():
 
 
 def _check_routing(case, idx, w):
+    """Indices bit-exact.  Weights within the tolerance the FP32 logits allow: the CUDA router
+    sums the d products in FP32 (|logit error| up to ~1e-5 at d = 5120), so s = sigmoid(logit)
+    moves by up to ~2.5e-6 and w = S s / sum(s) by ~1e-5 relative.  The block's router reads
+    its own BF16 copy of the normed input, which may sit one BF16 ulp (2^-8 relative) away from
+    the oracle's in a few elements; that moves a logit by up to ~4e-4 and w by ~5e-4."""
     idx = idx.cpu().numpy()
     assert np.array_equal(idx, case.idx), np.argwhere(idx != case.idx)[:5]
-    np.testing.assert_allclose(w.cpu().numpy(), case.w, rtol=2e-6, atol=1e-7)
+    rtol = 1e-3 if case.wl.block else 1e-5
+    np.testing.assert_allclose(w.cpu().numpy(), case.w, rtol=rtol, atol=1e-7)
 
 
 # ------------------------------------------------------------------ small cases, every token
