@@ -97,6 +97,26 @@ BEAM_API beam_status beam_moe_route(const beam_moe_shape* shape, const void* hid
                            const float* bias, int32_t* topk_idx, float* topk_w, float* logits_out,
                            void* ws, size_t ws_bytes, beam_stream stream);
 
+/* Router only, like beam_moe_route, for callers that cannot allocate device memory and have
+ * no workspace to pass: for example a serving engine that has handed all device memory to its
+ * own pool, or a host process that forbids device allocation (and the device-wide
+ * synchronisation cudaMalloc / cudaFree may cause) on its request path.  The pages have no
+ * counterpart to this entry point; it exists only for such callers.
+ *
+ * Scratch space is one static array of 16 MiB + 8 KiB in this library's device image; every
+ * GPU that loads the library holds a copy until the process exits.  It bounds T to at most
+ * 512 tokens (any supported d and E); larger T returns BEAM_ERR_UNSUPPORTED with the reason in
+ * beam_moe_last_cuda_error().  Nothing is allocated: the first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress), so make that first call before any
+ * stream capture.  All calls share the array and it keeps the last call's contents (each call
+ * clears what must start at zero): calls that overlap on the GPU -- on different streams, or
+ * from different host threads -- race on it and must be serialised by the caller.
+ * Arguments, layouts and outputs are those of beam_moe_route. */
+BEAM_API beam_status beam_moe_route_static(const beam_moe_shape* shape, const void* hidden,
+                                           const float* router_w, const float* bias,
+                                           int32_t* topk_idx, float* topk_w, float* logits_out,
+                                           beam_stream stream);
+
 /* Whole MoE layer forward.
  *   hidden           BF16 [T, d]
  *   router_w, bias   as for beam_moe_route

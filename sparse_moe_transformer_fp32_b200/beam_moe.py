@@ -29,7 +29,7 @@ EXPORTED = [
     "beam_moe_expert_counts", "beam_moe_set_wait_limit_ns", "beam_moe_get_wait_limit_ns",
     "beam_moe_launch_count", "beam_moe_profile_enable", "beam_moe_profile_reset",
     "beam_moe_kernel_count", "beam_moe_kernel_name", "beam_moe_profile_read",
-    "beam_moe_abi_version",
+    "beam_moe_abi_version", "beam_moe_route_static",
 ]
 
 
@@ -85,6 +85,7 @@ def lib():
     L.beam_moe_forward.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.beam_moe_block.argtypes = [shp, vp, vp, vp, f32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                  sz, vp]
+    L.beam_moe_route_static.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp]
     L.beam_moe_sync_status.argtypes = [vp, vp]
     L.beam_status_string.argtypes = [ctypes.c_int]
     L.beam_status_string.restype = ctypes.c_char_p
@@ -98,7 +99,8 @@ def lib():
     L.beam_moe_kernel_name.restype = ctypes.c_char_p
     L.beam_moe_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int64),
                                         ctypes.POINTER(ctypes.c_double)]
-    for name in ("beam_moe_route", "beam_moe_forward", "beam_moe_block", "beam_moe_sync_status",
+    for name in ("beam_moe_route", "beam_moe_route_static", "beam_moe_forward", "beam_moe_block",
+                 "beam_moe_sync_status",
                  "beam_moe_expert_counts", "beam_moe_profile_read"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -179,6 +181,22 @@ def beam_moe_route(shape, hidden, router_w, bias, topk_idx, topk_w, logits_out=N
     _check(lib().beam_moe_route(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
                                 _stream(stream)), "beam_moe_route")
     return ws
+
+
+def beam_moe_route_static(shape, hidden, router_w, bias, topk_idx, topk_w, logits_out=None,
+                          stream=None):
+    """beam_moe_route without a workspace: for callers that cannot allocate device memory.
+    Scratch is the library's static per-GPU array (T <= 512); calls that overlap on the GPU
+    race on it.  The first call on a device must come before any stream capture."""
+    T, d, E, k = shape.T, shape.d, shape.E, shape.top_k
+    args = [_ptr(hidden, torch.bfloat16, "hidden", (T, d)),
+            _ptr(router_w, torch.float32, "router_w", (E, d)),
+            _ptr(bias, torch.float32, "bias", (E,)),
+            _ptr(topk_idx, torch.int32, "topk_idx", (T, k)),
+            _ptr(topk_w, torch.float32, "topk_w", (T, k)),
+            _ptr(logits_out, torch.float32, "logits_out", (T, E), optional=True)]
+    _check(lib().beam_moe_route_static(ctypes.byref(shape), *args, _stream(stream)),
+           "beam_moe_route_static")
 
 
 def beam_moe_forward(shape, hidden, router_w, bias, w_gate, w_up, w_down, out, topk_idx=None,

@@ -382,11 +382,95 @@ bool any_misaligned(std::initializer_list<const void*> ps) {
   return false;
 }
 
+// ------------------------------------------------------------------ router without a workspace
+//
+// Scratch for beam_moe_route_static: one array per GPU, defined at file scope, so that the
+// entry point needs neither a caller workspace nor any allocation.  Host code may not use the
+// array's name as a device address (on the host it names a shadow variable); the device
+// address is obtained once per device with cudaGetSymbolAddress and kept in static_scratch.
+// Sized for the largest route plan with T <= kStaticRouteMaxTokens at any supported d and E:
+// status words, per-expert counters, the transposed router weight (<= 256 x 8192 FP32) and
+// up to 16 split-K partial logit arrays of T x 256 FP32.
+constexpr int kStaticRouteMaxTokens = 512;
+constexpr size_t kStaticRouteScratchBytes = (size_t(16) << 20) + 8192;
+static __device__ __align__(256) unsigned char g_static_route_scratch[kStaticRouteScratchBytes];
+
+// Offsets of the route-only plan inside the static scratch (status first, as in a workspace).
+Layout plan_route_static(const beam_moe_shape& s) {
+  Layout L{};
+  L.R = static_cast<int64_t>(s.T) * s.top_k;
+  const int64_t kblocks = s.d / kRK;
+  const int S = router_split(s);
+  L.kchunk = static_cast<int>(ceil_div(kblocks, S) * kRK);
+  L.S = static_cast<int>(ceil_div(s.d, L.kchunk));
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o = align_up(o + (bytes ? bytes : 1), 256);
+    return r;
+  };
+  L.status = take(256);
+  L.cnt = take(sizeof(int32_t) * s.E);
+  L.wt = take(sizeof(float) * static_cast<size_t>(s.E) * s.d);
+  L.part = take(sizeof(float) * static_cast<size_t>(L.S) * s.T * s.E);
+  L.total = o;
+  return L;
+}
+
+// Device address of this GPU's copy of the static scratch, looked up on first use per device.
+beam_status static_scratch(void** out) {
+  static void* addr[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= 64) return BEAM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_route_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return BEAM_OK;
+}
+
 }  // namespace
 
 extern "C" {
 
 int beam_moe_abi_version(void) { return 1; }
+
+beam_status beam_moe_route_static(const beam_moe_shape* shape, const void* hidden,
+                                  const float* router_w, const float* bias, int32_t* topk_idx,
+                                  float* topk_w, float* logits_out, beam_stream stream) {
+  beam_status b = check_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (any_misaligned({hidden, router_w, topk_idx, topk_w}) || !bias ||
+      (logits_out && !aligned16(logits_out)))
+    return BEAM_ERR_INVALID_ARG;
+  if (shape->T > kStaticRouteMaxTokens) {
+    std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,
+                  "beam_moe_route_static: T = %d exceeds the static-scratch limit of %d tokens",
+                  shape->T, kStaticRouteMaxTokens);
+    return BEAM_ERR_UNSUPPORTED;
+  }
+  const Layout L = plan_route_static(*shape);
+  if (L.total > kStaticRouteScratchBytes) {
+    std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,
+                  "beam_moe_route_static: needs %zu bytes of scratch, the static array holds %zu",
+                  L.total, kStaticRouteScratchBytes);
+    return BEAM_ERR_UNSUPPORTED;
+  }
+  if (shape->T == 0) return BEAM_OK;
+  DeviceInfo* dev;
+  if ((b = device_info(&dev)) != BEAM_OK) return b;
+  void* scratch = nullptr;
+  if ((b = static_scratch(&scratch)) != BEAM_OK) return b;
+  return run_router(*shape, L, static_cast<const __nv_bfloat16*>(hidden), router_w, bias, topk_idx,
+                    topk_w, logits_out, false, scratch, reinterpret_cast<cudaStream_t>(stream));
+}
 
 size_t beam_moe_workspace_size(const beam_moe_shape* shape) {
   if (check_shape(shape) != BEAM_OK) return 0;
