@@ -338,14 +338,18 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   BEAM_LAUNCH(kKPermute, st, launch_permute(pa, st));
 
   const uint64_t R = static_cast<uint64_t>(L.R);
-  CUtensorMap tm_xp, tm_g, tm_u, tm_act, tm_d;
+  ATensorMaps tm_xp, tm_act;
+  CUtensorMap tm_g, tm_u, tm_d;
   beam_status b;
-  if ((b = make_map(&tm_xp, pa.xp, s.d, R, kBM)) != BEAM_OK) return b;
+  for (int i = 0; i < kNumABoxes; ++i) {
+    if ((b = make_map(&tm_xp.m[i], pa.xp, s.d, R, a_box_rows(i))) != BEAM_OK) return b;
+    if ((b = make_map(&tm_act.m[i], at<void>(ws, L.act), s.I, R, a_box_rows(i))) != BEAM_OK)
+      return b;
+  }
   if ((b = make_map(&tm_g, w_gate, s.d, static_cast<uint64_t>(s.E) * s.I, kN1Half)) != BEAM_OK)
     return b;
   if ((b = make_map(&tm_u, w_up, s.d, static_cast<uint64_t>(s.E) * s.I, kN1Half)) != BEAM_OK)
     return b;
-  if ((b = make_map(&tm_act, at<void>(ws, L.act), s.I, R, kBM)) != BEAM_OK) return b;
   if ((b = make_map(&tm_d, w_down, s.I, static_cast<uint64_t>(s.E) * s.d, kN2)) != BEAM_OK)
     return b;
 
@@ -360,6 +364,9 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   g1.n_tiles_n = s.I / kN1Half;
   g1.k_blocks = s.d / kBK;
   g1.b_rows_per_expert = s.I;
+  // Weights-as-M tiles pay off only when nearly every tile is tiny (decode-sized calls, a few
+  // rows per expert); with larger tiles in the mix they measured slower.
+  g1.swap_max_rows = L.R <= 8 * static_cast<int64_t>(s.E) ? kSwapMaxRows : 0;
   const int64_t max_tiles1 = L.mt_cap * g1.n_tiles_n;
   const int grid1 = static_cast<int>(max_tiles1 < dev.sms ? max_tiles1 : dev.sms);
   BEAM_LAUNCH(kKGemmGateUp, st, launch_gemm_gate_up(tm_xp, tm_g, tm_u, g1, grid1, st));

@@ -20,6 +20,7 @@ constexpr int kN1Half = 128;    // gate (and up) columns per GEMM1 tile -> UMMA 
 constexpr int kN2 = 256;        // output columns per GEMM2 tile -> UMMA N = 256
 constexpr int kUmmaN = 256;
 constexpr int kBand = 8;        // m-tiles per raster band (L2 reuse of weight tiles)
+constexpr int kSwapMaxRows = 32;   // m-tiles with at most this many rows may run weights-as-M
 constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kTmemCols = 512;     // two 256-column FP32 accumulators
 
@@ -54,6 +55,17 @@ enum : uint32_t {
   kWhereCombine = 7,
   kWhereSelect = 8,
 };
+
+// Four views of the same row-major A operand (Xp or act) whose TMA boxes are 16, 32, 64 and
+// 128 rows high: a tile loads only as many rows as it has (rounded up to the next box).
+constexpr int kNumABoxes = 4;
+struct ATensorMaps {
+  CUtensorMap m[kNumABoxes];
+};
+__host__ __device__ constexpr int a_box_rows(int box) { return 16 << box; }
+__host__ __device__ constexpr int a_box_for_rows(int nrows) {
+  return nrows <= 16 ? 0 : nrows <= 32 ? 1 : nrows <= 64 ? 2 : 3;
+}
 
 struct MTile {
   int32_t e;      // expert
@@ -115,6 +127,7 @@ struct GemmArgs {
   int n_tiles_n;           // tiles along N per m-tile
   int k_blocks;            // K / kBK
   int b_rows_per_expert;   // rows of one expert in the 2-D weight view (I or d)
+  int swap_max_rows;       // m-tiles with at most this many rows run weights-as-M (0: none)
 };
 
 struct CombineArgs {
@@ -146,10 +159,10 @@ cudaError_t launch_router_gemm(const RouterGemmArgs& a, int S, cudaStream_t s);
 cudaError_t launch_router_select(const SelectArgs& a, cudaStream_t s);
 cudaError_t launch_dispatch_scan(const DispatchArgs& a, cudaStream_t s);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
-cudaError_t launch_gemm_gate_up(const CUtensorMap& tmA, const CUtensorMap& tmG,
+cudaError_t launch_gemm_gate_up(const ATensorMaps& tmA, const CUtensorMap& tmG,
                                 const CUtensorMap& tmU, const GemmArgs& a, int grid,
                                 cudaStream_t s);
-cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmD, const GemmArgs& a,
+cudaError_t launch_gemm_down(const ATensorMaps& tmA, const CUtensorMap& tmD, const GemmArgs& a,
                              int grid, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_combine_block(const CombineArgs& a, cudaStream_t s);
@@ -305,6 +318,19 @@ __device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]
         "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// 32 lanes x 16 consecutive FP32 columns (load and wait in one statement, as above).
+__device__ __forceinline__ void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
       : "memory");
 }

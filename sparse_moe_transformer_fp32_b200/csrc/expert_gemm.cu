@@ -13,7 +13,8 @@
 //       Y[rows, n-slice] = bf16( act[rows, :] . W_down,e[n-slice, :]^T )
 //
 // Kernel structure (persistent, one CTA per SM, 192 threads):
-//   warp 0     one thread issues TMA loads of the A and B tiles into a 4-stage ring
+//   warp 0     one thread issues TMA loads of the A (token rows) and B (weight) tiles into a
+//              4-stage ring; the A load covers only the tile's rows (16/32/64/128-row boxes)
 //   warp 1     allocates 512 TMEM columns; one thread issues tcgen05.mma (M=128, N=256,
 //              K=16, BF16 -> FP32) into one of two 256-column accumulators and commits
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp owns its 32-lane quarter),
@@ -21,6 +22,14 @@
 //              released so the MMA of the next tile overlaps this epilogue
 // Tiles are visited in bands of kBand m-tiles, slice-major inside a band, so the CTAs running
 // at the same time share A rows and weight slices through L2.
+//
+// In calls where nearly every m-tile is tiny (decode sizes: a few rows per expert), a tile with
+// at most swap_max_rows rows swaps the operand roles: the two 128-row halves of the weight tile become M and the
+// tile's rows, padded to a multiple of 16, become N:
+//       D_lo[128 x Np] = W[0:128, :] . X^T,   D_hi[128 x Np] = W[128:256, :] . X^T
+// so the MMA work follows the rows that exist instead of a full 128-row tile.  The same shared
+// memory stage serves both forms; the epilogue then owns one weight row per thread and writes
+// one value per token row.
 //
 // Every wait is bounded (globaltimer); on a timeout the kernel records it in the workspace
 // status word, raises a CTA-wide abort flag, waits for its own TMA loads and MMAs to finish,
@@ -42,6 +51,13 @@ __device__ __forceinline__ void decode_tile(int t, int m_tiles, int n_tiles, int
   mt = base + (r - n * gm);
 }
 
+__device__ __forceinline__ MTile load_tile(const GemmArgs& a, int t, int m_tiles, int n_tiles,
+                                           int& n) {
+  int mt;
+  decode_tile(t, m_tiles, n_tiles, mt, n);
+  return a.mtiles[mt];
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -49,24 +65,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
 
-template <bool kSwiGLU>
+template <bool kSwiGLU, bool kSwap>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    expert_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+    expert_gemm_kernel(const __grid_constant__ ATensorMaps tmA,
                        const __grid_constant__ CUtensorMap tmB0,
                        const __grid_constant__ CUtensorMap tmB1, const GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;  // 128-byte swizzle atoms need 1 KB alignment
   uint8_t* smem = smem_raw + (sbase - raw);
+  // [kStages x (A 16 KB | B 32 KB)][barriers][TMEM address][abort flag]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  constexpr int kBarFull = 0, kBarEmpty = kStages, kBarTFull = 2 * kStages,
+                kBarTEmpty = kBarTFull + 2, kBarDrain = kBarTEmpty + 2, kNumBars = kBarDrain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  auto full_bar = [&](int s) { return smem_u32(bars + s); };
-  auto empty_bar = [&](int s) { return smem_u32(bars + kStages + s); };
-  auto tfull_bar = [&](int i) { return smem_u32(bars + 2 * kStages + i); };
-  auto tempty_bar = [&](int i) { return smem_u32(bars + 2 * kStages + 2 + i); };
-  const uint32_t drain_bar = smem_u32(bars + 2 * kStages + 4);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tiles = *a.mt_count;
@@ -79,19 +93,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(bar(kBarFull + s), 1);
+      mbar_init(bar(kBarEmpty + s), 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(tfull_bar(i), 1);
-      mbar_init(tempty_bar(i), 4);
+      mbar_init(bar(kBarTFull + i), 1);
+      mbar_init(bar(kBarTEmpty + i), 4);
     }
-    mbar_init(drain_bar, 1);
+    mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
+    for (int i = 0; i < kNumABoxes; ++i) tma_prefetch_desc(&tmA.m[i]);
     tma_prefetch_desc(&tmB0);
     if (kSwiGLU) tma_prefetch_desc(&tmB1);
   }
@@ -110,27 +124,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0, filled = 0, last_parity = 0;
       bool ok = true;
+      // the next tile's descriptor is loaded one tile ahead, off the critical path
+      int n = 0;
+      MTile m = load_tile(a, blockIdx.x, m_tiles, n_tiles, n);
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        int mt, n;
-        decode_tile(t, m_tiles, n_tiles, mt, n);
-        const MTile m = a.mtiles[mt];
+        int n_next = 0;
+        const MTile m_next = load_tile(a, t + gridDim.x < ntiles ? t + gridDim.x : t, m_tiles,
+                                       n_tiles, n_next);
         const int brow = m.e * a.b_rows_per_expert + n * kNSlice;
+        // rows of A beyond the box are left from earlier stages: they only feed accumulator
+        // rows that are never stored
+        const int a_box = a_box_for_rows(m.nrows);
+        const uint32_t a_bytes = static_cast<uint32_t>(a_box_rows(a_box)) * kBK * 2;
         for (int kb = 0; kb < a.k_blocks; ++kb) {
-          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, limit, a.status,
+          if (!mbar_wait_bounded(bar(kBarEmpty + stage), phase ^ 1u, abort_flag, limit, a.status,
                                  kWhereProducerEmpty)) {
             ok = false;
             break;
           }
           const uint32_t sA = sbase + stage * kStageBytes;
           const uint32_t sB = sA + kStageABytes;
-          mbar_arrive_expect_tx(full_bar(stage), kStageBytes);
-          tma_load_2d(sA, &tmA, full_bar(stage), kb * kBK, m.row0);
-          if (kSwiGLU) {
-            tma_load_2d(sB, &tmB0, full_bar(stage), kb * kBK, brow);
-            tma_load_2d(sB + kStageBBytes / 2, &tmB1, full_bar(stage), kb * kBK, brow);
-          } else {
-            tma_load_2d(sB, &tmB0, full_bar(stage), kb * kBK, brow);
-          }
+          const uint32_t fb = bar(kBarFull + stage);
+          mbar_arrive_expect_tx(fb, a_bytes + kStageBBytes);
+          tma_load_2d(sA, &tmA.m[a_box], fb, kb * kBK, m.row0);
+          tma_load_2d(sB, &tmB0, fb, kb * kBK, brow);
+          if (kSwiGLU) tma_load_2d(sB + kStageBBytes / 2, &tmB1, fb, kb * kBK, brow);
           filled |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -138,29 +156,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             phase ^= 1u;
           }
         }
+        m = m_next;
+        n = n_next;
       }
       // every load this thread issued must land before the CTA may exit
       int no_abort = 0;
       for (int s = 0; s < kStages; ++s)
         if ((filled >> s) & 1u)
-          mbar_wait_bounded(full_bar(s), (last_parity >> s) & 1u, &no_abort, drain_limit,
+          mbar_wait_bounded(bar(kBarFull + s), (last_parity >> s) & 1u, &no_abort, drain_limit,
                             a.status, kWhereDrain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16_f32(kBM, kUmmaN);
+      constexpr uint32_t idesc_full = umma_idesc_bf16_f32(kBM, kUmmaN);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
+      int n_unused = 0;
+      int nrows = load_tile(a, blockIdx.x, m_tiles, n_tiles, n_unused).nrows;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, limit, a.status,
+        const int nrows_next = load_tile(a, t + gridDim.x < ntiles ? t + gridDim.x : t, m_tiles,
+                                         n_tiles, n_unused).nrows;
+        const bool swap = kSwap && nrows <= a.swap_max_rows;
+        const uint32_t idesc = swap ? umma_idesc_bf16_f32(kBM, (nrows + 15) & ~15) : idesc_full;
+        if (!mbar_wait_bounded(bar(kBarTEmpty + acc), acc_phase ^ 1u, abort_flag, limit, a.status,
                                kWhereMmaTmemEmpty))
           break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kUmmaN);
         for (int kb = 0; kb < a.k_blocks; ++kb) {
-          if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, limit, a.status,
+          if (!mbar_wait_bounded(bar(kBarFull + stage), phase, abort_flag, limit, a.status,
                                  kWhereMmaFull)) {
             ok = false;
             break;
@@ -169,28 +195,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t sA = sbase + stage * kStageBytes;
           const uint64_t adesc = smem_desc_k_sw128(sA);
           const uint64_t bdesc = smem_desc_k_sw128(sA + kStageABytes);
+          if (swap) {
+            const uint64_t bdesc_hi = smem_desc_k_sw128(sA + kStageABytes + kStageBBytes / 2);
 #pragma unroll
-          for (int k = 0; k < kBK / kUmmaK; ++k)  // +32 bytes along K per step: +2 in addr>>4
-            umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
-          umma_commit(empty_bar(stage));
+            for (int k = 0; k < kBK / kUmmaK; ++k) {
+              const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
+              umma_bf16(d_tmem, bdesc + 2u * k, adesc + 2u * k, idesc, accum);
+              umma_bf16(d_tmem + 128u, bdesc_hi + 2u * k, adesc + 2u * k, idesc, accum);
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < kBK / kUmmaK; ++k)  // +32 bytes along K per step: +2 in addr>>4
+              umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(bar(kBarEmpty + stage));
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(tfull_bar(acc));
+        umma_commit(bar(kBarTFull + acc));
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
+        nrows = nrows_next;
       }
       // all MMAs this thread issued must complete before TMEM is freed
       int no_abort = 0;
-      umma_commit(drain_bar);
-      mbar_wait_bounded(drain_bar, 0, &no_abort, drain_limit, a.status, kWhereDrain);
+      umma_commit(bar(kBarDrain));
+      mbar_wait_bounded(bar(kBarDrain), 0, &no_abort, drain_limit, a.status, kWhereDrain);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;  // TMEM lane quarter this warp may access (warps 2..5)
     const int row = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -200,18 +237,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const MTile m = a.mtiles[mt];
       int ok = 0;
       if (lane == 0)
-        ok = mbar_wait_bounded(tfull_bar(acc), acc_phase, abort_flag, limit, a.status,
+        ok = mbar_wait_bounded(bar(kBarTFull + acc), acc_phase, abort_flag, limit, a.status,
                                kWhereEpiTmemFull);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       // the phase has completed: each lane observes it (returns at once)
-      ok = mbar_wait_bounded(tfull_bar(acc), acc_phase, abort_flag, limit, a.status,
+      ok = mbar_wait_bounded(bar(kBarTFull + acc), acc_phase, abort_flag, limit, a.status,
                              kWhereEpiTmemFull);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
 
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(acc * kUmmaN);
+      if (kSwap && m.nrows <= a.swap_max_rows) {
+        // weights-as-M tile: this thread owns weight row `row` of each 128-row half; TMEM
+        // column j holds token row j of the tile
+        const int npad = (m.nrows + 15) & ~15;
+        __nv_bfloat16* base = a.out + static_cast<size_t>(m.row0) * a.out_ld + n * kNSlice + row;
+#pragma unroll 1
+        for (int c0 = 0; c0 < npad; c0 += 16) {
+          uint32_t lo[16], hi[16];
+          tmem_ld16_sync(tb + c0, lo);
+          tmem_ld16_sync(tb + 128 + c0, hi);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int r = c0 + j;
+            if (r < m.nrows) {
+              __nv_bfloat16* o = base + static_cast<size_t>(r) * a.out_ld;
+              if (kSwiGLU) {
+                o[0] = __float2bfloat16_rn(silu(__uint_as_float(lo[j])) * __uint_as_float(hi[j]));
+              } else {
+                o[0] = __float2bfloat16_rn(__uint_as_float(lo[j]));
+                o[128] = __float2bfloat16_rn(__uint_as_float(hi[j]));
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarTEmpty + acc));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+        continue;
+      }
       const bool valid = row < m.nrows;
       __nv_bfloat16* dst =
           a.out + static_cast<size_t>(m.row0 + (valid ? row : 0)) * a.out_ld + n * kNSlice;
@@ -252,7 +320,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (lane == 0) mbar_arrive(bar(kBarTEmpty + acc));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -269,23 +337,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }  // namespace
 
 cudaError_t prepare_gemm_kernels() {
-  cudaError_t e = cudaFuncSetAttribute(expert_gemm_kernel<true>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(expert_gemm_kernel<false>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
+  const void* kernels[] = {reinterpret_cast<const void*>(expert_gemm_kernel<true, false>),
+                           reinterpret_cast<const void*>(expert_gemm_kernel<true, true>),
+                           reinterpret_cast<const void*>(expert_gemm_kernel<false, false>),
+                           reinterpret_cast<const void*>(expert_gemm_kernel<false, true>)};
+  for (const void* k : kernels) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
-cudaError_t launch_gemm_gate_up(const CUtensorMap& tmA, const CUtensorMap& tmG,
+cudaError_t launch_gemm_gate_up(const ATensorMaps& tmA, const CUtensorMap& tmG,
                                 const CUtensorMap& tmU, const GemmArgs& a, int grid,
                                 cudaStream_t s) {
-  expert_gemm_kernel<true><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmG, tmU, a);
+  if (a.swap_max_rows > 0)
+    expert_gemm_kernel<true, true><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmG, tmU, a);
+  else
+    expert_gemm_kernel<true, false><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmG, tmU, a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmD, const GemmArgs& a,
+cudaError_t launch_gemm_down(const ATensorMaps& tmA, const CUtensorMap& tmD, const GemmArgs& a,
                              int grid, cudaStream_t s) {
-  expert_gemm_kernel<false><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmD, tmD, a);
+  if (a.swap_max_rows > 0)
+    expert_gemm_kernel<false, true><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmD, tmD, a);
+  else
+    expert_gemm_kernel<false, false><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmD, tmD, a);
   return cudaGetLastError();
 }
 
