@@ -12,6 +12,9 @@
 //   GEMM2 (down): for each m-tile and each 256-column slice n of d,
 //       Y[rows, n-slice] = bf16( act[rows, :] . W_down,e[n-slice, :]^T )
 //
+// An m-tile of at most 64 rows issues M = 64 MMAs (accumulator rows in lanes 0..15 of each
+// 32-lane quarter of TMEM), so absent rows cost no tensor-core work.
+//
 // Kernel structure (persistent, one CTA per SM, 192 threads):
 //   warp 0     one thread issues TMA loads of the A (token rows) and B (weight) tiles into a
 //              4-stage ring; the A load covers only the tile's rows (16/32/64/128-row boxes)
@@ -170,6 +173,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_full = umma_idesc_bf16_f32(kBM, kUmmaN);
+      // tiles of at most 64 rows use M = 64: half the datapath lanes, no work on absent rows
+      constexpr uint32_t idesc_m64 = umma_idesc_bf16_f32(64, kUmmaN);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -179,7 +184,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int nrows_next = load_tile(a, t + gridDim.x < ntiles ? t + gridDim.x : t, m_tiles,
                                          n_tiles, n_unused).nrows;
         const bool swap = kSwap && nrows <= a.swap_max_rows;
-        const uint32_t idesc = swap ? umma_idesc_bf16_f32(kBM, (nrows + 15) & ~15) : idesc_full;
+        const uint32_t idesc = swap ? umma_idesc_bf16_f32(kBM, (nrows + 15) & ~15)
+                               : nrows <= 64 ? idesc_m64 : idesc_full;
         if (!mbar_wait_bounded(bar(kBarTEmpty + acc), acc_phase ^ 1u, abort_flag, limit, a.status,
                                kWhereMmaTmemEmpty))
           break;
@@ -280,9 +286,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (acc == 0) acc_phase ^= 1u;
         continue;
       }
-      const bool valid = row < m.nrows;
+      // M = 128: accumulator row r sits in TMEM lane r.  M = 64 (tiles of at most 64 rows):
+      // row r sits in lane (r % 16) + 32 * (r / 16), i.e. lanes 0..15 of each warp's quarter.
+      const int trow = m.nrows <= 64 ? (lane < 16 ? q * 16 + lane : kBM) : row;
+      const bool valid = trow < m.nrows;
       __nv_bfloat16* dst =
-          a.out + static_cast<size_t>(m.row0 + (valid ? row : 0)) * a.out_ld + n * kNSlice;
+          a.out + static_cast<size_t>(m.row0 + (valid ? trow : 0)) * a.out_ld + n * kNSlice;
       if (kSwiGLU) {
 #pragma unroll 1
         for (int c = 0; c < kN1Half; c += 32) {
