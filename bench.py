@@ -299,6 +299,17 @@ def oracle_sample_rate(wl, router_w, bias, hidden_cpu, weights_dev, n_tokens: in
     return n_tokens * repeats / dt, dt, oracle.hardware_threads()
 
 
+def oracle_dense_rate(wl, hidden_cpu, weights_dev, n_tokens: int):
+    import oracle
+    oracle.build()
+    n = min(n_tokens, wl.T)
+    mats = tuple(m[0].cpu() for m in weights_dev)
+    t0 = time.perf_counter()
+    oracle.dense_mlp(range(n), hidden_cpu[:n], *mats)
+    dt = time.perf_counter() - t0
+    return n / dt, dt, oracle.hardware_threads()
+
+
 # ------------------------------------------------------------------ the CUDA arm
 
 def replica_workload(wl, rank):
@@ -321,6 +332,8 @@ def run_cuda(args, rank, world, local):
         bias = W.router_bias(wl).to(dev)
         weights = W.expert_weights(wl, dev)
         mine = replica_workload(wl, rank)
+        if wl.dense:
+            ds = bm.dense_shape(wl.T, wl.d, wl.I)
         if wl.block:
             x_cpu = W.residual_x(mine)
             g_pre, g_post = (g.to(dev) for g in W.norm_gains(wl))
@@ -332,13 +345,16 @@ def run_cuda(args, rank, world, local):
             h = h_cpu.to(dev)
             out = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
             inp_cpu, inp, res = h_cpu, h, out
-        ws = bm.workspace(s, dev)
+        ws = bm.dense_workspace(ds, dev) if wl.dense else bm.workspace(s, dev)
         stream = torch.cuda.current_stream(dev)
 
         def step(src=None, dst=None):
             src = inp if src is None else src
             dst = res if dst is None else dst
-            if wl.block:
+            if wl.dense:
+                bm.beam_dense_forward(ds, src, weights[0][0], weights[1][0], weights[2][0], dst,
+                                      ws=ws)
+            elif wl.block:
                 bm.beam_moe_block(s, src, g_pre, g_post, wl.eps, wl.k_resid, router_w, bias,
                                   *weights, dst, ws=ws)
             else:
@@ -350,7 +366,8 @@ def run_cuda(args, rank, world, local):
         st = bm.beam_moe_sync_status(ws)
         if st != bm.BEAM_OK:
             raise SystemExit(f"bench.py: device status {bm.status_string(st)}")
-        counts = bm.beam_moe_expert_counts(s, ws)
+        counts = (torch.tensor([wl.T], dtype=torch.int32) if wl.dense
+                  else bm.beam_moe_expert_counts(s, ws))
         touched = int((counts > 0).sum())
 
         # ---- timed region (device time, max over ranks)
@@ -384,31 +401,55 @@ def run_cuda(args, rank, world, local):
         value = tokens_all / (ms_total / 1e3)
         ms_per_step = ms_total / args.steps
 
-        # ---- end to end: pinned host input -> device -> layer -> host result, every step
+        # ---- end to end: pinned host input -> device -> layer -> host result, every step.
+        # Copies run on their own streams with two buffers each, so step i's upload and
+        # step i-1's download overlap step i's layer; events order every reuse of a buffer.
         e2e = None
         if not args.no_e2e:
             host_in = inp_cpu.pin_memory()
-            host_out = torch.empty(res.shape, dtype=res.dtype).pin_memory()
-            dev_in = torch.empty_like(inp)
-            for _ in range(3):
-                dev_in.copy_(host_in, non_blocking=True)
-                step(dev_in, res)
-                host_out.copy_(res, non_blocking=True)
+            host_out = [torch.empty(res.shape, dtype=res.dtype).pin_memory() for _ in range(2)]
+            dev_in = [torch.empty_like(inp) for _ in range(2)]
+            dev_out = [torch.empty_like(res) for _ in range(2)]
+            s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+            mk = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+            in_done, comp_done, out_done = mk(), mk(), mk()
+
+            def pipelined(n):
+                for i in range(n):
+                    b = i % 2
+                    if i >= 2:
+                        s_in.wait_event(comp_done[b])      # step i-2 finished reading dev_in[b]
+                    with torch.cuda.stream(s_in):
+                        dev_in[b].copy_(host_in, non_blocking=True)
+                    in_done[b].record(s_in)
+                    stream.wait_event(in_done[b])
+                    if i >= 2:
+                        stream.wait_event(out_done[b])     # dev_out[b] of step i-2 copied out
+                    step(dev_in[b], dev_out[b])
+                    comp_done[b].record(stream)
+                    s_out.wait_event(comp_done[b])
+                    with torch.cuda.stream(s_out):
+                        host_out[b].copy_(dev_out[b], non_blocking=True)
+                    out_done[b].record(s_out)
+                for b in range(2):
+                    stream.wait_event(out_done[b])
+
+            pipelined(3)
             barrier(dist, dev)
             torch.cuda.synchronize(dev)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for _ in range(args.steps):
-                dev_in.copy_(host_in, non_blocking=True)
-                step(dev_in, res)
-                host_out.copy_(res, non_blocking=True)
+            s_in.wait_event(e0)
+            s_out.wait_event(e0)
+            pipelined(args.steps)
             e1.record(stream)
             torch.cuda.synchronize(dev)
             barrier(dist, dev)
             e_ms = max_over_ranks(dist, e0.elapsed_time(e1), dev)
             e2e = {"value": tokens_all / (e_ms / 1e3), "unit": "tokens/s",
                    "h2d_bytes_per_step": host_in.numel() * host_in.element_size(),
-                   "d2h_bytes_per_step": host_out.numel() * host_out.element_size()}
+                   "d2h_bytes_per_step": host_out[0].numel() * host_out[0].element_size(),
+                   "overlap": "uploads and downloads on their own streams, double-buffered"}
 
         result = None
         if rank == 0:
@@ -441,10 +482,15 @@ def run_cuda(args, rank, world, local):
             roof["hbm_frac"] = (wk["bytes"] / avg_s / 1e9) / peaks["hbm_gbs"]
 
             step_s = ms_per_step / 1e3
-            flops_step = 6 * wl.T * wl.top_k * wl.d * wl.I
+            flops_step = 6 * wl.T * wl.top_k * wl.d * wl.I  # top_k = 1 for the dense MLP
             bytes_step = layer_min_bytes(wl, touched)
             cpu = None
-            if not args.no_cpu_baseline and world == 1:
+            if not args.no_cpu_baseline and world == 1 and wl.dense:
+                rate, secs, cores = oracle_dense_rate(wl, inp_cpu, weights, args.cpu_sample_tokens)
+                cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                       "sample": f"first {args.cpu_sample_tokens} tokens of the dense workload, "
+                                 f"SwiGLU MLP in double-accumulating C++; {secs:.2f} s"}
+            elif not args.no_cpu_baseline and world == 1:
                 rate, secs, cores = oracle_sample_rate(
                     wl, W.router_weight(wl), W.router_bias(wl),
                     inp_cpu if not wl.block else _block_h(wl, mine, g_pre), weights,

@@ -146,6 +146,34 @@ BEAM_API beam_status beam_moe_block(const beam_moe_shape* shape, const float* x,
                            const void* w_down, float* x_out, int32_t* topk_idx, float* topk_w,
                            void* ws, size_t ws_bytes, beam_stream stream);
 
+/* Dense SwiGLU MLP of Beam's first three decoder layers: out = W_down (silu(W_gate h) * (W_up h)),
+ * BF16 weights, FP32 accumulation and activation, BF16 output; no routing.
+ *   hidden  BF16 [T, d];  w_gate, w_up BF16 [I, d];  w_down BF16 [d, I];  out BF16 [T, d]
+ * Runs the same tensor-core GEMMs as the experts, with every token in one group.  Shapes:
+ * d % 256 == 0, d <= 8192, I % 128 == 0, 0 <= T < 2^31.
+ * Cites: "Beam" model doc, Overview ("The first 3 layers use a dense SwiGLU MLP") and
+ * BeamConfig (intermediate_size = 20480, hidden_act = silu). */
+typedef struct {
+  int32_t T;  /* tokens */
+  int32_t d;  /* hidden_size */
+  int32_t I;  /* intermediate_size */
+} beam_dense_shape;
+
+BEAM_API size_t beam_dense_workspace_size(const beam_dense_shape* shape);
+BEAM_API beam_status beam_dense_forward(const beam_dense_shape* shape, const void* hidden,
+                                        const void* w_gate, const void* w_up, const void* w_down,
+                                        void* out, void* ws, size_t ws_bytes, beam_stream stream);
+
+/* Selection-bias update from the expert loads of the last beam_moe_forward / beam_moe_block
+ * call made with `ws` (same shape):  bias[e] += gamma * sign(mean_load - load[e]), sign(0) = 0,
+ * mean_load = T * top_k / E.  Under-loaded experts gain bias, over-loaded ones lose it; the
+ * caller supplies gamma from its (e.g. cosine-decayed) schedule.
+ * Cites: archdb "Beam-1.0-501B-A23B", load-balancing entry (auxiliary-loss-free bias with
+ * cosine-decayed bias updates); news article "Reflection lança o Beam" (router follows
+ * DeepSeek-V3's scheme); "Beam" model doc, Notes (no auxiliary loss). */
+BEAM_API beam_status beam_moe_bias_update(const beam_moe_shape* shape, const void* ws,
+                                          float* bias, float gamma, beam_stream stream);
+
 /* Synchronises `stream`, reads and clears the device status word kept in `ws`, and
  * returns BEAM_OK, BEAM_ERR_TIMEOUT or BEAM_ERR_DEVICE_ASSERT (or BEAM_ERR_CUDA if the
  * stream itself reports an error).  `ws` must have been used with a call of this shape

@@ -57,6 +57,7 @@ def lib():
         L.oracle_residual.argtypes = [i64, vp, vp, i32, vp]
         L.oracle_residual_coefficients.argtypes = [i32, ctypes.POINTER(ctypes.c_double),
                                                    ctypes.POINTER(ctypes.c_double)]
+        L.oracle_bias_update.argtypes = [i32, vp, i64, vp, f32, vp]
         _lib = L
     return _lib
 
@@ -209,6 +210,23 @@ def residual_coefficients(k: int):
     cx, cf = ctypes.c_double(), ctypes.c_double()
     lib().oracle_residual_coefficients(k, ctypes.byref(cx), ctypes.byref(cf))
     return cx.value, cf.value
+
+
+def bias_update(counts, bias, gamma: float, slots: int) -> np.ndarray:
+    """bias + gamma * sign(slots / E - counts) (FP32)."""
+    c = _np(counts, np.int32)
+    b = _np(bias, np.float32)
+    out = np.empty_like(b)
+    lib().oracle_bias_update(b.size, _p(c), int(slots), _p(b), gamma, _p(out))
+    return out
+
+
+def dense_mlp(tokens, h, w_gate, w_up, w_down, nthreads: int = 0) -> np.ndarray:
+    """Dense SwiGLU MLP (FP32 out) for the listed tokens: one expert, weight 1."""
+    hb = bf16_bits(h)
+    idx = np.zeros((hb.shape[0], 1), np.int32)
+    w = np.ones((hb.shape[0], 1), np.float32)
+    return moe_tokens(tokens, hb, idx, w, {0: (w_gate, w_up, w_down)}, nthreads)
 
 
 # ---------------------------------------------------------------- whole layer / block

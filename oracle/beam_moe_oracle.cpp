@@ -273,6 +273,19 @@ void oracle_residual(int64_t n, const float* x, const float* f, int k, float* ou
     out[i] = static_cast<float>(static_cast<double>(x[i]) * cx + static_cast<double>(f[i]) * cf);
 }
 
+// Selection-bias update after one step (auxiliary-loss-free balancing): experts that got fewer
+// than the mean number of slots gain gamma, experts that got more lose gamma:
+//   bias'[e] = fl32( bias[e] + gamma * sign(slots / E - counts[e]) ),  sign(0) = 0.
+void oracle_bias_update(int E, const int32_t* counts, int64_t slots, const float* bias,
+                        float gamma, float* bias_out) {
+  const double mean = static_cast<double>(slots) / static_cast<double>(E);
+  for (int e = 0; e < E; ++e) {
+    const double c = static_cast<double>(counts[e]);
+    const float sgn = c < mean ? 1.0f : (c > mean ? -1.0f : 0.0f);
+    bias_out[e] = bias[e] + gamma * sgn;
+  }
+}
+
 void oracle_residual_coefficients(int k, double* cx, double* cf) {
   const double kk = static_cast<double>(k);
   *cx = std::sqrt((kk - 1.0) / kk);

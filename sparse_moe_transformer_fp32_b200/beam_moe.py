@@ -29,7 +29,8 @@ EXPORTED = [
     "beam_moe_expert_counts", "beam_moe_set_wait_limit_ns", "beam_moe_get_wait_limit_ns",
     "beam_moe_launch_count", "beam_moe_profile_enable", "beam_moe_profile_reset",
     "beam_moe_kernel_count", "beam_moe_kernel_name", "beam_moe_profile_read",
-    "beam_moe_abi_version", "beam_moe_route_static",
+    "beam_moe_abi_version", "beam_moe_route_static", "beam_dense_workspace_size",
+    "beam_dense_forward", "beam_moe_bias_update",
 ]
 
 
@@ -51,6 +52,10 @@ class beam_moe_shape(ctypes.Structure):
 
     def __repr__(self):
         return "beam_moe_shape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class beam_dense_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("I", ctypes.c_int32)]
 
 
 def make_shape(T, d, E, n_group, topk_group, top_k, I, routed_scaling_factor=2.5,
@@ -86,6 +91,11 @@ def lib():
     L.beam_moe_block.argtypes = [shp, vp, vp, vp, f32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                  sz, vp]
     L.beam_moe_route_static.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp]
+    dshp = ctypes.POINTER(beam_dense_shape)
+    L.beam_dense_workspace_size.argtypes = [dshp]
+    L.beam_dense_workspace_size.restype = sz
+    L.beam_dense_forward.argtypes = [dshp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.beam_moe_bias_update.argtypes = [shp, vp, vp, f32, vp]
     L.beam_moe_sync_status.argtypes = [vp, vp]
     L.beam_status_string.argtypes = [ctypes.c_int]
     L.beam_status_string.restype = ctypes.c_char_p
@@ -100,7 +110,7 @@ def lib():
     L.beam_moe_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int64),
                                         ctypes.POINTER(ctypes.c_double)]
     for name in ("beam_moe_route", "beam_moe_route_static", "beam_moe_forward", "beam_moe_block",
-                 "beam_moe_sync_status",
+                 "beam_moe_sync_status", "beam_dense_forward", "beam_moe_bias_update",
                  "beam_moe_expert_counts", "beam_moe_profile_read"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -236,6 +246,40 @@ def beam_moe_block(shape, x, g_pre, g_post, eps, k_resid, router_w, bias, w_gate
     _check(lib().beam_moe_block(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
                                 _stream(stream)), "beam_moe_block")
     return ws
+
+
+def dense_shape(T, d, I) -> beam_dense_shape:
+    return beam_dense_shape(T, d, I)
+
+
+def dense_workspace(shape: beam_dense_shape, device="cuda") -> torch.Tensor:
+    n = int(lib().beam_dense_workspace_size(ctypes.byref(shape)))
+    if n == 0:
+        raise BeamError(BEAM_ERR_UNSUPPORTED, "beam_dense_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def beam_dense_forward(shape, hidden, w_gate, w_up, w_down, out, ws=None, stream=None):
+    T, d, I = shape.T, shape.d, shape.I
+    args = [_ptr(hidden, torch.bfloat16, "hidden", (T, d)),
+            _ptr(w_gate, torch.bfloat16, "w_gate", (I, d)),
+            _ptr(w_up, torch.bfloat16, "w_up", (I, d)),
+            _ptr(w_down, torch.bfloat16, "w_down", (d, I)),
+            _ptr(out, torch.bfloat16, "out", (T, d))]
+    if ws is None:
+        ws = dense_workspace(shape, hidden.device)
+    _ptr(ws, torch.uint8, "ws")
+    _check(lib().beam_dense_forward(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
+                                    _stream(stream)), "beam_dense_forward")
+    return ws
+
+
+def beam_moe_bias_update(shape, ws, bias, gamma: float, stream=None) -> None:
+    """bias += gamma * sign(mean load - load) from the loads of the last forward on ``ws``."""
+    _check(lib().beam_moe_bias_update(ctypes.byref(shape), _ptr(ws, torch.uint8, "ws"),
+                                      _ptr(bias, torch.float32, "bias", (shape.E,)),
+                                      ctypes.c_float(gamma), _stream(stream)),
+           "beam_moe_bias_update")
 
 
 def beam_moe_sync_status(ws, stream=None) -> int:

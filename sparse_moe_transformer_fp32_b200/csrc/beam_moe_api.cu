@@ -33,11 +33,14 @@ enum KernelId {
   kKCombineBlock,
   kKPreNorm,
   kKRouterTranspose,
+  kKDenseTiles,
+  kKBiasUpdate,
   kNumKernels
 };
 const char* const kKernelNames[kNumKernels] = {
     "router_gemm", "router_select", "dispatch_scan", "permute", "expert_gemm_gate_up",
-    "expert_gemm_down", "combine", "combine_block", "prenorm", "router_transpose"};
+    "expert_gemm_down", "combine", "combine_block", "prenorm", "router_transpose", "dense_tiles",
+    "bias_update"};
 
 struct Profiler {
   std::mutex mu;
@@ -443,6 +446,38 @@ beam_status static_scratch(void** out) {
   return BEAM_OK;
 }
 
+// ------------------------------------------------------------------ dense SwiGLU MLP
+
+beam_status check_dense_shape(const beam_dense_shape* s) {
+  if (!s) return BEAM_ERR_INVALID_ARG;
+  if (s->T < 0 || s->d <= 0 || s->I <= 0) return BEAM_ERR_INVALID_ARG;
+  if (s->d % 256 != 0 || s->d > kMaxD || s->I % 128 != 0 || s->I > (1 << 20))
+    return BEAM_ERR_UNSUPPORTED;
+  return BEAM_OK;
+}
+
+struct DenseLayout {
+  size_t status, mt_count, mtiles, act, total;
+  int64_t mt_cap;
+};
+
+DenseLayout plan_dense(const beam_dense_shape& s) {
+  DenseLayout L{};
+  L.mt_cap = ceil_div(s.T, kBM);
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o = align_up(o + (bytes ? bytes : 1), 1024);
+    return r;
+  };
+  L.status = take(256);
+  L.mt_count = take(16);
+  L.mtiles = take(sizeof(MTile) * L.mt_cap);
+  L.act = take(sizeof(__nv_bfloat16) * static_cast<size_t>(s.T) * s.I);
+  L.total = o;
+  return L;
+}
+
 }  // namespace
 
 extern "C" {
@@ -613,6 +648,84 @@ beam_status beam_moe_block(const beam_moe_shape* shape, const float* x, const fl
   ca.k = shape->top_k;
   ca.R = static_cast<int>(L.R);
   BEAM_LAUNCH(kKCombineBlock, st, launch_combine_block(ca, st));
+  return BEAM_OK;
+}
+
+size_t beam_dense_workspace_size(const beam_dense_shape* shape) {
+  if (check_dense_shape(shape) != BEAM_OK) return 0;
+  return plan_dense(*shape).total;
+}
+
+beam_status beam_dense_forward(const beam_dense_shape* shape, const void* hidden,
+                               const void* w_gate, const void* w_up, const void* w_down,
+                               void* out, void* ws, size_t ws_bytes, beam_stream stream) {
+  beam_status b = check_dense_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (any_misaligned({hidden, w_gate, w_up, w_down, out})) return BEAM_ERR_INVALID_ARG;
+  const DenseLayout L = plan_dense(*shape);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < L.total)
+    return BEAM_ERR_WORKSPACE;
+  if (shape->T == 0) return BEAM_OK;
+  DeviceInfo* dev;
+  if ((b = device_info(&dev)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const beam_dense_shape& s = *shape;
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  cudaError_t e = cudaMemsetAsync(status, 0, 16, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  MTile* mtiles = at<MTile>(ws, L.mtiles);
+  int32_t* mt_count = at<int32_t>(ws, L.mt_count);
+  BEAM_LAUNCH(kKDenseTiles, st, launch_dense_tiles(s.T, mtiles, mt_count, st));
+
+  ATensorMaps tm_h, tm_act;
+  CUtensorMap tm_g, tm_u, tm_d;
+  void* act = at<void>(ws, L.act);
+  for (int i = 0; i < kNumABoxes; ++i) {
+    if ((b = make_map(&tm_h.m[i], hidden, s.d, s.T, a_box_rows(i))) != BEAM_OK) return b;
+    if ((b = make_map(&tm_act.m[i], act, s.I, s.T, a_box_rows(i))) != BEAM_OK) return b;
+  }
+  if ((b = make_map(&tm_g, w_gate, s.d, s.I, kN1Half)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_u, w_up, s.d, s.I, kN1Half)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_d, w_down, s.I, s.d, kN2)) != BEAM_OK) return b;
+
+  GemmArgs g1{};
+  g1.mtiles = mtiles;
+  g1.mt_count = mt_count;
+  g1.out = static_cast<__nv_bfloat16*>(act);
+  g1.status = status;
+  g1.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  g1.out_ld = s.I;
+  g1.n_tiles_n = s.I / kN1Half;
+  g1.k_blocks = s.d / kBK;
+  g1.b_rows_per_expert = s.I;
+  g1.swap_max_rows = 0;
+  const int64_t t1 = L.mt_cap * g1.n_tiles_n;
+  BEAM_LAUNCH(kKGemmGateUp, st,
+              launch_gemm_gate_up(tm_h, tm_g, tm_u, g1, static_cast<int>(t1 < dev->sms ? t1 : dev->sms), st));
+  GemmArgs g2 = g1;
+  g2.out = static_cast<__nv_bfloat16*>(out);
+  g2.out_ld = s.d;
+  g2.n_tiles_n = s.d / kN2;
+  g2.k_blocks = s.I / kBK;
+  g2.b_rows_per_expert = s.d;
+  const int64_t t2 = L.mt_cap * g2.n_tiles_n;
+  BEAM_LAUNCH(kKGemmDown, st,
+              launch_gemm_down(tm_act, tm_d, g2, static_cast<int>(t2 < dev->sms ? t2 : dev->sms), st));
+  return BEAM_OK;
+}
+
+beam_status beam_moe_bias_update(const beam_moe_shape* shape, const void* ws, float* bias,
+                                 float gamma, beam_stream stream) {
+  beam_status b = check_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (!ws || !bias || !std::isfinite(gamma)) return BEAM_ERR_INVALID_ARG;
+  if (shape->T == 0) return BEAM_OK;
+  const Layout L = plan(*shape);
+  const float mean = static_cast<float>(static_cast<double>(L.R) / shape->E);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  BEAM_LAUNCH(kKBiasUpdate, st,
+              launch_bias_update(reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + L.cnt),
+                                 bias, shape->E, mean, gamma, st));
   return BEAM_OK;
 }
 

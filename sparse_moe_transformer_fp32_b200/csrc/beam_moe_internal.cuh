@@ -167,6 +167,9 @@ cudaError_t launch_gemm_down(const ATensorMaps& tmA, const CUtensorMap& tmD, con
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_combine_block(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_prenorm(const PreNormArgs& a, cudaStream_t s);
+cudaError_t launch_dense_tiles(int T, MTile* mtiles, int32_t* mt_count, cudaStream_t s);
+cudaError_t launch_bias_update(const int32_t* cnt, float* bias, int E, float mean, float gamma,
+                               cudaStream_t s);
 cudaError_t prepare_gemm_kernels();  // opt-in shared memory sizes (once per device)
 
 // ------------------------------------------------------------------ device helpers

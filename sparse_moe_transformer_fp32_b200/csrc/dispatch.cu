@@ -84,7 +84,44 @@ __global__ void __launch_bounds__(256) permute_kernel(const PermuteArgs a) {
   }
 }
 
+// Dense MLP: every token belongs to the single group 0; tiles of up to kBM consecutive rows.
+__global__ void dense_tiles_kernel(int T, MTile* mtiles, int32_t* mt_count) {
+  const int n = (T + kBM - 1) / kBM;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    MTile t;
+    t.e = 0;
+    t.row0 = i * kBM;
+    t.nrows = min(kBM, T - i * kBM);
+    t.pad = 0;
+    mtiles[i] = t;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *mt_count = n;
+}
+
+// bias[e] += gamma * sign(mean - cnt[e])
+__global__ void bias_update_kernel(const int32_t* cnt, float* bias, int E, float mean,
+                                   float gamma) {
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < E; e += gridDim.x * blockDim.x) {
+    const float c = static_cast<float>(cnt[e]);
+    const float sgn = c < mean ? 1.f : (c > mean ? -1.f : 0.f);
+    bias[e] += gamma * sgn;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_dense_tiles(int T, MTile* mtiles, int32_t* mt_count, cudaStream_t s) {
+  const int n = (T + kBM - 1) / kBM;
+  const int blocks = (n + 255) / 256 < 1 ? 1 : (n + 255) / 256;
+  dense_tiles_kernel<<<blocks, 256, 0, s>>>(T, mtiles, mt_count);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bias_update(const int32_t* cnt, float* bias, int E, float mean, float gamma,
+                               cudaStream_t s) {
+  bias_update_kernel<<<1, 256, 0, s>>>(cnt, bias, E, mean, gamma);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_dispatch_scan(const DispatchArgs& a, cudaStream_t s) {
   dispatch_scan_kernel<<<1, 256, 0, s>>>(a);

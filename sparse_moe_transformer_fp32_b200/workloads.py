@@ -15,6 +15,7 @@ rms_norm_eps 1e-6).  The five workloads are:
 * ``prefill`` T=4096,  Beam shapes, near-uniform expert load
 * ``skewed``  T=16384, Beam shapes, bias 0.5/rank over a seeded permutation
 * ``block``   T=8192,  Beam shapes, FP32 residual input with sandwich norms
+* ``dense``   T=4096,  dense SwiGLU MLP of the first layers (d=5120, intermediate 20480)
 
 Distributions: hidden ~N(0,1) rounded to BF16; router weight FP32 normal with
 the stated standard deviation; expert weights BF16 normal with variance
@@ -52,6 +53,7 @@ class Workload:
     scale: float = 2.5        # routed_scaling_factor
     norm_topk_prob: bool = True
     block: bool = False       # sandwich RMSNorms + depth-scaled residual around the layer
+    dense: bool = False       # dense SwiGLU MLP (one "expert", no routing)
     eps: float = 1e-6
     k_resid: int = 10
 
@@ -74,6 +76,9 @@ WORKLOADS = {
     "skewed": Workload("skewed", T=16384, seed=3, bias_kind="inv_rank", bias_range=0.5, **_BEAM),
     "block": Workload("block", T=8192, seed=4, bias_kind="uniform", bias_range=0.05, block=True,
                       **_BEAM),
+    # Beam's first three layers: dense SwiGLU MLP, intermediate_size 20480
+    "dense": Workload("dense", T=4096, d=5120, E=1, n_group=1, topk_group=1, top_k=1, I=20480,
+                      seed=5, router_std=0.0, bias_kind="uniform", bias_range=0.0, dense=True),
 }
 
 # tensor ids for seed derivation

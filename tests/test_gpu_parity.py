@@ -191,3 +191,32 @@ def test_wait_timeout_is_reported_and_context_survives():
     _check_routing(case, idx, w)
     ref = H.oracle_out(case, weights, range(0, case.wl.T, 37), batch=64)
     H.assert_close_out(out2[::37].float().cpu().numpy(), ref, "after timeout")
+
+
+# ------------------------------------------------------------------ dense SwiGLU MLP and bias update
+
+@pytest.mark.parametrize("T,d,I", [(200, 256, 1024), (1, 512, 384), (129, 5120, 20480)])
+def test_dense_mlp_every_token(T, d, I):
+    import dataclasses
+    wl = dataclasses.replace(W.WORKLOADS["dense"], T=T, d=d, I=I)
+    h = W.hidden(wl)
+    mats = tuple(W.expert_weight(wl, m, 0, "cuda") for m in ("gate", "up", "down"))
+    out = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    s = bm.dense_shape(T, d, I)
+    bm.beam_dense_forward(s, h.cuda(), *mats, out)
+    torch.cuda.synchronize()
+    toks = list(range(T)) if T <= 200 else sorted({0, T - 1, 1, T // 2, T // 3, 2 * T // 3})
+    ref = oracle.dense_mlp(toks, h, *(m.cpu() for m in mats))
+    H.assert_close_out(out[toks].float().cpu().numpy(), ref, f"dense T={T} d={d} I={I}")
+
+
+def test_bias_update_matches_oracle():
+    case = H.make_case(W.WORKLOADS["tiny"].with_tokens(300))
+    weights = H.device_weights(case.wl)
+    _, _, _, ws = H.run_forward(case, weights)
+    s = bm.shape_of(case.wl)
+    bias = case.bias.cuda().clone()
+    bm.beam_moe_bias_update(s, ws, bias, 1e-3)
+    counts = np.bincount(case.idx.reshape(-1), minlength=case.wl.E)
+    ref = oracle.bias_update(counts, case.bias, 1e-3, case.wl.R)
+    assert np.array_equal(bias.cpu().numpy().view(np.uint32), ref.view(np.uint32))

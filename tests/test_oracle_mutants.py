@@ -43,6 +43,8 @@ MUTANTS = {
     "combine_drops_slot": ("      for (int j = 0; j < k; ++j)\n        acc += static_cast<double>(w[t * k + j])",
                            "      for (int j = 1; j < k; ++j)\n        acc += static_cast<double>(w[t * k + j])"),
     "bf16_truncates": ("if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;", ""),
+    "bias_update_sign_flipped": ("const float sgn = c < mean ? 1.0f : (c > mean ? -1.0f : 0.0f);",
+                                 "const float sgn = c < mean ? -1.0f : (c > mean ? 1.0f : 0.0f);"),
 }
 
 PIN_TESTS = [
@@ -59,6 +61,7 @@ PIN_TESTS = [
     (pins.test_residual_after_104_contributions_weighs_each_equally, [()]),
     (pins.test_rmsnorm_matches_torch_and_closed_form, [()]),
     (pins.test_bf16_rounding_matches_torch, [()]),
+    (pins.test_bias_update_hand_example_and_invariants, [()]),
 ]
 
 
@@ -81,7 +84,8 @@ def test_mutant_is_caught(tmp_path, monkeypatch, name):
     mut = ctypes.CDLL(so)
     for fn in ("oracle_hardware_threads", "oracle_f32_to_bf16", "oracle_bf16_to_f32",
                "oracle_router_logits", "oracle_route", "oracle_expert_mlp", "oracle_moe_tokens",
-               "oracle_rmsnorm", "oracle_residual", "oracle_residual_coefficients"):
+               "oracle_rmsnorm", "oracle_residual", "oracle_residual_coefficients",
+               "oracle_bias_update"):
         f, g = getattr(real, fn), getattr(mut, fn)
         g.argtypes, g.restype = f.argtypes, f.restype
     monkeypatch.setattr(oracle, "_lib", mut)

@@ -265,3 +265,27 @@ def test_beam_config_accounting():
     assert (beam.d, beam.I, beam.E, beam.top_k, beam.n_group, beam.topk_group, beam.scale) == (
         c["hidden_size"], c["moe_intermediate_size"], c["num_experts"], c["num_experts_per_tok"],
         c["n_group"], c["topk_group"], c["routed_scaling_factor"])
+
+
+def test_bias_update_hand_example_and_invariants():
+    with open(os.path.join(GOLDEN, "bias_update_example.json")) as f:
+        c = json.load(f)
+    got = oracle.bias_update(np.array(c["counts"]), np.array(c["bias"], np.float32), c["gamma"],
+                             c["slots"])
+    assert got.tolist() == c["expected"]
+    # repeated updates move an always-overloaded expert's bias down and an idle one's up,
+    # by exactly gamma per step, and leave the total unchanged when loads are symmetric
+    counts = np.array([10, 0, 5, 5])
+    b = np.zeros(4, np.float32)
+    for _ in range(8):
+        b = oracle.bias_update(counts, b, 0.25, 20)
+    assert b.tolist() == [-2.0, 2.0, 0.0, 0.0]
+
+
+def test_dense_mlp_is_one_expert_with_unit_weight():
+    wl = W.WORKLOADS["tiny"]
+    h = W.hidden(wl)[:6]
+    mats = tuple(W.expert_weight(wl, m, 5) for m in ("gate", "up", "down"))
+    out = oracle.dense_mlp(range(6), h, *mats)
+    ref = _torch_swiglu_f64(h, *mats).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-5, atol=1e-6)
