@@ -220,3 +220,61 @@ def test_bias_update_matches_oracle():
     counts = np.bincount(case.idx.reshape(-1), minlength=case.wl.E)
     ref = oracle.bias_update(counts, case.bias, 1e-3, case.wl.R)
     assert np.array_equal(bias.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+# ------------------------------------------------------------------ other shapes and edge cases
+
+_TINY = W.WORKLOADS["tiny"]
+
+
+@pytest.mark.parametrize("name,changes", [
+    ("E64_G4_Gk2_k6", dict(T=300, d=512, E=64, n_group=4, topk_group=2, top_k=6, I=256)),
+    ("no_group_limit", dict(T=100, d=256, E=32, n_group=4, topk_group=4, top_k=8, I=128)),
+    ("top1", dict(T=150, d=256, E=16, n_group=4, topk_group=1, top_k=1, I=128)),
+    ("one_group", dict(T=90, d=256, E=16, n_group=1, topk_group=1, top_k=4, I=256)),
+    ("one_expert_per_group", dict(T=77, d=256, E=8, n_group=8, topk_group=3, top_k=3, I=128)),
+    ("d8192", dict(T=40, d=8192, E=8, n_group=2, topk_group=1, top_k=2, I=128)),
+    ("many_tokens", dict(T=20000, d=256, E=16, n_group=4, topk_group=2, top_k=4, I=128)),
+])
+def test_forward_other_shapes(name, changes):
+    import dataclasses
+    wl = dataclasses.replace(_TINY, name=name, **changes)
+    case = H.make_case(wl)
+    weights = H.device_weights(wl)
+    out, idx, w, _ = H.run_forward(case, weights)
+    _check_routing(case, idx, w)
+    toks = list(range(wl.T)) if wl.T <= 300 else H.sample_tokens(case, 40)
+    ref = H.oracle_out(case, weights, toks, batch=64)
+    H.assert_close_out(out[toks].float().cpu().numpy(), ref, name)
+
+
+def test_block_at_maximum_hidden_size():
+    import dataclasses
+    wl = dataclasses.replace(_TINY, name="block_d8192", block=True, T=33, d=8192, E=8, n_group=2,
+                             topk_group=1, top_k=2, I=128)
+    case = H.make_case(wl)
+    weights = H.device_weights(wl)
+    x_out, idx, w, _ = H.run_block(case, weights)
+    _check_routing(case, idx, w)
+    moe = H.oracle_out(case, weights, range(wl.T), batch=64)
+    ref = oracle.block_tail(case.x, moe, case.g_post, wl.eps, wl.k_resid)
+    cx, cf = oracle.residual_coefficients(wl.k_resid)
+    got = x_out.cpu().numpy()
+    H.assert_close_out((got - cx * case.x.numpy()) / cf, (ref - cx * case.x.numpy()) / cf,
+                       "block d8192")
+
+
+@pytest.mark.parametrize("T", [1, 7])
+def test_beam_shape_few_tokens(beam_weights, T):
+    case = H.make_case(W.WORKLOADS["decode"].with_tokens(T))
+    out, idx, w, _ = H.run_forward(case, beam_weights)
+    _check_routing(case, idx, w)
+    ref = H.oracle_out(case, beam_weights, range(T))
+    H.assert_close_out(out.float().cpu().numpy(), ref, f"beam T={T}")
+
+
+def test_full_size_forward_is_deterministic(beam_weights):
+    case = H.make_case(W.WORKLOADS["prefill"])
+    out1, _, _, ws = H.run_forward(case, beam_weights)
+    out2, _, _, _ = H.run_forward(case, beam_weights, ws=ws)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
