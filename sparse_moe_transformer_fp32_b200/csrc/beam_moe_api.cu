@@ -247,6 +247,7 @@ beam_status make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
 
 struct DeviceInfo {
   int sms = 0;
+  int pair_grid = 0;  // CTAs of co-resident SM-pair clusters
   bool prepared = false;
 };
 
@@ -264,6 +265,9 @@ beam_status device_info(DeviceInfo** out) {
     if (e != cudaSuccess) return cuda_fail(e);
     e = prepare_gemm_kernels();
     if (e != cudaSuccess) return cuda_fail(e);
+    e = prepare_gemm_2sm_kernels();
+    if (e != cudaSuccess) return cuda_fail(e);
+    d.pair_grid = max_pair_grid(d.sms);
     d.prepared = true;
   }
   *out = &d;
@@ -318,12 +322,16 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
                         const __nv_bfloat16* h, const int32_t* idx, const void* w_gate,
                         const void* w_up, const void* w_down, void* ws, cudaStream_t st) {
   uint32_t* status = at<uint32_t>(ws, L.status);
+  // Calls averaging at least 256 rows per expert run their expert GEMMs on SM pairs
+  // (cta_group::2, 256-row tiles): half the operand traffic per SM for the same tensor work.
+  const bool pairs = L.R >= static_cast<int64_t>(kPairMinRowsPerExpert) * s.E && dev.pair_grid >= 2;
   DispatchArgs da{};
   da.cnt = at<int32_t>(ws, L.cnt);
   da.off = at<int32_t>(ws, L.off);
   da.mt_count = at<int32_t>(ws, L.mt_count);
   da.mtiles = at<MTile>(ws, L.mtiles);
   da.E = s.E;
+  da.tile_rows = pairs ? 2 * kBM : kBM;
   BEAM_LAUNCH(kKDispatchScan, st, launch_dispatch_scan(da, st));
 
   PermuteArgs pa{};
@@ -371,8 +379,15 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   // rows per expert); with larger tiles in the mix they measured slower.
   g1.swap_max_rows = L.R <= 8 * static_cast<int64_t>(s.E) ? kSwapMaxRows : 0;
   const int64_t max_tiles1 = L.mt_cap * g1.n_tiles_n;
-  const int grid1 = static_cast<int>(max_tiles1 < dev.sms ? max_tiles1 : dev.sms);
-  BEAM_LAUNCH(kKGemmGateUp, st, launch_gemm_gate_up(tm_xp, tm_g, tm_u, g1, grid1, st));
+  if (pairs) {
+    g1.swap_max_rows = 0;
+    const int64_t want = 2 * max_tiles1;
+    const int grid = static_cast<int>(want < dev.pair_grid ? want : dev.pair_grid) & ~1;
+    BEAM_LAUNCH(kKGemmGateUp, st, launch_gemm_gate_up_2sm(tm_xp, tm_g, tm_u, g1, grid, st));
+  } else {
+    const int grid1 = static_cast<int>(max_tiles1 < dev.sms ? max_tiles1 : dev.sms);
+    BEAM_LAUNCH(kKGemmGateUp, st, launch_gemm_gate_up(tm_xp, tm_g, tm_u, g1, grid1, st));
+  }
 
   GemmArgs g2 = g1;
   g2.out = at<__nv_bfloat16>(ws, L.y);
@@ -381,8 +396,17 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   g2.k_blocks = s.I / kBK;
   g2.b_rows_per_expert = s.d;
   const int64_t max_tiles2 = L.mt_cap * g2.n_tiles_n;
-  const int grid2 = static_cast<int>(max_tiles2 < dev.sms ? max_tiles2 : dev.sms);
-  BEAM_LAUNCH(kKGemmDown, st, launch_gemm_down(tm_act, tm_d, g2, grid2, st));
+  if (pairs) {
+    CUtensorMap tm_d_half;  // each SM of a pair loads 128 of the tile's 256 weight rows
+    if ((b = make_map(&tm_d_half, w_down, s.I, static_cast<uint64_t>(s.E) * s.d, kBM)) != BEAM_OK)
+      return b;
+    const int64_t want = 2 * max_tiles2;
+    const int grid = static_cast<int>(want < dev.pair_grid ? want : dev.pair_grid) & ~1;
+    BEAM_LAUNCH(kKGemmDown, st, launch_gemm_down_2sm(tm_act, tm_d_half, g2, grid, st));
+  } else {
+    const int grid2 = static_cast<int>(max_tiles2 < dev.sms ? max_tiles2 : dev.sms);
+    BEAM_LAUNCH(kKGemmDown, st, launch_gemm_down(tm_act, tm_d, g2, grid2, st));
+  }
   return BEAM_OK;
 }
 

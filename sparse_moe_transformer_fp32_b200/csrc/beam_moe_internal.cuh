@@ -20,6 +20,7 @@ constexpr int kN1Half = 128;    // gate (and up) columns per GEMM1 tile -> UMMA 
 constexpr int kN2 = 256;        // output columns per GEMM2 tile -> UMMA N = 256
 constexpr int kUmmaN = 256;
 constexpr int kBand = 8;        // m-tiles per raster band (L2 reuse of weight tiles)
+constexpr int kPairMinRowsPerExpert = 256;  // calls at or above this mean use SM-pair GEMMs
 constexpr int kSwapMaxRows = 32;   // m-tiles with at most this many rows may run weights-as-M
 constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kTmemCols = 512;     // two 256-column FP32 accumulators
@@ -104,6 +105,7 @@ struct DispatchArgs {
   int32_t* mt_count;    // [1] number of m-tiles
   MTile* mtiles;        // [capacity]
   int E;
+  int tile_rows;        // rows per m-tile: 128 (one SM) or 256 (an SM pair)
 };
 
 struct PermuteArgs {
@@ -164,6 +166,13 @@ cudaError_t launch_gemm_gate_up(const ATensorMaps& tmA, const CUtensorMap& tmG,
                                 cudaStream_t s);
 cudaError_t launch_gemm_down(const ATensorMaps& tmA, const CUtensorMap& tmD, const GemmArgs& a,
                              int grid, cudaStream_t s);
+cudaError_t launch_gemm_gate_up_2sm(const ATensorMaps& tmA, const CUtensorMap& tmG,
+                                    const CUtensorMap& tmU, const GemmArgs& a, int grid,
+                                    cudaStream_t s);
+cudaError_t launch_gemm_down_2sm(const ATensorMaps& tmA, const CUtensorMap& tmD,
+                                 const GemmArgs& a, int grid, cudaStream_t s);
+cudaError_t prepare_gemm_2sm_kernels();
+int max_pair_grid(int sms);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_combine_block(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_prenorm(const PreNormArgs& a, cudaStream_t s);

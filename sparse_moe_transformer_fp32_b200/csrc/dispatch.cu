@@ -32,7 +32,8 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a
   __shared__ int warp_tot[8];
   const int e = threadIdx.x;
   const int c = e < a.E ? a.cnt[e] : 0;
-  const int m = (c + kBM - 1) / kBM;
+  const int tr = a.tile_rows;
+  const int m = (c + tr - 1) / tr;
   const int c_incl = block_inclusive_scan(c, warp_tot);
   const int m_incl = block_inclusive_scan(m, warp_tot);
   const int c_excl = c_incl - c, m_excl = m_incl - m;
@@ -44,8 +45,8 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a
   for (int i = 0; i < m; ++i) {
     MTile t;
     t.e = e;
-    t.row0 = c_excl + i * kBM;
-    t.nrows = min(kBM, c - i * kBM);
+    t.row0 = c_excl + i * tr;
+    t.nrows = min(tr, c - i * tr);
     t.pad = 0;
     a.mtiles[m_excl + i] = t;
   }
