@@ -199,6 +199,14 @@ BEAM_API beam_status beam_moe_expert_counts(const beam_moe_shape* shape, const v
 BEAM_API void beam_moe_set_wait_limit_ns(uint64_t ns);
 BEAM_API uint64_t beam_moe_get_wait_limit_ns(void);
 
+/* Expert GEMMs on SM pairs (tcgen05 cta_group::2, 256-row tiles; one cluster of two CTAs
+ * per tile) for beam_moe_forward / beam_moe_block calls averaging at least 256 rows per
+ * expert.  Off by default: on a power-capped B200 those calls are bound by tensor throughput,
+ * and 256-row tiles add padded rows, so the single-SM 128-row kernel measured faster.  The
+ * setting applies to calls made after it. */
+BEAM_API void beam_moe_set_sm_pairs(int enable);
+BEAM_API int beam_moe_get_sm_pairs(void);
+
 /* Total kernels this library has launched in this process. */
 BEAM_API uint64_t beam_moe_launch_count(void);
 

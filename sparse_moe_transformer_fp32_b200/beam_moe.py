@@ -30,7 +30,8 @@ EXPORTED = [
     "beam_moe_launch_count", "beam_moe_profile_enable", "beam_moe_profile_reset",
     "beam_moe_kernel_count", "beam_moe_kernel_name", "beam_moe_profile_read",
     "beam_moe_abi_version", "beam_moe_route_static", "beam_dense_workspace_size",
-    "beam_dense_forward", "beam_moe_bias_update",
+    "beam_dense_forward", "beam_moe_bias_update", "beam_moe_set_sm_pairs",
+    "beam_moe_get_sm_pairs",
 ]
 
 
@@ -104,6 +105,8 @@ def lib():
     L.beam_moe_set_wait_limit_ns.argtypes = [u64]
     L.beam_moe_get_wait_limit_ns.restype = u64
     L.beam_moe_launch_count.restype = u64
+    L.beam_moe_set_sm_pairs.argtypes = [ctypes.c_int]
+    L.beam_moe_get_sm_pairs.restype = ctypes.c_int
     L.beam_moe_profile_enable.argtypes = [ctypes.c_int]
     L.beam_moe_kernel_name.argtypes = [ctypes.c_int]
     L.beam_moe_kernel_name.restype = ctypes.c_char_p
@@ -300,6 +303,14 @@ def beam_moe_set_wait_limit_ns(ns: int) -> None:
 
 def beam_moe_get_wait_limit_ns() -> int:
     return int(lib().beam_moe_get_wait_limit_ns())
+
+
+def beam_moe_set_sm_pairs(enable: bool) -> None:
+    lib().beam_moe_set_sm_pairs(1 if enable else 0)
+
+
+def beam_moe_get_sm_pairs() -> bool:
+    return bool(lib().beam_moe_get_sm_pairs())
 
 
 def beam_moe_launch_count() -> int:

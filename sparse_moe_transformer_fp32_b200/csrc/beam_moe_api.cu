@@ -18,6 +18,7 @@ using namespace beam;
 
 std::atomic<uint64_t> g_wait_limit_ns{4000000000ull};
 std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_sm_pairs{0};
 thread_local char g_last_cuda_error[256] = "";
 
 // ------------------------------------------------------------------ kernel ids and timing
@@ -322,9 +323,12 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
                         const __nv_bfloat16* h, const int32_t* idx, const void* w_gate,
                         const void* w_up, const void* w_down, void* ws, cudaStream_t st) {
   uint32_t* status = at<uint32_t>(ws, L.status);
-  // Calls averaging at least 256 rows per expert run their expert GEMMs on SM pairs
-  // (cta_group::2, 256-row tiles): half the operand traffic per SM for the same tensor work.
-  const bool pairs = L.R >= static_cast<int64_t>(kPairMinRowsPerExpert) * s.E && dev.pair_grid >= 2;
+  // With SM pairs enabled, calls averaging at least 256 rows per expert run their expert GEMMs
+  // on SM pairs (cta_group::2, 256-row tiles): half the operand bytes per SM for the same tensor
+  // work, but 256-row tiles pad more rows.
+  const bool pairs = g_sm_pairs.load(std::memory_order_relaxed) != 0 &&
+                     L.R >= static_cast<int64_t>(kPairMinRowsPerExpert) * s.E &&
+                     dev.pair_grid >= 2;
   DispatchArgs da{};
   da.cnt = at<int32_t>(ws, L.cnt);
   da.off = at<int32_t>(ws, L.off);
@@ -559,6 +563,8 @@ const char* beam_status_string(beam_status s) {
 const char* beam_moe_last_cuda_error(void) { return g_last_cuda_error; }
 
 void beam_moe_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+void beam_moe_set_sm_pairs(int enable) { g_sm_pairs.store(enable ? 1 : 0); }
+int beam_moe_get_sm_pairs(void) { return g_sm_pairs.load(); }
 uint64_t beam_moe_get_wait_limit_ns(void) { return g_wait_limit_ns.load(); }
 uint64_t beam_moe_launch_count(void) { return g_launches.load(); }
 

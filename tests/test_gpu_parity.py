@@ -282,12 +282,29 @@ def test_full_size_forward_is_deterministic(beam_weights):
 
 @pytest.mark.parametrize("T", [1024, 1500, 4000])
 def test_forward_sm_pair_path(T):
-    """T * top_k >= 256 * E runs the expert GEMMs on SM pairs (cta_group::2, 256-row tiles);
-    T = 1500 leaves experts whose last pair tile has no rows for the second SM."""
+    """With SM pairs on, T * top_k >= 256 * E runs the expert GEMMs on SM pairs (cta_group::2,
+    256-row tiles); T = 1500 leaves experts whose last pair tile has no rows for the second SM."""
     case = H.make_case(W.WORKLOADS["tiny"].with_tokens(T))
     weights = H.device_weights(case.wl)
-    out, idx, w, _ = H.run_forward(case, weights)
+    bm.beam_moe_set_sm_pairs(True)
+    try:
+        out, idx, w, _ = H.run_forward(case, weights)
+    finally:
+        bm.beam_moe_set_sm_pairs(False)
     _check_routing(case, idx, w)
     toks = H.sample_tokens(case, 64)
     ref = H.oracle_out(case, weights, toks, batch=64)
     H.assert_close_out(out[toks].float().cpu().numpy(), ref, f"pairs T={T}")
+
+
+def test_sm_pair_path_on_beam_shapes(beam_weights):
+    case = H.make_case(W.WORKLOADS["prefill"].with_tokens(8192))
+    bm.beam_moe_set_sm_pairs(True)
+    try:
+        out, idx, w, _ = H.run_forward(case, beam_weights)
+    finally:
+        bm.beam_moe_set_sm_pairs(False)
+    _check_routing(case, idx, w)
+    toks = H.sample_tokens(case, 8)
+    ref = H.oracle_out(case, beam_weights, toks)
+    H.assert_close_out(out[toks].float().cpu().numpy(), ref, "pairs beam")
