@@ -36,7 +36,7 @@
  *  - Supported shapes: d % 256 == 0, d <= 8192, I % 128 == 0, 1 <= E <= 256,
  *    E % 4 == 0, E % n_group == 0, n_group <= 32, 1 <= topk_group <= n_group, 1 <= top_k <= 8,
  *    top_k <= topk_group * E / n_group, T >= 0, T * top_k < 2^31.  Others return
- *    BEAM_ERR_UNSUPPORTED.  T == 0 is a no-op.
+ *    BEAM_ERR_UNSUPPORTED.  T == 0 is a no-op that reads no pointer (they may be NULL).
  */
 #ifndef BEAM_MOE_H_
 #define BEAM_MOE_H_

@@ -517,6 +517,7 @@ beam_status beam_moe_route_static(const beam_moe_shape* shape, const void* hidde
                                   float* topk_w, float* logits_out, beam_stream stream) {
   beam_status b = check_shape(shape);
   if (b != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
   if (any_misaligned({hidden, router_w, topk_idx, topk_w}) || !bias ||
       (logits_out && !aligned16(logits_out)))
     return BEAM_ERR_INVALID_ARG;
@@ -533,7 +534,6 @@ beam_status beam_moe_route_static(const beam_moe_shape* shape, const void* hidde
                   L.total, kStaticRouteScratchBytes);
     return BEAM_ERR_UNSUPPORTED;
   }
-  if (shape->T == 0) return BEAM_OK;
   DeviceInfo* dev;
   if ((b = device_info(&dev)) != BEAM_OK) return b;
   void* scratch = nullptr;
@@ -573,12 +573,12 @@ beam_status beam_moe_route(const beam_moe_shape* shape, const void* hidden, cons
                            void* ws, size_t ws_bytes, beam_stream stream) {
   beam_status b = check_shape(shape);
   if (b != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
   if (any_misaligned({hidden, router_w, topk_idx, topk_w}) || !bias ||
       (logits_out && !aligned16(logits_out)))
     return BEAM_ERR_INVALID_ARG;
   const Layout L = plan(*shape);
   if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
-  if (shape->T == 0) return BEAM_OK;
   DeviceInfo* dev;
   if ((b = device_info(&dev)) != BEAM_OK) return b;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -592,12 +592,12 @@ beam_status beam_moe_forward(const beam_moe_shape* shape, const void* hidden, co
                              void* ws, size_t ws_bytes, beam_stream stream) {
   beam_status b = check_shape(shape);
   if (b != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
   if (any_misaligned({hidden, router_w, w_gate, w_up, w_down, out}) || !bias ||
       (topk_idx && !aligned16(topk_idx)) || (topk_w && !aligned16(topk_w)))
     return BEAM_ERR_INVALID_ARG;
   const Layout L = plan(*shape);
   if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
-  if (shape->T == 0) return BEAM_OK;
   DeviceInfo* dev;
   if ((b = device_info(&dev)) != BEAM_OK) return b;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -629,6 +629,7 @@ beam_status beam_moe_block(const beam_moe_shape* shape, const float* x, const fl
                            void* ws, size_t ws_bytes, beam_stream stream) {
   beam_status b = check_shape(shape);
   if (b != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
   if (any_misaligned({x, g_pre, g_post, router_w, w_gate, w_up, w_down, x_out}) || !bias ||
       (topk_idx && !aligned16(topk_idx)) || (topk_w && !aligned16(topk_w)))
     return BEAM_ERR_INVALID_ARG;
@@ -641,7 +642,6 @@ beam_status beam_moe_block(const beam_moe_shape* shape, const float* x, const fl
   }
   const Layout L = plan(*shape);
   if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
-  if (shape->T == 0) return BEAM_OK;
   DeviceInfo* dev;
   if ((b = device_info(&dev)) != BEAM_OK) return b;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -691,11 +691,11 @@ beam_status beam_dense_forward(const beam_dense_shape* shape, const void* hidden
                                void* out, void* ws, size_t ws_bytes, beam_stream stream) {
   beam_status b = check_dense_shape(shape);
   if (b != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
   if (any_misaligned({hidden, w_gate, w_up, w_down, out})) return BEAM_ERR_INVALID_ARG;
   const DenseLayout L = plan_dense(*shape);
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < L.total)
     return BEAM_ERR_WORKSPACE;
-  if (shape->T == 0) return BEAM_OK;
   DeviceInfo* dev;
   if ((b = device_info(&dev)) != BEAM_OK) return b;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -748,8 +748,8 @@ beam_status beam_moe_bias_update(const beam_moe_shape* shape, const void* ws, fl
                                  float gamma, beam_stream stream) {
   beam_status b = check_shape(shape);
   if (b != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
   if (!ws || !bias || !std::isfinite(gamma)) return BEAM_ERR_INVALID_ARG;
-  if (shape->T == 0) return BEAM_OK;
   const Layout L = plan(*shape);
   const float mean = static_cast<float>(static_cast<double>(L.R) / shape->E);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

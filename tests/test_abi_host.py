@@ -89,6 +89,7 @@ def test_forward_rejects_bad_arguments(L):
     assert fwd(L, s, ws=FAKE + 128) == bm.BEAM_ERR_WORKSPACE
     assert fwd(L, s, ws_bytes=bm.beam_moe_workspace_size(s) - 1) == bm.BEAM_ERR_WORKSPACE
     assert fwd(L, beam(0)) == bm.BEAM_OK  # nothing to do, nothing launched
+    assert fwd(L, beam(0), hidden=None, out=None, ws=None) == bm.BEAM_OK
 
 
 def test_route_and_block_reject_bad_arguments(L):

@@ -5,6 +5,8 @@ relative L2 1e-2 and max |err| 5e-2 * RMS of the oracle's.  Small cases are comp
 token; the full-size workloads are compared on every token's routing and on sampled tokens'
 outputs, in the same launch configuration the benchmark times.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -308,3 +310,21 @@ def test_sm_pair_path_on_beam_shapes(beam_weights):
     toks = H.sample_tokens(case, 8)
     ref = H.oracle_out(case, beam_weights, toks)
     H.assert_close_out(out[toks].float().cpu().numpy(), ref, "pairs beam")
+
+
+def test_maximum_size_beam_call(beam_weights):
+    """T = 65536 at Beam shapes: 524,288 slots, expert-contiguous buffers of 2.7e9 elements
+    (past 32-bit element offsets).  Routing on every token, outputs on sampled tokens."""
+    case = H.make_case(W.WORKLOADS["prefill"].with_tokens(65536))
+    out, idx, w, _ = H.run_forward(case, beam_weights)
+    _check_routing(case, idx, w)
+    toks = H.sample_tokens(case, 8)
+    ref = H.oracle_out(case, beam_weights, toks)
+    H.assert_close_out(out[toks].float().cpu().numpy(), ref, "T=65536")
+
+
+def test_zero_tokens_reads_nothing():
+    s = bm.shape_of(W.WORKLOADS["prefill"], 0)
+    L = bm.lib()
+    assert L.beam_moe_forward(ctypes.byref(s), None, None, None, None, None, None, None, None,
+                              None, None, 0, None) == bm.BEAM_OK
