@@ -130,6 +130,27 @@ def test_decode_every_token(beam_weights):
     H.assert_close_out(out.float().cpu().numpy(), ref, "decode")
 
 
+@pytest.mark.parametrize("name", ["decode", "prefill", "skewed"])
+def test_full_size_logits_within_fp32_dot_error(name):
+    """Every router logit at the Beam shapes against the oracle's (exact sum rounded once to
+    FP32).  An FP32 dot product of length 5120 with h ~ N(0, 1) and W_r ~ N(0, 0.01^2) carries
+    a rounding error of order sqrt(d) * 2^-24 * |partial sums| ~ 1e-6; the bound 1e-5 leaves
+    room for the summation order and is the one the weight tolerance above is derived from.
+    A router that summed all d products into one tensor-core accumulator would miss it (that
+    error grows with the chain length, to ~6e-5 at d = 5120)."""
+    case = H.make_case(W.WORKLOADS[name])
+    wl = case.wl
+    s = bm.shape_of(wl)
+    idx = torch.empty(wl.T, wl.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(wl.T, wl.top_k, dtype=torch.float32, device="cuda")
+    logits = torch.empty(wl.T, wl.E, dtype=torch.float32, device="cuda")
+    ws = bm.beam_moe_route(s, case.h.cuda(), case.router_w.cuda(), case.bias.cuda(), idx, w, logits)
+    assert bm.beam_moe_sync_status(ws) == bm.BEAM_OK
+    _check_routing(case, idx, w)
+    err = np.abs(logits.cpu().numpy().astype(np.float64) - case.logits.astype(np.float64))
+    assert err.max() <= 1e-5, f"{name}: max |logit error| {err.max():.3e}"
+
+
 @pytest.mark.parametrize("name,n_sample", [("prefill", 12), ("skewed", 12)])
 def test_full_size_routing_all_tokens_output_sampled(beam_weights, name, n_sample):
     case = H.make_case(W.WORKLOADS[name])
