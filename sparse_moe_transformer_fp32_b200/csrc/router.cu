@@ -246,60 +246,90 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   }
 }
 
-// ---------------------------------------------------------------- selection: one warp per token
+// ---------------------------------------------------------------- selection
 //
-// Each lane owns up to 8 consecutive experts (lane * per_lane ...).  The token's scores are
-// also kept in shared memory so that any lane can read any expert's score.  Group scores are
-// computed by lane g for group g (sequential scan of its E/G experts); the kept groups come
-// from a rank count over all group scores; the top_k experts are taken in top_k rounds of a
-// warp-wide maximum over 64-bit keys (order-preserving score bits, then inverted expert id, so
-// that the lower id wins a tie).
+// A block of 256 threads takes 8 tokens.  First the whole block forms the 8 x E logits (the
+// K-split partials added in z order, loads of four splits in flight), scores s = sigmoid and
+// biased scores sb = s + b into shared memory.  Then one warp per token:
+//   group scores   lane g scans group g's E/G biased scores (sum of the top two); lanes start
+//                  at different offsets of their groups so that the reads hit distinct banks
+//   kept groups    rank of each group score among all (higher first, lower index on ties)
+//   top-k          lane l holds experts l*c .. l*c+c-1 (c = ceil(E/32)); k rounds of a warp
+//                  maximum of the lanes' best candidate scores (order-preserving bits, redux),
+//                  then a warp minimum of the expert ids holding it (lower id wins a tie)
+//   output         ascending expert id: lane order, then a prefix sum of the lanes' counts;
+//                  the weights' denominator is summed in that order
 
 __device__ __forceinline__ uint32_t ordered_bits(float f) {
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) {
-  __shared__ float s_sh[8][kMaxE];
-  __shared__ float sb_sh[8][kMaxE];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= a.T) return;
-  const int E = a.E, G = a.G, P = E / G;
-  const int per_lane = (E + 31) / 32;
-  float* s_w = s_sh[warp];
-  float* sb_w = sb_sh[warp];
+constexpr int kSelTokens = 8;
+constexpr int kSelLogitsPerThread = kSelTokens * kMaxE / 256;
 
-  // logits (sum of the split-K partials in z order), scores, biased scores
-  float my_sb[kMaxE / 32];
+__global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) {
+  __shared__ float s_sh[kSelTokens][kMaxE];
+  __shared__ float sb_sh[kSelTokens][kMaxE];
+  __shared__ int sel_sh[kSelTokens][kMaxTopK];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = a.E, G = a.G, P = E / G;
+  const int t0 = blockIdx.x * kSelTokens;
+  const int ntok = min(kSelTokens, a.T - t0);
+
+  // ---- logits, scores and biased scores of the block's tokens
+  {
+    const int n = ntok * E;
+    const size_t zs = static_cast<size_t>(a.T) * E;
+    const float* base = a.part + static_cast<size_t>(t0) * E;
+    float l[kSelLogitsPerThread];
 #pragma unroll
-  for (int i = 0; i < kMaxE / 32; ++i) {
-    my_sb[i] = -CUDART_INF_F;
-    const int e = lane * per_lane + i;
-    if (i < per_lane && e < E) {
-      const float* p = a.part + static_cast<size_t>(t) * E + e;
-      const size_t zs = static_cast<size_t>(a.T) * E;
-      float l = 0.f;
-#pragma unroll 4
-      for (int z = 0; z < a.S; ++z) l += p[z * zs];
-      if (a.logits_out) a.logits_out[static_cast<size_t>(t) * E + e] = l;
-      const float s = 1.0f / (1.0f + expf(-l));
-      const float sb = s + a.bias[e];
-      s_w[e] = s;
-      sb_w[e] = sb;
-      my_sb[i] = sb;
+    for (int j = 0; j < kSelLogitsPerThread; ++j) l[j] = 0.f;
+#pragma unroll 1
+    for (int z0 = 0; z0 < a.S; z0 += 4) {
+      float v[4][kSelLogitsPerThread];
+#pragma unroll
+      for (int zz = 0; zz < 4; ++zz)
+#pragma unroll
+        for (int j = 0; j < kSelLogitsPerThread; ++j) {
+          const int i = threadIdx.x + 256 * j;
+          v[zz][j] = (z0 + zz < a.S && i < n) ? base[(z0 + zz) * zs + i] : 0.f;
+        }
+#pragma unroll
+      for (int zz = 0; zz < 4; ++zz)
+#pragma unroll
+        for (int j = 0; j < kSelLogitsPerThread; ++j)
+          if (z0 + zz < a.S) l[j] += v[zz][j];
+    }
+#pragma unroll
+    for (int j = 0; j < kSelLogitsPerThread; ++j) {
+      const int i = threadIdx.x + 256 * j;
+      if (i < n) {
+        const int tl = i / E, e = i - tl * E;
+        if (a.logits_out) a.logits_out[static_cast<size_t>(t0) * E + i] = l[j];
+        const float s = 1.0f / (1.0f + expf(-l[j]));
+        s_sh[tl][e] = s;
+        sb_sh[tl][e] = s + a.bias[e];
+      }
     }
   }
-  __syncwarp();
+  __syncthreads();
+  if (warp >= ntok) return;
+  const int t = t0 + warp;
+  const float* sw = s_sh[warp];
+  const float* sbw = sb_sh[warp];
 
-  // group scores: lane g scans group g
+  // ---- group scores: lane g takes group g
   float gs = -CUDART_INF_F;
   if (lane < G) {
+    const float* grp = sbw + lane * P;
+    const int o = lane % P;
     float m1 = -CUDART_INF_F, m2 = -CUDART_INF_F;
-#pragma unroll 1
-    for (int e = lane * P; e < (lane + 1) * P; ++e) {
-      const float v = sb_w[e];
+#pragma unroll 8
+    for (int j = 0; j < P; ++j) {
+      int jj = j + o;
+      if (jj >= P) jj -= P;
+      const float v = grp[jj];
       if (v > m1) {
         m2 = m1;
         m1 = v;
@@ -309,73 +339,95 @@ __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) 
     }
     gs = P >= 2 ? m1 + m2 : m1;
   }
-  // rank of my group among all groups (higher score first, lower index on ties)
-  int rank = 0;
-#pragma unroll 1
+  int grank = 0;
+#pragma unroll 8
   for (int g2 = 0; g2 < G; ++g2) {
     const float o = __shfl_sync(0xffffffffu, gs, g2);
-    if (lane < G && (o > gs || (o == gs && g2 < lane))) ++rank;
+    if (lane < G && (o > gs || (o == gs && g2 < lane))) ++grank;
   }
-  const uint32_t kept = __ballot_sync(0xffffffffu, lane < G && rank < a.Gk);
+  const uint32_t kept = __ballot_sync(0xffffffffu, lane < G && grank < a.Gk);
 
-  // candidate keys of my experts (0 = not a candidate)
-  uint64_t key[kMaxE / 32];
+  // ---- this lane's candidates
+  const int c = (E + 31) / 32;
+  const int e0 = lane * c;
+  uint32_t bits[kMaxE / 32];
+  uint32_t avail = 0;
+  {
+    int g = e0 / P, r = e0 - g * P;
 #pragma unroll
-  for (int i = 0; i < kMaxE / 32; ++i) {
-    const int e = lane * per_lane + i;
-    key[i] = 0;
-    if (i < per_lane && e < E && ((kept >> (e / P)) & 1u))
-      key[i] = (static_cast<uint64_t>(ordered_bits(my_sb[i])) << 32) |
-               static_cast<uint64_t>(0xffffffffu - static_cast<uint32_t>(e));
-  }
-  int sel[kMaxTopK];
-#pragma unroll
-  for (int r = 0; r < kMaxTopK; ++r) {
-    sel[r] = 0x7fffffff;
-    if (r < a.k) {
-      uint64_t best = 0;
-#pragma unroll
-      for (int i = 0; i < kMaxE / 32; ++i) best = key[i] > best ? key[i] : best;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
-        best = o > best ? o : best;
+    for (int i = 0; i < kMaxE / 32; ++i) {
+      bits[i] = 0;
+      if (i < c && e0 + i < E) {
+        if ((kept >> g) & 1u) {
+          bits[i] = ordered_bits(sbw[e0 + i]);
+          avail |= 1u << i;
+        }
+        if (++r == P) {
+          r = 0;
+          ++g;
+        }
       }
-      const int e = best ? static_cast<int>(0xffffffffu - static_cast<uint32_t>(best)) : -1;
-      sel[r] = e < 0 ? 0x7fffffff : e;
-#pragma unroll
-      for (int i = 0; i < kMaxE / 32; ++i)
-        if (key[i] == best) key[i] = 0;
     }
   }
-  // ascending expert id (insertion sort, identical on every lane)
+  auto local_best = [&](uint32_t& best, int& bi) {
+    best = 0;
+    bi = 0;
 #pragma unroll
-  for (int r = 1; r < kMaxTopK; ++r)
-#pragma unroll
-    for (int q = r; q > 0; --q)
-      if (sel[q] < sel[q - 1]) {
-        const int tmp = sel[q];
-        sel[q] = sel[q - 1];
-        sel[q - 1] = tmp;
+    for (int i = 0; i < kMaxE / 32; ++i)
+      if (((avail >> i) & 1u) && bits[i] > best) {  // strict: the lower id keeps a tie
+        best = bits[i];
+        bi = i;
       }
+  };
+  uint32_t best;
+  int bi;
+  local_best(best, bi);
+  uint32_t chosen = 0;
+  bool short_of_candidates = false;
+#pragma unroll 1
+  for (int r = 0; r < a.k; ++r) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+    if (m == 0u) {  // no candidate left: cannot happen for a validated shape
+      short_of_candidates = true;
+      break;
+    }
+    const uint32_t mine = best == m ? static_cast<uint32_t>(e0 + bi) : 0xffffffffu;
+    const uint32_t win = __reduce_min_sync(0xffffffffu, mine);
+    if (mine == win) {
+      chosen |= 1u << bi;
+      avail &= ~(1u << bi);
+      local_best(best, bi);
+    }
+  }
+
+  // ---- ascending expert ids: lanes in order, each lane's experts in order
+  const int cnt = __popc(chosen);
+  int incl = cnt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  int pos = incl - cnt;
+#pragma unroll
+  for (int i = 0; i < kMaxE / 32; ++i)
+    if ((chosen >> i) & 1u) sel_sh[warp][pos++] = e0 + i;
+  __syncwarp();
   float denom = 0.f;
 #pragma unroll
   for (int r = 0; r < kMaxTopK; ++r)
-    if (r < a.k && sel[r] < E) denom += s_w[sel[r]];
-
-#pragma unroll
-  for (int r = 0; r < kMaxTopK; ++r) {
-    if (r < a.k && lane == r) {
-      const int e = sel[r];
-      const size_t slot = static_cast<size_t>(t) * a.k + r;
-      if (e < 0 || e >= E) {  // no candidate left: cannot happen for a validated shape
-        record_status(a.status, kDevAssert, kWhereSelect);
-        a.idx[slot] = 0;
-        a.w[slot] = 0.f;
-        if (a.cnt) a.rank[slot] = -1;
-        continue;
-      }
-      const float s = s_w[e];
+    if (r < total) denom += sw[sel_sh[warp][r]];
+  if (lane < a.k) {
+    const size_t slot = static_cast<size_t>(t) * a.k + lane;
+    if (lane >= total) {
+      if (lane == total && short_of_candidates) record_status(a.status, kDevAssert, kWhereSelect);
+      a.idx[slot] = 0;
+      a.w[slot] = 0.f;
+      if (a.cnt) a.rank[slot] = -1;
+    } else {
+      const int e = sel_sh[warp][lane];
+      const float s = sw[e];
       a.idx[slot] = e;
       a.w[slot] = a.norm ? a.scale * s / denom : a.scale * s;
       if (a.cnt) a.rank[slot] = atomicAdd(a.cnt + e, 1);
@@ -409,7 +461,7 @@ cudaError_t launch_router_gemm(const CUtensorMap& tmH, const CUtensorMap& tmW,
 }
 
 cudaError_t launch_router_select(const SelectArgs& a, cudaStream_t s) {
-  router_select_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(a);
+  router_select_kernel<<<(a.T + kSelTokens - 1) / kSelTokens, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -258,6 +258,11 @@ _TINY = W.WORKLOADS["tiny"]
     ("one_expert_per_group", dict(T=77, d=256, E=8, n_group=8, topk_group=3, top_k=3, I=128)),
     ("d8192", dict(T=40, d=8192, E=8, n_group=2, topk_group=1, top_k=2, I=128)),
     ("many_tokens", dict(T=20000, d=256, E=16, n_group=4, topk_group=2, top_k=4, I=128)),
+    # groups that straddle the selection's per-lane expert runs (ceil(E/32) experts a lane)
+    ("E48_G8", dict(T=200, d=256, E=48, n_group=8, topk_group=3, top_k=5, I=128)),
+    ("E200_G8", dict(T=130, d=256, E=200, n_group=8, topk_group=2, top_k=8, I=128)),
+    ("E256_G32", dict(T=64, d=256, E=256, n_group=32, topk_group=4, top_k=8, I=128)),
+    ("E20_G5", dict(T=70, d=256, E=20, n_group=5, topk_group=2, top_k=3, I=128)),
 ])
 def test_forward_other_shapes(name, changes):
     import dataclasses
