@@ -237,7 +237,6 @@ def kernel_work(wl, touched: int):
     w_gu = touched * 2 * I * d * bf
     w_dn = touched * d * I * bf
     return {
-        "router_split": {"flops": 0, "bytes": E * d * f4 + 3 * E * d * bf},
         "router_gemm": {"flops": 2 * T * d * E, "bytes": T * d * bf + E * d * f4 + T * E * f4},
         "router_select": {"flops": 0, "bytes": T * E * f4 + 2 * R * f4},
         "permute": {"flops": 0, "bytes": T * d * bf + R * d * bf},

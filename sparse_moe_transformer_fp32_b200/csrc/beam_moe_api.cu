@@ -5,7 +5,6 @@
 
 #include <cudaTypedefs.h>
 
-#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -34,14 +33,14 @@ enum KernelId {
   kKCombine,
   kKCombineBlock,
   kKPreNorm,
-  kKRouterSplit,
+  kKRouterTranspose,
   kKDenseTiles,
   kKBiasUpdate,
   kNumKernels
 };
 const char* const kKernelNames[kNumKernels] = {
     "router_gemm", "router_select", "dispatch_scan", "permute", "expert_gemm_gate_up",
-    "expert_gemm_down", "combine", "combine_block", "prenorm", "router_split", "dense_tiles",
+    "expert_gemm_down", "combine", "combine_block", "prenorm", "router_transpose", "dense_tiles",
     "bias_update"};
 
 struct Profiler {
@@ -129,25 +128,29 @@ beam_status check_shape(const beam_moe_shape* s) {
 
 struct Layout {
   size_t status, cnt, off, mt_count, mtiles, rank, rowmap, idx, w, wt, part, h, xp, act, y, total;
-  int S, kb_per_split;  // router K splits and K blocks (of kBK) per split
+  int S, kchunk;
   int64_t R, mt_cap;
 };
 
-// Router split-K factor S from a simple cost model of the tcgen05 logits kernel on a 148-SM
-// B200 (one CTA per SM): waves of (token tile, expert tile, K split) CTAs, each streaming its
-// K blocks through L2 at ~0.7 us per 64 KB stage plus ~3 us of setup and epilogue, plus the
-// traffic of writing and re-reading S partial logit arrays.  At most max_s splits.
-int router_split(const beam_moe_shape& s, int max_s) {
-  const int64_t tiles = ceil_div(s.T, kRouterM) * ceil_div(s.E, kRouterN);
-  const int64_t kblocks = s.d / kBK;
-  const double t_kb = 0.7e-6, t_cta = 3e-6, hbm = 6.5e12;
+// Router split-K factor S from a simple cost model: the FFMA time of the waves of
+// (token tile, expert tile, K chunk) blocks over the resident router blocks of a 148-SM B200,
+// plus the traffic of writing and re-reading S partial logit arrays.  K chunks are a multiple
+// of the router's K step.
+int router_split(const beam_moe_shape& s) {
+  const int64_t tiles = ceil_div(s.T, kRM) * ceil_div(s.E, kRN);
+  const int64_t kblocks = s.d / kRK;
+  const double block_flops_per_k = 2.0 * kRM * kRN;
+  const double slot_rate = 70e12 / kRouterSlots;  // FP32 FLOP/s per resident block
+  const double hbm = 6.5e12;
   int best = 1;
   double best_t = 1e30;
-  for (int S = 1; S <= max_s && S <= kblocks; ++S) {
+  for (int S = 1; S <= 16 && S <= kblocks; ++S) {
     const int64_t per = ceil_div(kblocks, S);
-    if (ceil_div(kblocks, per) != S) continue;
+    const int64_t Sx = ceil_div(kblocks, per);
+    if (Sx != S) continue;
     const double waves = static_cast<double>(ceil_div(tiles * S, kRouterSlots));
-    const double t = waves * (per * t_kb + t_cta) + static_cast<double>(S) * s.T * s.E * 8.0 / hbm;
+    const double t = waves * per * kRK * block_flops_per_k / slot_rate +
+                     static_cast<double>(S) * s.T * s.E * 8.0 / hbm;
     if (t < best_t * 0.97) {  // a larger split must win clearly
       best_t = t;
       best = S;
@@ -160,9 +163,10 @@ Layout plan(const beam_moe_shape& s) {
   Layout L{};
   const int64_t T = s.T, R = T * s.top_k;
   L.R = R;
-  const int64_t kblocks = s.d / kBK;
-  L.kb_per_split = static_cast<int>(ceil_div(kblocks, router_split(s, 64)));
-  L.S = static_cast<int>(ceil_div(kblocks, L.kb_per_split));
+  const int64_t kblocks = s.d / kRK;
+  const int S = router_split(s);
+  L.kchunk = static_cast<int>(ceil_div(kblocks, S) * kRK);
+  L.S = static_cast<int>(ceil_div(s.d, L.kchunk));
   L.mt_cap = ceil_div(R, kBM) + s.E;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -179,7 +183,7 @@ Layout plan(const beam_moe_shape& s) {
   L.rowmap = take(sizeof(int32_t) * R);
   L.idx = take(sizeof(int32_t) * R);
   L.w = take(sizeof(float) * R);
-  L.wt = take(3 * sizeof(__nv_bfloat16) * static_cast<size_t>(s.E) * s.d);
+  L.wt = take(sizeof(float) * static_cast<size_t>(s.E) * s.d);
   L.part = take(sizeof(float) * static_cast<size_t>(L.S) * T * s.E);
   L.h = take(sizeof(__nv_bfloat16) * T * s.d);
   L.xp = take(sizeof(__nv_bfloat16) * R * s.d);
@@ -240,27 +244,6 @@ beam_status make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
   return BEAM_OK;
 }
 
-// The three BF16 terms of the router weight, [3, E, d] (d contiguous), as one 3-D view whose
-// box holds kRouterN rows of all three terms; rows past E read as zeros.
-beam_status make_router_w_map(CUtensorMap* m, const void* base, uint64_t d, uint64_t E) {
-  auto fn = encode_fn();
-  if (!fn) return cuda_fail(cudaErrorNotSupported);
-  const cuuint64_t dims[3] = {d, E, 3};
-  const cuuint64_t strides[2] = {d * 2, E * d * 2};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kRouterN), 3};
-  const cuuint32_t es[3] = {1, 1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
-                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled: %d",
-                  static_cast<int>(r));
-    return BEAM_ERR_CUDA;
-  }
-  return BEAM_OK;
-}
-
 // ------------------------------------------------------------------ per-device state
 
 struct DeviceInfo {
@@ -285,8 +268,6 @@ beam_status device_info(DeviceInfo** out) {
     if (e != cudaSuccess) return cuda_fail(e);
     e = prepare_gemm_2sm_kernels();
     if (e != cudaSuccess) return cuda_fail(e);
-    e = prepare_router_kernels();
-    if (e != cudaSuccess) return cuda_fail(e);
     d.pair_grid = max_pair_grid(d.sms);
     d.prepared = true;
   }
@@ -296,30 +277,25 @@ beam_status device_info(DeviceInfo** out) {
 
 // ------------------------------------------------------------------ launch sequences
 
-// Router: weight split, logits partials, then selection (+ counts and ranks when dispatching).
-beam_status run_router(const beam_moe_shape& s, const Layout& L, const DeviceInfo& dev,
-                       const __nv_bfloat16* h, const float* router_w, const float* bias,
-                       int32_t* idx, float* w, float* logits_out, bool dispatch, void* ws,
-                       cudaStream_t st) {
-  __nv_bfloat16* w3 = at<__nv_bfloat16>(ws, L.wt);
-  CUtensorMap tm_h, tm_w;
-  beam_status b;
-  if ((b = make_map(&tm_h, h, s.d, s.T, kRouterM)) != BEAM_OK) return b;
-  if ((b = make_router_w_map(&tm_w, w3, s.d, s.E)) != BEAM_OK) return b;
-  RouterMmaArgs ga{};
+// Router: logits partials, then selection (+ counts and ranks when dispatching).
+beam_status run_router(const beam_moe_shape& s, const Layout& L, const __nv_bfloat16* h,
+                       const float* router_w, const float* bias, int32_t* idx, float* w,
+                       float* logits_out, bool dispatch, void* ws, cudaStream_t st) {
+  RouterGemmArgs ga{};
+  ga.h = h;
+  ga.WT = at<float>(ws, L.wt);
   ga.part = at<float>(ws, L.part);
   ga.zero_counts = at<int32_t>(ws, L.cnt);
-  ga.status = at<uint32_t>(ws, L.status);
-  ga.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   ga.T = s.T;
+  ga.d = s.d;
   ga.E = s.E;
-  ga.k_blocks = s.d / kBK;
-  ga.kb_per_split = L.kb_per_split;
+  ga.kchunk = L.kchunk;
   // the status words reflect the latest call: cleared before the first kernel runs
   cudaError_t e = cudaMemsetAsync(at<uint32_t>(ws, L.status), 0, 16, st);
   if (e != cudaSuccess) return cuda_fail(e);
-  BEAM_LAUNCH(kKRouterSplit, st, launch_router_split(router_w, w3, s.E, s.d, dev.sms, st));
-  BEAM_LAUNCH(kKRouterGemm, st, launch_router_gemm(tm_h, tm_w, ga, st));
+  BEAM_LAUNCH(kKRouterTranspose, st,
+              launch_router_transpose(router_w, at<float>(ws, L.wt), s.E, s.d, st));
+  BEAM_LAUNCH(kKRouterGemm, st, launch_router_gemm(ga, L.S, st));
 
   SelectArgs sa{};
   sa.part = ga.part;
@@ -451,9 +427,8 @@ bool any_misaligned(std::initializer_list<const void*> ps) {
 // array's name as a device address (on the host it names a shadow variable); the device
 // address is obtained once per device with cudaGetSymbolAddress and kept in static_scratch.
 // Sized for the largest route plan with T <= kStaticRouteMaxTokens at any supported d and E:
-// status words, per-expert counters, the three BF16 terms of the router weight (<= 3 x 256 x
-// 8192) and as many split-K partial logit arrays of T x E FP32 as fit in the rest (>= 8 at
-// T = 512, E = 256).
+// status words, per-expert counters, the transposed router weight (<= 256 x 8192 FP32) and
+// up to 16 split-K partial logit arrays of T x 256 FP32.
 constexpr int kStaticRouteMaxTokens = 512;
 constexpr size_t kStaticRouteScratchBytes = (size_t(16) << 20) + 8192;
 static __device__ __align__(256) unsigned char g_static_route_scratch[kStaticRouteScratchBytes];
@@ -462,15 +437,10 @@ static __device__ __align__(256) unsigned char g_static_route_scratch[kStaticRou
 Layout plan_route_static(const beam_moe_shape& s) {
   Layout L{};
   L.R = static_cast<int64_t>(s.T) * s.top_k;
-  const int64_t kblocks = s.d / kBK;
-  // as many K splits as the scratch left after the weight terms holds (at least one)
-  const size_t fixed = 256 + align_up(sizeof(int32_t) * s.E, 256) +
-                       align_up(3 * sizeof(__nv_bfloat16) * s.E * s.d, 256);
-  const size_t per_split = sizeof(float) * static_cast<size_t>(s.T) * s.E;
-  const size_t room = kStaticRouteScratchBytes > fixed ? kStaticRouteScratchBytes - fixed : 0;
-  const int max_s = static_cast<int>(std::max<size_t>(1, std::min<size_t>(64, room / per_split)));
-  L.kb_per_split = static_cast<int>(ceil_div(kblocks, router_split(s, max_s)));
-  L.S = static_cast<int>(ceil_div(kblocks, L.kb_per_split));
+  const int64_t kblocks = s.d / kRK;
+  const int S = router_split(s);
+  L.kchunk = static_cast<int>(ceil_div(kblocks, S) * kRK);
+  L.S = static_cast<int>(ceil_div(s.d, L.kchunk));
   size_t o = 0;
   auto take = [&](size_t bytes) {
     const size_t r = o;
@@ -479,7 +449,7 @@ Layout plan_route_static(const beam_moe_shape& s) {
   };
   L.status = take(256);
   L.cnt = take(sizeof(int32_t) * s.E);
-  L.wt = take(3 * sizeof(__nv_bfloat16) * static_cast<size_t>(s.E) * s.d);
+  L.wt = take(sizeof(float) * static_cast<size_t>(s.E) * s.d);
   L.part = take(sizeof(float) * static_cast<size_t>(L.S) * s.T * s.E);
   L.total = o;
   return L;
@@ -568,9 +538,8 @@ beam_status beam_moe_route_static(const beam_moe_shape* shape, const void* hidde
   if ((b = device_info(&dev)) != BEAM_OK) return b;
   void* scratch = nullptr;
   if ((b = static_scratch(&scratch)) != BEAM_OK) return b;
-  return run_router(*shape, L, *dev, static_cast<const __nv_bfloat16*>(hidden), router_w, bias,
-                    topk_idx, topk_w, logits_out, false, scratch,
-                    reinterpret_cast<cudaStream_t>(stream));
+  return run_router(*shape, L, static_cast<const __nv_bfloat16*>(hidden), router_w, bias, topk_idx,
+                    topk_w, logits_out, false, scratch, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t beam_moe_workspace_size(const beam_moe_shape* shape) {
@@ -613,8 +582,8 @@ beam_status beam_moe_route(const beam_moe_shape* shape, const void* hidden, cons
   DeviceInfo* dev;
   if ((b = device_info(&dev)) != BEAM_OK) return b;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return run_router(*shape, L, *dev, static_cast<const __nv_bfloat16*>(hidden), router_w, bias,
-                    topk_idx, topk_w, logits_out, false, ws, st);
+  return run_router(*shape, L, static_cast<const __nv_bfloat16*>(hidden), router_w, bias, topk_idx,
+                    topk_w, logits_out, false, ws, st);
 }
 
 beam_status beam_moe_forward(const beam_moe_shape* shape, const void* hidden, const float* router_w,
@@ -635,8 +604,8 @@ beam_status beam_moe_forward(const beam_moe_shape* shape, const void* hidden, co
   int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
   float* w = topk_w ? topk_w : at<float>(ws, L.w);
   const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(hidden);
-  b = run_router(*shape, L, *dev, h, router_w, bias, idx, w, nullptr, true, ws, st);
-  if (b != BEAM_OK) return b;
+  if ((b = run_router(*shape, L, h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
+    return b;
   if ((b = run_experts(*shape, L, *dev, h, idx, w_gate, w_up, w_down, ws, st)) != BEAM_OK)
     return b;
   CombineArgs ca{};
@@ -688,8 +657,8 @@ beam_status beam_moe_block(const beam_moe_shape* shape, const float* x, const fl
 
   int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
   float* w = topk_w ? topk_w : at<float>(ws, L.w);
-  b = run_router(*shape, L, *dev, pn.h, router_w, bias, idx, w, nullptr, true, ws, st);
-  if (b != BEAM_OK) return b;
+  if ((b = run_router(*shape, L, pn.h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
+    return b;
   if ((b = run_experts(*shape, L, *dev, pn.h, idx, w_gate, w_up, w_down, ws, st)) != BEAM_OK)
     return b;
   const double kk = static_cast<double>(k_resid);

@@ -30,16 +30,9 @@ constexpr int kStageBBytes = kUmmaN * kBK * 2;     // 32 KB
 constexpr int kStageBytes = kStageABytes + kStageBBytes;
 constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*align*/;
 
-// router logits GEMM (tcgen05, three BF16 terms of the FP32 router weight)
-constexpr int kRouterM = 128;       // tokens per tile = UMMA M
-constexpr int kRouterN = 128;       // experts per tile = UMMA N = TMEM columns
-constexpr int kRouterStages = 3;
-constexpr int kRouterChunk = 2;     // K blocks (24 MMAs) per accumulator hand-over
-constexpr int kRouterThreads = 192; // warp 0 TMA, warp 1 MMA, warps 2..5 chunk sums
-constexpr int kRouterStageABytes = kRouterM * kBK * 2;                   // 16 KB
-constexpr int kRouterStageBytes = kRouterStageABytes + 3 * kRouterN * kBK * 2;  // 64 KB
-constexpr int kRouterSmemBytes = kRouterStages * kRouterStageBytes + 1024 + 1024;
-constexpr int kRouterSlots = 148;   // resident router CTAs on a 148-SM B200 (one per SM)
+// router GEMM tiling (FP32 FFMA)
+constexpr int kRM = 128, kRN = 128, kRK = 16, kRThreads = 256, kRBStages = 3;
+constexpr int kRouterSlots = 2 * 148;  // resident router blocks on a 148-SM B200
 
 constexpr int kMaxTopK = 8;
 constexpr int kMaxE = 256;
@@ -84,14 +77,12 @@ struct MTile {
 
 // ------------------------------------------------------------------ kernel arguments
 
-struct RouterMmaArgs {
+struct RouterGemmArgs {
+  const __nv_bfloat16* h;  // [T, d]
+  const float* WT;         // [d, E] (transposed router weight)
   float* part;             // [S, T, E]
-  int32_t* zero_counts;    // [E] zeroed by CTA (0,0,0), or null
-  uint32_t* status;
-  uint64_t wait_limit_ns;
-  int T, E;
-  int k_blocks;            // d / kBK
-  int kb_per_split;        // K blocks per split (grid z)
+  int32_t* zero_counts;    // [E] zeroed by block (0,0,0), or null
+  int T, d, E, kchunk;
 };
 
 struct SelectArgs {
@@ -165,11 +156,8 @@ struct PreNormArgs {
 
 // ------------------------------------------------------------------ launchers (one per kernel)
 
-cudaError_t launch_router_split(const float* W, __nv_bfloat16* Ws, int E, int d, int sms,
-                                cudaStream_t s);
-cudaError_t launch_router_gemm(const CUtensorMap& tmH, const CUtensorMap& tmW,
-                               const RouterMmaArgs& a, cudaStream_t s);
-cudaError_t prepare_router_kernels();  // opt-in shared memory size (once per device)
+cudaError_t launch_router_transpose(const float* W, float* WT, int E, int d, cudaStream_t s);
+cudaError_t launch_router_gemm(const RouterGemmArgs& a, int S, cudaStream_t s);
 cudaError_t launch_router_select(const SelectArgs& a, cudaStream_t s);
 cudaError_t launch_dispatch_scan(const DispatchArgs& a, cudaStream_t s);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
@@ -285,16 +273,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
-      : "memory");
-}
-
-// 3-D tiled load of a box at (x, y, z) (x innermost), completing on mbarrier `bar`.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, uint32_t bar,
-                                            int32_t x, int32_t y, int32_t z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 

@@ -1,4 +1,4 @@
-// Router of the Beam sparse-MoE layer: FP32 logits on the tensor cores, then sigmoid scores,
+// Router of the Beam sparse-MoE layer: FP32 logits on the CUDA cores, then sigmoid scores,
 // selection-only bias, group-limited top-k and normalised, scaled weights.
 //
 // Transformers model doc "Beam", Overview: the router scores experts with a sigmoid, balances
@@ -14,235 +14,145 @@
 namespace beam {
 namespace {
 
-// ---------------------------------------------------------------- W_r split
+// ---------------------------------------------------------------- W_r transpose
 //
-// The logits run on the tensor cores as BF16 x BF16 products with FP32 accumulation.  h is
-// BF16 already; the FP32 router weight is written as the sum of three BF16 terms
-//     w1 = bf16(W),  w2 = bf16(W - w1),  w3 = bf16(W - w1 - w2)
-// (round to nearest even).  Each difference is exact in FP32 and each rounding leaves at most
-// 2^-8 of what it rounds, so |W - (w1 + w2 + w3)| <= 2^-24 |W|: the FP32 weight itself, up to
-// its own unit roundoff.  Products of BF16 values are exact in FP32, so h . W = h . w1 +
-// h . w2 + h . w3 is an FP32-accumulated FP32 dot product.  Ws is [3, E, d] BF16, written
-// into the workspace on every call (7.9 MB at Beam shapes).
-__global__ void __launch_bounds__(256) router_split_kernel(const float4* __restrict__ W,
-                                                           uint2* __restrict__ Ws, size_t n4) {
-  for (size_t i = static_cast<size_t>(blockIdx.x) * 256 + threadIdx.x; i < n4;
-       i += static_cast<size_t>(gridDim.x) * 256) {
-    const float4 v = W[i];
-    float r[4] = {v.x, v.y, v.z, v.w};
+// The logits GEMM streams the router weight along the expert index; a transposed copy
+// W_rT [d, E] (5 MB at Beam shapes) is written into the workspace on every call.
+__global__ void __launch_bounds__(256) router_transpose_kernel(const float* __restrict__ W,
+                                                               float* __restrict__ WT, int E, int d) {
+  __shared__ float tile[32][33];
+  const int e0 = blockIdx.y * 32, k0 = blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
 #pragma unroll
-    for (int term = 0; term < 3; ++term) {
-      uint32_t p[2];
+  for (int r = ty; r < 32; r += 8) {
+    const int e = e0 + r;
+    tile[r][tx] = e < E ? W[static_cast<size_t>(e) * d + k0 + tx] : 0.f;
+  }
+  __syncthreads();
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const __nv_bfloat16 lo = __float2bfloat16_rn(r[2 * j]);
-        const __nv_bfloat16 hi = __float2bfloat16_rn(r[2 * j + 1]);
-        r[2 * j] -= __bfloat162float(lo);
-        r[2 * j + 1] -= __bfloat162float(hi);
-        p[j] = static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
-               (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
-      }
-      Ws[term * n4 + i] = make_uint2(p[0], p[1]);
-    }
+  for (int r = ty; r < 32; r += 8) {
+    const int e = e0 + tx;
+    if (e < E) WT[static_cast<size_t>(k0 + r) * E + e] = tile[tx][r];
   }
 }
 
-// ---------------------------------------------------------------- logits: tcgen05 GEMM
+// ---------------------------------------------------------------- logits: FP32 FFMA GEMM
 //
-// part[z, t, e] = sum over the K blocks of split z of h[t, :] . (w1 + w2 + w3)[e, :]
-// One CTA per (128-token tile, 128-expert tile, K split), 192 threads:
-//   warp 0     one thread issues TMA loads into a 3-stage ring; a stage holds the 128 x 64 BF16
-//              h tile and one 3-D box with the three 128 x 64 weight-term tiles (64 KB)
-//   warp 1     allocates 256 TMEM columns (two 128-column accumulators); one thread issues 12
-//              tcgen05.mma (M=128, N=128, K=16) per stage, the three terms into the same
-//              accumulator, and hands the accumulator over every kRouterChunk stages
-//   warps 2-5  add each handed-over accumulator into FP32 registers (one token row per thread,
-//              its warp's 32-lane TMEM quarter), then store the row's partial logits
-// The tensor cores accumulate with less care than round-to-nearest FP32 adds: the logit error
-// grows with the number of MMAs summed into one accumulator (measured ~1e-6 per 24 MMAs at
-// d = 5120, ~6e-5 when all 960 of a full-K tile are chained).  Chunks of 24 MMAs summed by
-// FP32 adds in a fixed order keep it at the level of a plain FP32 dot product.
-// Rows past T and experts past E are zero-filled by TMA and never stored.  The selection
-// kernel adds the K-split partials in a fixed order, so the result is deterministic.
-// Waits are bounded as in the expert GEMMs: a timeout is recorded in the status word, the CTA
-// drains its own TMA loads and MMAs, frees TMEM and returns.
-constexpr uint64_t kRouterMinDrainNs = 1000000000ull;
+// part[z, t, e] = sum_{j in K-chunk z} float(h[t, j]) * W[e, j].  Block tile 128 tokens x 128
+// experts x 16 K, 256 threads, each an 8 x 8 register tile (rows ty*4.., 64+ty*4..; columns
+// tx*4.., 64+tx*4..).  h is staged through registers (BF16 -> FP32, transposed into As[k][t]
+// with a warp covering 32 consecutive tokens, so the stores are conflict-free); W_rT streams
+// into a 3-stage cp.async ring.  Split-K over gridDim.z fills the machine for small T; the
+// selection kernel adds the partial sums in a fixed order.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_1() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
 
-__global__ void __launch_bounds__(kRouterThreads, 1)
-    router_mma_kernel(const __grid_constant__ CUtensorMap tmH,
-                      const __grid_constant__ CUtensorMap tmW, const RouterMmaArgs a) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t sbase = (raw + 1023u) & ~1023u;
-  uint8_t* smem = smem_raw + (sbase - raw);
-  // [kRouterStages x (h 16 KB | w1, w2, w3 48 KB)][barriers][TMEM address][abort flag]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRouterStages * kRouterStageBytes);
-  constexpr int kBarFull = 0, kBarEmpty = kRouterStages, kBarCFull = 2 * kRouterStages,
-                kBarCEmpty = kBarCFull + 2, kBarDrain = kBarCEmpty + 2, kNumBars = kBarDrain + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  auto bar = [&](int i) { return smem_u32(bars + i); };
+__global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterGemmArgs a) {
+  __shared__ __align__(16) float As[2][kRK][kRM];
+  __shared__ __align__(16) float Bs[kRBStages][kRK][kRN];
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kRouterM, n0 = blockIdx.y * kRouterN;
-  const int kb0 = blockIdx.z * a.kb_per_split;
-  const int kb1 = min(a.k_blocks, kb0 + a.kb_per_split);
-  const int nchunks = (kb1 - kb0 + kRouterChunk - 1) / kRouterChunk;
-  const uint64_t limit = a.wait_limit_ns;
-  const uint64_t drain_limit = limit > kRouterMinDrainNs ? limit : kRouterMinDrainNs;
+  const int tid = threadIdx.x;
+  const int m0 = blockIdx.x * kRM;
+  const int n0 = blockIdx.y * kRN;
+  const int kbeg = blockIdx.z * a.kchunk;
+  const int kend = min(a.d, kbeg + a.kchunk);
+  const int nk = (kend - kbeg) / kRK;
 
   if (a.zero_counts && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) a.zero_counts[e] = 0;
+    for (int e = tid; e < a.E; e += blockDim.x) a.zero_counts[e] = 0;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kRouterStages; ++s) {
-      mbar_init(bar(kBarFull + s), 1);
-      mbar_init(bar(kBarEmpty + s), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(kBarCFull + i), 1);
-      mbar_init(bar(kBarCEmpty + i), 4);
-    }
-    mbar_init(bar(kBarDrain), 1);
-    *abort_flag = 0;
-    fence_mbarrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmH);
-    tma_prefetch_desc(&tmW);
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 2 * kRouterN);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
+  const int tx = tid & 15;
+  const int ty = tid >> 4;
+  // A staging: one 16-byte chunk (8 K values) of one token per thread and K tile
+  const int a_row = tid & (kRM - 1);
+  const int a_kp = (tid >> 7) * 8;
+  const int a_t = m0 + a_row;
+  const __nv_bfloat16* a_src = a.h + static_cast<size_t>(a_t < a.T ? a_t : 0) * a.d + a_kp;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, filled = 0, last_parity = 0;
-      for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait_bounded(bar(kBarEmpty + stage), phase ^ 1u, abort_flag, limit, a.status,
-                               kWhereProducerEmpty))
-          break;
-        const uint32_t sA = sbase + stage * kRouterStageBytes;
-        const uint32_t fb = bar(kBarFull + stage);
-        mbar_arrive_expect_tx(fb, kRouterStageBytes);
-        tma_load_2d(sA, &tmH, fb, kb * kBK, m0);
-        tma_load_3d(sA + kRouterStageABytes, &tmW, fb, kb * kBK, n0, 0);
-        filled |= 1u << stage;
-        last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == kRouterStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-      // every load this thread issued must land before the CTA may exit
-      int no_abort = 0;
-      for (int s = 0; s < kRouterStages; ++s)
-        if ((filled >> s) & 1u)
-          mbar_wait_bounded(bar(kBarFull + s), (last_parity >> s) & 1u, &no_abort, drain_limit,
-                            a.status, kWhereDrain);
+  auto load_a = [&](int k0) -> uint4 {
+    return a_t < a.T ? *reinterpret_cast<const uint4*>(a_src + k0) : make_uint4(0, 0, 0, 0);
+  };
+  auto store_a = [&](int buf, uint4 v) {
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      As[buf][a_kp + 2 * q][a_row] = __uint_as_float(w4[q] << 16);
+      As[buf][a_kp + 2 * q + 1][a_row] = __uint_as_float(w4[q] & 0xffff0000u);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16_f32(kRouterM, kRouterN);
-      constexpr uint32_t kTermBytes = kRouterN * kBK * 2;
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int c = 0; c < nchunks && ok; ++c) {
-        const int buf = c & 1;
-        const uint32_t cphase = static_cast<uint32_t>(c >> 1) & 1u;
-        if (!mbar_wait_bounded(bar(kBarCEmpty + buf), cphase ^ 1u, abort_flag, limit, a.status,
-                               kWhereMmaTmemEmpty))
-          break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kRouterN);
-        const int c0 = kb0 + c * kRouterChunk;
-        const int c1 = min(kb1, c0 + kRouterChunk);
-        for (int kb = c0; kb < c1; ++kb) {
-          if (!mbar_wait_bounded(bar(kBarFull + stage), phase, abort_flag, limit, a.status,
-                                 kWhereMmaFull)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sA = sbase + stage * kRouterStageBytes;
-          const uint64_t adesc = smem_desc_k_sw128(sA);
+  };
+  auto issue_b = [&](int stage, int k0) {
 #pragma unroll
-          for (int term = 0; term < 3; ++term) {
-            const uint64_t bdesc = smem_desc_k_sw128(sA + kRouterStageABytes + term * kTermBytes);
-#pragma unroll
-            for (int k = 0; k < kBK / kUmmaK; ++k)  // +32 bytes along K per step: +2 in addr>>4
-              umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc,
-                        (kb != c0 || term != 0 || k != 0) ? 1u : 0u);
-          }
-          umma_commit(bar(kBarEmpty + stage));
-          if (++stage == kRouterStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (ok) umma_commit(bar(kBarCFull + buf));
-      }
-      // all MMAs this thread issued must complete before TMEM is freed
-      int no_abort = 0;
-      umma_commit(bar(kBarDrain));
-      mbar_wait_bounded(bar(kBarDrain), 0, &no_abort, drain_limit, a.status, kWhereDrain);
+    for (int i = 0; i < (kRK * kRN / 4) / kRThreads; ++i) {
+      const int c = tid + i * kRThreads;
+      const int k = c / (kRN / 4), n4 = (c % (kRN / 4)) * 4;
+      const int e = n0 + n4;
+      const bool ok = e < a.E;  // E % 4 == 0: a chunk is wholly in or out
+      const float* src = a.WT + static_cast<size_t>(k0 + k) * a.E + (ok ? e : 0);
+      cp_async16(smem_u32(&Bs[stage][k][n4]), src, ok ? 16 : 0);
     }
-  } else {
-    // ------------------------------------------------------------ chunk sums, then stores
-    const int q = warp & 3;  // TMEM lane quarter this warp may access (warps 2..5)
-    const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    float acc[kRouterN];
+  };
+
+  float acc[8][8];
 #pragma unroll
-    for (int j = 0; j < kRouterN; ++j) acc[j] = 0.f;
-    bool ok = true;
-    for (int c = 0; c < nchunks; ++c) {
-      const int buf = c & 1;
-      const uint32_t cphase = static_cast<uint32_t>(c >> 1) & 1u;
-      ok = mbar_wait_bounded(bar(kBarCFull + buf), cphase, abort_flag, limit, a.status,
-                             kWhereEpiTmemFull);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int g = 0; g < kRouterN / 32; ++g) {
-        uint32_t v[32];
-        tmem_ld32_sync(tq + static_cast<uint32_t>(buf * kRouterN + g * 32), v);
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  if (nk > 0) {
+    issue_b(0, kbeg);
+    cp_async_commit();
+    if (nk > 1) issue_b(1, kbeg + kRK);
+    cp_async_commit();
+    store_a(0, load_a(kbeg));
+  }
+#pragma unroll 1
+  for (int kt = 0; kt < nk; ++kt) {
+    cp_async_wait_1();  // this tile's B has landed (one newer group may be in flight)
+    __syncthreads();    // ... for every thread, and As[kt & 1] is stored
+    if (kt + 2 < nk) issue_b((kt + 2) % kRBStages, kbeg + (kt + 2) * kRK);
+    cp_async_commit();
+    uint4 next = make_uint4(0, 0, 0, 0);
+    if (kt + 1 < nk) next = load_a(kbeg + (kt + 1) * kRK);
+    const int buf = kt & 1, st = kt % kRBStages;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc[g * 32 + j] += __uint_as_float(v[j]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarCEmpty + buf));
+    for (int kk = 0; kk < kRK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[st][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[st][kk][64 + tx * 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
-    const int t = m0 + q * 32 + lane;
-    if (ok && t < a.T) {
-      float* prow = a.part + (static_cast<size_t>(blockIdx.z) * a.T + t) * a.E;
-#pragma unroll
-      for (int j = 0; j < kRouterN; j += 4) {
-        const int e = n0 + j;  // E % 4 == 0: a group of four is wholly in or out
-        if (e < a.E)
-          *reinterpret_cast<float4*>(prow + e) =
-              make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-      }
-    }
+    if (kt + 1 < nk) store_a(buf ^ 1, next);
   }
 
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * kRouterN);
+  float* part = a.part + static_cast<size_t>(blockIdx.z) * a.T * a.E;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+    if (t >= a.T) continue;
+    float* prow = part + static_cast<size_t>(t) * a.E;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int e = n0 + half * 64 + tx * 4;
+      if (e < a.E) {
+        const float* v = &acc[i][half * 4];
+        *reinterpret_cast<float4*>(prow + e) = make_float4(v[0], v[1], v[2], v[3]);
+      }
+    }
   }
 }
 
@@ -437,26 +347,15 @@ __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) 
 
 }  // namespace
 
-cudaError_t launch_router_split(const float* W, __nv_bfloat16* Ws, int E, int d, int sms,
-                                cudaStream_t s) {
-  const size_t n4 = static_cast<size_t>(E) * d / 4;
-  const size_t want = (n4 + 255) / 256;
-  const int grid = static_cast<int>(want < static_cast<size_t>(4 * sms) ? want : 4 * sms);
-  router_split_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(W),
-                                           reinterpret_cast<uint2*>(Ws), n4);
+cudaError_t launch_router_transpose(const float* W, float* WT, int E, int d, cudaStream_t s) {
+  const dim3 grid(d / 32, (E + 31) / 32);
+  router_transpose_kernel<<<grid, 256, 0, s>>>(W, WT, E, d);
   return cudaGetLastError();
 }
 
-cudaError_t prepare_router_kernels() {
-  return cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              kRouterSmemBytes);
-}
-
-cudaError_t launch_router_gemm(const CUtensorMap& tmH, const CUtensorMap& tmW,
-                               const RouterMmaArgs& a, cudaStream_t s) {
-  const dim3 grid((a.T + kRouterM - 1) / kRouterM, (a.E + kRouterN - 1) / kRouterN,
-                  (a.k_blocks + a.kb_per_split - 1) / a.kb_per_split);
-  router_mma_kernel<<<grid, kRouterThreads, kRouterSmemBytes, s>>>(tmH, tmW, a);
+cudaError_t launch_router_gemm(const RouterGemmArgs& a, int S, cudaStream_t s) {
+  const dim3 grid((a.T + kRM - 1) / kRM, (a.E + kRN - 1) / kRN, S);
+  router_gemm_kernel<<<grid, kRThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -135,9 +135,7 @@ def test_full_size_logits_within_fp32_dot_error(name):
     """Every router logit at the Beam shapes against the oracle's (exact sum rounded once to
     FP32).  An FP32 dot product of length 5120 with h ~ N(0, 1) and W_r ~ N(0, 0.01^2) carries
     a rounding error of order sqrt(d) * 2^-24 * |partial sums| ~ 1e-6; the bound 1e-5 leaves
-    room for the summation order and is the one the weight tolerance above is derived from.
-    A router that summed all d products into one tensor-core accumulator would miss it (that
-    error grows with the chain length, to ~6e-5 at d = 5120)."""
+    room for the summation order and is the one the weight tolerance above is derived from."""
     case = H.make_case(W.WORKLOADS[name])
     wl = case.wl
     s = bm.shape_of(wl)
