@@ -58,6 +58,14 @@ def lib():
         L.oracle_residual_coefficients.argtypes = [i32, ctypes.POINTER(ctypes.c_double),
                                                    ctypes.POINTER(ctypes.c_double)]
         L.oracle_bias_update.argtypes = [i32, vp, i64, vp, f32, vp]
+        L.oracle_f32_to_e4m3.argtypes = [i64, vp, vp]
+        L.oracle_e4m3_to_f32.argtypes = [i64, vp, vp]
+        L.oracle_quantize_rows_e4m3.argtypes = [i64, i64, vp, vp, vp, i32]
+        L.oracle_linear_fp8.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, i32]
+        L.oracle_expert_mlp_fp8.argtypes = [i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.oracle_moe_tokens_fp8.argtypes = [i64, vp, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp,
+                                            vp, vp, vp, i32]
+        L.oracle_moe_tokens_fp8.restype = i32
         _lib = L
     return _lib
 
@@ -247,3 +255,87 @@ def block_tail(x_rows, moe_out_rows, g_post, eps: float, k_resid: int, nthreads:
     """x' = x*sqrt((k-1)/k) + rmsnorm(out)*g_post / sqrt(k) for the given rows."""
     o = rmsnorm(moe_out_rows, g_post, eps, nthreads)
     return residual(x_rows, o, k_resid)
+
+
+# ------------------------------------------------------------------ FP8 (E4M3) expert weights
+
+def f32_to_e4m3(x) -> np.ndarray:
+    """E4M3 codes (uint8) of FP32 values: round to nearest even, saturate to +-448."""
+    a = np.ascontiguousarray(_np(x, np.float32))
+    out = np.empty(a.shape, np.uint8)
+    lib().oracle_f32_to_e4m3(a.size, _p(a), _p(out))
+    return out
+
+
+def e4m3_to_f32(codes) -> np.ndarray:
+    c = np.ascontiguousarray(np.asarray(codes, np.uint8))
+    out = np.empty(c.shape, np.float32)
+    lib().oracle_e4m3_to_f32(c.size, _p(c), _p(out))
+    return out
+
+
+def quantize_rows_e4m3(x, nthreads: int = 0):
+    """Row-wise E4M3 quantisation of a BF16 matrix [rows, cols] -> (codes uint8, scales f32)."""
+    b = np.ascontiguousarray(bf16_bits(x))
+    rows, cols = b.shape
+    q = np.empty((rows, cols), np.uint8)
+    s = np.empty(rows, np.float32)
+    lib().oracle_quantize_rows_e4m3(rows, cols, _p(b), _p(q), _p(s), nthreads)
+    return q, s
+
+
+def linear_fp8(xq, sx, wq, sw, nthreads: int = 0) -> np.ndarray:
+    """y[r, c] = fl32(sx_r * sw_c * sum_j xq[r, j] wq[c, j]) on decoded E4M3 codes."""
+    xq = np.ascontiguousarray(np.asarray(xq, np.uint8))
+    wq = np.ascontiguousarray(np.asarray(wq, np.uint8))
+    sx = np.ascontiguousarray(np.asarray(sx, np.float32))
+    sw = np.ascontiguousarray(np.asarray(sw, np.float32))
+    rows, K = xq.shape
+    n_out = wq.shape[0]
+    y = np.empty((rows, n_out), np.float32)
+    lib().oracle_linear_fp8(rows, n_out, K, _p(xq), _p(sx), _p(wq), _p(sw), _p(y), nthreads)
+    return y
+
+
+def expert_mlp_fp8(x, gq, sg, uq, su, dq, sd, return_act: bool = False):
+    """One E4M3 SwiGLU expert on one BF16 row x [d]; weights as (codes, row scales)."""
+    xb = np.ascontiguousarray(bf16_bits(x).reshape(-1))
+    d = xb.size
+    I = gq.shape[0]
+    arrs = [_np(a, t) for a, t in
+            ((gq, np.uint8), (sg, np.float32), (uq, np.uint8), (su, np.float32),
+             (dq, np.uint8), (sd, np.float32))]
+    y = np.empty(d, np.float32)
+    a = np.empty(I, np.uint16)
+    lib().oracle_expert_mlp_fp8(d, I, _p(xb), *[_p(v) for v in arrs], _p(y), _p(a))
+    return (y, a) if return_act else y
+
+
+def moe_tokens_fp8(tokens, h, idx, w, experts, nthreads: int = 0) -> np.ndarray:
+    """MoE output rows for `tokens` with E4M3 experts; experts maps e -> (gq, sg, uq, su, dq, sd)
+    (codes uint8 [I, d] / [d, I], row scales f32)."""
+    tokens = np.ascontiguousarray(np.asarray(tokens, np.int64))
+    hb = np.ascontiguousarray(bf16_bits(h))
+    T, d = hb.shape
+    idx = _np(idx, np.int32)
+    w = _np(w, np.float32)
+    k = idx.shape[1]
+    E = int(idx.max()) + 1 if idx.size else 0
+    E = max([E] + [int(e) + 1 for e in experts])
+    keep = []
+    ptrs = [(ctypes.c_void_p * E)() for _ in range(6)]
+    I = None
+    for e, parts in experts.items():
+        dt = (np.uint8, np.float32) * 3
+        arrs = [_np(a, t) for a, t in zip(parts, dt)]
+        keep.append(arrs)
+        I = arrs[0].shape[0]
+        for i, a in enumerate(arrs):
+            ptrs[i][e] = a.ctypes.data
+    out = np.empty((tokens.size, d), np.float32)
+    r = lib().oracle_moe_tokens_fp8(tokens.size, _p(tokens), d, I, k, _p(hb), _p(idx), _p(w),
+                                    *[ctypes.cast(p, ctypes.c_void_p) for p in ptrs], _p(out),
+                                    nthreads)
+    if r != 0:
+        raise ValueError("moe_tokens_fp8: a token uses an expert that was not supplied")
+    return out

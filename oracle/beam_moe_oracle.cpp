@@ -28,6 +28,15 @@
 // lower group / expert index.  Selected experts are reported in ascending id
 // order with their weights permuted alongside; the combine sums in that order.
 //
+// FP8 expert weights (a reading; the pages name FP8 and NVFP4 checkpoints but no scale
+// format -- news article "Reflection lança o Beam", section "Onde o Beam economiza ...";
+// review page "обзор модели «Бим»", weights and vLLM-recipe entries): E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities,
+// largest finite 448), one FP32 scale per matrix row (per output channel of a weight, per
+// token row of an activation): s = fl32(amax / 448), q = e4m3(fl32(x / s)) rounded to
+// nearest even and saturated to +-448.  The SwiGLU expert then runs as above with every
+// GEMM input quantised that way; products of codes are exact and summed in double, and the
+// two row scales are applied before the single rounding to FP32.
+//
 // Plain loops, no BLAS, no intrinsics; std::thread over tokens.
 
 #include <algorithm>
@@ -84,6 +93,80 @@ void parallel_for(int64_t n, int nthreads, F body) {
 }
 
 double sigmoid(double x) { return 1.0 / (1.0 + std::exp(-x)); }
+
+// E4M3 code -> value.  Exponent field 0 holds the subnormals m/8 * 2^-6; S.1111.111 is NaN.
+double e4m3_value(uint8_t b) {
+  const int sgn = b >> 7, e = (b >> 3) & 15, m = b & 7;
+  if (e == 15 && m == 7) return std::nan("");
+  const double v = e == 0 ? std::ldexp(m / 8.0, -6) : std::ldexp(1.0 + m / 8.0, e - 7);
+  return sgn ? -v : v;
+}
+
+// Value -> E4M3 code, round to nearest with ties to the even code, saturating to +-448.
+uint8_t e4m3_code(float f) {
+  if (std::isnan(f)) return 0x7f;
+  const uint8_t sgn = std::signbit(f) ? 0x80 : 0x00;
+  const double a = std::fabs(static_cast<double>(f));
+  uint8_t mag;
+  if (a >= 448.0) {
+    mag = 0x7e;
+  } else if (a < std::ldexp(1.0, -6)) {
+    // subnormal range: steps of 2^-9; rounding up to 8 steps gives the smallest normal (code 8)
+    mag = static_cast<uint8_t>(std::nearbyint(a / std::ldexp(1.0, -9)));
+  } else {
+    int ex;
+    std::frexp(a, &ex);  // a = f * 2^ex, f in [0.5, 1): a in [2^(ex-1), 2^ex)
+    const int E = ex - 1;
+    double r = std::nearbyint(a / std::ldexp(1.0, E - 3));  // 8 .. 16 steps of 2^(E-3)
+    int Eb = E + 7;
+    if (r == 16.0) {
+      r = 8.0;
+      ++Eb;
+    }
+    const int code = (Eb << 3) | (static_cast<int>(r) - 8);
+    mag = static_cast<uint8_t>(code > 0x7e ? 0x7e : code);
+  }
+  return static_cast<uint8_t>(sgn | mag);
+}
+
+// Quantises one BF16 row of n values: s = fl32(amax / 448), q_j = e4m3(fl32(x_j / s)).
+// An all-zero row gets s = 0 and zero codes.
+float quantize_row(int64_t n, const uint16_t* x, uint8_t* q) {
+  float amax = 0.0f;
+  for (int64_t j = 0; j < n; ++j) amax = std::max(amax, std::fabs(bf16_bits_to_float(x[j])));
+  const float s = amax / 448.0f;
+  for (int64_t j = 0; j < n; ++j)
+    q[j] = s > 0.0f ? e4m3_code(bf16_bits_to_float(x[j]) / s) : 0;
+  return s;
+}
+
+// y_c = fl32( sx * sw_c * sum_j value(xq_j) * value(Wq[c, j]) ) for c < n_out; Wq is [n_out, K].
+void linear_fp8_row(int64_t K, int64_t n_out, const uint8_t* xq, float sx, const uint8_t* Wq,
+                    const float* sw, float* y) {
+  std::vector<double> xv(K);
+  for (int64_t j = 0; j < K; ++j) xv[j] = e4m3_value(xq[j]);
+  for (int64_t c = 0; c < n_out; ++c) {
+    const uint8_t* w = Wq + c * K;
+    double acc = 0.0;
+    for (int64_t j = 0; j < K; ++j) acc += xv[j] * e4m3_value(w[j]);
+    y[c] = static_cast<float>(static_cast<double>(sx) * static_cast<double>(sw[c]) * acc);
+  }
+}
+
+// out[n, c] = fl32( sum_j w[t, j] * ys[n, j, c] ) over the k slots in their order, t = tokens[n].
+void combine_slots(int64_t ntok, const int64_t* tokens, int64_t d, int k, const float* w,
+                   const float* ys, float* out) {
+  for (int64_t n = 0; n < ntok; ++n) {
+    const int64_t t = tokens[n];
+    for (int64_t c = 0; c < d; ++c) {
+      double acc = 0.0;
+      for (int j = 0; j < k; ++j)
+        acc += static_cast<double>(w[t * k + j]) *
+               static_cast<double>(ys[(static_cast<size_t>(n) * k + j) * d + c]);
+      out[n * d + c] = static_cast<float>(acc);
+    }
+  }
+}
 
 }  // namespace
 
@@ -237,16 +320,84 @@ int oracle_moe_tokens(int64_t ntok, const int64_t* tokens, int64_t d, int64_t I,
     const int e = idx[t * k + j];
     oracle_expert_mlp(d, I, h + t * d, Wg[e], Wu[e], Wd[e], ys.data() + item * d, nullptr);
   });
-  for (int64_t n = 0; n < ntok; ++n) {
-    const int64_t t = tokens[n];
-    for (int64_t c = 0; c < d; ++c) {
-      double acc = 0.0;
-      for (int j = 0; j < k; ++j)
-        acc += static_cast<double>(w[t * k + j]) *
-               static_cast<double>(ys[(static_cast<size_t>(n) * k + j) * d + c]);
-      out[n * d + c] = static_cast<float>(acc);
-    }
+  combine_slots(ntok, tokens, d, k, w, ys.data(), out);
+  return 0;
+}
+
+void oracle_f32_to_e4m3(int64_t n, const float* in, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_code(in[i]);
+}
+
+void oracle_e4m3_to_f32(int64_t n, const uint8_t* in, float* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = static_cast<float>(e4m3_value(in[i]));
+}
+
+// Row-wise E4M3 quantisation of a BF16 matrix [rows, cols] (see quantize_row).
+void oracle_quantize_rows_e4m3(int64_t rows, int64_t cols, const uint16_t* x, uint8_t* q,
+                               float* scale, int nthreads) {
+  parallel_for(rows, nthreads,
+               [&](int64_t r) { scale[r] = quantize_row(cols, x + r * cols, q + r * cols); });
+}
+
+// FP8 linear layer on quantised rows: y[r, c] = fl32( sx_r * sw_c * sum_j xq[r, j] Wq[c, j] )
+// with codes decoded exactly; xq [rows, K], Wq [n_out, K].
+void oracle_linear_fp8(int64_t rows, int64_t n_out, int64_t K, const uint8_t* xq,
+                       const float* sx, const uint8_t* Wq, const float* sw, float* y,
+                       int nthreads) {
+  parallel_for(rows, nthreads, [&](int64_t r) {
+    linear_fp8_row(K, n_out, xq + r * K, sx[r], Wq, sw, y + r * n_out);
+  });
+}
+
+// One SwiGLU expert with E4M3 weights on one input row x [d] (BF16):
+//   (xq, sx) = quantize(x)
+//   g = linear_fp8(xq, sx; Wgq, sg),  u = linear_fp8(xq, sx; Wuq, su)      [I]
+//   a_i = bf16( fl32(silu(g_i)) * u_i )
+//   (aq, sa) = quantize(a)
+//   y = linear_fp8(aq, sa; Wdq, sd)                                          [d]
+// Wgq, Wuq [I, d] with row scales sg, su [I]; Wdq [d, I] with row scales sd [d].
+// a_out [I] (BF16 bits, before its quantisation) may be NULL.
+void oracle_expert_mlp_fp8(int64_t d, int64_t I, const uint16_t* x, const uint8_t* Wgq,
+                           const float* sg, const uint8_t* Wuq, const float* su,
+                           const uint8_t* Wdq, const float* sd, float* y, uint16_t* a_out) {
+  std::vector<uint8_t> xq(d), aq(I);
+  const float sx = quantize_row(d, x, xq.data());
+  std::vector<float> g(I), u(I);
+  linear_fp8_row(d, I, xq.data(), sx, Wgq, sg, g.data());
+  linear_fp8_row(d, I, xq.data(), sx, Wuq, su, u.data());
+  std::vector<uint16_t> a(I);
+  for (int64_t i = 0; i < I; ++i) {
+    const float act =
+        static_cast<float>(static_cast<double>(g[i]) * sigmoid(static_cast<double>(g[i])));
+    a[i] = float_to_bf16_bits(act * u[i]);
   }
+  if (a_out) std::copy(a.begin(), a.end(), a_out);
+  const float sa = quantize_row(I, a.data(), aq.data());
+  linear_fp8_row(I, d, aq.data(), sa, Wdq, sd, y);
+}
+
+// MoE output for a list of tokens with E4M3 experts; as oracle_moe_tokens otherwise.
+int oracle_moe_tokens_fp8(int64_t ntok, const int64_t* tokens, int64_t d, int64_t I, int k,
+                          const uint16_t* h, const int32_t* idx, const float* w,
+                          const uint8_t* const* Wgq, const float* const* sg,
+                          const uint8_t* const* Wuq, const float* const* su,
+                          const uint8_t* const* Wdq, const float* const* sd, float* out,
+                          int nthreads) {
+  for (int64_t n = 0; n < ntok; ++n)
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[tokens[n] * k + j];
+      if (!Wgq[e] || !sg[e] || !Wuq[e] || !su[e] || !Wdq[e] || !sd[e]) return -1;
+    }
+  std::vector<float> ys(static_cast<size_t>(ntok) * k * d);
+  parallel_for(ntok * k, nthreads, [&](int64_t item) {
+    const int64_t n = item / k;
+    const int j = static_cast<int>(item % k);
+    const int64_t t = tokens[n];
+    const int e = idx[t * k + j];
+    oracle_expert_mlp_fp8(d, I, h + t * d, Wgq[e], sg[e], Wuq[e], su[e], Wdq[e], sd[e],
+                          ys.data() + item * d, nullptr);
+  });
+  combine_slots(ntok, tokens, d, k, w, ys.data(), out);
   return 0;
 }
 

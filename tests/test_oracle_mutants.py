@@ -1,7 +1,7 @@
 """Planted mistakes: each mutant copy of the oracle must fail at least one pin.
 
 A mutant is the oracle's C++ source with one plausible error written into it
-(a dropped term, a wrong index, a swapped operand, a wrong convention).  It is
+(a dropped term, a wrong index, a swapped operand, a wrong convention, a wrong rounding).  It is
 compiled into a temporary library on the CPU, swapped in for the real one, and
 the pins in test_oracle_pins are run against it.  Every mutant must be caught.
 """
@@ -12,6 +12,7 @@ import subprocess
 import pytest
 
 import oracle
+from tests import test_oracle_fp8_pins as fp8
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "beam_moe_oracle.cpp")
@@ -45,6 +46,15 @@ MUTANTS = {
     "bf16_truncates": ("if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;", ""),
     "bias_update_sign_flipped": ("const float sgn = c < mean ? 1.0f : (c > mean ? -1.0f : 0.0f);",
                                  "const float sgn = c < mean ? -1.0f : (c > mean ? 1.0f : 0.0f);"),
+    "e4m3_truncates": ("double r = std::nearbyint(a / std::ldexp(1.0, E - 3));",
+                       "double r = std::floor(a / std::ldexp(1.0, E - 3));"),
+    "e4m3_subnormal_step": ("std::nearbyint(a / std::ldexp(1.0, -9))",
+                            "std::nearbyint(a / std::ldexp(1.0, -10))"),
+    "fp8_scale_divisor": ("const float s = amax / 448.0f;", "const float s = amax / 240.0f;"),
+    "fp8_weight_scale_not_per_row": ("static_cast<double>(sx) * static_cast<double>(sw[c]) * acc",
+                                     "static_cast<double>(sx) * static_cast<double>(sw[0]) * acc"),
+    "fp8_down_reads_input_codes": ("linear_fp8_row(I, d, aq.data(), sa, Wdq, sd, y);",
+                                   "linear_fp8_row(I, d, xq.data(), sx, Wdq, sd, y);"),
 }
 
 PIN_TESTS = [
@@ -62,6 +72,16 @@ PIN_TESTS = [
     (pins.test_rmsnorm_matches_torch_and_closed_form, [()]),
     (pins.test_bf16_rounding_matches_torch, [()]),
     (pins.test_bias_update_hand_example_and_invariants, [()]),
+    (fp8.test_e4m3_decode_matches_torch_for_all_codes, [()]),
+    (fp8.test_e4m3_encode_matches_torch_in_range_and_on_ties, [()]),
+    (fp8.test_e4m3_saturates_and_keeps_nan, [()]),
+    (fp8.test_quantize_rows_matches_torch_conversion_and_error_bounds, [()]),
+    (fp8.test_quantize_rows_is_exact_on_representable_rows, [()]),
+    (fp8.test_linear_fp8_equals_router_logits_on_exact_operands, [()]),
+    (fp8.test_linear_fp8_general_scales_match_float64, [()]),
+    (fp8.test_expert_mlp_fp8_gate_up_equal_bf16_expert_on_exact_operands, [()]),
+    (fp8.test_expert_mlp_fp8_down_scales_are_per_output_row, [()]),
+    (fp8.test_moe_tokens_fp8_is_weighted_sum_of_fp8_experts, [()]),
 ]
 
 
@@ -85,7 +105,9 @@ def test_mutant_is_caught(tmp_path, monkeypatch, name):
     for fn in ("oracle_hardware_threads", "oracle_f32_to_bf16", "oracle_bf16_to_f32",
                "oracle_router_logits", "oracle_route", "oracle_expert_mlp", "oracle_moe_tokens",
                "oracle_rmsnorm", "oracle_residual", "oracle_residual_coefficients",
-               "oracle_bias_update"):
+               "oracle_bias_update", "oracle_f32_to_e4m3", "oracle_e4m3_to_f32",
+               "oracle_quantize_rows_e4m3", "oracle_linear_fp8", "oracle_expert_mlp_fp8",
+               "oracle_moe_tokens_fp8"):
         f, g = getattr(real, fn), getattr(mut, fn)
         g.argtypes, g.restype = f.argtypes, f.restype
     monkeypatch.setattr(oracle, "_lib", mut)
