@@ -37,6 +37,7 @@ import torch  # noqa: E402
 from sparse_moe_transformer_fp32_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at Beam shape T=4096 BF16; % BF16 tensor peak / % HBM BW"
+METRIC_FP8 = "MoE-layer tokens/s at Beam shape with FP8 E4M3 expert weights; % FP8 tensor peak / % HBM BW"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0, "source": "fallback"}
 N_SMS = 148
@@ -58,6 +59,8 @@ def parse_args(argv=None):
                    help="tokens in the oracle's bounded sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--fp8", action="store_true",
+                   help="E4M3 expert weights (beam_moe_forward_fp8); layer workloads only")
     p.add_argument("--route-only", action="store_true",
                    help="time beam_moe_route alone (router profiling; not the layer metric)")
     p.add_argument("--dry-run", action="store_true",
@@ -229,11 +232,25 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ algorithmic work
 
-def kernel_work(wl, touched: int):
-    """Algorithmic bytes and FLOPs per launch of each kernel (the minimum each must move)."""
+def kernel_work(wl, touched: int, fp8: bool = False):
+    """Algorithmic bytes and FLOPs per launch of each kernel (the minimum each must move).
+    With fp8 the weights and the GEMM inputs are one-byte E4M3 codes (row scales ignored)."""
     T, d, E, k, I = wl.T, wl.d, wl.E, wl.top_k, wl.I
     R = T * k
     bf, f4 = 2, 4
+    if fp8:
+        q = 1
+        return {
+            "router_gemm": {"flops": 2 * T * d * E, "bytes": T * d * bf + E * d * f4 + T * E * f4},
+            "router_select": {"flops": 0, "bytes": T * E * f4 + 2 * R * f4},
+            "permute": {"flops": 0, "bytes": T * d * bf + R * d * q},
+            "expert_gemm_gate_up": {"flops": 4 * R * d * I,
+                                    "bytes": touched * 2 * I * d * q + R * d * q + R * I * bf},
+            "quantize_e4m3": {"flops": 0, "bytes": R * I * bf + R * I * q},
+            "expert_gemm_down": {"flops": 2 * R * d * I,
+                                 "bytes": touched * d * I * q + R * I * q + R * d * bf},
+            "combine": {"flops": 2 * R * d, "bytes": R * d * bf + T * d * bf},
+        }
     w_gu = touched * 2 * I * d * bf
     w_dn = touched * d * I * bf
     return {
@@ -248,9 +265,9 @@ def kernel_work(wl, touched: int):
     }
 
 
-def layer_min_bytes(wl, touched: int):
+def layer_min_bytes(wl, touched: int, fp8: bool = False):
     T, d, I = wl.T, wl.d, wl.I
-    b = touched * 3 * d * I * 2 + T * d * 2 * 2
+    b = touched * 3 * d * I * (1 if fp8 else 2) + T * d * 2 * 2
     if wl.block:
         b += 2 * T * d * 4
     return b
@@ -299,6 +316,28 @@ def oracle_sample_rate(wl, router_w, bias, hidden_cpu, weights_dev, n_tokens: in
     return n_tokens * repeats / dt, dt, oracle.hardware_threads()
 
 
+def oracle_fp8_sample_rate(wl, router_w, bias, hidden_cpu, weights_dev, n_tokens: int):
+    """Tokens/s of the CPU oracle's E4M3 layer on the first n tokens; the oracle converts the
+    experts those tokens use from the BF16 weights first (not timed: a one-off conversion)."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    h = hidden_cpu[:n_tokens]
+    sample = wl.with_tokens(n_tokens)
+    _, idx, w, _, _ = oracle.layer_routing(h, router_w, bias, sample)
+    experts = {}
+    for e in sorted({int(e) for e in idx.reshape(-1)}):
+        parts = []
+        for m in weights_dev:
+            parts += list(oracle.quantize_rows_e4m3(m[e].cpu()))
+        experts[e] = tuple(parts)
+    t0 = time.perf_counter()
+    _, idx, w, _, _ = oracle.layer_routing(h, router_w, bias, sample)
+    oracle.moe_tokens_fp8(np.arange(n_tokens), h, idx, w, experts)
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt, oracle.hardware_threads()
+
+
 def oracle_dense_rate(wl, hidden_cpu, weights_dev, n_tokens: int):
     import oracle
     oracle.build()
@@ -345,7 +384,18 @@ def run_cuda(args, rank, world, local):
             h = h_cpu.to(dev)
             out = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
             inp_cpu, inp, res = h_cpu, h, out
-        ws = bm.dense_workspace(ds, dev) if wl.dense else bm.workspace(s, dev)
+        fp8 = None
+        if args.fp8:
+            if wl.dense or wl.block:
+                raise SystemExit("bench.py: --fp8 applies to the layer workloads")
+            fp8 = []
+            for m in weights:
+                fp8 += list(bm.beam_moe_quantize_e4m3(m))
+            torch.cuda.synchronize(dev)
+        if wl.dense:
+            ws = bm.dense_workspace(ds, dev)
+        else:
+            ws = bm.fp8_workspace(s, dev) if fp8 else bm.workspace(s, dev)
         stream = torch.cuda.current_stream(dev)
 
         def step(src=None, dst=None):
@@ -357,6 +407,8 @@ def run_cuda(args, rank, world, local):
             elif wl.block:
                 bm.beam_moe_block(s, src, g_pre, g_post, wl.eps, wl.k_resid, router_w, bias,
                                   *weights, dst, ws=ws)
+            elif fp8:
+                bm.beam_moe_forward_fp8(s, src, router_w, bias, *fp8, dst, ws=ws)
             else:
                 bm.beam_moe_forward(s, src, router_w, bias, *weights, dst, ws=ws)
 
@@ -453,7 +505,7 @@ def run_cuda(args, rank, world, local):
 
         result = None
         if rank == 0:
-            work = kernel_work(wl, touched)
+            work = kernel_work(wl, touched, fp8=bool(fp8))
             per_kernel = {k: {"launches": n, "ms_per_launch": (ms / n if n else None)}
                           for k, (n, ms) in prof.items() if n}
             dom = max((k for k in per_kernel), key=lambda k: prof[k][1])
@@ -462,6 +514,8 @@ def run_cuda(args, rank, world, local):
             wk = work[dom]
             hbm_t = wk["bytes"] / (peaks["hbm_gbs"] * 1e9)
             ten_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+            if fp8:
+                ten_peak *= 2  # FP8 dense tensor rate: the measured BF16 rate x the nominal 2
             if dom == "router_gemm":
                 clk = float(peaks.get("sm_max_mhz", 1965.0))
                 alu_peak = N_SMS * FFMA_PER_SM_PER_CLK * 2 * clk * 1e6 / 1e12
@@ -476,16 +530,26 @@ def run_cuda(args, rank, world, local):
             roof["frac"] = roof["achieved"] / roof["peak"]
             roof["kernel"] = dom
             roof["peak_source"] = peaks.get("source", "measured")
-            roof["traffic"] = traffic_from_profile(dom, wl.name)
+            if fp8 and roof["bound"] == "tensor":
+                roof["peak_source"] += " bf16 x 2 (nominal FP8:BF16 ratio)"
+            roof["traffic"] = traffic_from_profile(dom, wl.name + ("-fp8" if fp8 else ""))
             roof["algorithmic_per_launch"] = wk["bytes"] if roof["bound"] == "hbm" else wk["flops"]
             roof["tensor_frac_of_sustained"] = (wk["flops"] / avg_s / 1e12) / ten_peak
             roof["hbm_frac"] = (wk["bytes"] / avg_s / 1e9) / peaks["hbm_gbs"]
 
             step_s = ms_per_step / 1e3
             flops_step = 6 * wl.T * wl.top_k * wl.d * wl.I  # top_k = 1 for the dense MLP
-            bytes_step = layer_min_bytes(wl, touched)
+            bytes_step = layer_min_bytes(wl, touched, fp8=bool(fp8))
             cpu = None
-            if not args.no_cpu_baseline and world == 1 and wl.dense:
+            if not args.no_cpu_baseline and world == 1 and fp8:
+                n_cpu = min(args.cpu_sample_tokens, 16)
+                rate, secs, cores = oracle_fp8_sample_rate(
+                    wl, W.router_weight(wl), W.router_bias(wl), inp_cpu, weights, n_cpu)
+                cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                       "sample": f"first {n_cpu} tokens of the {wl.name} workload, full E4M3 "
+                                 f"layer (router logits, routing, {wl.top_k} E4M3 SwiGLU experts "
+                                 f"each, combine) in double-accumulating C++; {secs:.2f} s"}
+            elif not args.no_cpu_baseline and world == 1 and wl.dense:
                 rate, secs, cores = oracle_dense_rate(wl, inp_cpu, weights, args.cpu_sample_tokens)
                 cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                        "sample": f"first {args.cpu_sample_tokens} tokens of the dense workload, "
@@ -500,18 +564,21 @@ def run_cuda(args, rank, world, local):
                                  f"full layer (router logits, routing, {wl.top_k} SwiGLU experts "
                                  f"each, combine) in double-accumulating C++; {secs:.2f} s"}
             result = {
-                "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "metric": METRIC_FP8 if fp8 else METRIC, "value": value, "unit": "tokens/s",
+                "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": f"{wl.name}: T={wl.T} d={wl.d} E={wl.E} n_group={wl.n_group} "
+                "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
+                "config": {"workload": f"{wl.name}{'-fp8' if fp8 else ''}: T={wl.T} d={wl.d} "
+                                       f"E={wl.E} n_group={wl.n_group} "
                                        f"topk_group={wl.topk_group} top_k={wl.top_k} I={wl.I}"
                                        + (" block" if wl.block else ""),
                            "tokens_per_gpu": wl.T, "global_tokens": wl.T * world,
                            "parallelism": f"replicas x{world} (data parallel over tokens)",
                            "l2": "inputs larger than L2: every step streams the touched experts' "
                                  f"weights ({touched} of {wl.E} experts, "
-                                 f"{touched * 3 * wl.d * wl.I * 2 / 1e9:.2f} GB) from HBM",
+                                 f"{touched * 3 * wl.d * wl.I * (1 if fp8 else 2) / 1e9:.2f} GB) "
+                                 "from HBM",
                            "touched_experts": touched,
                            "max_expert_load": int(counts.max()),
                            "top16_share": float(counts.sort(descending=True).values[:16].sum()
@@ -526,7 +593,7 @@ def run_cuda(args, rank, world, local):
                 "cpu_baseline": cpu,
             }
         barrier(dist, dev)
-        del weights
+        del weights, fp8
     return result
 
 

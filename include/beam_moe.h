@@ -131,6 +131,42 @@ BEAM_API beam_status beam_moe_forward(const beam_moe_shape* shape, const void* h
                              const void* w_down, void* out, int32_t* topk_idx, float* topk_w,
                              void* ws, size_t ws_bytes, beam_stream stream);
 
+/* ---- FP8 (E4M3) expert weights
+ *
+ * The pages name FP8 and NVFP4 checkpoints of the model (news article "Reflection lança o
+ * Beam", section "Onde o Beam economiza ..."; review page "обзор модели «Бим»", weights and
+ * vLLM-recipe entries) but no scale format.  This path reads the plainest one the tensor cores
+ * take directly: E4M3 codes with one FP32 scale per row, s = fl32(amax / 448) and
+ * q = e4m3(fl32(x / s)) rounded to nearest even, saturating to +-448 (an all-zero row has
+ * s = 0 and zero codes).  Weights are quantised per output channel, activations per token
+ * row: the token rows entering the gate/up GEMM and the SwiGLU activation (after its BF16
+ * rounding) entering the down GEMM.  Each GEMM multiplies codes on the tensor cores with FP32
+ * accumulation and applies both row scales in its epilogue.  Routing is unchanged. */
+
+/* Row-wise E4M3 quantisation of a BF16 matrix x [rows, cols] (row-major) into codes q
+ * [rows, cols] (uint8) and scales scale [rows] (FP32), on `stream`.  Used once per model to
+ * convert the expert weights: w_gate and w_up as [E * I, d], w_down as [E * d, I].
+ * cols must be a positive multiple of 16; x and q 16-byte aligned and not overlapping.
+ * Returns BEAM_ERR_INVALID_ARG otherwise; rows == 0 is a no-op. */
+BEAM_API beam_status beam_moe_quantize_e4m3(const void* x, int64_t rows, int32_t cols, void* q,
+                                            float* scale, beam_stream stream);
+
+/* Workspace bytes for beam_moe_forward_fp8 (0 for an unsupported shape). */
+BEAM_API size_t beam_moe_fp8_workspace_size(const beam_moe_shape* shape);
+
+/* beam_moe_forward with E4M3 expert weights.
+ *   w_gate, w_up     E4M3 [E, I, d] with row scales gate_scale, up_scale FP32 [E * I]
+ *   w_down           E4M3 [E, d, I] with row scales down_scale FP32 [E * d]
+ *   (as written by beam_moe_quantize_e4m3); every other argument as for beam_moe_forward,
+ *   with ws sized by beam_moe_fp8_workspace_size.  Scale arrays must be 16-byte aligned. */
+BEAM_API beam_status beam_moe_forward_fp8(const beam_moe_shape* shape, const void* hidden,
+                                          const float* router_w, const float* bias,
+                                          const void* w_gate, const float* gate_scale,
+                                          const void* w_up, const float* up_scale,
+                                          const void* w_down, const float* down_scale, void* out,
+                                          int32_t* topk_idx, float* topk_w, void* ws,
+                                          size_t ws_bytes, beam_stream stream);
+
 /* MoE block: x' = x * sqrt((k_resid-1)/k_resid) + RMSNorm(MoE(bf16(RMSNorm(x) g_pre))) g_post
  *                 / sqrt(k_resid), RMSNorm(v) = v / sqrt(mean(v^2) + eps), all FP32.
  *   x       FP32 [T, d] residual stream in

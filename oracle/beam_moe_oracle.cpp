@@ -143,12 +143,14 @@ float quantize_row(int64_t n, const uint16_t* x, uint8_t* q) {
 // y_c = fl32( sx * sw_c * sum_j value(xq_j) * value(Wq[c, j]) ) for c < n_out; Wq is [n_out, K].
 void linear_fp8_row(int64_t K, int64_t n_out, const uint8_t* xq, float sx, const uint8_t* Wq,
                     const float* sw, float* y) {
+  double value[256];  // e4m3_value of every code, looked up below
+  for (int b = 0; b < 256; ++b) value[b] = e4m3_value(static_cast<uint8_t>(b));
   std::vector<double> xv(K);
-  for (int64_t j = 0; j < K; ++j) xv[j] = e4m3_value(xq[j]);
+  for (int64_t j = 0; j < K; ++j) xv[j] = value[xq[j]];
   for (int64_t c = 0; c < n_out; ++c) {
     const uint8_t* w = Wq + c * K;
     double acc = 0.0;
-    for (int64_t j = 0; j < K; ++j) acc += xv[j] * e4m3_value(w[j]);
+    for (int64_t j = 0; j < K; ++j) acc += xv[j] * value[w[j]];
     y[c] = static_cast<float>(static_cast<double>(sx) * static_cast<double>(sw[c]) * acc);
   }
 }

@@ -31,7 +31,8 @@ EXPORTED = [
     "beam_moe_kernel_count", "beam_moe_kernel_name", "beam_moe_profile_read",
     "beam_moe_abi_version", "beam_moe_route_static", "beam_dense_workspace_size",
     "beam_dense_forward", "beam_moe_bias_update", "beam_moe_set_sm_pairs",
-    "beam_moe_get_sm_pairs",
+    "beam_moe_get_sm_pairs", "beam_moe_quantize_e4m3", "beam_moe_fp8_workspace_size",
+    "beam_moe_forward_fp8",
 ]
 
 
@@ -97,6 +98,11 @@ def lib():
     L.beam_dense_workspace_size.restype = sz
     L.beam_dense_forward.argtypes = [dshp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.beam_moe_bias_update.argtypes = [shp, vp, vp, f32, vp]
+    L.beam_moe_quantize_e4m3.argtypes = [vp, ctypes.c_int64, i32, vp, vp, vp]
+    L.beam_moe_fp8_workspace_size.argtypes = [shp]
+    L.beam_moe_fp8_workspace_size.restype = sz
+    L.beam_moe_forward_fp8.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                       sz, vp]
     L.beam_moe_sync_status.argtypes = [vp, vp]
     L.beam_status_string.argtypes = [ctypes.c_int]
     L.beam_status_string.restype = ctypes.c_char_p
@@ -114,7 +120,8 @@ def lib():
                                         ctypes.POINTER(ctypes.c_double)]
     for name in ("beam_moe_route", "beam_moe_route_static", "beam_moe_forward", "beam_moe_block",
                  "beam_moe_sync_status", "beam_dense_forward", "beam_moe_bias_update",
-                 "beam_moe_expert_counts", "beam_moe_profile_read"):
+                 "beam_moe_expert_counts", "beam_moe_profile_read", "beam_moe_quantize_e4m3",
+                 "beam_moe_forward_fp8"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -227,6 +234,61 @@ def beam_moe_forward(shape, hidden, router_w, bias, w_gate, w_up, w_down, out, t
     ws = _ws(shape, ws, hidden.device)
     _check(lib().beam_moe_forward(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
                                   _stream(stream)), "beam_moe_forward")
+    return ws
+
+
+# ------------------------------------------------------------------ FP8 (E4M3) expert weights
+
+def beam_moe_fp8_workspace_size(shape: beam_moe_shape) -> int:
+    return lib().beam_moe_fp8_workspace_size(ctypes.byref(shape))
+
+
+def fp8_workspace(shape: beam_moe_shape, device="cuda") -> torch.Tensor:
+    n = beam_moe_fp8_workspace_size(shape)
+    if n == 0:
+        raise BeamError(BEAM_ERR_UNSUPPORTED, "beam_moe_fp8_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def beam_moe_quantize_e4m3(x, q=None, scale=None, stream=None):
+    """Row-wise E4M3 codes and FP32 scales of a BF16 matrix (the last dimension is the row);
+    returns (q uint8 of x's shape, scale float32 of x's shape without the last dimension)."""
+    if x.dim() < 2:
+        raise ValueError("x must have at least two dimensions")
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    if q is None:
+        q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    args = [_ptr(x, torch.bfloat16, "x", tuple(x.shape)), ctypes.c_int64(rows),
+            ctypes.c_int32(cols), _ptr(q, torch.uint8, "q", tuple(x.shape)),
+            _ptr(scale, torch.float32, "scale", tuple(x.shape[:-1]))]
+    _check(lib().beam_moe_quantize_e4m3(*args, _stream(stream)), "beam_moe_quantize_e4m3")
+    return q, scale
+
+
+def beam_moe_forward_fp8(shape, hidden, router_w, bias, w_gate, gate_scale, w_up, up_scale,
+                         w_down, down_scale, out, topk_idx=None, topk_w=None, ws=None,
+                         stream=None):
+    T, d, E, k, I = shape.T, shape.d, shape.E, shape.top_k, shape.I
+    args = [_ptr(hidden, torch.bfloat16, "hidden", (T, d)),
+            _ptr(router_w, torch.float32, "router_w", (E, d)),
+            _ptr(bias, torch.float32, "bias", (E,)),
+            _ptr(w_gate, torch.uint8, "w_gate", (E, I, d)),
+            _ptr(gate_scale, torch.float32, "gate_scale", (E, I)),
+            _ptr(w_up, torch.uint8, "w_up", (E, I, d)),
+            _ptr(up_scale, torch.float32, "up_scale", (E, I)),
+            _ptr(w_down, torch.uint8, "w_down", (E, d, I)),
+            _ptr(down_scale, torch.float32, "down_scale", (E, d)),
+            _ptr(out, torch.bfloat16, "out", (T, d)),
+            _ptr(topk_idx, torch.int32, "topk_idx", (T, k), optional=True),
+            _ptr(topk_w, torch.float32, "topk_w", (T, k), optional=True)]
+    if ws is None:
+        ws = fp8_workspace(shape, hidden.device)
+    _ptr(ws, torch.uint8, "ws")
+    _check(lib().beam_moe_forward_fp8(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
+                                      _stream(stream)), "beam_moe_forward_fp8")
     return ws
 
 

@@ -36,12 +36,13 @@ enum KernelId {
   kKRouterTranspose,
   kKDenseTiles,
   kKBiasUpdate,
+  kKQuantize,
   kNumKernels
 };
 const char* const kKernelNames[kNumKernels] = {
     "router_gemm", "router_select", "dispatch_scan", "permute", "expert_gemm_gate_up",
     "expert_gemm_down", "combine", "combine_block", "prenorm", "router_transpose", "dense_tiles",
-    "bias_update"};
+    "bias_update", "quantize_e4m3"};
 
 struct Profiler {
   std::mutex mu;
@@ -128,6 +129,7 @@ beam_status check_shape(const beam_moe_shape* s) {
 
 struct Layout {
   size_t status, cnt, off, mt_count, mtiles, rank, rowmap, idx, w, wt, part, h, xp, act, y, total;
+  size_t xs = 0, act8 = 0, as = 0;  // FP8 path: row scales of Xp, E4M3 act, act row scales
   int S, kchunk;
   int64_t R, mt_cap;
 };
@@ -193,6 +195,23 @@ Layout plan(const beam_moe_shape& s) {
   return L;
 }
 
+// FP8 path: the BF16 layout (whose Xp region holds the E4M3 rows, half its size) plus the row
+// scales of Xp, the E4M3 activation and its row scales.
+Layout plan_fp8(const beam_moe_shape& s) {
+  Layout L = plan(s);
+  size_t o = L.total;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o = align_up(o + (bytes ? bytes : 1), 1024);
+    return r;
+  };
+  L.xs = take(sizeof(float) * L.R);
+  L.act8 = take(static_cast<size_t>(L.R) * s.I);
+  L.as = take(sizeof(float) * L.R);
+  L.total = o;
+  return L;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <class T>
@@ -222,17 +241,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D BF16 view [outer, inner] (inner contiguous), box [box_outer, 64] with 128-byte swizzle;
-// rows past `outer` read as zeros.
+// 2-D view [outer, inner] (inner contiguous) of BF16 (elem_bytes 2) or E4M3 (1) elements, box
+// [box_outer rows, 128 bytes] with 128-byte swizzle; rows past `outer` read as zeros.
 beam_status make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-                     uint32_t box_outer) {
+                     uint32_t box_outer, int elem_bytes = 2) {
   auto fn = encode_fn();
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_outer};
+  const cuuint64_t strides[1] = {inner * elem_bytes};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), box_outer};
   const cuuint32_t es[2] = {1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+  const CUtensorMapDataType dt =
+      elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims,
                         strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -318,15 +339,25 @@ beam_status run_router(const beam_moe_shape& s, const Layout& L, const __nv_bflo
   return BEAM_OK;
 }
 
-// Dispatch, the two expert GEMMs; leaves Y and rowmap in the workspace.
+// Row scales of E4M3 expert weights (gate and up [E * I], down [E * d]); see beam_moe_forward_fp8.
+struct Fp8Scales {
+  const float* gate;
+  const float* up;
+  const float* down;
+};
+
+// Dispatch, the two expert GEMMs; leaves Y and rowmap in the workspace.  With f8 the weights
+// are E4M3 codes: the permute writes E4M3 rows of Xp with their scales, and the activation is
+// quantised between the two GEMMs.
 beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceInfo& dev,
                         const __nv_bfloat16* h, const int32_t* idx, const void* w_gate,
-                        const void* w_up, const void* w_down, void* ws, cudaStream_t st) {
+                        const void* w_up, const void* w_down, void* ws, cudaStream_t st,
+                        const Fp8Scales* f8 = nullptr) {
   uint32_t* status = at<uint32_t>(ws, L.status);
   // With SM pairs enabled, calls averaging at least 256 rows per expert run their expert GEMMs
   // on SM pairs (cta_group::2, 256-row tiles): half the operand bytes per SM for the same tensor
   // work, but 256-row tiles pad more rows.
-  const bool pairs = g_sm_pairs.load(std::memory_order_relaxed) != 0 &&
+  const bool pairs = !f8 && g_sm_pairs.load(std::memory_order_relaxed) != 0 &&
                      L.R >= static_cast<int64_t>(kPairMinRowsPerExpert) * s.E &&
                      dev.pair_grid >= 2;
   DispatchArgs da{};
@@ -344,7 +375,9 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   pa.rank = at<int32_t>(ws, L.rank);
   pa.off = da.off;
   pa.rowmap = at<int32_t>(ws, L.rowmap);
-  pa.xp = at<__nv_bfloat16>(ws, L.xp);
+  pa.xp = f8 ? nullptr : at<__nv_bfloat16>(ws, L.xp);
+  pa.xq = f8 ? at<uint8_t>(ws, L.xp) : nullptr;
+  pa.xs = f8 ? at<float>(ws, L.xs) : nullptr;
   pa.status = status;
   pa.T = s.T;
   pa.d = s.d;
@@ -356,17 +389,18 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   ATensorMaps tm_xp, tm_act;
   CUtensorMap tm_g, tm_u, tm_d;
   beam_status b;
+  const int eb = f8 ? 1 : 2;  // bytes per element of the GEMM operands
+  const void* a1 = at<void>(ws, L.xp);
+  const void* a2 = at<void>(ws, f8 ? L.act8 : L.act);
   for (int i = 0; i < kNumABoxes; ++i) {
-    if ((b = make_map(&tm_xp.m[i], pa.xp, s.d, R, a_box_rows(i))) != BEAM_OK) return b;
-    if ((b = make_map(&tm_act.m[i], at<void>(ws, L.act), s.I, R, a_box_rows(i))) != BEAM_OK)
-      return b;
+    if ((b = make_map(&tm_xp.m[i], a1, s.d, R, a_box_rows(i), eb)) != BEAM_OK) return b;
+    if ((b = make_map(&tm_act.m[i], a2, s.I, R, a_box_rows(i), eb)) != BEAM_OK) return b;
   }
-  if ((b = make_map(&tm_g, w_gate, s.d, static_cast<uint64_t>(s.E) * s.I, kN1Half)) != BEAM_OK)
-    return b;
-  if ((b = make_map(&tm_u, w_up, s.d, static_cast<uint64_t>(s.E) * s.I, kN1Half)) != BEAM_OK)
-    return b;
-  if ((b = make_map(&tm_d, w_down, s.I, static_cast<uint64_t>(s.E) * s.d, kN2)) != BEAM_OK)
-    return b;
+  const uint64_t EI = static_cast<uint64_t>(s.E) * s.I, Ed = static_cast<uint64_t>(s.E) * s.d;
+  if ((b = make_map(&tm_g, w_gate, s.d, EI, kN1Half, eb)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_u, w_up, s.d, EI, kN1Half, eb)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_d, w_down, s.I, Ed, kN2, eb)) != BEAM_OK) return b;
+  const int k_elems = 128 / eb;  // K elements per 128-byte pipeline stage
 
   const uint64_t limit = g_wait_limit_ns.load(std::memory_order_relaxed);
   GemmArgs g1{};
@@ -377,8 +411,13 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   g1.wait_limit_ns = limit;
   g1.out_ld = s.I;
   g1.n_tiles_n = s.I / kN1Half;
-  g1.k_blocks = s.d / kBK;
+  g1.k_blocks = s.d / k_elems;
   g1.b_rows_per_expert = s.I;
+  if (f8) {
+    g1.a_scale = pa.xs;
+    g1.b_scale0 = f8->gate;
+    g1.b_scale1 = f8->up;
+  }
   // Weights-as-M tiles pay off only when nearly every tile is tiny (decode-sized calls, a few
   // rows per expert); with larger tiles in the mix they measured slower.
   g1.swap_max_rows = L.R <= 8 * static_cast<int64_t>(s.E) ? kSwapMaxRows : 0;
@@ -390,15 +429,25 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
     BEAM_LAUNCH(kKGemmGateUp, st, launch_gemm_gate_up_2sm(tm_xp, tm_g, tm_u, g1, grid, st));
   } else {
     const int grid1 = static_cast<int>(max_tiles1 < dev.sms ? max_tiles1 : dev.sms);
-    BEAM_LAUNCH(kKGemmGateUp, st, launch_gemm_gate_up(tm_xp, tm_g, tm_u, g1, grid1, st));
+    BEAM_LAUNCH(kKGemmGateUp, st,
+                launch_gemm_gate_up(tm_xp, tm_g, tm_u, g1, grid1, st, f8 != nullptr));
   }
+  if (f8)
+    BEAM_LAUNCH(kKQuantize, st,
+                launch_quantize_rows(at<__nv_bfloat16>(ws, L.act), L.R, s.I,
+                                     at<uint8_t>(ws, L.act8), at<float>(ws, L.as), st));
 
   GemmArgs g2 = g1;
   g2.out = at<__nv_bfloat16>(ws, L.y);
   g2.out_ld = s.d;
   g2.n_tiles_n = s.d / kN2;
-  g2.k_blocks = s.I / kBK;
+  g2.k_blocks = s.I / k_elems;
   g2.b_rows_per_expert = s.d;
+  if (f8) {
+    g2.a_scale = at<float>(ws, L.as);
+    g2.b_scale0 = f8->down;
+    g2.b_scale1 = nullptr;
+  }
   const int64_t max_tiles2 = L.mt_cap * g2.n_tiles_n;
   if (pairs) {
     CUtensorMap tm_d_half;  // each SM of a pair loads 128 of the tile's 256 weight rows
@@ -409,7 +458,7 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
     BEAM_LAUNCH(kKGemmDown, st, launch_gemm_down_2sm(tm_act, tm_d_half, g2, grid, st));
   } else {
     const int grid2 = static_cast<int>(max_tiles2 < dev.sms ? max_tiles2 : dev.sms);
-    BEAM_LAUNCH(kKGemmDown, st, launch_gemm_down(tm_act, tm_d, g2, grid2, st));
+    BEAM_LAUNCH(kKGemmDown, st, launch_gemm_down(tm_act, tm_d, g2, grid2, st, f8 != nullptr));
   }
   return BEAM_OK;
 }
@@ -608,6 +657,67 @@ beam_status beam_moe_forward(const beam_moe_shape* shape, const void* hidden, co
     return b;
   if ((b = run_experts(*shape, L, *dev, h, idx, w_gate, w_up, w_down, ws, st)) != BEAM_OK)
     return b;
+  CombineArgs ca{};
+  ca.y = at<__nv_bfloat16>(ws, L.y);
+  ca.rowmap = at<int32_t>(ws, L.rowmap);
+  ca.w = w;
+  ca.out = static_cast<__nv_bfloat16*>(out);
+  ca.status = at<uint32_t>(ws, L.status);
+  ca.T = shape->T;
+  ca.d = shape->d;
+  ca.k = shape->top_k;
+  ca.R = static_cast<int>(L.R);
+  BEAM_LAUNCH(kKCombine, st, launch_combine(ca, st));
+  return BEAM_OK;
+}
+
+size_t beam_moe_fp8_workspace_size(const beam_moe_shape* shape) {
+  if (check_shape(shape) != BEAM_OK) return 0;
+  return plan_fp8(*shape).total;
+}
+
+beam_status beam_moe_quantize_e4m3(const void* x, int64_t rows, int32_t cols, void* q,
+                                   float* scale, beam_stream stream) {
+  if (rows < 0 || cols <= 0 || cols % 16 != 0) return BEAM_ERR_INVALID_ARG;
+  if (rows == 0) return BEAM_OK;
+  if (any_misaligned({x, q}) || !scale) return BEAM_ERR_INVALID_ARG;
+  const uintptr_t xb = reinterpret_cast<uintptr_t>(x), qb = reinterpret_cast<uintptr_t>(q);
+  const uint64_t xbytes = static_cast<uint64_t>(rows) * cols * 2;
+  if (qb < xb + xbytes && xb < qb + static_cast<uint64_t>(rows) * cols)
+    return BEAM_ERR_INVALID_ARG;  // the codes may not overwrite the input
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  BEAM_LAUNCH(kKQuantize, st,
+              launch_quantize_rows(static_cast<const __nv_bfloat16*>(x), rows, cols,
+                                   static_cast<uint8_t*>(q), scale, st));
+  return BEAM_OK;
+}
+
+beam_status beam_moe_forward_fp8(const beam_moe_shape* shape, const void* hidden,
+                                 const float* router_w, const float* bias, const void* w_gate,
+                                 const float* gate_scale, const void* w_up, const float* up_scale,
+                                 const void* w_down, const float* down_scale, void* out,
+                                 int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                                 beam_stream stream) {
+  beam_status b = check_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
+  if (any_misaligned({hidden, router_w, w_gate, w_up, w_down, out, gate_scale, up_scale,
+                      down_scale}) ||
+      !bias || (topk_idx && !aligned16(topk_idx)) || (topk_w && !aligned16(topk_w)))
+    return BEAM_ERR_INVALID_ARG;
+  const Layout L = plan_fp8(*shape);
+  if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
+  DeviceInfo* dev;
+  if ((b = device_info(&dev)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
+  float* w = topk_w ? topk_w : at<float>(ws, L.w);
+  const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(hidden);
+  if ((b = run_router(*shape, L, h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
+    return b;
+  const Fp8Scales f8{gate_scale, up_scale, down_scale};
+  b = run_experts(*shape, L, *dev, h, idx, w_gate, w_up, w_down, ws, st, &f8);
+  if (b != BEAM_OK) return b;
   CombineArgs ca{};
   ca.y = at<__nv_bfloat16>(ws, L.y);
   ca.rowmap = at<int32_t>(ws, L.rowmap);

@@ -114,7 +114,9 @@ struct PermuteArgs {
   const int32_t* rank;     // [T, k]
   const int32_t* off;      // [E + 1]
   int32_t* rowmap;         // [T, k] out: row of slot (t, j) in the expert-contiguous buffers
-  __nv_bfloat16* xp;       // [R, d] out
+  __nv_bfloat16* xp;       // [R, d] out (BF16 path), or null
+  uint8_t* xq;             // [R, d] out: E4M3 codes (FP8 path), or null
+  float* xs;               // [R] out: row scales (FP8 path)
   uint32_t* status;
   int T, d, k, E;
 };
@@ -130,6 +132,10 @@ struct GemmArgs {
   int k_blocks;            // K / kBK
   int b_rows_per_expert;   // rows of one expert in the 2-D weight view (I or d)
   int swap_max_rows;       // m-tiles with at most this many rows run weights-as-M (0: none)
+  // FP8 instances only: D = acc * a_scale[A row] * b_scale[B row] (b_scale1: the up slice)
+  const float* a_scale;
+  const float* b_scale0;
+  const float* b_scale1;
 };
 
 struct CombineArgs {
@@ -163,9 +169,11 @@ cudaError_t launch_dispatch_scan(const DispatchArgs& a, cudaStream_t s);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
 cudaError_t launch_gemm_gate_up(const ATensorMaps& tmA, const CUtensorMap& tmG,
                                 const CUtensorMap& tmU, const GemmArgs& a, int grid,
-                                cudaStream_t s);
+                                cudaStream_t s, bool fp8 = false);
 cudaError_t launch_gemm_down(const ATensorMaps& tmA, const CUtensorMap& tmD, const GemmArgs& a,
-                             int grid, cudaStream_t s);
+                             int grid, cudaStream_t s, bool fp8 = false);
+cudaError_t launch_quantize_rows(const __nv_bfloat16* x, int64_t rows, int cols, uint8_t* q,
+                                 float* scale, cudaStream_t s);
 cudaError_t launch_gemm_gate_up_2sm(const ATensorMaps& tmA, const CUtensorMap& tmG,
                                     const CUtensorMap& tmU, const GemmArgs& a, int grid,
                                     cudaStream_t s);
@@ -308,6 +316,17 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, E4M3 x E4M3 -> FP32, issued by one thread.
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives once on `bar` when every tcgen05 operation this thread issued before has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile(
@@ -367,6 +386,12 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::f8f6f4: D FP32 (bits 4..5 = 1), A and B E4M3 (format 0 in
+// bits 7..9 and 10..12), both K-major, N >> 3 in 17..22, M >> 4 in 24..28.
+__host__ __device__ constexpr uint32_t umma_idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 #endif  // __CUDACC__

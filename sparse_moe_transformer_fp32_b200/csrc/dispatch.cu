@@ -9,6 +9,8 @@
 // combine reads rows back through rowmap in a fixed slot order.
 #include "beam_moe_internal.cuh"
 
+#include <cuda_fp8.h>
+
 namespace beam {
 namespace {
 
@@ -52,6 +54,39 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a
   }
 }
 
+// ---- E4M3 row quantisation helpers (FP8 expert weights; see quantize_rows_kernel)
+//
+// s = fl32(amax / 448) over the row, q = e4m3(fl32(x / s)) with round-to-nearest-even and
+// saturation (cvt.rn.satfinite); an all-zero row has s = 0 and zero codes.
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Scale of a row of nvec 8-element chunks read by the 32 lanes of a warp (all lanes return it).
+__device__ __forceinline__ float row_scale_e4m3(const uint4* src, int nvec, int lane) {
+  float amax = 0.f;
+  for (int c = lane; c < nvec; c += 32) {
+    const uint4 v = src[c];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+  }
+  // non-negative floats order like their bit patterns
+  amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+  return amax / 448.0f;
+}
+
+__device__ __forceinline__ uint2 quantize8_e4m3(const uint4 v, float s) {
+  if (s == 0.f) return make_uint2(0u, 0u);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t p[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    p[i] = __nv_cvt_float2_to_fp8x2(make_float2(bf16_lo(w[i]) / s, bf16_hi(w[i]) / s),
+                                    __NV_SATFINITE, __NV_E4M3);
+  return make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+}
+
 // One warp per token: the row is read once and written to each of its top_k destinations.
 __global__ void __launch_bounds__(256) permute_kernel(const PermuteArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -75,14 +110,45 @@ __global__ void __launch_bounds__(256) permute_kernel(const PermuteArgs a) {
 
   const uint4* src = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(t) * a.d);
   const int nvec = a.d / 8;
+  if (!a.xq) {
+    for (int c = lane; c < nvec; c += 32) {
+      const uint4 v = src[c];
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j) {
+        if (j < a.k && rows[j] >= 0)
+          reinterpret_cast<uint4*>(a.xp + static_cast<size_t>(rows[j]) * a.d)[c] = v;
+      }
+    }
+    return;
+  }
+  // FP8 path: the token row is quantised once (s = amax / 448, q = e4m3(x / s)) and its codes
+  // and scale written to each of its rows
+  const float s = row_scale_e4m3(src, nvec, lane);
+  if (lane < a.k && row >= 0) a.xs[row] = s;
   for (int c = lane; c < nvec; c += 32) {
-    const uint4 v = src[c];
+    const uint2 q = quantize8_e4m3(src[c], s);
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
       if (j < a.k && rows[j] >= 0)
-        reinterpret_cast<uint4*>(a.xp + static_cast<size_t>(rows[j]) * a.d)[c] = v;
+        reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(rows[j]) * a.d)[c] = q;
     }
   }
+}
+
+// Row-wise E4M3 quantisation of a BF16 matrix [rows, cols]: one warp per row.
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                                            int64_t rows, int cols,
+                                                            uint8_t* __restrict__ q,
+                                                            float* __restrict__ scale) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const uint4* src = reinterpret_cast<const uint4*>(x + r * cols);
+  const int nvec = cols / 8;
+  const float s = row_scale_e4m3(src, nvec, lane);
+  if (lane == 0) scale[r] = s;
+  uint2* dst = reinterpret_cast<uint2*>(q + r * cols);
+  for (int c = lane; c < nvec; c += 32) dst[c] = quantize8_e4m3(src[c], s);
 }
 
 // Dense MLP: every token belongs to the single group 0; tiles of up to kBM consecutive rows.
@@ -121,6 +187,15 @@ cudaError_t launch_dense_tiles(int T, MTile* mtiles, int32_t* mt_count, cudaStre
 cudaError_t launch_bias_update(const int32_t* cnt, float* bias, int E, float mean, float gamma,
                                cudaStream_t s) {
   bias_update_kernel<<<1, 256, 0, s>>>(cnt, bias, E, mean, gamma);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_rows(const __nv_bfloat16* x, int64_t rows, int cols, uint8_t* q,
+                                 float* scale, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  const int64_t blocks = (rows + 7) / 8;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  quantize_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, rows, cols, q, scale);
   return cudaGetLastError();
 }
 

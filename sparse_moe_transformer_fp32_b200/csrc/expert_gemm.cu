@@ -68,7 +68,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
 
-template <bool kSwiGLU, bool kSwap>
+// FP8 epilogue: v0[j] *= sa * s0[j] and, when s1 is given, v1[j] *= sa * s1[j], for 32
+// consecutive columns (s0, s1 16-byte aligned; the same addresses across the warp).
+__device__ __forceinline__ void scale_columns(uint32_t (&v0)[32], uint32_t (&v1)[32], float sa,
+                                              const float* s0, const float* s1) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 a4 = reinterpret_cast<const float4*>(s0)[q];
+    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v0[4 * q + i] = __float_as_uint(__uint_as_float(v0[4 * q + i]) * sa * av[i]);
+    if (s1) {
+      const float4 b4 = reinterpret_cast<const float4*>(s1)[q];
+      const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v1[4 * q + i] = __float_as_uint(__uint_as_float(v1[4 * q + i]) * sa * bv[i]);
+    }
+  }
+}
+
+template <bool kSwiGLU, bool kSwap, bool kFp8>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     expert_gemm_kernel(const __grid_constant__ ATensorMaps tmA,
                        const __grid_constant__ CUtensorMap tmB0,
@@ -93,6 +112,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint64_t limit = a.wait_limit_ns;
   const uint64_t drain_limit = limit > kMinDrainNs ? limit : kMinDrainNs;
   constexpr int kNSlice = kSwiGLU ? kN1Half : kN2;
+  constexpr int kKElems = kFp8 ? 2 * kBK : kBK;  // K elements in one 128-byte stage row
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -149,9 +169,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t sB = sA + kStageABytes;
           const uint32_t fb = bar(kBarFull + stage);
           mbar_arrive_expect_tx(fb, a_bytes + kStageBBytes);
-          tma_load_2d(sA, &tmA.m[a_box], fb, kb * kBK, m.row0);
-          tma_load_2d(sB, &tmB0, fb, kb * kBK, brow);
-          if (kSwiGLU) tma_load_2d(sB + kStageBBytes / 2, &tmB1, fb, kb * kBK, brow);
+          tma_load_2d(sA, &tmA.m[a_box], fb, kb * kKElems, m.row0);
+          tma_load_2d(sB, &tmB0, fb, kb * kKElems, brow);
+          if (kSwiGLU) tma_load_2d(sB + kStageBBytes / 2, &tmB1, fb, kb * kKElems, brow);
           filled |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -172,9 +192,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_full = umma_idesc_bf16_f32(kBM, kUmmaN);
+      auto make_idesc = [](int M, int N) {
+        return kFp8 ? umma_idesc_e4m3_f32(M, N) : umma_idesc_bf16_f32(M, N);
+      };
+      // one MMA covers 32 bytes of K: 16 BF16 or 32 E4M3 elements
+      auto mma = [](uint32_t d, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
+        if constexpr (kFp8)
+          umma_e4m3(d, ad, bd, id, acc);
+        else
+          umma_bf16(d, ad, bd, id, acc);
+      };
+      const uint32_t idesc_full = make_idesc(kBM, kUmmaN);
       // tiles of at most 64 rows use M = 64: half the datapath lanes, no work on absent rows
-      constexpr uint32_t idesc_m64 = umma_idesc_bf16_f32(64, kUmmaN);
+      const uint32_t idesc_m64 = make_idesc(64, kUmmaN);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -184,7 +214,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int nrows_next = load_tile(a, t + gridDim.x < ntiles ? t + gridDim.x : t, m_tiles,
                                          n_tiles, n_unused).nrows;
         const bool swap = kSwap && nrows <= a.swap_max_rows;
-        const uint32_t idesc = swap ? umma_idesc_bf16_f32(kBM, (nrows + 15) & ~15)
+        const uint32_t idesc = swap ? make_idesc(kBM, (nrows + 15) & ~15)
                                : nrows <= 64 ? idesc_m64 : idesc_full;
         if (!mbar_wait_bounded(bar(kBarTEmpty + acc), acc_phase ^ 1u, abort_flag, limit, a.status,
                                kWhereMmaTmemEmpty))
@@ -206,13 +236,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int k = 0; k < kBK / kUmmaK; ++k) {
               const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
-              umma_bf16(d_tmem, bdesc + 2u * k, adesc + 2u * k, idesc, accum);
-              umma_bf16(d_tmem + 128u, bdesc_hi + 2u * k, adesc + 2u * k, idesc, accum);
+              mma(d_tmem, bdesc + 2u * k, adesc + 2u * k, idesc, accum);
+              mma(d_tmem + 128u, bdesc_hi + 2u * k, adesc + 2u * k, idesc, accum);
             }
           } else {
 #pragma unroll
             for (int k = 0; k < kBK / kUmmaK; ++k)  // +32 bytes along K per step: +2 in addr>>4
-              umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+              mma(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           umma_commit(bar(kBarEmpty + stage));
           if (++stage == kStages) {
@@ -260,6 +290,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // column j holds token row j of the tile
         const int npad = (m.nrows + 15) & ~15;
         __nv_bfloat16* base = a.out + static_cast<size_t>(m.row0) * a.out_ld + n * kNSlice + row;
+        // FP8: this thread's weight rows (gate and up of one column, or two down columns)
+        float sb_lo = 1.f, sb_hi = 1.f;
+        if constexpr (kFp8) {
+          const int64_t brow = static_cast<int64_t>(m.e) * a.b_rows_per_expert + n * kNSlice + row;
+          sb_lo = a.b_scale0[brow];
+          sb_hi = kSwiGLU ? a.b_scale1[brow] : a.b_scale0[brow + 128];
+        }
 #pragma unroll 1
         for (int c0 = 0; c0 < npad; c0 += 16) {
           uint32_t lo[16], hi[16];
@@ -270,11 +307,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int r = c0 + j;
             if (r < m.nrows) {
               __nv_bfloat16* o = base + static_cast<size_t>(r) * a.out_ld;
+              float vlo = __uint_as_float(lo[j]), vhi = __uint_as_float(hi[j]);
+              if constexpr (kFp8) {
+                const float sa = a.a_scale[m.row0 + r];
+                vlo = vlo * sa * sb_lo;
+                vhi = vhi * sa * sb_hi;
+              }
               if (kSwiGLU) {
-                o[0] = __float2bfloat16_rn(silu(__uint_as_float(lo[j])) * __uint_as_float(hi[j]));
+                o[0] = __float2bfloat16_rn(silu(vlo) * vhi);
               } else {
-                o[0] = __float2bfloat16_rn(__uint_as_float(lo[j]));
-                o[128] = __float2bfloat16_rn(__uint_as_float(hi[j]));
+                o[0] = __float2bfloat16_rn(vlo);
+                o[128] = __float2bfloat16_rn(vhi);
               }
             }
           }
@@ -292,12 +335,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const bool valid = trow < m.nrows;
       __nv_bfloat16* dst =
           a.out + static_cast<size_t>(m.row0 + (valid ? trow : 0)) * a.out_ld + n * kNSlice;
+      // FP8: this row's scale and the first weight row of the slice
+      float sa = 1.f;
+      int64_t brow0 = 0;
+      if constexpr (kFp8) {
+        sa = valid ? a.a_scale[m.row0 + trow] : 0.f;
+        brow0 = static_cast<int64_t>(m.e) * a.b_rows_per_expert + n * kNSlice;
+      }
       if (kSwiGLU) {
 #pragma unroll 1
         for (int c = 0; c < kN1Half; c += 32) {
           uint32_t g[32], u[32];
           tmem_ld32_sync(tb + c, g);
           tmem_ld32_sync(tb + kN1Half + c, u);
+          if constexpr (kFp8) scale_columns(g, u, sa, a.b_scale0 + brow0 + c, a.b_scale1 + brow0 + c);
           uint32_t p[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -316,6 +367,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int c = 0; c < kN2; c += 32) {
           uint32_t y[32];
           tmem_ld32_sync(tb + c, y);
+          if constexpr (kFp8) scale_columns(y, y, sa, a.b_scale0 + brow0 + c, nullptr);
           uint32_t p[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j)
@@ -346,10 +398,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }  // namespace
 
 cudaError_t prepare_gemm_kernels() {
-  const void* kernels[] = {reinterpret_cast<const void*>(expert_gemm_kernel<true, false>),
-                           reinterpret_cast<const void*>(expert_gemm_kernel<true, true>),
-                           reinterpret_cast<const void*>(expert_gemm_kernel<false, false>),
-                           reinterpret_cast<const void*>(expert_gemm_kernel<false, true>)};
+  const void* kernels[] = {reinterpret_cast<const void*>(expert_gemm_kernel<true, false, false>),
+                           reinterpret_cast<const void*>(expert_gemm_kernel<true, true, false>),
+                           reinterpret_cast<const void*>(expert_gemm_kernel<false, false, false>),
+                           reinterpret_cast<const void*>(expert_gemm_kernel<false, true, false>),
+                           reinterpret_cast<const void*>(expert_gemm_kernel<true, false, true>),
+                           reinterpret_cast<const void*>(expert_gemm_kernel<true, true, true>),
+                           reinterpret_cast<const void*>(expert_gemm_kernel<false, false, true>),
+                           reinterpret_cast<const void*>(expert_gemm_kernel<false, true, true>)};
   for (const void* k : kernels) {
     const cudaError_t e =
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
@@ -358,22 +414,35 @@ cudaError_t prepare_gemm_kernels() {
   return cudaSuccess;
 }
 
+namespace {
+template <bool kSwiGLU, bool kFp8>
+void launch_gemm(const ATensorMaps& tmA, const CUtensorMap& tmB0, const CUtensorMap& tmB1,
+                 const GemmArgs& a, int grid, cudaStream_t s) {
+  if (a.swap_max_rows > 0)
+    expert_gemm_kernel<kSwiGLU, true, kFp8>
+        <<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB0, tmB1, a);
+  else
+    expert_gemm_kernel<kSwiGLU, false, kFp8>
+        <<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB0, tmB1, a);
+}
+}  // namespace
+
 cudaError_t launch_gemm_gate_up(const ATensorMaps& tmA, const CUtensorMap& tmG,
                                 const CUtensorMap& tmU, const GemmArgs& a, int grid,
-                                cudaStream_t s) {
-  if (a.swap_max_rows > 0)
-    expert_gemm_kernel<true, true><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmG, tmU, a);
+                                cudaStream_t s, bool fp8) {
+  if (fp8)
+    launch_gemm<true, true>(tmA, tmG, tmU, a, grid, s);
   else
-    expert_gemm_kernel<true, false><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmG, tmU, a);
+    launch_gemm<true, false>(tmA, tmG, tmU, a, grid, s);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_down(const ATensorMaps& tmA, const CUtensorMap& tmD, const GemmArgs& a,
-                             int grid, cudaStream_t s) {
-  if (a.swap_max_rows > 0)
-    expert_gemm_kernel<false, true><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmD, tmD, a);
+                             int grid, cudaStream_t s, bool fp8) {
+  if (fp8)
+    launch_gemm<false, true>(tmA, tmD, tmD, a, grid, s);
   else
-    expert_gemm_kernel<false, false><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmD, tmD, a);
+    launch_gemm<false, false>(tmA, tmD, tmD, a, grid, s);
   return cudaGetLastError();
 }
 

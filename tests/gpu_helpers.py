@@ -162,3 +162,71 @@ def sample_tokens(case: Case, n: int, seed: int = 0):
     while len(picks) < min(n, T):
         picks.add(int(rng.integers(0, T)))
     return sorted(picks)
+
+
+# ------------------------------------------------------------------ FP8 (E4M3) expert weights
+
+def device_weights_fp8(weights):
+    """E4M3 codes and row scales of BF16 expert weights, quantised by the CUDA path:
+    (gate codes, gate scales, up codes, up scales, down codes, down scales)."""
+    out = []
+    for m in weights:
+        q, s = bm.beam_moe_quantize_e4m3(m)
+        out += [q, s]
+    torch.cuda.synchronize()
+    return tuple(out)
+
+
+def oracle_experts_fp8(weights, experts, gpu_fp8=None):
+    """The oracle's own E4M3 quantisation of the listed experts (from the BF16 weights); when
+    the CUDA path's codes are given, they must equal the oracle's bit for bit."""
+    res = {}
+    for e in experts:
+        parts = []
+        for m_i, m in enumerate(weights):
+            q, s = oracle.quantize_rows_e4m3(m[e].cpu())
+            if gpu_fp8 is not None:
+                gq = gpu_fp8[2 * m_i][e].cpu().numpy()
+                gs = gpu_fp8[2 * m_i + 1][e].cpu().numpy()
+                assert np.array_equal(gq, q), f"expert {e} matrix {m_i}: E4M3 codes differ"
+                assert np.array_equal(gs, s), f"expert {e} matrix {m_i}: scales differ"
+            parts += [q, s]
+        res[e] = tuple(parts)
+    return res
+
+
+def run_forward_fp8(case: Case, fp8, ws=None):
+    wl = case.wl
+    s = bm.shape_of(wl)
+    dev = "cuda"
+    out = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(wl.T, wl.top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(wl.T, wl.top_k, dtype=torch.float32, device=dev)
+    ws = bm.beam_moe_forward_fp8(s, case.h.to(dev), case.router_w.to(dev), case.bias.to(dev),
+                                 *fp8, out, idx, w, ws=ws)
+    st = bm.beam_moe_sync_status(ws)
+    assert st == bm.BEAM_OK, bm.status_string(st)
+    return out, idx, w, ws
+
+
+def oracle_out_fp8(case: Case, weights, tokens, gpu_fp8=None, batch: int = 4):
+    """Oracle MoE output (FP32) of the E4M3 path for ``tokens``; the oracle quantises the BF16
+    weights of the experts each batch uses (and checks the CUDA path's codes against its own)."""
+    tokens = list(tokens)
+    out = np.empty((len(tokens), case.wl.d), np.float32)
+    checked = set()
+    for b0 in range(0, len(tokens), batch):
+        tb = tokens[b0:b0 + batch]
+        ex = sorted({int(e) for t in tb for e in case.idx[t]})
+        experts = oracle_experts_fp8(weights, ex, None)
+        if gpu_fp8 is not None:
+            for e in ex:
+                if e in checked:
+                    continue
+                checked.add(e)
+                for m_i in range(3):
+                    assert np.array_equal(gpu_fp8[2 * m_i][e].cpu().numpy(), experts[e][2 * m_i])
+                    assert np.array_equal(gpu_fp8[2 * m_i + 1][e].cpu().numpy(),
+                                          experts[e][2 * m_i + 1])
+        out[b0:b0 + len(tb)] = oracle.moe_tokens_fp8(tb, case.h, case.idx, case.w, experts)
+    return out

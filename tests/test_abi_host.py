@@ -138,3 +138,34 @@ def test_binding_rejects_cpu_tensors(L):
     with pytest.raises(ValueError):
         bm.beam_moe_route(s, h, torch.zeros(w.E, w.d), torch.zeros(w.E),
                           torch.zeros(w.T, w.top_k, dtype=torch.int32), torch.zeros(w.T, w.top_k))
+
+
+def test_fp8_entry_points_validate_before_launching(L):
+    s = beam(4096)
+    fp8 = bm.beam_moe_fp8_workspace_size(s)
+    R = 4096 * 8
+    # the BF16 layout plus Xp row scales, the E4M3 activation and its row scales
+    assert fp8 >= bm.beam_moe_workspace_size(s) + R * (4 + 2560 + 4)
+    assert L.beam_moe_fp8_workspace_size(None) == 0
+    assert bm.beam_moe_fp8_workspace_size(beam(64, d=100)) == 0
+    A = 1 << 20  # a fake, 16-byte aligned address: never dereferenced on these paths
+    q = ctypes.c_void_p
+    quant = L.beam_moe_quantize_e4m3
+    assert quant(q(A), 0, 512, q(A + (1 << 24)), q(A), None) == bm.BEAM_OK  # no rows: no-op
+    for rows, cols, x, out, sc in ((4, 24, A, A << 4, A),        # cols not a multiple of 16
+                                   (4, 0, A, A << 4, A),         # no columns
+                                   (-1, 64, A, A << 4, A),       # negative rows
+                                   (4, 64, A + 8, A << 4, A),    # misaligned input
+                                   (4, 64, A, (A << 4) + 4, A),  # misaligned codes
+                                   (4, 64, A, A << 4, 0),        # no scale array
+                                   (4, 64, A, A + 64, A)):       # codes overlap the input
+        assert quant(q(x), rows, cols, q(out), q(sc) if sc else None, None) == \
+            bm.BEAM_ERR_INVALID_ARG, (rows, cols)
+    fwd = L.beam_moe_forward_fp8
+    args = [q(A)] * 13
+    assert fwd(ctypes.byref(beam(0)), *[None] * 13, 0, None) == bm.BEAM_OK
+    assert fwd(ctypes.byref(beam(64, d=100)), *args, 1 << 30, None) == bm.BEAM_ERR_UNSUPPORTED
+    misaligned = list(args)
+    misaligned[5] = q(A + 4)  # up_scale
+    assert fwd(ctypes.byref(beam(64)), *misaligned, 1 << 30, None) == bm.BEAM_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(beam(64)), *args[:12], None, 16, None) == bm.BEAM_ERR_WORKSPACE

@@ -1,0 +1,126 @@
+"""Parity of the FP8 (E4M3) expert-weight path (called through the C ABI) with the oracle.
+
+The oracle quantises the seeded BF16 weights itself; the CUDA path's codes and scales must
+equal the oracle's bit for bit (integer decisions taken in FP32 on both sides).  Routing is the
+BF16 path's (indices bit-exact).  Outputs: relative L2 <= 1e-2 and max |err| <= 5e-2 * RMS
+against the oracle's FP8 layer, which multiplies the same codes exactly in double; the GPU
+accumulates in FP32 on the tensor cores, and an activation value that lands on the other side
+of a BF16 or E4M3 rounding boundary moves one code of its row.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_moe_transformer_fp32_b200 import beam_moe as bm
+from sparse_moe_transformer_fp32_b200 import workloads as W
+from tests import gpu_helpers as H
+from tests.test_gpu_parity import _check_routing
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    from sparse_moe_transformer_fp32_b200 import build
+    build.build()
+    bm.lib()
+    yield
+    torch.cuda.empty_cache()
+
+
+def test_quantize_e4m3_bit_exact_with_edge_rows():
+    rng = np.random.default_rng(0)
+    x = rng.normal(0, 1, (300, 512)).astype(np.float32)
+    x[1] = 0.0                          # all-zero row: scale 0, codes 0
+    x[2] *= 1e-30                       # tiny row (scale far below 1)
+    x[3, :] = 1e-2
+    x[3, 7] = 1e3                       # one outlier: the other codes subnormal (2 * 2^-9)
+    x[4] = np.where(np.arange(512) % 2 == 0, 448.0, -448.0)
+    x[5] *= 3e37                        # huge row
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    q, s = bm.beam_moe_quantize_e4m3(xb.cuda())
+    q_ref, s_ref = oracle.quantize_rows_e4m3(xb)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+def test_quantize_e4m3_bit_exact_beam_expert():
+    wl = W.WORKLOADS["prefill"]
+    for kind in ("gate", "down"):
+        m = W.expert_weight(wl, kind, 17, "cuda")
+        q, s = bm.beam_moe_quantize_e4m3(m)
+        q_ref, s_ref = oracle.quantize_rows_e4m3(m.cpu())
+        assert np.array_equal(s.cpu().numpy(), s_ref), kind
+        assert np.array_equal(q.cpu().numpy(), q_ref), kind
+
+
+def test_quantize_e4m3_rejects_bad_arguments():
+    x = torch.zeros(4, 24, dtype=torch.bfloat16, device="cuda")  # 24 columns: not a multiple of 16
+    with pytest.raises(bm.BeamError):
+        bm.beam_moe_quantize_e4m3(x)
+
+
+def test_forward_fp8_tiny_every_token():
+    case = H.make_case(W.WORKLOADS["tiny"])
+    weights = H.device_weights(case.wl)
+    fp8 = H.device_weights_fp8(weights)
+    out, idx, w, _ = H.run_forward_fp8(case, fp8)
+    _check_routing(case, idx, w)
+    ref = H.oracle_out_fp8(case, weights, range(case.wl.T), fp8, batch=64)
+    H.assert_close_out(out.float().cpu().numpy(), ref, "fp8 tiny")
+
+
+@pytest.mark.parametrize("T", [1, 33, 300])
+def test_forward_fp8_ragged_token_counts(T):
+    case = H.make_case(W.WORKLOADS["tiny"].with_tokens(T))
+    weights = H.device_weights(case.wl)
+    fp8 = H.device_weights_fp8(weights)
+    out, idx, w, _ = H.run_forward_fp8(case, fp8)
+    _check_routing(case, idx, w)
+    ref = H.oracle_out_fp8(case, weights, range(T), fp8, batch=64)
+    H.assert_close_out(out.float().cpu().numpy(), ref, f"fp8 tiny T={T}")
+
+
+def test_forward_fp8_differs_from_bf16_by_quantisation_only():
+    """Same inputs through both paths: the FP8 layer stays within a few percent of the BF16
+    layer (E4M3 keeps 4 significant bits), and is not identical to it."""
+    case = H.make_case(W.WORKLOADS["tiny"])
+    weights = H.device_weights(case.wl)
+    fp8 = H.device_weights_fp8(weights)
+    out8, _, _, _ = H.run_forward_fp8(case, fp8)
+    out16, _, _, _ = H.run_forward(case, weights)
+    a, b = out8.float().cpu().numpy(), out16.float().cpu().numpy()
+    r = H.rel_l2(a, b)
+    assert 1e-3 < r < 8e-2, r
+
+
+@pytest.fixture(scope="module")
+def beam_fp8():
+    wl = W.WORKLOADS["prefill"]
+    weights = H.device_weights(wl)
+    fp8 = H.device_weights_fp8(weights)
+    yield weights, fp8
+    del weights, fp8
+    torch.cuda.empty_cache()
+
+
+def test_forward_fp8_decode_every_token(beam_fp8):
+    weights, fp8 = beam_fp8
+    case = H.make_case(W.WORKLOADS["decode"])
+    out, idx, w, _ = H.run_forward_fp8(case, fp8)
+    _check_routing(case, idx, w)
+    ref = H.oracle_out_fp8(case, weights, range(case.wl.T), fp8, batch=8)
+    H.assert_close_out(out.float().cpu().numpy(), ref, "fp8 decode")
+
+
+def test_forward_fp8_prefill_sampled(beam_fp8):
+    weights, fp8 = beam_fp8
+    case = H.make_case(W.WORKLOADS["prefill"])
+    out, idx, w, _ = H.run_forward_fp8(case, fp8)
+    _check_routing(case, idx, w)
+    toks = H.sample_tokens(case, 8)
+    ref = H.oracle_out_fp8(case, weights, toks, fp8, batch=8)
+    H.assert_close_out(out[toks].float().cpu().numpy(), ref, "fp8 prefill")
