@@ -241,6 +241,8 @@ def kernel_work(wl, touched: int, fp8: bool = False):
     if fp8:
         q = 1
         return {
+            "router_transpose": {"flops": 0, "bytes": 2 * E * d * f4},
+            "dispatch_scan": {"flops": 0, "bytes": E * 16},
             "router_gemm": {"flops": 2 * T * d * E, "bytes": T * d * bf + E * d * f4 + T * E * f4},
             "router_select": {"flops": 0, "bytes": T * E * f4 + 2 * R * f4},
             "permute": {"flops": 0, "bytes": T * d * bf + R * d * q},
@@ -254,6 +256,8 @@ def kernel_work(wl, touched: int, fp8: bool = False):
     w_gu = touched * 2 * I * d * bf
     w_dn = touched * d * I * bf
     return {
+        "router_transpose": {"flops": 0, "bytes": 2 * E * d * f4},
+        "dispatch_scan": {"flops": 0, "bytes": E * 16},
         "router_gemm": {"flops": 2 * T * d * E, "bytes": T * d * bf + E * d * f4 + T * E * f4},
         "router_select": {"flops": 0, "bytes": T * E * f4 + 2 * R * f4},
         "permute": {"flops": 0, "bytes": T * d * bf + R * d * bf},
@@ -508,7 +512,7 @@ def run_cuda(args, rank, world, local):
             work = kernel_work(wl, touched, fp8=bool(fp8))
             per_kernel = {k: {"launches": n, "ms_per_launch": (ms / n if n else None)}
                           for k, (n, ms) in prof.items() if n}
-            dom = max((k for k in per_kernel), key=lambda k: prof[k][1])
+            dom = max((k for k in per_kernel if k in work), key=lambda k: prof[k][1])
             n_dom, ms_dom = prof[dom]
             avg_s = ms_dom / n_dom / 1e3
             wk = work[dom]

@@ -66,7 +66,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
+// SiLU with the fast reciprocal division (about two ulp): the epilogue's arithmetic is on the
+// critical path when the K loop is short (E4M3 operands), and the result is rounded to BF16.
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // FP8 epilogue: v0[j] *= sa * s0[j] and, when s1 is given, v1[j] *= sa * s1[j], for 32
 // consecutive columns (s0, s1 16-byte aligned; the same addresses across the warp).
