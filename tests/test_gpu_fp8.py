@@ -124,3 +124,31 @@ def test_forward_fp8_prefill_sampled(beam_fp8):
     toks = H.sample_tokens(case, 8)
     ref = H.oracle_out_fp8(case, weights, toks, fp8, batch=8)
     H.assert_close_out(out[toks].float().cpu().numpy(), ref, "fp8 prefill")
+
+
+@pytest.mark.parametrize("name,changes", [
+    ("E48_G8", dict(T=200, d=256, E=48, n_group=8, topk_group=3, top_k=5, I=128)),
+    ("d8192", dict(T=40, d=8192, E=8, n_group=2, topk_group=1, top_k=2, I=128)),
+    ("one_expert_per_group", dict(T=77, d=256, E=8, n_group=8, topk_group=3, top_k=3, I=128)),
+    ("many_tokens", dict(T=20000, d=256, E=16, n_group=4, topk_group=2, top_k=4, I=256)),
+])
+def test_forward_fp8_other_shapes(name, changes):
+    import dataclasses
+    wl = dataclasses.replace(W.WORKLOADS["tiny"], name=name, **changes)
+    case = H.make_case(wl)
+    weights = H.device_weights(wl)
+    fp8 = H.device_weights_fp8(weights)
+    out, idx, w, _ = H.run_forward_fp8(case, fp8)
+    _check_routing(case, idx, w)
+    toks = list(range(wl.T)) if wl.T <= 300 else H.sample_tokens(case, 40)
+    ref = H.oracle_out_fp8(case, weights, toks, fp8, batch=64)
+    H.assert_close_out(out[toks].float().cpu().numpy(), ref, f"fp8 {name}")
+
+
+def test_forward_fp8_deterministic():
+    case = H.make_case(W.WORKLOADS["tiny"].with_tokens(300))
+    weights = H.device_weights(case.wl)
+    fp8 = H.device_weights_fp8(weights)
+    out1, _, _, ws = H.run_forward_fp8(case, fp8)
+    out2, _, _, _ = H.run_forward_fp8(case, fp8, ws=ws)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
