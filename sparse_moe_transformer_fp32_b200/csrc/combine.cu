@@ -61,17 +61,37 @@ __device__ __forceinline__ void load_slots(const CombineArgs& a, int t, int* row
   __syncthreads();
 }
 
+// kPrefetch: all k row loads are issued before the sums that consume them (which stay in slot
+// order); it helps the layer combine and costs the block form occupancy (more registers), so
+// the block form loads a row at a time.
+template <bool kPrefetch>
 __device__ __forceinline__ void combine_vec(const CombineArgs& a, const int* rows, const float* ws,
                                             int c, float (&acc)[8]) {
 #pragma unroll
   for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-  for (int j = 0; j < a.k; ++j) {
-    const uint4 v =
-        reinterpret_cast<const uint4*>(a.y + static_cast<size_t>(rows[j]) * a.d)[c];
-    float f[8];
-    unpack_bf16x8(v, f);
+  if constexpr (!kPrefetch) {
+    for (int j = 0; j < a.k; ++j) {
+      const uint4 v =
+          reinterpret_cast<const uint4*>(a.y + static_cast<size_t>(rows[j]) * a.d)[c];
+      float f[8];
+      unpack_bf16x8(v, f);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) acc[q] = fmaf(ws[j], f[q], acc[q]);
+      for (int q = 0; q < 8; ++q) acc[q] = fmaf(ws[j], f[q], acc[q]);
+    }
+    return;
+  }
+  uint4 v[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (j < a.k) v[j] = reinterpret_cast<const uint4*>(a.y + static_cast<size_t>(rows[j]) * a.d)[c];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    if (j < a.k) {
+      float f[8];
+      unpack_bf16x8(v[j], f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = fmaf(ws[j], f[q], acc[q]);
+    }
   }
 }
 
@@ -84,7 +104,7 @@ __global__ void __launch_bounds__(kCThreads) combine_kernel(const CombineArgs a)
   uint4* out = reinterpret_cast<uint4*>(a.out + static_cast<size_t>(t) * a.d);
   for (int c = threadIdx.x; c < nvec; c += kCThreads) {
     float acc[8];
-    combine_vec(a, rows, ws, c, acc);
+    combine_vec<true>(a, rows, ws, c, acc);
     out[c] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
                         pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
   }
@@ -103,7 +123,7 @@ __global__ void __launch_bounds__(kCThreads) combine_block_kernel(const CombineA
   for (int v = 0; v < kMaxVec; ++v) {
     const int c = threadIdx.x + v * kCThreads;
     if (c < nvec) {
-      combine_vec(a, rows, ws, c, o[v]);
+      combine_vec<false>(a, rows, ws, c, o[v]);
 #pragma unroll
       for (int q = 0; q < 8; ++q) ss = fmaf(o[v][q], o[v][q], ss);
     }

@@ -152,3 +152,27 @@ def test_forward_fp8_deterministic():
     out1, _, _, ws = H.run_forward_fp8(case, fp8)
     out2, _, _, _ = H.run_forward_fp8(case, fp8, ws=ws)
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_forward_fp8_wait_timeout_is_reported_and_context_survives():
+    """With a zero wait limit the E4M3 GEMMs give up at their first open barrier, record the
+    timeout and drain; the next call is correct."""
+    case = H.make_case(W.WORKLOADS["tiny"].with_tokens(512))
+    weights = H.device_weights(case.wl)
+    fp8 = H.device_weights_fp8(weights)
+    s = bm.shape_of(case.wl)
+    out = torch.empty(case.wl.T, case.wl.d, dtype=torch.bfloat16, device="cuda")
+    old = bm.beam_moe_get_wait_limit_ns()
+    bm.beam_moe_set_wait_limit_ns(0)
+    try:
+        ws = bm.beam_moe_forward_fp8(s, case.h.cuda(), case.router_w.cuda(), case.bias.cuda(),
+                                     *fp8, out)
+        st = bm.beam_moe_sync_status(ws)
+    finally:
+        bm.beam_moe_set_wait_limit_ns(old)
+    assert st == bm.BEAM_ERR_TIMEOUT, bm.status_string(st)
+    out2, idx, w, _ = H.run_forward_fp8(case, fp8)
+    _check_routing(case, idx, w)
+    toks = list(range(0, case.wl.T, 37))
+    ref = H.oracle_out_fp8(case, weights, toks, fp8, batch=64)
+    H.assert_close_out(out2[toks].float().cpu().numpy(), ref, "fp8 after timeout")
