@@ -59,6 +59,9 @@ def parse_args(argv=None):
                    help="tokens in the oracle's bounded sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--sm-pairs", action="store_true",
+                   help="enable the SM-pair (cta_group::2) expert GEMMs for calls with >= 256 "
+                        "rows per expert (off by default)")
     p.add_argument("--fp8", action="store_true",
                    help="E4M3 expert weights (beam_moe_forward_fp8); layer workloads only")
     p.add_argument("--route-only", action="store_true",
@@ -367,6 +370,7 @@ def run_cuda(args, rank, world, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     bm.lib()  # fails loudly if the extension is missing
+    bm.beam_moe_set_sm_pairs(bool(args.sm_pairs))
     wl = selected_workload(args)
     peaks = load_peaks()
     with process_group(world, "nccl") as dist:
@@ -573,7 +577,8 @@ def run_cuda(args, rank, world, local):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
-                "config": {"workload": f"{wl.name}{'-fp8' if fp8 else ''}: T={wl.T} d={wl.d} "
+                "config": {"workload": f"{wl.name}{'-fp8' if fp8 else ''}"
+                                       f"{'-smpairs' if args.sm_pairs else ''}: T={wl.T} d={wl.d} "
                                        f"E={wl.E} n_group={wl.n_group} "
                                        f"topk_group={wl.topk_group} top_k={wl.top_k} I={wl.I}"
                                        + (" block" if wl.block else ""),

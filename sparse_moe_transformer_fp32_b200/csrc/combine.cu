@@ -78,19 +78,20 @@ __device__ __forceinline__ void combine_vec(const CombineArgs& a, const int* row
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[q] = fmaf(ws[j], f[q], acc[q]);
     }
-    return;
-  }
-  uint4 v[kMaxTopK];
+  } else {
+    uint4 v[kMaxTopK];
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j)
-    if (j < a.k) v[j] = reinterpret_cast<const uint4*>(a.y + static_cast<size_t>(rows[j]) * a.d)[c];
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (j < a.k)
+        v[j] = reinterpret_cast<const uint4*>(a.y + static_cast<size_t>(rows[j]) * a.d)[c];
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
-    if (j < a.k) {
-      float f[8];
-      unpack_bf16x8(v[j], f);
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j < a.k) {
+        float f[8];
+        unpack_bf16x8(v[j], f);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] = fmaf(ws[j], f[q], acc[q]);
+        for (int q = 0; q < 8; ++q) acc[q] = fmaf(ws[j], f[q], acc[q]);
+      }
     }
   }
 }

@@ -101,11 +101,17 @@ __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterG
     }
   };
 
-  float acc[8][8];
+  // Packed FMAs (fma.rn.f32x2: two IEEE FMAs, so every logit sees the same sequence of
+  // roundings as with scalar fmaf, in half the instructions).  Rows are paired (2r, 2r + 1)
+  // and columns (2c, 2c + 1); a row pair times a column pair gives the diagonal products,
+  // times the swapped column pair the anti-diagonal ones:
+  //   dg[r][c] = (acc[2r][2c],     acc[2r + 1][2c + 1])
+  //   ad[r][c] = (acc[2r][2c + 1], acc[2r + 1][2c])
+  float2 dg[4][4], ad[4][4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int r = 0; r < 4; ++r)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int c = 0; c < 4; ++c) dg[r][c] = ad[r][c] = make_float2(0.f, 0.f);
 
   if (nk > 0) {
     issue_b(0, kbeg);
@@ -129,16 +135,34 @@ __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterG
       const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
       const float4 b0 = *reinterpret_cast<const float4*>(&Bs[st][kk][tx * 4]);
       const float4 b1 = *reinterpret_cast<const float4*>(&Bs[st][kk][64 + tx * 4]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      const float2 ap[4] = {make_float2(a0.x, a0.y), make_float2(a0.z, a0.w),
+                            make_float2(a1.x, a1.y), make_float2(a1.z, a1.w)};
+      const float2 bp[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w),
+                            make_float2(b1.x, b1.y), make_float2(b1.z, b1.w)};
+      const float2 bs[4] = {make_float2(b0.y, b0.x), make_float2(b0.w, b0.z),
+                            make_float2(b1.y, b1.x), make_float2(b1.w, b1.z)};
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int c = 0; c < 4; ++c) {
+          dg[r][c] = __ffma2_rn(ap[r], bp[c], dg[r][c]);
+          ad[r][c] = __ffma2_rn(ap[r], bs[c], ad[r][c]);
+        }
     }
     if (kt + 1 < nk) store_a(buf ^ 1, next);
   }
 
+  // acc[i][j] back from the pairs: rows i = 2r + s, columns j = 2c + u
+  float acc[8][8];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      acc[2 * r][2 * c] = dg[r][c].x;
+      acc[2 * r + 1][2 * c + 1] = dg[r][c].y;
+      acc[2 * r][2 * c + 1] = ad[r][c].x;
+      acc[2 * r + 1][2 * c] = ad[r][c].y;
+    }
   float* part = a.part + static_cast<size_t>(blockIdx.z) * a.T * a.E;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
