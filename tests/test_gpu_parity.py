@@ -6,6 +6,7 @@ token; the full-size workloads are compared on every token's routing and on samp
 outputs, in the same launch configuration the benchmark times.
 """
 import ctypes
+import dataclasses
 
 import numpy as np
 import pytest
@@ -352,3 +353,44 @@ def test_zero_tokens_reads_nothing():
     L = bm.lib()
     assert L.beam_moe_forward(ctypes.byref(s), None, None, None, None, None, None, None, None,
                               None, None, 0, None) == bm.BEAM_OK
+
+
+def test_forward_replays_from_a_cuda_graph():
+    """The forward is launches only (no allocation, no host synchronisation), so it can be
+    captured once and replayed: replays on new input contents match eager calls bit for bit."""
+    wl = W.WORKLOADS["tiny"].with_tokens(300)
+    case = H.make_case(wl)
+    weights = H.device_weights(wl)
+    fp8 = H.device_weights_fp8(weights)
+    s = bm.shape_of(wl)
+    dev = "cuda"
+    h_static = case.h.to(dev).clone()
+    rw, b = case.router_w.to(dev), case.bias.to(dev)
+    out16 = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
+    out8 = torch.empty_like(out16)
+    ws16, ws8 = bm.workspace(s), bm.fp8_workspace(s)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # first calls outside the capture set up per-device state
+        bm.beam_moe_forward(s, h_static, rw, b, *weights, out16, ws=ws16)
+        bm.beam_moe_forward_fp8(s, h_static, rw, b, *fp8, out8, ws=ws8)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        bm.beam_moe_forward(s, h_static, rw, b, *weights, out16, ws=ws16)
+        bm.beam_moe_forward_fp8(s, h_static, rw, b, *fp8, out8, ws=ws8)
+    for seed in (5, 6):
+        h_new = W.hidden(dataclasses.replace(wl, seed=seed)).to(dev)
+        h_static.copy_(h_new)
+        g.replay()
+        torch.cuda.synchronize()
+        assert bm.beam_moe_sync_status(ws16) == bm.BEAM_OK
+        ref16 = torch.empty_like(out16)
+        ref8 = torch.empty_like(out8)
+        bm.beam_moe_forward(s, h_new, rw, b, *weights, ref16)
+        bm.beam_moe_forward_fp8(s, h_new, rw, b, *fp8, ref8)
+        torch.cuda.synchronize()
+        assert torch.equal(out16.view(torch.int16), ref16.view(torch.int16)), seed
+        assert torch.equal(out8.view(torch.int16), ref8.view(torch.int16)), seed
+    del g
