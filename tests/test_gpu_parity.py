@@ -394,3 +394,28 @@ def test_forward_replays_from_a_cuda_graph():
         assert torch.equal(out16.view(torch.int16), ref16.view(torch.int16)), seed
         assert torch.equal(out8.view(torch.int16), ref8.view(torch.int16)), seed
     del g
+
+
+def test_concurrent_forwards_on_two_streams():
+    """Two forwards with their own workspaces running at the same time on two streams (kernels
+    of one may share SMs with the other's) give the same bits as each run alone."""
+    wl = W.WORKLOADS["tiny"].with_tokens(600)
+    weights = H.device_weights(wl)
+    s = bm.shape_of(wl)
+    cases = [H.make_case(dataclasses.replace(wl, seed=sd)) for sd in (11, 12)]
+    alone = [H.run_forward(c, weights)[0] for c in cases]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs, wss = [], []
+    for c, st in zip(cases, streams):
+        outs.append(torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda"))
+        wss.append(bm.workspace(s))
+    torch.cuda.synchronize()
+    for _ in range(5):
+        for c, st, o, ws in zip(cases, streams, outs, wss):
+            with torch.cuda.stream(st):
+                bm.beam_moe_forward(s, c.h.cuda(), c.router_w.cuda(), c.bias.cuda(), *weights, o,
+                                    ws=ws)
+    torch.cuda.synchronize()
+    for o, a, ws in zip(outs, alone, wss):
+        assert bm.beam_moe_sync_status(ws) == bm.BEAM_OK
+        assert torch.equal(o.view(torch.int16), a.view(torch.int16))
