@@ -255,6 +255,9 @@ def kernel_work(wl, touched: int, fp8: bool = False):
             "expert_gemm_down": {"flops": 2 * R * d * I,
                                  "bytes": touched * d * I * q + R * I * q + R * d * bf},
             "combine": {"flops": 2 * R * d, "bytes": R * d * bf + T * d * bf},
+            "combine_block": {"flops": 2 * R * d, "bytes": R * d * bf + 3 * T * d * f4},
+            "prenorm": {"flops": 3 * T * d, "bytes": T * d * f4 + T * d * bf},
+            "dense_tiles": {"flops": 0, "bytes": 16 * (T // 128 + 1)},
         }
     w_gu = touched * 2 * I * d * bf
     w_dn = touched * d * I * bf
@@ -394,14 +397,12 @@ def run_cuda(args, rank, world, local):
             inp_cpu, inp, res = h_cpu, h, out
         fp8 = None
         if args.fp8:
-            if wl.dense or wl.block:
-                raise SystemExit("bench.py: --fp8 applies to the layer workloads")
             fp8 = []
             for m in weights:
-                fp8 += list(bm.beam_moe_quantize_e4m3(m))
+                fp8 += list(bm.beam_moe_quantize_e4m3(m[0] if wl.dense else m))
             torch.cuda.synchronize(dev)
         if wl.dense:
-            ws = bm.dense_workspace(ds, dev)
+            ws = bm.dense_fp8_workspace(ds, dev) if fp8 else bm.dense_workspace(ds, dev)
         else:
             ws = bm.fp8_workspace(s, dev) if fp8 else bm.workspace(s, dev)
         stream = torch.cuda.current_stream(dev)
@@ -409,9 +410,14 @@ def run_cuda(args, rank, world, local):
         def step(src=None, dst=None):
             src = inp if src is None else src
             dst = res if dst is None else dst
-            if wl.dense:
+            if wl.dense and fp8:
+                bm.beam_dense_forward_fp8(ds, src, *fp8, dst, ws=ws)
+            elif wl.dense:
                 bm.beam_dense_forward(ds, src, weights[0][0], weights[1][0], weights[2][0], dst,
                                       ws=ws)
+            elif wl.block and fp8:
+                bm.beam_moe_block_fp8(s, src, g_pre, g_post, wl.eps, wl.k_resid, router_w, bias,
+                                      *fp8, dst, ws=ws)
             elif wl.block:
                 bm.beam_moe_block(s, src, g_pre, g_post, wl.eps, wl.k_resid, router_w, bias,
                                   *weights, dst, ws=ws)
@@ -549,7 +555,9 @@ def run_cuda(args, rank, world, local):
             flops_step = 6 * wl.T * wl.top_k * wl.d * wl.I  # top_k = 1 for the dense MLP
             bytes_step = layer_min_bytes(wl, touched, fp8=bool(fp8))
             cpu = None
-            if not args.no_cpu_baseline and world == 1 and fp8:
+            if fp8 and (wl.dense or wl.block):
+                pass  # the E4M3 CPU baseline is timed on the layer workloads only
+            elif not args.no_cpu_baseline and world == 1 and fp8:
                 n_cpu = min(args.cpu_sample_tokens, 16)
                 rate, secs, cores = oracle_fp8_sample_rate(
                     wl, W.router_weight(wl), W.router_bias(wl), inp_cpu, weights, n_cpu)

@@ -167,6 +167,17 @@ BEAM_API beam_status beam_moe_forward_fp8(const beam_moe_shape* shape, const voi
                                           int32_t* topk_idx, float* topk_w, void* ws,
                                           size_t ws_bytes, beam_stream stream);
 
+/* beam_moe_block with E4M3 expert weights (codes and row scales as for beam_moe_forward_fp8);
+ * every other argument as for beam_moe_block, with ws sized by beam_moe_fp8_workspace_size. */
+BEAM_API beam_status beam_moe_block_fp8(const beam_moe_shape* shape, const float* x,
+                                        const float* g_pre, const float* g_post, float eps,
+                                        int32_t k_resid, const float* router_w, const float* bias,
+                                        const void* w_gate, const float* gate_scale,
+                                        const void* w_up, const float* up_scale,
+                                        const void* w_down, const float* down_scale,
+                                        float* x_out, int32_t* topk_idx, float* topk_w, void* ws,
+                                        size_t ws_bytes, beam_stream stream);
+
 /* MoE block: x' = x * sqrt((k_resid-1)/k_resid) + RMSNorm(MoE(bf16(RMSNorm(x) g_pre))) g_post
  *                 / sqrt(k_resid), RMSNorm(v) = v / sqrt(mean(v^2) + eps), all FP32.
  *   x       FP32 [T, d] residual stream in
@@ -199,6 +210,20 @@ BEAM_API size_t beam_dense_workspace_size(const beam_dense_shape* shape);
 BEAM_API beam_status beam_dense_forward(const beam_dense_shape* shape, const void* hidden,
                                         const void* w_gate, const void* w_up, const void* w_down,
                                         void* out, void* ws, size_t ws_bytes, beam_stream stream);
+
+/* Workspace bytes for beam_dense_forward_fp8 (0 for an unsupported shape). */
+BEAM_API size_t beam_dense_fp8_workspace_size(const beam_dense_shape* shape);
+
+/* beam_dense_forward with E4M3 weights: w_gate, w_up E4M3 [I, d] with row scales gate_scale,
+ * up_scale FP32 [I]; w_down E4M3 [d, I] with row scales down_scale FP32 [d] (as written by
+ * beam_moe_quantize_e4m3; scale arrays 16-byte aligned).  The token rows and the SwiGLU
+ * activation are quantised per row as in beam_moe_forward_fp8. */
+BEAM_API beam_status beam_dense_forward_fp8(const beam_dense_shape* shape, const void* hidden,
+                                            const void* w_gate, const float* gate_scale,
+                                            const void* w_up, const float* up_scale,
+                                            const void* w_down, const float* down_scale,
+                                            void* out, void* ws, size_t ws_bytes,
+                                            beam_stream stream);
 
 /* Selection-bias update from the expert loads of the last beam_moe_forward / beam_moe_block
  * call made with `ws` (same shape):  bias[e] += gamma * sign(mean_load - load[e]), sign(0) = 0,

@@ -32,7 +32,8 @@ EXPORTED = [
     "beam_moe_abi_version", "beam_moe_route_static", "beam_dense_workspace_size",
     "beam_dense_forward", "beam_moe_bias_update", "beam_moe_set_sm_pairs",
     "beam_moe_get_sm_pairs", "beam_moe_quantize_e4m3", "beam_moe_fp8_workspace_size",
-    "beam_moe_forward_fp8",
+    "beam_moe_forward_fp8", "beam_moe_block_fp8", "beam_dense_fp8_workspace_size",
+    "beam_dense_forward_fp8",
 ]
 
 
@@ -97,12 +98,16 @@ def lib():
     L.beam_dense_workspace_size.argtypes = [dshp]
     L.beam_dense_workspace_size.restype = sz
     L.beam_dense_forward.argtypes = [dshp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.beam_dense_fp8_workspace_size.argtypes = [dshp]
+    L.beam_dense_fp8_workspace_size.restype = sz
+    L.beam_dense_forward_fp8.argtypes = [dshp] + [vp] * 9 + [sz, vp]
     L.beam_moe_bias_update.argtypes = [shp, vp, vp, f32, vp]
     L.beam_moe_quantize_e4m3.argtypes = [vp, ctypes.c_int64, i32, vp, vp, vp]
     L.beam_moe_fp8_workspace_size.argtypes = [shp]
     L.beam_moe_fp8_workspace_size.restype = sz
     L.beam_moe_forward_fp8.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                        sz, vp]
+    L.beam_moe_block_fp8.argtypes = [shp, vp, vp, vp, f32, i32] + [vp] * 12 + [sz, vp]
     L.beam_moe_sync_status.argtypes = [vp, vp]
     L.beam_status_string.argtypes = [ctypes.c_int]
     L.beam_status_string.restype = ctypes.c_char_p
@@ -121,7 +126,7 @@ def lib():
     for name in ("beam_moe_route", "beam_moe_route_static", "beam_moe_forward", "beam_moe_block",
                  "beam_moe_sync_status", "beam_dense_forward", "beam_moe_bias_update",
                  "beam_moe_expert_counts", "beam_moe_profile_read", "beam_moe_quantize_e4m3",
-                 "beam_moe_forward_fp8"):
+                 "beam_moe_forward_fp8", "beam_moe_block_fp8", "beam_dense_forward_fp8"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -336,6 +341,59 @@ def beam_dense_forward(shape, hidden, w_gate, w_up, w_down, out, ws=None, stream
     _ptr(ws, torch.uint8, "ws")
     _check(lib().beam_dense_forward(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
                                     _stream(stream)), "beam_dense_forward")
+    return ws
+
+
+def beam_moe_block_fp8(shape, x, g_pre, g_post, eps, k_resid, router_w, bias, w_gate, gate_scale,
+                       w_up, up_scale, w_down, down_scale, x_out, topk_idx=None, topk_w=None,
+                       ws=None, stream=None):
+    T, d, E, k, I = shape.T, shape.d, shape.E, shape.top_k, shape.I
+    args = [_ptr(x, torch.float32, "x", (T, d)),
+            _ptr(g_pre, torch.float32, "g_pre", (d,)),
+            _ptr(g_post, torch.float32, "g_post", (d,)),
+            ctypes.c_float(eps), ctypes.c_int32(k_resid),
+            _ptr(router_w, torch.float32, "router_w", (E, d)),
+            _ptr(bias, torch.float32, "bias", (E,)),
+            _ptr(w_gate, torch.uint8, "w_gate", (E, I, d)),
+            _ptr(gate_scale, torch.float32, "gate_scale", (E, I)),
+            _ptr(w_up, torch.uint8, "w_up", (E, I, d)),
+            _ptr(up_scale, torch.float32, "up_scale", (E, I)),
+            _ptr(w_down, torch.uint8, "w_down", (E, d, I)),
+            _ptr(down_scale, torch.float32, "down_scale", (E, d)),
+            _ptr(x_out, torch.float32, "x_out", (T, d)),
+            _ptr(topk_idx, torch.int32, "topk_idx", (T, k), optional=True),
+            _ptr(topk_w, torch.float32, "topk_w", (T, k), optional=True)]
+    if ws is None:
+        ws = fp8_workspace(shape, x.device)
+    _ptr(ws, torch.uint8, "ws")
+    _check(lib().beam_moe_block_fp8(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
+                                    _stream(stream)), "beam_moe_block_fp8")
+    return ws
+
+
+def dense_fp8_workspace(shape: beam_dense_shape, device="cuda") -> torch.Tensor:
+    n = int(lib().beam_dense_fp8_workspace_size(ctypes.byref(shape)))
+    if n == 0:
+        raise BeamError(BEAM_ERR_UNSUPPORTED, "beam_dense_fp8_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def beam_dense_forward_fp8(shape, hidden, w_gate, gate_scale, w_up, up_scale, w_down, down_scale,
+                           out, ws=None, stream=None):
+    T, d, I = shape.T, shape.d, shape.I
+    args = [_ptr(hidden, torch.bfloat16, "hidden", (T, d)),
+            _ptr(w_gate, torch.uint8, "w_gate", (I, d)),
+            _ptr(gate_scale, torch.float32, "gate_scale", (I,)),
+            _ptr(w_up, torch.uint8, "w_up", (I, d)),
+            _ptr(up_scale, torch.float32, "up_scale", (I,)),
+            _ptr(w_down, torch.uint8, "w_down", (d, I)),
+            _ptr(down_scale, torch.float32, "down_scale", (d,)),
+            _ptr(out, torch.bfloat16, "out", (T, d))]
+    if ws is None:
+        ws = dense_fp8_workspace(shape, hidden.device)
+    _ptr(ws, torch.uint8, "ws")
+    _check(lib().beam_dense_forward_fp8(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
+                                        _stream(stream)), "beam_dense_forward_fp8")
     return ws
 
 

@@ -535,6 +535,7 @@ beam_status check_dense_shape(const beam_dense_shape* s) {
 
 struct DenseLayout {
   size_t status, mt_count, mtiles, act, total;
+  size_t hq = 0, hs = 0, act8 = 0, as = 0;  // E4M3 form: quantised rows and their scales
   int64_t mt_cap;
 };
 
@@ -553,6 +554,220 @@ DenseLayout plan_dense(const beam_dense_shape& s) {
   L.act = take(sizeof(__nv_bfloat16) * static_cast<size_t>(s.T) * s.I);
   L.total = o;
   return L;
+}
+
+// E4M3 dense MLP: the BF16 layout plus the quantised token rows, the quantised activation and
+// their row scales.
+DenseLayout plan_dense_fp8(const beam_dense_shape& s) {
+  DenseLayout L = plan_dense(s);
+  size_t o = L.total;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o = align_up(o + (bytes ? bytes : 1), 1024);
+    return r;
+  };
+  L.hq = take(static_cast<size_t>(s.T) * s.d);
+  L.hs = take(sizeof(float) * s.T);
+  L.act8 = take(static_cast<size_t>(s.T) * s.I);
+  L.as = take(sizeof(float) * s.T);
+  L.total = o;
+  return L;
+}
+
+
+// ------------------------------------------------------------------ entry-point bodies
+//
+// The BF16 and E4M3 forms of each entry point share one body; f8 (non-null) carries the row
+// scales of E4M3 expert weights.
+
+bool misaligned_fp8(const Fp8Scales* f8) {
+  return f8 && any_misaligned({f8->gate, f8->up, f8->down});
+}
+
+beam_status forward_impl(const beam_moe_shape* shape, const void* hidden, const float* router_w,
+                         const float* bias, const void* w_gate, const void* w_up,
+                         const void* w_down, void* out, int32_t* topk_idx, float* topk_w,
+                         void* ws, size_t ws_bytes, beam_stream stream, const Fp8Scales* f8) {
+  beam_status b = check_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
+  if (any_misaligned({hidden, router_w, w_gate, w_up, w_down, out}) || misaligned_fp8(f8) ||
+      !bias || (topk_idx && !aligned16(topk_idx)) || (topk_w && !aligned16(topk_w)))
+    return BEAM_ERR_INVALID_ARG;
+  const Layout L = f8 ? plan_fp8(*shape) : plan(*shape);
+  if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
+  DeviceInfo* dev;
+  if ((b = device_info(&dev)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
+  float* w = topk_w ? topk_w : at<float>(ws, L.w);
+  const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(hidden);
+  if ((b = run_router(*shape, L, h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
+    return b;
+  if ((b = run_experts(*shape, L, *dev, h, idx, w_gate, w_up, w_down, ws, st, f8)) != BEAM_OK)
+    return b;
+  CombineArgs ca{};
+  ca.y = at<__nv_bfloat16>(ws, L.y);
+  ca.rowmap = at<int32_t>(ws, L.rowmap);
+  ca.w = w;
+  ca.out = static_cast<__nv_bfloat16*>(out);
+  ca.status = at<uint32_t>(ws, L.status);
+  ca.T = shape->T;
+  ca.d = shape->d;
+  ca.k = shape->top_k;
+  ca.R = static_cast<int>(L.R);
+  BEAM_LAUNCH(kKCombine, st, launch_combine(ca, st));
+  return BEAM_OK;
+}
+
+beam_status block_impl(const beam_moe_shape* shape, const float* x, const float* g_pre,
+                       const float* g_post, float eps, int32_t k_resid, const float* router_w,
+                       const float* bias, const void* w_gate, const void* w_up,
+                       const void* w_down, float* x_out, int32_t* topk_idx, float* topk_w,
+                       void* ws, size_t ws_bytes, beam_stream stream, const Fp8Scales* f8) {
+  beam_status b = check_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
+  if (any_misaligned({x, g_pre, g_post, router_w, w_gate, w_up, w_down, x_out}) ||
+      misaligned_fp8(f8) || !bias || (topk_idx && !aligned16(topk_idx)) ||
+      (topk_w && !aligned16(topk_w)))
+    return BEAM_ERR_INVALID_ARG;
+  if (!(eps > 0.f) || !std::isfinite(eps) || k_resid < 1) return BEAM_ERR_INVALID_ARG;
+  if (x_out != x) {  // in place or disjoint
+    const char* a0 = reinterpret_cast<const char*>(x);
+    const char* b0 = reinterpret_cast<const char*>(x_out);
+    const size_t n = sizeof(float) * static_cast<size_t>(shape->T) * shape->d;
+    if (a0 < b0 + n && b0 < a0 + n) return BEAM_ERR_INVALID_ARG;
+  }
+  const Layout L = f8 ? plan_fp8(*shape) : plan(*shape);
+  if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
+  DeviceInfo* dev;
+  if ((b = device_info(&dev)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  PreNormArgs pn{};
+  pn.x = x;
+  pn.g_pre = g_pre;
+  pn.h = at<__nv_bfloat16>(ws, L.h);
+  pn.eps = eps;
+  pn.T = shape->T;
+  pn.d = shape->d;
+  BEAM_LAUNCH(kKPreNorm, st, launch_prenorm(pn, st));
+
+  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
+  float* w = topk_w ? topk_w : at<float>(ws, L.w);
+  if ((b = run_router(*shape, L, pn.h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
+    return b;
+  if ((b = run_experts(*shape, L, *dev, pn.h, idx, w_gate, w_up, w_down, ws, st, f8)) != BEAM_OK)
+    return b;
+  const double kk = static_cast<double>(k_resid);
+  CombineArgs ca{};
+  ca.y = at<__nv_bfloat16>(ws, L.y);
+  ca.rowmap = at<int32_t>(ws, L.rowmap);
+  ca.w = w;
+  ca.x = x;
+  ca.g_post = g_post;
+  ca.x_out = x_out;
+  ca.eps = eps;
+  ca.coef_x = static_cast<float>(std::sqrt((kk - 1.0) / kk));
+  ca.coef_f = static_cast<float>(1.0 / std::sqrt(kk));
+  ca.status = at<uint32_t>(ws, L.status);
+  ca.T = shape->T;
+  ca.d = shape->d;
+  ca.k = shape->top_k;
+  ca.R = static_cast<int>(L.R);
+  BEAM_LAUNCH(kKCombineBlock, st, launch_combine_block(ca, st));
+  return BEAM_OK;
+}
+
+// Dense SwiGLU MLP: one "expert" holding every token.  The E4M3 form quantises the token rows
+// and the activation per row, as the MoE path does.
+beam_status dense_impl(const beam_dense_shape* shape, const void* hidden, const void* w_gate,
+                       const void* w_up, const void* w_down, void* out, void* ws,
+                       size_t ws_bytes, beam_stream stream, const Fp8Scales* f8) {
+  beam_status b = check_dense_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
+  if (any_misaligned({hidden, w_gate, w_up, w_down, out}) || misaligned_fp8(f8))
+    return BEAM_ERR_INVALID_ARG;
+  const DenseLayout L = f8 ? plan_dense_fp8(*shape) : plan_dense(*shape);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < L.total)
+    return BEAM_ERR_WORKSPACE;
+  DeviceInfo* dev;
+  if ((b = device_info(&dev)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const beam_dense_shape& s = *shape;
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  cudaError_t e = cudaMemsetAsync(status, 0, 16, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  MTile* mtiles = at<MTile>(ws, L.mtiles);
+  int32_t* mt_count = at<int32_t>(ws, L.mt_count);
+  BEAM_LAUNCH(kKDenseTiles, st, launch_dense_tiles(s.T, mtiles, mt_count, st));
+
+  void* act = at<void>(ws, L.act);
+  const void* a1 = hidden;
+  const void* a2 = act;
+  if (f8) {
+    BEAM_LAUNCH(kKQuantize, st,
+                launch_quantize_rows(static_cast<const __nv_bfloat16*>(hidden), s.T, s.d,
+                                     at<uint8_t>(ws, L.hq), at<float>(ws, L.hs), st));
+    a1 = at<void>(ws, L.hq);
+    a2 = at<void>(ws, L.act8);
+  }
+  const int eb = f8 ? 1 : 2;
+  const int k_elems = 128 / eb;
+  ATensorMaps tm_h, tm_act;
+  CUtensorMap tm_g, tm_u, tm_d;
+  for (int i = 0; i < kNumABoxes; ++i) {
+    if ((b = make_map(&tm_h.m[i], a1, s.d, s.T, a_box_rows(i), eb)) != BEAM_OK) return b;
+    if ((b = make_map(&tm_act.m[i], a2, s.I, s.T, a_box_rows(i), eb)) != BEAM_OK) return b;
+  }
+  if ((b = make_map(&tm_g, w_gate, s.d, s.I, kN1Half, eb)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_u, w_up, s.d, s.I, kN1Half, eb)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_d, w_down, s.I, s.d, kN2, eb)) != BEAM_OK) return b;
+
+  GemmArgs g1{};
+  g1.mtiles = mtiles;
+  g1.mt_count = mt_count;
+  g1.out = static_cast<__nv_bfloat16*>(act);
+  g1.status = status;
+  g1.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  g1.out_ld = s.I;
+  g1.n_tiles_n = s.I / kN1Half;
+  g1.k_blocks = s.d / k_elems;
+  g1.b_rows_per_expert = s.I;
+  g1.swap_max_rows = 0;
+  if (f8) {
+    g1.a_scale = at<float>(ws, L.hs);
+    g1.b_scale0 = f8->gate;
+    g1.b_scale1 = f8->up;
+  }
+  const int64_t t1 = L.mt_cap * g1.n_tiles_n;
+  BEAM_LAUNCH(kKGemmGateUp, st,
+              launch_gemm_gate_up(tm_h, tm_g, tm_u, g1,
+                                  static_cast<int>(t1 < dev->sms ? t1 : dev->sms), st,
+                                  f8 != nullptr));
+  if (f8)
+    BEAM_LAUNCH(kKQuantize, st,
+                launch_quantize_rows(static_cast<const __nv_bfloat16*>(act), s.T, s.I,
+                                     at<uint8_t>(ws, L.act8), at<float>(ws, L.as), st));
+  GemmArgs g2 = g1;
+  g2.out = static_cast<__nv_bfloat16*>(out);
+  g2.out_ld = s.d;
+  g2.n_tiles_n = s.d / kN2;
+  g2.k_blocks = s.I / k_elems;
+  g2.b_rows_per_expert = s.d;
+  if (f8) {
+    g2.a_scale = at<float>(ws, L.as);
+    g2.b_scale0 = f8->down;
+    g2.b_scale1 = nullptr;
+  }
+  const int64_t t2 = L.mt_cap * g2.n_tiles_n;
+  BEAM_LAUNCH(kKGemmDown, st,
+              launch_gemm_down(tm_act, tm_d, g2,
+                               static_cast<int>(t2 < dev->sms ? t2 : dev->sms), st,
+                               f8 != nullptr));
+  return BEAM_OK;
 }
 
 }  // namespace
@@ -635,41 +850,6 @@ beam_status beam_moe_route(const beam_moe_shape* shape, const void* hidden, cons
                     topk_w, logits_out, false, ws, st);
 }
 
-beam_status beam_moe_forward(const beam_moe_shape* shape, const void* hidden, const float* router_w,
-                             const float* bias, const void* w_gate, const void* w_up,
-                             const void* w_down, void* out, int32_t* topk_idx, float* topk_w,
-                             void* ws, size_t ws_bytes, beam_stream stream) {
-  beam_status b = check_shape(shape);
-  if (b != BEAM_OK) return b;
-  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
-  if (any_misaligned({hidden, router_w, w_gate, w_up, w_down, out}) || !bias ||
-      (topk_idx && !aligned16(topk_idx)) || (topk_w && !aligned16(topk_w)))
-    return BEAM_ERR_INVALID_ARG;
-  const Layout L = plan(*shape);
-  if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
-  DeviceInfo* dev;
-  if ((b = device_info(&dev)) != BEAM_OK) return b;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
-  float* w = topk_w ? topk_w : at<float>(ws, L.w);
-  const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(hidden);
-  if ((b = run_router(*shape, L, h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
-    return b;
-  if ((b = run_experts(*shape, L, *dev, h, idx, w_gate, w_up, w_down, ws, st)) != BEAM_OK)
-    return b;
-  CombineArgs ca{};
-  ca.y = at<__nv_bfloat16>(ws, L.y);
-  ca.rowmap = at<int32_t>(ws, L.rowmap);
-  ca.w = w;
-  ca.out = static_cast<__nv_bfloat16*>(out);
-  ca.status = at<uint32_t>(ws, L.status);
-  ca.T = shape->T;
-  ca.d = shape->d;
-  ca.k = shape->top_k;
-  ca.R = static_cast<int>(L.R);
-  BEAM_LAUNCH(kKCombine, st, launch_combine(ca, st));
-  return BEAM_OK;
-}
 
 size_t beam_moe_fp8_workspace_size(const beam_moe_shape* shape) {
   if (check_shape(shape) != BEAM_OK) return 0;
@@ -692,44 +872,25 @@ beam_status beam_moe_quantize_e4m3(const void* x, int64_t rows, int32_t cols, vo
   return BEAM_OK;
 }
 
+
+
+beam_status beam_moe_forward(const beam_moe_shape* shape, const void* hidden, const float* router_w,
+                             const float* bias, const void* w_gate, const void* w_up,
+                             const void* w_down, void* out, int32_t* topk_idx, float* topk_w,
+                             void* ws, size_t ws_bytes, beam_stream stream) {
+  return forward_impl(shape, hidden, router_w, bias, w_gate, w_up, w_down, out, topk_idx, topk_w,
+                      ws, ws_bytes, stream, nullptr);
+}
+
 beam_status beam_moe_forward_fp8(const beam_moe_shape* shape, const void* hidden,
                                  const float* router_w, const float* bias, const void* w_gate,
                                  const float* gate_scale, const void* w_up, const float* up_scale,
                                  const void* w_down, const float* down_scale, void* out,
                                  int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
                                  beam_stream stream) {
-  beam_status b = check_shape(shape);
-  if (b != BEAM_OK) return b;
-  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
-  if (any_misaligned({hidden, router_w, w_gate, w_up, w_down, out, gate_scale, up_scale,
-                      down_scale}) ||
-      !bias || (topk_idx && !aligned16(topk_idx)) || (topk_w && !aligned16(topk_w)))
-    return BEAM_ERR_INVALID_ARG;
-  const Layout L = plan_fp8(*shape);
-  if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
-  DeviceInfo* dev;
-  if ((b = device_info(&dev)) != BEAM_OK) return b;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
-  float* w = topk_w ? topk_w : at<float>(ws, L.w);
-  const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(hidden);
-  if ((b = run_router(*shape, L, h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
-    return b;
   const Fp8Scales f8{gate_scale, up_scale, down_scale};
-  b = run_experts(*shape, L, *dev, h, idx, w_gate, w_up, w_down, ws, st, &f8);
-  if (b != BEAM_OK) return b;
-  CombineArgs ca{};
-  ca.y = at<__nv_bfloat16>(ws, L.y);
-  ca.rowmap = at<int32_t>(ws, L.rowmap);
-  ca.w = w;
-  ca.out = static_cast<__nv_bfloat16*>(out);
-  ca.status = at<uint32_t>(ws, L.status);
-  ca.T = shape->T;
-  ca.d = shape->d;
-  ca.k = shape->top_k;
-  ca.R = static_cast<int>(L.R);
-  BEAM_LAUNCH(kKCombine, st, launch_combine(ca, st));
-  return BEAM_OK;
+  return forward_impl(shape, hidden, router_w, bias, w_gate, w_up, w_down, out, topk_idx, topk_w,
+                      ws, ws_bytes, stream, &f8);
 }
 
 beam_status beam_moe_block(const beam_moe_shape* shape, const float* x, const float* g_pre,
@@ -737,58 +898,40 @@ beam_status beam_moe_block(const beam_moe_shape* shape, const float* x, const fl
                            const float* bias, const void* w_gate, const void* w_up,
                            const void* w_down, float* x_out, int32_t* topk_idx, float* topk_w,
                            void* ws, size_t ws_bytes, beam_stream stream) {
-  beam_status b = check_shape(shape);
-  if (b != BEAM_OK) return b;
-  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
-  if (any_misaligned({x, g_pre, g_post, router_w, w_gate, w_up, w_down, x_out}) || !bias ||
-      (topk_idx && !aligned16(topk_idx)) || (topk_w && !aligned16(topk_w)))
-    return BEAM_ERR_INVALID_ARG;
-  if (!(eps > 0.f) || !std::isfinite(eps) || k_resid < 1) return BEAM_ERR_INVALID_ARG;
-  if (x_out != x) {  // in place or disjoint
-    const char* a0 = reinterpret_cast<const char*>(x);
-    const char* b0 = reinterpret_cast<const char*>(x_out);
-    const size_t n = sizeof(float) * static_cast<size_t>(shape->T) * shape->d;
-    if (a0 < b0 + n && b0 < a0 + n) return BEAM_ERR_INVALID_ARG;
-  }
-  const Layout L = plan(*shape);
-  if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
-  DeviceInfo* dev;
-  if ((b = device_info(&dev)) != BEAM_OK) return b;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return block_impl(shape, x, g_pre, g_post, eps, k_resid, router_w, bias, w_gate, w_up, w_down,
+                    x_out, topk_idx, topk_w, ws, ws_bytes, stream, nullptr);
+}
 
-  PreNormArgs pn{};
-  pn.x = x;
-  pn.g_pre = g_pre;
-  pn.h = at<__nv_bfloat16>(ws, L.h);
-  pn.eps = eps;
-  pn.T = shape->T;
-  pn.d = shape->d;
-  BEAM_LAUNCH(kKPreNorm, st, launch_prenorm(pn, st));
+beam_status beam_moe_block_fp8(const beam_moe_shape* shape, const float* x, const float* g_pre,
+                               const float* g_post, float eps, int32_t k_resid,
+                               const float* router_w, const float* bias, const void* w_gate,
+                               const float* gate_scale, const void* w_up, const float* up_scale,
+                               const void* w_down, const float* down_scale, float* x_out,
+                               int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                               beam_stream stream) {
+  const Fp8Scales f8{gate_scale, up_scale, down_scale};
+  return block_impl(shape, x, g_pre, g_post, eps, k_resid, router_w, bias, w_gate, w_up, w_down,
+                    x_out, topk_idx, topk_w, ws, ws_bytes, stream, &f8);
+}
 
-  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
-  float* w = topk_w ? topk_w : at<float>(ws, L.w);
-  if ((b = run_router(*shape, L, pn.h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
-    return b;
-  if ((b = run_experts(*shape, L, *dev, pn.h, idx, w_gate, w_up, w_down, ws, st)) != BEAM_OK)
-    return b;
-  const double kk = static_cast<double>(k_resid);
-  CombineArgs ca{};
-  ca.y = at<__nv_bfloat16>(ws, L.y);
-  ca.rowmap = at<int32_t>(ws, L.rowmap);
-  ca.w = w;
-  ca.x = x;
-  ca.g_post = g_post;
-  ca.x_out = x_out;
-  ca.eps = eps;
-  ca.coef_x = static_cast<float>(std::sqrt((kk - 1.0) / kk));
-  ca.coef_f = static_cast<float>(1.0 / std::sqrt(kk));
-  ca.status = at<uint32_t>(ws, L.status);
-  ca.T = shape->T;
-  ca.d = shape->d;
-  ca.k = shape->top_k;
-  ca.R = static_cast<int>(L.R);
-  BEAM_LAUNCH(kKCombineBlock, st, launch_combine_block(ca, st));
-  return BEAM_OK;
+beam_status beam_dense_forward(const beam_dense_shape* shape, const void* hidden,
+                               const void* w_gate, const void* w_up, const void* w_down,
+                               void* out, void* ws, size_t ws_bytes, beam_stream stream) {
+  return dense_impl(shape, hidden, w_gate, w_up, w_down, out, ws, ws_bytes, stream, nullptr);
+}
+
+size_t beam_dense_fp8_workspace_size(const beam_dense_shape* shape) {
+  if (check_dense_shape(shape) != BEAM_OK) return 0;
+  return plan_dense_fp8(*shape).total;
+}
+
+beam_status beam_dense_forward_fp8(const beam_dense_shape* shape, const void* hidden,
+                                   const void* w_gate, const float* gate_scale, const void* w_up,
+                                   const float* up_scale, const void* w_down,
+                                   const float* down_scale, void* out, void* ws, size_t ws_bytes,
+                                   beam_stream stream) {
+  const Fp8Scales f8{gate_scale, up_scale, down_scale};
+  return dense_impl(shape, hidden, w_gate, w_up, w_down, out, ws, ws_bytes, stream, &f8);
 }
 
 size_t beam_dense_workspace_size(const beam_dense_shape* shape) {
@@ -796,63 +939,6 @@ size_t beam_dense_workspace_size(const beam_dense_shape* shape) {
   return plan_dense(*shape).total;
 }
 
-beam_status beam_dense_forward(const beam_dense_shape* shape, const void* hidden,
-                               const void* w_gate, const void* w_up, const void* w_down,
-                               void* out, void* ws, size_t ws_bytes, beam_stream stream) {
-  beam_status b = check_dense_shape(shape);
-  if (b != BEAM_OK) return b;
-  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
-  if (any_misaligned({hidden, w_gate, w_up, w_down, out})) return BEAM_ERR_INVALID_ARG;
-  const DenseLayout L = plan_dense(*shape);
-  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < L.total)
-    return BEAM_ERR_WORKSPACE;
-  DeviceInfo* dev;
-  if ((b = device_info(&dev)) != BEAM_OK) return b;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const beam_dense_shape& s = *shape;
-  uint32_t* status = at<uint32_t>(ws, L.status);
-  cudaError_t e = cudaMemsetAsync(status, 0, 16, st);
-  if (e != cudaSuccess) return cuda_fail(e);
-  MTile* mtiles = at<MTile>(ws, L.mtiles);
-  int32_t* mt_count = at<int32_t>(ws, L.mt_count);
-  BEAM_LAUNCH(kKDenseTiles, st, launch_dense_tiles(s.T, mtiles, mt_count, st));
-
-  ATensorMaps tm_h, tm_act;
-  CUtensorMap tm_g, tm_u, tm_d;
-  void* act = at<void>(ws, L.act);
-  for (int i = 0; i < kNumABoxes; ++i) {
-    if ((b = make_map(&tm_h.m[i], hidden, s.d, s.T, a_box_rows(i))) != BEAM_OK) return b;
-    if ((b = make_map(&tm_act.m[i], act, s.I, s.T, a_box_rows(i))) != BEAM_OK) return b;
-  }
-  if ((b = make_map(&tm_g, w_gate, s.d, s.I, kN1Half)) != BEAM_OK) return b;
-  if ((b = make_map(&tm_u, w_up, s.d, s.I, kN1Half)) != BEAM_OK) return b;
-  if ((b = make_map(&tm_d, w_down, s.I, s.d, kN2)) != BEAM_OK) return b;
-
-  GemmArgs g1{};
-  g1.mtiles = mtiles;
-  g1.mt_count = mt_count;
-  g1.out = static_cast<__nv_bfloat16*>(act);
-  g1.status = status;
-  g1.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
-  g1.out_ld = s.I;
-  g1.n_tiles_n = s.I / kN1Half;
-  g1.k_blocks = s.d / kBK;
-  g1.b_rows_per_expert = s.I;
-  g1.swap_max_rows = 0;
-  const int64_t t1 = L.mt_cap * g1.n_tiles_n;
-  BEAM_LAUNCH(kKGemmGateUp, st,
-              launch_gemm_gate_up(tm_h, tm_g, tm_u, g1, static_cast<int>(t1 < dev->sms ? t1 : dev->sms), st));
-  GemmArgs g2 = g1;
-  g2.out = static_cast<__nv_bfloat16*>(out);
-  g2.out_ld = s.d;
-  g2.n_tiles_n = s.d / kN2;
-  g2.k_blocks = s.I / kBK;
-  g2.b_rows_per_expert = s.d;
-  const int64_t t2 = L.mt_cap * g2.n_tiles_n;
-  BEAM_LAUNCH(kKGemmDown, st,
-              launch_gemm_down(tm_act, tm_d, g2, static_cast<int>(t2 < dev->sms ? t2 : dev->sms), st));
-  return BEAM_OK;
-}
 
 beam_status beam_moe_bias_update(const beam_moe_shape* shape, const void* ws, float* bias,
                                  float gamma, beam_stream stream) {

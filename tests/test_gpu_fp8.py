@@ -176,3 +176,51 @@ def test_forward_fp8_wait_timeout_is_reported_and_context_survives():
     toks = list(range(0, case.wl.T, 37))
     ref = H.oracle_out_fp8(case, weights, toks, fp8, batch=64)
     H.assert_close_out(out2[toks].float().cpu().numpy(), ref, "fp8 after timeout")
+
+
+def test_block_fp8_every_token():
+    import dataclasses
+    wl = dataclasses.replace(W.WORKLOADS["tiny"], block=True, T=96)
+    case = H.make_case(wl)
+    weights = H.device_weights(wl)
+    fp8 = H.device_weights_fp8(weights)
+    s = bm.shape_of(wl)
+    dev = "cuda"
+    x = case.x.to(dev)
+    x_out = torch.empty_like(x)
+    idx = torch.empty(wl.T, wl.top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(wl.T, wl.top_k, dtype=torch.float32, device=dev)
+    ws = bm.beam_moe_block_fp8(s, x, case.g_pre.to(dev), case.g_post.to(dev), wl.eps, wl.k_resid,
+                               case.router_w.to(dev), case.bias.to(dev), *fp8, x_out, idx, w)
+    assert bm.beam_moe_sync_status(ws) == bm.BEAM_OK
+    _check_routing(case, idx, w)
+    moe = H.oracle_out_fp8(case, weights, range(wl.T), fp8, batch=96)
+    ref = oracle.block_tail(case.x, moe, case.g_post, wl.eps, wl.k_resid)
+    cx, cf = oracle.residual_coefficients(wl.k_resid)
+    got = x_out.cpu().numpy()
+    # the residual term dominates x'; compare the MoE contribution
+    H.assert_close_out((got - cx * case.x.numpy()) / cf, (ref - cx * case.x.numpy()) / cf,
+                       "fp8 block")
+
+
+@pytest.mark.parametrize("T,d,I", [(200, 256, 1024), (1, 512, 384), (129, 5120, 20480)])
+def test_dense_fp8_every_token(T, d, I):
+    import dataclasses
+    wl = dataclasses.replace(W.WORKLOADS["dense"], T=T, d=d, I=I)
+    h = W.hidden(wl)
+    mats = tuple(W.expert_weight(wl, m, 0, "cuda") for m in ("gate", "up", "down"))
+    q = []
+    for m in mats:
+        q += list(bm.beam_moe_quantize_e4m3(m))
+    out = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    s = bm.dense_shape(T, d, I)
+    bm.beam_dense_forward_fp8(s, h.cuda(), *q, out)
+    torch.cuda.synchronize()
+    ref_q = []
+    for i, m in enumerate(mats):
+        rq, rs = oracle.quantize_rows_e4m3(m.cpu())
+        assert np.array_equal(q[2 * i].cpu().numpy(), rq) and np.array_equal(q[2 * i + 1].cpu().numpy(), rs)
+        ref_q += [rq, rs]
+    toks = list(range(T)) if T <= 200 else sorted({0, T - 1, 1, T // 2, T // 3, 2 * T // 3})
+    ref = np.stack([oracle.expert_mlp_fp8(h[t], *ref_q) for t in toks])
+    H.assert_close_out(out[toks].float().cpu().numpy(), ref, f"fp8 dense T={T} d={d} I={I}")
