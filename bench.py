@@ -648,11 +648,17 @@ def run_reference(args, rank, world, local):
         ex = sorted({int(e) for e in idx.reshape(-1)})
         experts = {e: tuple(W.expert_weight(wl, m, e, dev).cpu() for m in ("gate", "up", "down"))
                    for e in ex}
+        if args.fp8:  # the oracle converts the experts itself (a one-off, not timed)
+            experts = {e: tuple(p for m in mats for p in oracle.quantize_rows_e4m3(m))
+                       for e, mats in experts.items()}
         return sample, experts
 
     def one_step(n, sample, experts):
         _, ix, ww, _, _ = oracle.layer_routing(h[:n], router_w, bias, sample)
-        oracle.moe_tokens(np.arange(n), h[:n], ix, ww, experts)
+        if args.fp8:
+            oracle.moe_tokens_fp8(np.arange(n), h[:n], ix, ww, experts)
+        else:
+            oracle.moe_tokens(np.arange(n), h[:n], ix, ww, experts)
 
     sample1, experts1 = prepare(1)
     t0 = time.perf_counter()
@@ -670,10 +676,12 @@ def run_reference(args, rank, world, local):
     dt = time.perf_counter() - t0
     value = n * args.steps / dt
     cores = oracle.hardware_threads()
-    desc = (f"first {n} tokens of the {wl.name} workload per step, full layer (router logits, "
-            f"routing, {wl.top_k} SwiGLU experts per token, combine) in double-accumulating C++ "
-            f"on {cores} host threads")
-    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+    kind = "E4M3 " if args.fp8 else ""
+    desc = (f"first {n} tokens of the {wl.name} workload per step, full {kind}layer (router "
+            f"logits, routing, {wl.top_k} {kind}SwiGLU experts per token, combine) in "
+            f"double-accumulating C++ on {cores} host threads")
+    return {"impl": "reference", "metric": METRIC_FP8 if args.fp8 else METRIC, "value": value,
+            "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
