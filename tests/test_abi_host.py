@@ -169,3 +169,36 @@ def test_fp8_entry_points_validate_before_launching(L):
     misaligned[5] = q(A + 4)  # up_scale
     assert fwd(ctypes.byref(beam(64)), *misaligned, 1 << 30, None) == bm.BEAM_ERR_INVALID_ARG
     assert fwd(ctypes.byref(beam(64)), *args[:12], None, 16, None) == bm.BEAM_ERR_WORKSPACE
+
+
+def test_fp8_block_and_dense_validate_before_launching(L):
+    A = 1 << 20
+    q = ctypes.c_void_p
+    s = beam(64)
+    blk = L.beam_moe_block_fp8
+    base = [q(A)] * 3 + [ctypes.c_float(1e-6), ctypes.c_int32(10)] + [q(A)] * 12
+    assert blk(ctypes.byref(beam(0)), *[None] * 3, ctypes.c_float(1e-6), ctypes.c_int32(10),
+               *[None] * 12, 0, None) == bm.BEAM_OK
+    bad_eps = list(base)
+    bad_eps[3] = ctypes.c_float(0.0)
+    assert blk(ctypes.byref(s), *bad_eps, 1 << 30, None) == bm.BEAM_ERR_INVALID_ARG
+    mis = list(base)
+    mis[8] = q(A + 8)  # gate_scale
+    assert blk(ctypes.byref(s), *mis, 1 << 30, None) == bm.BEAM_ERR_INVALID_ARG
+    # x_out overlapping x without being x
+    ov = list(base)
+    ov[13] = q(A + 64)
+    assert blk(ctypes.byref(s), *ov, 1 << 30, None) == bm.BEAM_ERR_INVALID_ARG
+    assert blk(ctypes.byref(s), *base[:16], None, 16, None) == bm.BEAM_ERR_WORKSPACE
+
+    ds = bm.dense_shape(256, 5120, 20480)
+    assert bm.lib().beam_dense_fp8_workspace_size(ctypes.byref(ds)) > \
+        bm.lib().beam_dense_workspace_size(ctypes.byref(ds)) + 256 * (5120 + 20480)
+    assert bm.lib().beam_dense_fp8_workspace_size(ctypes.byref(bm.dense_shape(4, 100, 128))) == 0
+    dns = L.beam_dense_forward_fp8
+    args = [q(A)] * 8  # hidden, w_gate, gate_scale, w_up, up_scale, w_down, down_scale, out
+    mis = list(args)
+    mis[4] = q(A + 4)  # up_scale
+    assert dns(ctypes.byref(ds), *mis, q(A), 1 << 30, None) == bm.BEAM_ERR_INVALID_ARG
+    assert dns(ctypes.byref(ds), *args, None, 16, None) == bm.BEAM_ERR_WORKSPACE
+    assert dns(ctypes.byref(bm.dense_shape(0, 5120, 20480)), *[None] * 9, 0, None) == bm.BEAM_OK
