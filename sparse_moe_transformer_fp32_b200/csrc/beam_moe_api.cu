@@ -136,9 +136,10 @@ struct Layout {
 
 // Router split-K factor S from a simple cost model: the FFMA time of the waves of
 // (token tile, expert tile, K chunk) blocks over the resident router blocks of a 148-SM B200,
-// plus the traffic of writing and re-reading S partial logit arrays.  K chunks are a multiple
-// of the router's K step.
-int router_split(const beam_moe_shape& s) {
+// plus the traffic of writing and re-reading S partial logit arrays and the selection kernel's
+// latency of adding them (one round of loads per four splits).  K chunks are a multiple of the
+// router's K step; at most max_s splits.
+int router_split(const beam_moe_shape& s, int max_s) {
   const int64_t tiles = ceil_div(s.T, kRM) * ceil_div(s.E, kRN);
   const int64_t kblocks = s.d / kRK;
   const double block_flops_per_k = 2.0 * kRM * kRN;
@@ -146,13 +147,14 @@ int router_split(const beam_moe_shape& s) {
   const double hbm = 6.5e12;
   int best = 1;
   double best_t = 1e30;
-  for (int S = 1; S <= 16 && S <= kblocks; ++S) {
+  for (int S = 1; S <= max_s && S <= kblocks; ++S) {
     const int64_t per = ceil_div(kblocks, S);
     const int64_t Sx = ceil_div(kblocks, per);
     if (Sx != S) continue;
     const double waves = static_cast<double>(ceil_div(tiles * S, kRouterSlots));
     const double t = waves * per * kRK * block_flops_per_k / slot_rate +
-                     static_cast<double>(S) * s.T * s.E * 8.0 / hbm;
+                     static_cast<double>(S) * s.T * s.E * 8.0 / hbm +
+                     static_cast<double>(ceil_div(S, 4)) * 0.8e-6;
     if (t < best_t * 0.97) {  // a larger split must win clearly
       best_t = t;
       best = S;
@@ -166,7 +168,7 @@ Layout plan(const beam_moe_shape& s) {
   const int64_t T = s.T, R = T * s.top_k;
   L.R = R;
   const int64_t kblocks = s.d / kRK;
-  const int S = router_split(s);
+  const int S = router_split(s, 64);
   L.kchunk = static_cast<int>(ceil_div(kblocks, S) * kRK);
   L.S = static_cast<int>(ceil_div(s.d, L.kchunk));
   L.mt_cap = ceil_div(R, kBM) + s.E;
@@ -487,7 +489,7 @@ Layout plan_route_static(const beam_moe_shape& s) {
   Layout L{};
   L.R = static_cast<int64_t>(s.T) * s.top_k;
   const int64_t kblocks = s.d / kRK;
-  const int S = router_split(s);
+  const int S = router_split(s, 16);  // the static scratch holds 16 partial arrays
   L.kchunk = static_cast<int>(ceil_div(kblocks, S) * kRK);
   L.S = static_cast<int>(ceil_div(s.d, L.kchunk));
   size_t o = 0;
