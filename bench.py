@@ -307,9 +307,10 @@ def traffic_from_profile(kernel: str, workload: str):
 
 # ------------------------------------------------------------------ oracle (CPU) timing
 
-def oracle_sample_rate(wl, router_w, bias, hidden_cpu, weights_dev, n_tokens: int, repeats=1):
+def oracle_sample_rate(wl, router_w, bias, hidden_cpu, weights_dev, n_tokens: int, repeats=1,
+                       nthreads: int = 0):
     """Tokens/s of the CPU oracle on the first n tokens (full layer: logits, routing, experts,
-    combine), expert weights copied from the device (not timed)."""
+    combine), expert weights copied from the device (not timed); nthreads 0 = all cores."""
     import numpy as np
     import oracle
     oracle.build()
@@ -320,10 +321,10 @@ def oracle_sample_rate(wl, router_w, bias, hidden_cpu, weights_dev, n_tokens: in
     experts = {e: tuple(m[e].cpu() for m in weights_dev) for e in ex}
     t0 = time.perf_counter()
     for _ in range(repeats):
-        _, idx, w, _, _ = oracle.layer_routing(h, router_w, bias, sample)
-        oracle.moe_tokens(np.arange(n_tokens), h, idx, w, experts)
+        _, idx, w, _, _ = oracle.layer_routing(h, router_w, bias, sample, nthreads=nthreads)
+        oracle.moe_tokens(np.arange(n_tokens), h, idx, w, experts, nthreads=nthreads)
     dt = time.perf_counter() - t0
-    return n_tokens * repeats / dt, dt, oracle.hardware_threads()
+    return n_tokens * repeats / dt, dt, nthreads or oracle.hardware_threads()
 
 
 def oracle_fp8_sample_rate(wl, router_w, bias, hidden_cpu, weights_dev, n_tokens: int):
@@ -555,6 +556,7 @@ def run_cuda(args, rank, world, local):
             flops_step = 6 * wl.T * wl.top_k * wl.d * wl.I  # top_k = 1 for the dense MLP
             bytes_step = layer_min_bytes(wl, touched, fp8=bool(fp8))
             cpu = None
+            result_extra = {}
             if fp8 and (wl.dense or wl.block):
                 pass  # the E4M3 CPU baseline is timed on the layer workloads only
             elif not args.no_cpu_baseline and world == 1 and fp8:
@@ -579,6 +581,14 @@ def run_cuda(args, rank, world, local):
                        "sample": f"first {args.cpu_sample_tokens} tokens of the {wl.name} workload, "
                                  f"full layer (router logits, routing, {wl.top_k} SwiGLU experts "
                                  f"each, combine) in double-accumulating C++; {secs:.2f} s"}
+                if wl.name in ("tiny", "decode"):  # the small configurations also on one core
+                    n1 = min(args.cpu_sample_tokens, wl.T)
+                    rate1, secs1, _ = oracle_sample_rate(
+                        wl, W.router_weight(wl), W.router_bias(wl), inp_cpu, weights, n1,
+                        nthreads=1)
+                    result_extra["cpu_baseline_1core"] = {
+                        "value": rate1, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                        "sample": f"first {n1} tokens, one host thread; {secs1:.2f} s"}
             result = {
                 "metric": METRIC_FP8 if fp8 else METRIC, "value": value, "unit": "tokens/s",
                 "n_gpus": world,
@@ -608,6 +618,7 @@ def run_cuda(args, rank, world, local):
                 "clocks": clocks.summary(),
                 "e2e": e2e,
                 "cpu_baseline": cpu,
+                **result_extra,
             }
         barrier(dist, dev)
         del weights, fp8
