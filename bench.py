@@ -314,6 +314,7 @@ def oracle_sample_rate(wl, router_w, bias, hidden_cpu, weights_dev, n_tokens: in
     import numpy as np
     import oracle
     oracle.build()
+    n_tokens = min(n_tokens, wl.T)
     h = hidden_cpu[:n_tokens]
     sample = wl.with_tokens(n_tokens)
     _, idx, w, _, _ = oracle.layer_routing(h, router_w, bias, sample)
@@ -333,6 +334,7 @@ def oracle_fp8_sample_rate(wl, router_w, bias, hidden_cpu, weights_dev, n_tokens
     import numpy as np
     import oracle
     oracle.build()
+    n_tokens = min(n_tokens, wl.T)
     h = hidden_cpu[:n_tokens]
     sample = wl.with_tokens(n_tokens)
     _, idx, w, _, _ = oracle.layer_routing(h, router_w, bias, sample)
@@ -578,7 +580,8 @@ def run_cuda(args, rank, world, local):
                     inp_cpu if not wl.block else _block_h(wl, mine, g_pre), weights,
                     args.cpu_sample_tokens)
                 cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                       "sample": f"first {args.cpu_sample_tokens} tokens of the {wl.name} workload, "
+                       "sample": f"first {min(args.cpu_sample_tokens, wl.T)} tokens of the "
+                                 f"{wl.name} workload, "
                                  f"full layer (router logits, routing, {wl.top_k} SwiGLU experts "
                                  f"each, combine) in double-accumulating C++; {secs:.2f} s"}
                 if wl.name in ("tiny", "decode"):  # the small configurations also on one core

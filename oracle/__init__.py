@@ -92,6 +92,12 @@ def _np(x, dtype):
     return x
 
 
+def _check_tokens(tokens: np.ndarray, n: int) -> None:
+    """Token ids index rows of h, idx and w: they must lie in [0, n)."""
+    if tokens.size and (tokens.min() < 0 or tokens.max() >= n):
+        raise ValueError(f"token ids must lie in [0, {n}); got {tokens.min()}..{tokens.max()}")
+
+
 def _p(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
@@ -174,6 +180,7 @@ def moe_tokens(tokens, h, idx, w, experts, nthreads: int = 0) -> np.ndarray:
     ix = _np(idx, np.int32)
     ww = _np(w, np.float32)
     T, d = hb.shape
+    _check_tokens(tok, min(T, ix.shape[0], ww.shape[0]))
     k = ix.shape[1]
     E = int(max(experts.keys())) + 1 if experts else 1
     E = max(E, int(ix.max()) + 1)
@@ -319,6 +326,7 @@ def moe_tokens_fp8(tokens, h, idx, w, experts, nthreads: int = 0) -> np.ndarray:
     T, d = hb.shape
     idx = _np(idx, np.int32)
     w = _np(w, np.float32)
+    _check_tokens(tokens, min(T, idx.shape[0], w.shape[0]))
     k = idx.shape[1]
     E = int(idx.max()) + 1 if idx.size else 0
     E = max([E] + [int(e) + 1 for e in experts])
