@@ -241,9 +241,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, letting the hardware park the thread until the phase completes or about
+// hint_ns nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of parity `parity` of barrier `bar` to complete.  Gives up when the
 // CTA-wide abort flag is raised, or after limit_ns, in which case it raises the flag and
 // records a timeout.  A limit of 0 gives up at the first check that finds the phase open.
+// After a few polls the thread is parked by the hardware between checks (suspend hint), so
+// long waits -- the epilogue's for a whole K loop -- issue few instructions.
 // Returns true when the phase completed.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int* abort_flag, uint64_t limit_ns,
@@ -255,7 +271,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   const uint64_t t0 = globaltimer_ns();
 #pragma unroll 1
   for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_hint(bar, parity, 1000u)) return true;
     if ((it & 7u) == 0u) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
