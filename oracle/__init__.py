@@ -66,6 +66,13 @@ def lib():
         L.oracle_moe_tokens_fp8.argtypes = [i64, vp, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp,
                                             vp, vp, vp, i32]
         L.oracle_moe_tokens_fp8.restype = i32
+        L.oracle_f32_to_e2m1.argtypes = [i64, vp, vp]
+        L.oracle_e2m1_to_f32.argtypes = [i64, vp, vp]
+        L.oracle_quantize_rows_nvfp4.argtypes = [i64, i64, vp, vp, vp, vp, i32]
+        L.oracle_linear_nvfp4.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, i32]
+        L.oracle_expert_mlp_nvfp4.argtypes = [i64, i64] + [vp] * 12
+        L.oracle_moe_tokens_nvfp4.argtypes = [i64, vp, i64, i64, i32, vp, vp, vp] + [vp] * 10 + [i32]
+        L.oracle_moe_tokens_nvfp4.restype = i32
         _lib = L
     return _lib
 
@@ -346,4 +353,95 @@ def moe_tokens_fp8(tokens, h, idx, w, experts, nthreads: int = 0) -> np.ndarray:
                                     nthreads)
     if r != 0:
         raise ValueError("moe_tokens_fp8: a token uses an expert that was not supplied")
+    return out
+
+
+# ------------------------------------------------------------------ NVFP4 expert weights
+
+def f32_to_e2m1(x) -> np.ndarray:
+    """E2M1 codes (uint8, low 4 bits) of FP32 values: round to nearest even, saturate to +-6."""
+    a = np.ascontiguousarray(_np(x, np.float32))
+    out = np.empty(a.shape, np.uint8)
+    lib().oracle_f32_to_e2m1(a.size, _p(a), _p(out))
+    return out
+
+
+def e2m1_to_f32(codes) -> np.ndarray:
+    c = np.ascontiguousarray(np.asarray(codes, np.uint8))
+    out = np.empty(c.shape, np.float32)
+    lib().oracle_e2m1_to_f32(c.size, _p(c), _p(out))
+    return out
+
+
+def quantize_rows_nvfp4(x, nthreads: int = 0):
+    """NVFP4 quantisation of a BF16 matrix [rows, cols] (cols a multiple of 16) ->
+    (codes uint8 [rows, cols], E4M3 block scales uint8 [rows, cols / 16], row scales f32)."""
+    b = np.ascontiguousarray(bf16_bits(x))
+    rows, cols = b.shape
+    if cols % 16:
+        raise ValueError("quantize_rows_nvfp4: cols must be a multiple of 16")
+    q = np.empty((rows, cols), np.uint8)
+    bs = np.empty((rows, cols // 16), np.uint8)
+    s = np.empty(rows, np.float32)
+    lib().oracle_quantize_rows_nvfp4(rows, cols, _p(b), _p(q), _p(bs), _p(s), nthreads)
+    return q, bs, s
+
+
+def linear_nvfp4(xq, xbs, sx, wq, wbs, sw, nthreads: int = 0) -> np.ndarray:
+    """y[r, c] = fl32(sx_r * sw_c * sum_b xbs[r, b] wbs[c, b] sum_{j in b} xq[r, j] wq[c, j])
+    on decoded codes (blocks of 16 along K)."""
+    xq, wq, xbs, wbs = (np.ascontiguousarray(np.asarray(a, np.uint8)) for a in (xq, wq, xbs, wbs))
+    sx = np.ascontiguousarray(np.asarray(sx, np.float32))
+    sw = np.ascontiguousarray(np.asarray(sw, np.float32))
+    rows, K = xq.shape
+    n_out = wq.shape[0]
+    y = np.empty((rows, n_out), np.float32)
+    lib().oracle_linear_nvfp4(rows, n_out, K, _p(xq), _p(xbs), _p(sx), _p(wq), _p(wbs), _p(sw),
+                              _p(y), nthreads)
+    return y
+
+
+_NVFP4_PARTS = (np.uint8, np.uint8, np.float32) * 3
+
+
+def expert_mlp_nvfp4(x, gate, up, down, return_act: bool = False):
+    """One NVFP4 SwiGLU expert on one BF16 row x [d]; gate, up, down are each
+    (codes, block scales, row scales) as returned by quantize_rows_nvfp4."""
+    xb = np.ascontiguousarray(bf16_bits(x).reshape(-1))
+    d = xb.size
+    I = gate[0].shape[0]
+    arrs = [_np(a, t) for a, t in zip((*gate, *up, *down), _NVFP4_PARTS)]
+    y = np.empty(d, np.float32)
+    a = np.empty(I, np.uint16)
+    lib().oracle_expert_mlp_nvfp4(d, I, _p(xb), *[_p(v) for v in arrs], _p(y), _p(a))
+    return (y, a) if return_act else y
+
+
+def moe_tokens_nvfp4(tokens, h, idx, w, experts, nthreads: int = 0) -> np.ndarray:
+    """MoE output rows for `tokens` with NVFP4 experts; experts maps e -> (gate, up, down), each
+    (codes, block scales, row scales) as returned by quantize_rows_nvfp4."""
+    tokens = np.ascontiguousarray(np.asarray(tokens, np.int64))
+    hb = np.ascontiguousarray(bf16_bits(h))
+    T, d = hb.shape
+    idx = _np(idx, np.int32)
+    w = _np(w, np.float32)
+    _check_tokens(tokens, min(T, idx.shape[0], w.shape[0]))
+    k = idx.shape[1]
+    E = int(idx.max()) + 1 if idx.size else 0
+    E = max([E] + [int(e) + 1 for e in experts])
+    keep = []
+    ptrs = [(ctypes.c_void_p * E)() for _ in range(9)]
+    I = None
+    for e, (gate, up, down) in experts.items():
+        arrs = [_np(a, t) for a, t in zip((*gate, *up, *down), _NVFP4_PARTS)]
+        keep.append(arrs)
+        I = arrs[0].shape[0]
+        for i, a in enumerate(arrs):
+            ptrs[i][e] = a.ctypes.data
+    out = np.empty((tokens.size, d), np.float32)
+    r = lib().oracle_moe_tokens_nvfp4(tokens.size, _p(tokens), d, I, k, _p(hb), _p(idx), _p(w),
+                                      *[ctypes.cast(p, ctypes.c_void_p) for p in ptrs], _p(out),
+                                      nthreads)
+    if r != 0:
+        raise ValueError("moe_tokens_nvfp4: a token uses an expert that was not supplied")
     return out

@@ -37,6 +37,17 @@
 // GEMM input quantised that way; products of codes are exact and summed in double, and the
 // two row scales are applied before the single rounding to FP32.
 //
+// NVFP4 expert weights (a reading, from the same passages): E2M1 codes (1 sign, 2 exponent
+// bits with bias 1, 1 mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6, no infinities),
+// two scales per value: one E4M3 scale per block of 16 consecutive elements of a row and one
+// FP32 scale per row.  With amax the row's largest magnitude and m_b the block's:
+//   s = fl32(amax / 2688)                       (2688 = 6 * 448, the two formats' maxima)
+//   bs_b = e4m3( fl32( fl32(m_b / s) / 6 ) )    (nearest even, saturating)
+//   q_j = e2m1( fl32( x_j / fl32(s * value(bs_b)) ) )   (nearest even, saturating to +-6)
+// and a block whose scale is zero (or a row with s = 0) gets zero codes.  The value of an
+// element is value(q_j) * value(bs_b) * s; a linear layer sums the exact products of codes and
+// block scales in double and applies the two row scales before the single rounding to FP32.
+//
 // Plain loops, no BLAS, no intrinsics; std::thread over tokens.
 
 #include <algorithm>
@@ -151,6 +162,76 @@ void linear_fp8_row(int64_t K, int64_t n_out, const uint8_t* xq, float sx, const
     const uint8_t* w = Wq + c * K;
     double acc = 0.0;
     for (int64_t j = 0; j < K; ++j) acc += xv[j] * value[w[j]];
+    y[c] = static_cast<float>(static_cast<double>(sx) * static_cast<double>(sw[c]) * acc);
+  }
+}
+
+// E2M1 code -> value.  Bit 3 is the sign; exponent field e = bits 2..1, mantissa bit 0:
+// e = 0 gives m * 0.5 (0 or 0.5), e > 0 gives 2^(e-1) * (1 + m/2).
+double e2m1_value(uint8_t c) {
+  const int e = (c >> 1) & 3, m = c & 1;
+  const double v = e == 0 ? 0.5 * m : std::ldexp(1.0 + 0.5 * m, e - 1);
+  return (c & 8) ? -v : v;
+}
+
+// Value -> E2M1 code, round to nearest with ties to the even code, saturating to +-6.  Inside
+// each binade the grid step is constant (0.5 below 2, 1 on [2, 4), 2 on [4, 6]), so the value
+// is rounded to a whole number of steps; an even step count is an even code.
+uint8_t e2m1_code(float f) {
+  const uint8_t sgn = std::signbit(f) ? 8 : 0;
+  const double a = std::fabs(static_cast<double>(f));
+  uint8_t mag;
+  if (a >= 6.0) {
+    mag = 7;
+  } else if (a < 2.0) {
+    mag = static_cast<uint8_t>(std::nearbyint(a / 0.5));  // 0..4 halves: codes 0..4
+  } else if (a < 4.0) {
+    mag = static_cast<uint8_t>(std::nearbyint(a) + 2.0);  // 2..4: codes 4..6
+  } else {
+    mag = static_cast<uint8_t>(std::nearbyint(a / 2.0) + 4.0);  // 2..3 (x2): codes 6..7
+  }
+  return static_cast<uint8_t>(sgn | mag);
+}
+
+// NVFP4 quantisation of one BF16 row of n values (n a multiple of 16): q [n] codes (one per
+// byte), bs [n / 16] E4M3 block-scale codes; returns the row scale s.
+float quantize_row_nvfp4(int64_t n, const uint16_t* x, uint8_t* q, uint8_t* bs) {
+  float amax = 0.0f;
+  for (int64_t j = 0; j < n; ++j) amax = std::max(amax, std::fabs(bf16_bits_to_float(x[j])));
+  const float s = amax / 2688.0f;
+  for (int64_t b = 0; b < n / 16; ++b) {
+    const uint16_t* xb = x + b * 16;
+    float mb = 0.0f;
+    for (int j = 0; j < 16; ++j) mb = std::max(mb, std::fabs(bf16_bits_to_float(xb[j])));
+    float t = 0.0f;
+    if (s > 0.0f) {
+      t = mb / s;
+      t = t / 6.0f;
+    }
+    bs[b] = s > 0.0f ? e4m3_code(t) : 0;
+    const float den = s * static_cast<float>(e4m3_value(bs[b]));
+    for (int j = 0; j < 16; ++j)
+      q[b * 16 + j] = den > 0.0f ? e2m1_code(bf16_bits_to_float(xb[j]) / den) : 0;
+  }
+  return s;
+}
+
+// y_c = fl32( sx * sw_c * sum_b value(xbs_b) value(Wbs[c, b]) sum_{j in b} value(xq_j)
+// value(Wq[c, j]) ) for c < n_out; Wq [n_out, K] codes, Wbs [n_out, K / 16] block scales.
+void linear_nvfp4_row(int64_t K, int64_t n_out, const uint8_t* xq, const uint8_t* xbs, float sx,
+                      const uint8_t* Wq, const uint8_t* Wbs, const float* sw, float* y) {
+  double v4[16];
+  for (int c = 0; c < 16; ++c) v4[c] = e2m1_value(static_cast<uint8_t>(c));
+  const int64_t nb = K / 16;
+  for (int64_t c = 0; c < n_out; ++c) {
+    const uint8_t* w = Wq + c * K;
+    const uint8_t* wb = Wbs + c * nb;
+    double acc = 0.0;
+    for (int64_t b = 0; b < nb; ++b) {
+      double part = 0.0;
+      for (int j = 0; j < 16; ++j) part += v4[xq[b * 16 + j] & 15] * v4[w[b * 16 + j] & 15];
+      acc += e4m3_value(xbs[b]) * e4m3_value(wb[b]) * part;
+    }
     y[c] = static_cast<float>(static_cast<double>(sx) * static_cast<double>(sw[c]) * acc);
   }
 }
@@ -398,6 +479,86 @@ int oracle_moe_tokens_fp8(int64_t ntok, const int64_t* tokens, int64_t d, int64_
     const int e = idx[t * k + j];
     oracle_expert_mlp_fp8(d, I, h + t * d, Wgq[e], sg[e], Wuq[e], su[e], Wdq[e], sd[e],
                           ys.data() + item * d, nullptr);
+  });
+  combine_slots(ntok, tokens, d, k, w, ys.data(), out);
+  return 0;
+}
+
+void oracle_f32_to_e2m1(int64_t n, const float* in, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e2m1_code(in[i]);
+}
+
+void oracle_e2m1_to_f32(int64_t n, const uint8_t* in, float* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = static_cast<float>(e2m1_value(in[i]));
+}
+
+// Row-wise NVFP4 quantisation of a BF16 matrix [rows, cols] (see quantize_row_nvfp4):
+// q [rows, cols] codes, bs [rows, cols / 16] block scales, scale [rows].
+void oracle_quantize_rows_nvfp4(int64_t rows, int64_t cols, const uint16_t* x, uint8_t* q,
+                                uint8_t* bs, float* scale, int nthreads) {
+  parallel_for(rows, nthreads, [&](int64_t r) {
+    scale[r] = quantize_row_nvfp4(cols, x + r * cols, q + r * cols, bs + r * (cols / 16));
+  });
+}
+
+// NVFP4 linear layer on quantised rows (see linear_nvfp4_row): xq [rows, K], xbs [rows, K/16],
+// sx [rows]; Wq [n_out, K], Wbs [n_out, K/16], sw [n_out]; y [rows, n_out].
+void oracle_linear_nvfp4(int64_t rows, int64_t n_out, int64_t K, const uint8_t* xq,
+                         const uint8_t* xbs, const float* sx, const uint8_t* Wq,
+                         const uint8_t* Wbs, const float* sw, float* y, int nthreads) {
+  parallel_for(rows, nthreads, [&](int64_t r) {
+    linear_nvfp4_row(K, n_out, xq + r * K, xbs + r * (K / 16), sx[r], Wq, Wbs, sw,
+                     y + r * n_out);
+  });
+}
+
+// One SwiGLU expert with NVFP4 weights on one BF16 input row, as oracle_expert_mlp_fp8 with
+// every quantisation in NVFP4: Wgq, Wuq [I, d] codes with block scales [I, d/16] and row
+// scales [I]; Wdq [d, I] with [d, I/16] and [d].  a_out [I] (BF16 bits before the activation's
+// quantisation) may be NULL.
+void oracle_expert_mlp_nvfp4(int64_t d, int64_t I, const uint16_t* x, const uint8_t* Wgq,
+                             const uint8_t* Wgb, const float* sg, const uint8_t* Wuq,
+                             const uint8_t* Wub, const float* su, const uint8_t* Wdq,
+                             const uint8_t* Wdb, const float* sd, float* y, uint16_t* a_out) {
+  std::vector<uint8_t> xq(d), xb(d / 16), aq(I), ab(I / 16);
+  const float sx = quantize_row_nvfp4(d, x, xq.data(), xb.data());
+  std::vector<float> g(I), u(I);
+  linear_nvfp4_row(d, I, xq.data(), xb.data(), sx, Wgq, Wgb, sg, g.data());
+  linear_nvfp4_row(d, I, xq.data(), xb.data(), sx, Wuq, Wub, su, u.data());
+  std::vector<uint16_t> a(I);
+  for (int64_t i = 0; i < I; ++i) {
+    const float act =
+        static_cast<float>(static_cast<double>(g[i]) * sigmoid(static_cast<double>(g[i])));
+    a[i] = float_to_bf16_bits(act * u[i]);
+  }
+  if (a_out) std::copy(a.begin(), a.end(), a_out);
+  const float sa = quantize_row_nvfp4(I, a.data(), aq.data(), ab.data());
+  linear_nvfp4_row(I, d, aq.data(), ab.data(), sa, Wdq, Wdb, sd, y);
+}
+
+// MoE output for a list of tokens with NVFP4 experts; as oracle_moe_tokens otherwise.
+int oracle_moe_tokens_nvfp4(int64_t ntok, const int64_t* tokens, int64_t d, int64_t I, int k,
+                            const uint16_t* h, const int32_t* idx, const float* w,
+                            const uint8_t* const* Wgq, const uint8_t* const* Wgb,
+                            const float* const* sg, const uint8_t* const* Wuq,
+                            const uint8_t* const* Wub, const float* const* su,
+                            const uint8_t* const* Wdq, const uint8_t* const* Wdb,
+                            const float* const* sd, float* out, int nthreads) {
+  for (int64_t n = 0; n < ntok; ++n)
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[tokens[n] * k + j];
+      if (!Wgq[e] || !Wgb[e] || !sg[e] || !Wuq[e] || !Wub[e] || !su[e] || !Wdq[e] || !Wdb[e] ||
+          !sd[e])
+        return -1;
+    }
+  std::vector<float> ys(static_cast<size_t>(ntok) * k * d);
+  parallel_for(ntok * k, nthreads, [&](int64_t item) {
+    const int64_t n = item / k;
+    const int j = static_cast<int>(item % k);
+    const int64_t t = tokens[n];
+    const int e = idx[t * k + j];
+    oracle_expert_mlp_nvfp4(d, I, h + t * d, Wgq[e], Wgb[e], sg[e], Wuq[e], Wub[e], su[e],
+                            Wdq[e], Wdb[e], sd[e], ys.data() + item * d, nullptr);
   });
   combine_slots(ntok, tokens, d, k, w, ys.data(), out);
   return 0;

@@ -13,6 +13,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_fp8_pins as fp8
+from tests import test_oracle_nvfp4_pins as fp4
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "beam_moe_oracle.cpp")
@@ -55,6 +56,21 @@ MUTANTS = {
                                      "static_cast<double>(sx) * static_cast<double>(sw[0]) * acc"),
     "fp8_down_reads_input_codes": ("linear_fp8_row(I, d, aq.data(), sa, Wdq, sd, y);",
                                    "linear_fp8_row(I, d, xq.data(), sx, Wdq, sd, y);"),
+    "e2m1_truncates": ("mag = static_cast<uint8_t>(std::nearbyint(a / 0.5));",
+                       "mag = static_cast<uint8_t>(std::floor(a / 0.5));"),
+    "e2m1_middle_binade_step": ("mag = static_cast<uint8_t>(std::nearbyint(a) + 2.0);",
+                                "mag = static_cast<uint8_t>(std::nearbyint(a / 2.0) * 2.0 + 2.0);"),
+    "e2m1_exponent_bias": ("std::ldexp(1.0 + 0.5 * m, e - 1)", "std::ldexp(1.0 + 0.5 * m, e)"),
+    "nvfp4_row_scale_divisor": ("const float s = amax / 2688.0f;", "const float s = amax / 448.0f;"),
+    "nvfp4_block_scale_divisor": ("      t = t / 6.0f;", "      t = t / 4.0f;"),
+    "nvfp4_block_max_is_row_max": ("    float mb = 0.0f;\n    for (int j = 0; j < 16; ++j) mb",
+                                   "    float mb = amax;\n    for (int j = 0; j < 16; ++j) mb"),
+    "nvfp4_linear_drops_input_block_scale": (
+        "acc += e4m3_value(xbs[b]) * e4m3_value(wb[b]) * part;",
+        "acc += e4m3_value(wb[b]) * part;"),
+    "nvfp4_down_reads_input_codes": (
+        "linear_nvfp4_row(I, d, aq.data(), ab.data(), sa, Wdq, Wdb, sd, y);",
+        "linear_nvfp4_row(I, d, xq.data(), xb.data(), sx, Wdq, Wdb, sd, y);"),
 }
 
 PIN_TESTS = [
@@ -82,6 +98,15 @@ PIN_TESTS = [
     (fp8.test_expert_mlp_fp8_gate_up_equal_bf16_expert_on_exact_operands, [()]),
     (fp8.test_expert_mlp_fp8_down_scales_are_per_output_row, [()]),
     (fp8.test_moe_tokens_fp8_is_weighted_sum_of_fp8_experts, [()]),
+    (fp4.test_e2m1_decode_matches_the_format_table, [()]),
+    (fp4.test_e2m1_encode_is_nearest_with_ties_to_even_and_saturates, [()]),
+    (fp4.test_quantize_rows_nvfp4_is_exact_on_representable_rows, [()]),
+    (fp4.test_quantize_rows_nvfp4_error_bounds_and_block_maxima, [()]),
+    (fp4.test_linear_nvfp4_matches_float64_on_decoded_operands, [()]),
+    (fp4.test_linear_nvfp4_equals_router_logits_on_exact_operands, [()]),
+    (fp4.test_expert_mlp_nvfp4_gate_up_equal_bf16_expert_on_exact_operands, [()]),
+    (fp4.test_expert_mlp_nvfp4_down_uses_the_quantised_activation, [()]),
+    (fp4.test_moe_tokens_nvfp4_is_weighted_sum_of_nvfp4_experts, [()]),
 ]
 
 
@@ -107,7 +132,9 @@ def test_mutant_is_caught(tmp_path, monkeypatch, name):
                "oracle_rmsnorm", "oracle_residual", "oracle_residual_coefficients",
                "oracle_bias_update", "oracle_f32_to_e4m3", "oracle_e4m3_to_f32",
                "oracle_quantize_rows_e4m3", "oracle_linear_fp8", "oracle_expert_mlp_fp8",
-               "oracle_moe_tokens_fp8"):
+               "oracle_moe_tokens_fp8", "oracle_f32_to_e2m1", "oracle_e2m1_to_f32",
+               "oracle_quantize_rows_nvfp4", "oracle_linear_nvfp4", "oracle_expert_mlp_nvfp4",
+               "oracle_moe_tokens_nvfp4"):
         f, g = getattr(real, fn), getattr(mut, fn)
         g.argtypes, g.restype = f.argtypes, f.restype
     monkeypatch.setattr(oracle, "_lib", mut)
