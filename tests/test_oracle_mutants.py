@@ -52,8 +52,9 @@ MUTANTS = {
     "e4m3_subnormal_step": ("std::nearbyint(a / std::ldexp(1.0, -9))",
                             "std::nearbyint(a / std::ldexp(1.0, -10))"),
     "fp8_scale_divisor": ("const float s = amax / 448.0f;", "const float s = amax / 240.0f;"),
-    "fp8_weight_scale_not_per_row": ("static_cast<double>(sx) * static_cast<double>(sw[c]) * acc",
-                                     "static_cast<double>(sx) * static_cast<double>(sw[0]) * acc"),
+    "fp8_weight_scale_not_per_row": (
+        "acc += xv[j] * value[w[j]];\n    y[c] = static_cast<float>(static_cast<double>(sx) * static_cast<double>(sw[c]) * acc",
+        "acc += xv[j] * value[w[j]];\n    y[c] = static_cast<float>(static_cast<double>(sx) * static_cast<double>(sw[0]) * acc"),
     "fp8_down_reads_input_codes": ("linear_fp8_row(I, d, aq.data(), sa, Wdq, sd, y);",
                                    "linear_fp8_row(I, d, xq.data(), sx, Wdq, sd, y);"),
     "e2m1_truncates": ("mag = static_cast<uint8_t>(std::nearbyint(a / 0.5));",
