@@ -178,6 +178,62 @@ BEAM_API beam_status beam_moe_block_fp8(const beam_moe_shape* shape, const float
                                         float* x_out, int32_t* topk_idx, float* topk_w, void* ws,
                                         size_t ws_bytes, beam_stream stream);
 
+/* ---- NVFP4 expert weights
+ *
+ * The other checkpoint format the pages name (same passages as the FP8 section, no scale
+ * format given).  This path reads it as E2M1 codes (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6)
+ * with two scales: an E4M3 scale per block of 16 consecutive elements of a row, and an FP32
+ * scale per row.  With amax the row's largest magnitude and m_b the block's:
+ *   s = fl32(amax / 2688),  bs_b = e4m3(fl32(fl32(m_b / s) / 6)),
+ *   q_j = e2m1(fl32(x_j / fl32(s * value(bs_b))))
+ * rounded to nearest even and saturating; a block whose scale is 0 gets zero codes.  Weights are
+ * quantised per output channel.  Token rows and the SwiGLU activation (after its BF16 rounding)
+ * are quantised per row the same way.  Each GEMM runs tcgen05 block-scaled MMAs
+ * (kind::mxf4nvf4, scales applied by the tensor cores, FP32 accumulation) and applies both row
+ * scales in its epilogue.  Routing is unchanged.
+ *
+ * Storage: codes two per byte, element 2i in the low nibble of byte i.  Block scales in
+ * 512-byte atoms covering 128 rows x 64 elements: the scale of row r (0..127) and block j
+ * (0..3) of an atom is byte (r % 32) * 16 + (r / 32) * 4 + j, and the atoms of one 128-row
+ * group follow each other in K order (atom (group g, K block b) at byte (g * K / 64 + b) * 512).
+ * This is the layout the tensor cores read scales in. */
+
+/* Converts BF16 weights to NVFP4 on `stream` (once per model).
+ *   a        BF16 [groups, rows, cols] (row-major)
+ *   b        NULL, or a second BF16 [groups, rows, cols]: the output then holds 2 * rows rows
+ *            per group, interleaving a and b in 64-row chunks (row 128c + w is a's row 64c + w
+ *            for w < 64, b's row 64c + w - 64 otherwise).  Pass w_gate and w_up [E, I, d] this
+ *            way for beam_moe_forward_nvfp4.  w_down [E, d, I] is passed alone (b = NULL).
+ *   codes         out: uint8 [groups * out_rows, cols / 2]
+ *   block_scales  out: E4M3 atoms, groups * out_rows * cols / 16 bytes
+ *   row_scales    out: FP32 [groups * out_rows]
+ * Requires cols a positive multiple of 256, rows a positive multiple of 64 (with b) or 128
+ * (without), every pointer 16-byte aligned, and no output overlapping an input; otherwise
+ * BEAM_ERR_INVALID_ARG.  groups == 0 is a no-op. */
+BEAM_API beam_status beam_moe_quantize_nvfp4(const void* a, const void* b, int64_t groups,
+                                             int32_t rows, int32_t cols, void* codes,
+                                             void* block_scales, float* row_scales,
+                                             beam_stream stream);
+
+/* Workspace bytes for beam_moe_forward_nvfp4 (0 for an unsupported shape; I must be a multiple
+ * of 256 besides the layer's shape rules). */
+BEAM_API size_t beam_moe_nvfp4_workspace_size(const beam_moe_shape* shape);
+
+/* beam_moe_forward with NVFP4 expert weights as written by beam_moe_quantize_nvfp4:
+ *   gate_up_*   w_gate and w_up interleaved: codes [E * 2I, d / 2], atoms, row scales [E * 2I]
+ *   down_*      w_down: codes [E * d, I / 2], atoms, row scales [E * d]
+ * Every other argument as for beam_moe_forward, with ws sized by
+ * beam_moe_nvfp4_workspace_size.  All weight and scale pointers must be 16-byte aligned. */
+BEAM_API beam_status beam_moe_forward_nvfp4(const beam_moe_shape* shape, const void* hidden,
+                                            const float* router_w, const float* bias,
+                                            const void* gate_up_codes,
+                                            const void* gate_up_block_scales,
+                                            const float* gate_up_scales, const void* down_codes,
+                                            const void* down_block_scales,
+                                            const float* down_scales, void* out,
+                                            int32_t* topk_idx, float* topk_w, void* ws,
+                                            size_t ws_bytes, beam_stream stream);
+
 /* MoE block: x' = x * sqrt((k_resid-1)/k_resid) + RMSNorm(MoE(bf16(RMSNorm(x) g_pre))) g_post
  *                 / sqrt(k_resid), RMSNorm(v) = v / sqrt(mean(v^2) + eps), all FP32.
  *   x       FP32 [T, d] residual stream in

@@ -33,7 +33,8 @@ EXPORTED = [
     "beam_dense_forward", "beam_moe_bias_update", "beam_moe_set_sm_pairs",
     "beam_moe_get_sm_pairs", "beam_moe_quantize_e4m3", "beam_moe_fp8_workspace_size",
     "beam_moe_forward_fp8", "beam_moe_block_fp8", "beam_dense_fp8_workspace_size",
-    "beam_dense_forward_fp8",
+    "beam_dense_forward_fp8", "beam_moe_quantize_nvfp4", "beam_moe_nvfp4_workspace_size",
+    "beam_moe_forward_nvfp4",
 ]
 
 
@@ -108,6 +109,10 @@ def lib():
     L.beam_moe_forward_fp8.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                        sz, vp]
     L.beam_moe_block_fp8.argtypes = [shp, vp, vp, vp, f32, i32] + [vp] * 12 + [sz, vp]
+    L.beam_moe_quantize_nvfp4.argtypes = [vp, vp, ctypes.c_int64, i32, i32, vp, vp, vp, vp]
+    L.beam_moe_nvfp4_workspace_size.argtypes = [shp]
+    L.beam_moe_nvfp4_workspace_size.restype = sz
+    L.beam_moe_forward_nvfp4.argtypes = [shp] + [vp] * 13 + [sz, vp]
     L.beam_moe_sync_status.argtypes = [vp, vp]
     L.beam_status_string.argtypes = [ctypes.c_int]
     L.beam_status_string.restype = ctypes.c_char_p
@@ -126,7 +131,8 @@ def lib():
     for name in ("beam_moe_route", "beam_moe_route_static", "beam_moe_forward", "beam_moe_block",
                  "beam_moe_sync_status", "beam_dense_forward", "beam_moe_bias_update",
                  "beam_moe_expert_counts", "beam_moe_profile_read", "beam_moe_quantize_e4m3",
-                 "beam_moe_forward_fp8", "beam_moe_block_fp8", "beam_dense_forward_fp8"):
+                 "beam_moe_forward_fp8", "beam_moe_block_fp8", "beam_dense_forward_fp8",
+                 "beam_moe_quantize_nvfp4", "beam_moe_forward_nvfp4"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -294,6 +300,66 @@ def beam_moe_forward_fp8(shape, hidden, router_w, bias, w_gate, gate_scale, w_up
     _ptr(ws, torch.uint8, "ws")
     _check(lib().beam_moe_forward_fp8(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
                                       _stream(stream)), "beam_moe_forward_fp8")
+    return ws
+
+
+# ------------------------------------------------------------------ NVFP4 expert weights
+
+def beam_moe_nvfp4_workspace_size(shape: beam_moe_shape) -> int:
+    return int(lib().beam_moe_nvfp4_workspace_size(ctypes.byref(shape)))
+
+
+def nvfp4_workspace(shape: beam_moe_shape, device="cuda") -> torch.Tensor:
+    n = beam_moe_nvfp4_workspace_size(shape)
+    if n == 0:
+        raise BeamError(BEAM_ERR_UNSUPPORTED, "beam_moe_nvfp4_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def beam_moe_quantize_nvfp4(a, b=None, stream=None):
+    """NVFP4 codes, block-scale atoms and row scales of BF16 weights a [groups, rows, cols]
+    (with b of the same shape: a and b interleaved in 64-row chunks, 2 * rows rows per group).
+    Returns (codes uint8 [groups, out_rows, cols / 2], atoms uint8 [groups, out_rows * cols / 16],
+    row scales float32 [groups, out_rows])."""
+    if a.dim() != 3:
+        raise ValueError("a must be [groups, rows, cols]")
+    groups, rows, cols = a.shape
+    out_rows = 2 * rows if b is not None else rows
+    codes = torch.empty((groups, out_rows, cols // 2), dtype=torch.uint8, device=a.device)
+    atoms = torch.empty((groups, out_rows * (cols // 16)), dtype=torch.uint8, device=a.device)
+    scales = torch.empty((groups, out_rows), dtype=torch.float32, device=a.device)
+    args = [_ptr(a, torch.bfloat16, "a", tuple(a.shape)),
+            _ptr(b, torch.bfloat16, "b", tuple(a.shape), optional=True),
+            ctypes.c_int64(groups), ctypes.c_int32(rows), ctypes.c_int32(cols),
+            codes.data_ptr(), atoms.data_ptr(), scales.data_ptr()]
+    _check(lib().beam_moe_quantize_nvfp4(*args, _stream(stream)), "beam_moe_quantize_nvfp4")
+    return codes, atoms, scales
+
+
+def beam_moe_forward_nvfp4(shape, hidden, router_w, bias, gate_up, down, out, topk_idx=None,
+                           topk_w=None, ws=None, stream=None):
+    """beam_moe_forward with NVFP4 experts: gate_up = beam_moe_quantize_nvfp4(w_gate, w_up),
+    down = beam_moe_quantize_nvfp4(w_down), each (codes, atoms, row scales)."""
+    T, d, E, k, I = shape.T, shape.d, shape.E, shape.top_k, shape.I
+    gc, ga, gs = gate_up
+    dc, da, ds = down
+    args = [_ptr(hidden, torch.bfloat16, "hidden", (T, d)),
+            _ptr(router_w, torch.float32, "router_w", (E, d)),
+            _ptr(bias, torch.float32, "bias", (E,)),
+            _ptr(gc, torch.uint8, "gate_up codes", (E, 2 * I, d // 2)),
+            _ptr(ga, torch.uint8, "gate_up block scales", (E, 2 * I * (d // 16))),
+            _ptr(gs, torch.float32, "gate_up scales", (E, 2 * I)),
+            _ptr(dc, torch.uint8, "down codes", (E, d, I // 2)),
+            _ptr(da, torch.uint8, "down block scales", (E, d * (I // 16))),
+            _ptr(ds, torch.float32, "down scales", (E, d)),
+            _ptr(out, torch.bfloat16, "out", (T, d)),
+            _ptr(topk_idx, torch.int32, "topk_idx", (T, k), optional=True),
+            _ptr(topk_w, torch.float32, "topk_w", (T, k), optional=True)]
+    if ws is None:
+        ws = nvfp4_workspace(shape, hidden.device)
+    _ptr(ws, torch.uint8, "ws")
+    _check(lib().beam_moe_forward_nvfp4(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
+                                        _stream(stream)), "beam_moe_forward_nvfp4")
     return ws
 
 

@@ -2,6 +2,7 @@
 // layout, TMA tensor maps, kernel launch sequence, device status, launch counting and timing.
 #include "beam_moe.h"
 #include "beam_moe_internal.cuh"
+#include "beam_moe_nvfp4.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -130,6 +131,7 @@ beam_status check_shape(const beam_moe_shape* s) {
 struct Layout {
   size_t status, cnt, off, mt_count, mtiles, rank, rowmap, idx, w, wt, part, h, xp, act, y, total;
   size_t xs = 0, act8 = 0, as = 0;  // FP8 path: row scales of Xp, E4M3 act, act row scales
+  size_t xsf = 0, asf = 0;           // NVFP4 path: block-scale atoms of Xp and of the act
   int S, kchunk;
   int64_t R, mt_cap;
 };
@@ -214,6 +216,27 @@ Layout plan_fp8(const beam_moe_shape& s) {
   return L;
 }
 
+// NVFP4 path: the BF16 layout (whose Xp region holds the code rows, a quarter of its size)
+// plus the row scales and block-scale atoms of Xp, the activation's codes, atoms and scales.
+// Atoms are kept per m-tile (one 128-row group each): mt_cap groups of K / 16 x 128 bytes.
+Layout plan_nvfp4(const beam_moe_shape& s) {
+  Layout L = plan(s);
+  size_t o = L.total;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o = align_up(o + (bytes ? bytes : 1), 1024);
+    return r;
+  };
+  const size_t groups = static_cast<size_t>(L.mt_cap);
+  L.xs = take(sizeof(float) * L.R);
+  L.xsf = take(groups * (s.d / 16) * 128);
+  L.act8 = take(static_cast<size_t>(L.R) * (s.I / 2));
+  L.asf = take(groups * (s.I / 16) * 128);
+  L.as = take(sizeof(float) * L.R);
+  L.total = o;
+  return L;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <class T>
@@ -290,6 +313,8 @@ beam_status device_info(DeviceInfo** out) {
     e = prepare_gemm_kernels();
     if (e != cudaSuccess) return cuda_fail(e);
     e = prepare_gemm_2sm_kernels();
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = prepare_gemm_nvfp4_kernels();
     if (e != cudaSuccess) return cuda_fail(e);
     d.pair_grid = max_pair_grid(d.sms);
     d.prepared = true;
@@ -465,6 +490,107 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   return BEAM_OK;
 }
 
+// NVFP4 expert weights as produced by beam_moe_quantize_nvfp4: gate and up interleaved in
+// 64-row chunks ([E, 2I] rows of d / 2 code bytes) and down ([E, d] rows of I / 2 bytes), each
+// with its block-scale atoms and row scales.
+struct Nvfp4Weights {
+  const void* gu_codes;
+  const void* gu_sf;
+  const float* gu_scale;
+  const void* d_codes;
+  const void* d_sf;
+  const float* d_scale;
+};
+
+// Dispatch and the two NVFP4 expert GEMMs; leaves Y and rowmap in the workspace.
+beam_status run_experts_nvfp4(const beam_moe_shape& s, const Layout& L, const DeviceInfo& dev,
+                              const __nv_bfloat16* h, const int32_t* idx, const Nvfp4Weights& w4,
+                              void* ws, cudaStream_t st) {
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  DispatchArgs da{};
+  da.cnt = at<int32_t>(ws, L.cnt);
+  da.off = at<int32_t>(ws, L.off);
+  da.mt_count = at<int32_t>(ws, L.mt_count);
+  da.mtiles = at<MTile>(ws, L.mtiles);
+  da.E = s.E;
+  da.tile_rows = kBM;
+  BEAM_LAUNCH(kKDispatchScan, st, launch_dispatch_scan(da, st));
+
+  Fp4PermuteArgs pa{};
+  pa.h = h;
+  pa.idx = idx;
+  pa.rank = at<int32_t>(ws, L.rank);
+  pa.cnt = da.cnt;
+  pa.off = da.off;
+  pa.rowmap = at<int32_t>(ws, L.rowmap);
+  pa.xq = at<uint8_t>(ws, L.xp);
+  pa.xsf = at<uint8_t>(ws, L.xsf);
+  pa.xs = at<float>(ws, L.xs);
+  pa.status = status;
+  pa.T = s.T;
+  pa.d = s.d;
+  pa.k = s.top_k;
+  pa.E = s.E;
+  BEAM_LAUNCH(kKPermute, st, launch_nvfp4_permute(pa, st));
+
+  const uint64_t R = static_cast<uint64_t>(L.R);
+  ATensorMaps tm_x, tm_a;
+  CUtensorMap tm_gu, tm_d;
+  beam_status b;
+  for (int i = 0; i < kNumABoxes; ++i) {
+    if ((b = make_map(&tm_x.m[i], pa.xq, s.d / 2, R, a_box_rows(i), 1)) != BEAM_OK) return b;
+    if ((b = make_map(&tm_a.m[i], at<void>(ws, L.act8), s.I / 2, R, a_box_rows(i), 1)) != BEAM_OK)
+      return b;
+  }
+  const uint64_t E2I = static_cast<uint64_t>(s.E) * 2 * s.I, Ed = static_cast<uint64_t>(s.E) * s.d;
+  if ((b = make_map(&tm_gu, w4.gu_codes, s.d / 2, E2I, kF4N, 1)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_d, w4.d_codes, s.I / 2, Ed, kF4N, 1)) != BEAM_OK) return b;
+
+  Fp4GemmArgs g1{};
+  g1.mtiles = da.mtiles;
+  g1.mt_count = da.mt_count;
+  g1.out = at<__nv_bfloat16>(ws, L.act);
+  g1.status = status;
+  g1.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  g1.out_ld = s.I;
+  g1.n_tiles_n = 2 * s.I / kF4N;
+  g1.k_blocks = s.d / kF4KElems;
+  g1.b_rows_per_expert = 2 * s.I;
+  g1.a_sf = pa.xsf;
+  g1.b_sf = static_cast<const uint8_t*>(w4.gu_sf);
+  g1.a_scale = pa.xs;
+  g1.b_scale = w4.gu_scale;
+  const int64_t max_tiles1 = L.mt_cap * g1.n_tiles_n;
+  const int grid1 = static_cast<int>(max_tiles1 < dev.sms ? max_tiles1 : dev.sms);
+  BEAM_LAUNCH(kKGemmGateUp, st, launch_gemm_nvfp4(true, tm_x, tm_gu, g1, grid1, st));
+
+  Fp4ActArgs qa{};
+  qa.x = g1.out;
+  qa.mtiles = da.mtiles;
+  qa.mt_count = da.mt_count;
+  qa.q = at<uint8_t>(ws, L.act8);
+  qa.sf = at<uint8_t>(ws, L.asf);
+  qa.s = at<float>(ws, L.as);
+  qa.cols = s.I;
+  qa.mt_cap = static_cast<int>(L.mt_cap);
+  BEAM_LAUNCH(kKQuantize, st, launch_nvfp4_act(qa, st));
+
+  Fp4GemmArgs g2 = g1;
+  g2.out = at<__nv_bfloat16>(ws, L.y);
+  g2.out_ld = s.d;
+  g2.n_tiles_n = s.d / kF4N;
+  g2.k_blocks = s.I / kF4KElems;
+  g2.b_rows_per_expert = s.d;
+  g2.a_sf = qa.sf;
+  g2.b_sf = static_cast<const uint8_t*>(w4.d_sf);
+  g2.a_scale = qa.s;
+  g2.b_scale = w4.d_scale;
+  const int64_t max_tiles2 = L.mt_cap * g2.n_tiles_n;
+  const int grid2 = static_cast<int>(max_tiles2 < dev.sms ? max_tiles2 : dev.sms);
+  BEAM_LAUNCH(kKGemmDown, st, launch_gemm_nvfp4(false, tm_a, tm_d, g2, grid2, st));
+  return BEAM_OK;
+}
+
 bool any_misaligned(std::initializer_list<const void*> ps) {
   for (const void* p : ps)
     if (!p || !aligned16(p)) return true;
@@ -608,6 +734,43 @@ beam_status forward_impl(const beam_moe_shape* shape, const void* hidden, const 
     return b;
   if ((b = run_experts(*shape, L, *dev, h, idx, w_gate, w_up, w_down, ws, st, f8)) != BEAM_OK)
     return b;
+  CombineArgs ca{};
+  ca.y = at<__nv_bfloat16>(ws, L.y);
+  ca.rowmap = at<int32_t>(ws, L.rowmap);
+  ca.w = w;
+  ca.out = static_cast<__nv_bfloat16*>(out);
+  ca.status = at<uint32_t>(ws, L.status);
+  ca.T = shape->T;
+  ca.d = shape->d;
+  ca.k = shape->top_k;
+  ca.R = static_cast<int>(L.R);
+  BEAM_LAUNCH(kKCombine, st, launch_combine(ca, st));
+  return BEAM_OK;
+}
+
+beam_status forward_nvfp4_impl(const beam_moe_shape* shape, const void* hidden,
+                               const float* router_w, const float* bias, const Nvfp4Weights& w4,
+                               void* out, int32_t* topk_idx, float* topk_w, void* ws,
+                               size_t ws_bytes, beam_stream stream) {
+  beam_status b = check_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (shape->I % kF4KElems != 0) return BEAM_ERR_UNSUPPORTED;
+  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
+  if (any_misaligned({hidden, router_w, w4.gu_codes, w4.gu_sf, w4.gu_scale, w4.d_codes, w4.d_sf,
+                      w4.d_scale, out}) ||
+      !bias || (topk_idx && !aligned16(topk_idx)) || (topk_w && !aligned16(topk_w)))
+    return BEAM_ERR_INVALID_ARG;
+  const Layout L = plan_nvfp4(*shape);
+  if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
+  DeviceInfo* dev;
+  if ((b = device_info(&dev)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
+  float* w = topk_w ? topk_w : at<float>(ws, L.w);
+  const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(hidden);
+  if ((b = run_router(*shape, L, h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
+    return b;
+  if ((b = run_experts_nvfp4(*shape, L, *dev, h, idx, w4, ws, st)) != BEAM_OK) return b;
   CombineArgs ca{};
   ca.y = at<__nv_bfloat16>(ws, L.y);
   ca.rowmap = at<int32_t>(ws, L.rowmap);
@@ -875,6 +1038,53 @@ beam_status beam_moe_quantize_e4m3(const void* x, int64_t rows, int32_t cols, vo
 }
 
 
+
+size_t beam_moe_nvfp4_workspace_size(const beam_moe_shape* shape) {
+  if (check_shape(shape) != BEAM_OK || shape->I % kF4KElems != 0) return 0;
+  return plan_nvfp4(*shape).total;
+}
+
+beam_status beam_moe_quantize_nvfp4(const void* a, const void* b, int64_t groups, int32_t rows,
+                                    int32_t cols, void* codes, void* block_scales,
+                                    float* row_scales, beam_stream stream) {
+  if (groups < 0 || rows <= 0 || cols <= 0 || cols % kF4KElems != 0 ||
+      rows % (b ? 64 : 128) != 0)
+    return BEAM_ERR_INVALID_ARG;
+  if (groups == 0) return BEAM_OK;
+  if (any_misaligned({a, codes, block_scales, row_scales}) || (b && !aligned16(b)))
+    return BEAM_ERR_INVALID_ARG;
+  const uint64_t in_bytes = static_cast<uint64_t>(groups) * rows * cols * 2;
+  const uint64_t out_rows = static_cast<uint64_t>(groups) * (b ? 2 * rows : rows);
+  const uint64_t outs[3][2] = {{reinterpret_cast<uintptr_t>(codes), out_rows * (cols / 2)},
+                               {reinterpret_cast<uintptr_t>(block_scales), out_rows * (cols / 16)},
+                               {reinterpret_cast<uintptr_t>(row_scales), out_rows * 4}};
+  for (const void* in : {a, b}) {
+    if (!in) continue;
+    const uint64_t ib = reinterpret_cast<uintptr_t>(in);
+    for (const auto& o : outs)
+      if (o[0] < ib + in_bytes && ib < o[0] + o[1]) return BEAM_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  BEAM_LAUNCH(kKQuantize, st,
+              launch_nvfp4_weights(static_cast<const __nv_bfloat16*>(a),
+                                   static_cast<const __nv_bfloat16*>(b), groups, rows, cols,
+                                   static_cast<uint8_t*>(codes),
+                                   static_cast<uint8_t*>(block_scales), row_scales, st));
+  return BEAM_OK;
+}
+
+beam_status beam_moe_forward_nvfp4(const beam_moe_shape* shape, const void* hidden,
+                                   const float* router_w, const float* bias,
+                                   const void* gate_up_codes, const void* gate_up_block_scales,
+                                   const float* gate_up_scales, const void* down_codes,
+                                   const void* down_block_scales, const float* down_scales,
+                                   void* out, int32_t* topk_idx, float* topk_w, void* ws,
+                                   size_t ws_bytes, beam_stream stream) {
+  const Nvfp4Weights w4{gate_up_codes, gate_up_block_scales, gate_up_scales,
+                        down_codes,    down_block_scales,    down_scales};
+  return forward_nvfp4_impl(shape, hidden, router_w, bias, w4, out, topk_idx, topk_w, ws,
+                            ws_bytes, stream);
+}
 
 beam_status beam_moe_forward(const beam_moe_shape* shape, const void* hidden, const float* router_w,
                              const float* bias, const void* w_gate, const void* w_up,

@@ -230,3 +230,98 @@ def oracle_out_fp8(case: Case, weights, tokens, gpu_fp8=None, batch: int = 4):
                                           experts[e][2 * m_i + 1])
         out[b0:b0 + len(tb)] = oracle.moe_tokens_fp8(tb, case.h, case.idx, case.w, experts)
     return out
+
+
+# ------------------------------------------------------------------ NVFP4 expert weights
+
+def device_weights_nvfp4(weights):
+    """NVFP4 form of BF16 expert weights, quantised by the CUDA path: ((gate|up interleaved
+    codes, atoms, row scales), (down codes, atoms, row scales))."""
+    wg, wu, wd = weights
+    gu = bm.beam_moe_quantize_nvfp4(wg, wu)
+    dn = bm.beam_moe_quantize_nvfp4(wd)
+    torch.cuda.synchronize()
+    return gu, dn
+
+
+def unpack_e2m1(packed: np.ndarray) -> np.ndarray:
+    """[..., n / 2] bytes -> [..., n] codes (element 2i in the low nibble of byte i)."""
+    lo, hi = packed & 0xF, packed >> 4
+    return np.stack([lo, hi], axis=-1).reshape(*packed.shape[:-1], packed.shape[-1] * 2)
+
+
+def atoms_to_rows(atoms: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """Block-scale atoms of `rows` (a multiple of 128) x `cols` -> [rows, cols / 16] codes:
+    byte (r % 32) * 16 + (r / 32) * 4 + (j % 4) of atom j / 4 of row group r / 128."""
+    a = atoms.reshape(rows // 128, cols // 64, 32, 4, 4)      # group, atom, m0, m1, block
+    return a.transpose(0, 3, 2, 1, 4).reshape(rows, cols // 16)
+
+
+def canonical_e2m1(q: np.ndarray) -> np.ndarray:
+    """Codes with -0 written as +0 (both are zero)."""
+    return np.where((q & 7) == 0, 0, q).astype(np.uint8)
+
+
+def nvfp4_expert_from_device(w4, e: int, I: int, d: int):
+    """The CUDA path's NVFP4 matrices of expert e in the oracle's layout: (gate, up, down),
+    each (codes [rows, cols], block scales [rows, cols / 16], row scales [rows])."""
+    (gc, ga, gs), (dc, da, ds) = w4
+    q = unpack_e2m1(gc[e].cpu().numpy())                       # [2I, d]
+    b = atoms_to_rows(ga[e].cpu().numpy(), 2 * I, d)           # [2I, d / 16]
+    s = gs[e].cpu().numpy()
+    def split(x):
+        x = x.reshape(I // 64, 2, 64, *x.shape[1:])
+        return x[:, 0].reshape(I, *x.shape[3:]), x[:, 1].reshape(I, *x.shape[3:])
+    (qg, qu), (bg, bu), (sg, su) = split(q), split(b), split(s)
+    qd = unpack_e2m1(dc[e].cpu().numpy())
+    bd = atoms_to_rows(da[e].cpu().numpy(), d, I)
+    sd = ds[e].cpu().numpy()
+    return (qg, bg, sg), (qu, bu, su), (qd, bd, sd)
+
+
+def oracle_experts_nvfp4(weights, experts, w4=None):
+    """The oracle's own NVFP4 quantisation of the listed experts (from the BF16 weights); when
+    the CUDA path's weights are given, they must equal the oracle's bit for bit (+-0 alike)."""
+    res = {}
+    for e in experts:
+        parts = tuple(oracle.quantize_rows_nvfp4(m[e].cpu()) for m in weights)
+        if w4 is not None:
+            I, d = weights[0].shape[1], weights[0].shape[2]
+            got = nvfp4_expert_from_device(w4, e, I, d)
+            for name, (q, b, s), (gq, gb, gs) in zip(("gate", "up", "down"), parts, got):
+                assert np.array_equal(canonical_e2m1(gq), canonical_e2m1(q)), f"{e} {name} codes"
+                assert np.array_equal(gb, b), f"expert {e} {name}: block scales differ"
+                assert np.array_equal(gs, s), f"expert {e} {name}: row scales differ"
+        res[e] = parts
+    return res
+
+
+def run_forward_nvfp4(case: Case, w4, ws=None):
+    wl = case.wl
+    s = bm.shape_of(wl)
+    dev = "cuda"
+    out = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(wl.T, wl.top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(wl.T, wl.top_k, dtype=torch.float32, device=dev)
+    ws = bm.beam_moe_forward_nvfp4(s, case.h.to(dev), case.router_w.to(dev), case.bias.to(dev),
+                                   w4[0], w4[1], out, idx, w, ws=ws)
+    st = bm.beam_moe_sync_status(ws)
+    assert st == bm.BEAM_OK, bm.status_string(st)
+    return out, idx, w, ws
+
+
+def oracle_out_nvfp4(case: Case, weights, tokens, w4=None, batch: int = 4):
+    """Oracle MoE output (FP32) of the NVFP4 path for ``tokens``; the oracle quantises the BF16
+    weights of the experts each batch uses (and checks the CUDA path's weights against them)."""
+    tokens = list(tokens)
+    out = np.empty((len(tokens), case.wl.d), np.float32)
+    checked = set()
+    for b0 in range(0, len(tokens), batch):
+        tb = tokens[b0:b0 + batch]
+        ex = sorted({int(e) for t in tb for e in case.idx[t]})
+        new = [e for e in ex if e not in checked]
+        experts = oracle_experts_nvfp4(weights, new, w4)
+        experts.update(oracle_experts_nvfp4(weights, [e for e in ex if e in checked], None))
+        checked.update(new)
+        out[b0:b0 + len(tb)] = oracle.moe_tokens_nvfp4(tb, case.h, case.idx, case.w, experts)
+    return out

@@ -202,3 +202,40 @@ def test_fp8_block_and_dense_validate_before_launching(L):
     assert dns(ctypes.byref(ds), *mis, q(A), 1 << 30, None) == bm.BEAM_ERR_INVALID_ARG
     assert dns(ctypes.byref(ds), *args, None, 16, None) == bm.BEAM_ERR_WORKSPACE
     assert dns(ctypes.byref(bm.dense_shape(0, 5120, 20480)), *[None] * 9, 0, None) == bm.BEAM_OK
+
+
+def test_nvfp4_entry_points_validate_before_launching(L):
+    s = beam(4096)
+    n = bm.beam_moe_nvfp4_workspace_size(s)
+    R = 4096 * 8
+    mt_cap = R // 128 + 256
+    # the BF16 layout plus Xp row scales and atoms, the act codes, atoms and row scales
+    assert n >= bm.beam_moe_workspace_size(s) + R * (4 + 1280 + 4) + mt_cap * 128 * (320 + 160)
+    assert L.beam_moe_nvfp4_workspace_size(None) == 0
+    assert bm.beam_moe_nvfp4_workspace_size(beam(64, I=128)) == 0   # I not a multiple of 256
+    A = 1 << 20  # a fake, 16-byte aligned address: never dereferenced on these paths
+    q = ctypes.c_void_p
+    quant = L.beam_moe_quantize_nvfp4
+    far = A << 6
+    assert quant(q(A), None, 0, 128, 256, q(far), q(far << 1), q(far << 2), None) == bm.BEAM_OK
+    for b, groups, rows, cols, codes in ((None, 2, 128, 320, far),   # cols not a multiple of 256
+                                         (None, 2, 64, 256, far),    # rows not a multiple of 128
+                                         (A << 3, 2, 32, 256, far),  # interleaved: rows % 64
+                                         (None, -1, 128, 256, far),  # negative groups
+                                         (None, 2, 0, 256, far),     # no rows
+                                         (None, 2, 128, 256, far + 4),  # misaligned codes
+                                         (A << 3 | 8, 2, 64, 256, far),  # misaligned b
+                                         (None, 2, 128, 256, A + 256)):  # codes overlap a
+        assert quant(q(A), q(b) if b else None, groups, rows, cols, q(codes), q(far << 1),
+                     q(far << 2), None) == bm.BEAM_ERR_INVALID_ARG, (b, groups, rows, cols)
+    # block scales overlapping the second input
+    assert quant(q(A), q(A << 3), 2, 64, 256, q(far), q((A << 3) + 64), q(far << 2), None) == \
+        bm.BEAM_ERR_INVALID_ARG
+    fwd = L.beam_moe_forward_nvfp4
+    args = [q(A)] * 13  # hidden .. topk_w, ws
+    assert fwd(ctypes.byref(beam(0)), *[None] * 13, 0, None) == bm.BEAM_OK
+    assert fwd(ctypes.byref(beam(64, I=128)), *args, 1 << 30, None) == bm.BEAM_ERR_UNSUPPORTED
+    misaligned = list(args)
+    misaligned[4] = q(A + 4)  # gate_up block scales
+    assert fwd(ctypes.byref(beam(64)), *misaligned, 1 << 30, None) == bm.BEAM_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(beam(64)), *args[:12], None, 16, None) == bm.BEAM_ERR_WORKSPACE
