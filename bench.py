@@ -38,6 +38,9 @@ from sparse_moe_transformer_fp32_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at Beam shape T=4096 BF16; % BF16 tensor peak / % HBM BW"
 METRIC_FP8 = "MoE-layer tokens/s at Beam shape with FP8 E4M3 expert weights; % FP8 tensor peak / % HBM BW"
+METRIC_NVFP4 = ("MoE-layer tokens/s at Beam shape with NVFP4 expert weights; % FP4 tensor peak / "
+                "% HBM BW")
+NVFP4_BYTES = 0.5 + 1.0 / 16  # one E2M1 code and a sixteenth of an E4M3 block scale per element
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0, "source": "fallback"}
 N_SMS = 148
@@ -64,6 +67,8 @@ def parse_args(argv=None):
                         "rows per expert (off by default)")
     p.add_argument("--fp8", action="store_true",
                    help="E4M3 expert weights (beam_moe_forward_fp8); layer workloads only")
+    p.add_argument("--nvfp4", action="store_true",
+                   help="NVFP4 expert weights (beam_moe_forward_nvfp4); layer workloads only")
     p.add_argument("--route-only", action="store_true",
                    help="time beam_moe_route alone (router profiling; not the layer metric)")
     p.add_argument("--dry-run", action="store_true",
@@ -71,6 +76,9 @@ def parse_args(argv=None):
     args = p.parse_args(argv)
     if args.warmup < 3 and not args.dry_run:
         p.error("--warmup must be >= 3")
+    if args.nvfp4 and (args.fp8 or W.WORKLOADS[args.workload].block
+                       or W.WORKLOADS[args.workload].dense):
+        p.error("--nvfp4 runs the layer workloads with NVFP4 weights only")
     return args
 
 
@@ -235,12 +243,28 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ algorithmic work
 
-def kernel_work(wl, touched: int, fp8: bool = False):
+def kernel_work(wl, touched: int, fp8: bool = False, nvfp4: bool = False):
     """Algorithmic bytes and FLOPs per launch of each kernel (the minimum each must move).
-    With fp8 the weights and the GEMM inputs are one-byte E4M3 codes (row scales ignored)."""
+    With fp8 the weights and the GEMM inputs are one-byte E4M3 codes (row scales ignored); with
+    nvfp4 they are half-byte E2M1 codes plus one E4M3 block scale per 16 elements."""
     T, d, E, k, I = wl.T, wl.d, wl.E, wl.top_k, wl.I
     R = T * k
     bf, f4 = 2, 4
+    if nvfp4:
+        q = NVFP4_BYTES
+        return {
+            "router_transpose": {"flops": 0, "bytes": 2 * E * d * f4},
+            "dispatch_scan": {"flops": 0, "bytes": E * 16},
+            "router_gemm": {"flops": 2 * T * d * E, "bytes": T * d * bf + E * d * f4 + T * E * f4},
+            "router_select": {"flops": 0, "bytes": T * E * f4 + 2 * R * f4},
+            "permute": {"flops": 0, "bytes": T * d * bf + R * d * q},
+            "expert_gemm_gate_up": {"flops": 4 * R * d * I,
+                                    "bytes": touched * 2 * I * d * q + R * d * q + R * I * bf},
+            "quantize_nvfp4": {"flops": 0, "bytes": R * I * bf + R * I * q},
+            "expert_gemm_down": {"flops": 2 * R * d * I,
+                                 "bytes": touched * d * I * q + R * I * q + R * d * bf},
+            "combine": {"flops": 2 * R * d, "bytes": R * d * bf + T * d * bf},
+        }
     if fp8:
         q = 1
         return {
@@ -275,17 +299,21 @@ def kernel_work(wl, touched: int, fp8: bool = False):
     }
 
 
-def layer_min_bytes(wl, touched: int, fp8: bool = False):
+def layer_min_bytes(wl, touched: int, fp8: bool = False, nvfp4: bool = False):
     T, d, I = wl.T, wl.d, wl.I
-    b = touched * 3 * d * I * (1 if fp8 else 2) + T * d * 2 * 2
+    b = touched * 3 * d * I * (NVFP4_BYTES if nvfp4 else 1 if fp8 else 2) + T * d * 2 * 2
     if wl.block:
         b += 2 * T * d * 4
     return b
 
 
-def traffic_from_profile(kernel: str, workload: str):
+GEMM_SOURCES = ("expert_gemm.cu", "beam_moe_internal.cuh")
+NVFP4_SOURCES = ("nvfp4.cu", "beam_moe_nvfp4.cuh", "beam_moe_internal.cuh")
+
+
+def traffic_from_profile(kernel: str, workload: str, sources=GEMM_SOURCES):
     """dram bytes per launch from the committed ncu summary, if it was taken on the current
-    kernel source (else None)."""
+    kernel source (the sha256 of `sources`, in order; else None)."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         text = open(path).read()
@@ -297,7 +325,7 @@ def traffic_from_profile(kernel: str, workload: str):
         return None
     src = os.path.join(ROOT, "sparse_moe_transformer_fp32_b200", "csrc")
     cur = hashlib.sha256()
-    for name in ("expert_gemm.cu", "beam_moe_internal.cuh"):
+    for name in sources:
         with open(os.path.join(src, name), "rb") as f:
             cur.update(f.read())
     if not cur.hexdigest().startswith(h.group(1)):
@@ -351,6 +379,25 @@ def oracle_fp8_sample_rate(wl, router_w, bias, hidden_cpu, weights_dev, n_tokens
     return n_tokens / dt, dt, oracle.hardware_threads()
 
 
+def oracle_nvfp4_sample_rate(wl, router_w, bias, hidden_cpu, weights_dev, n_tokens: int):
+    """Tokens/s of the CPU oracle's NVFP4 layer on the first n tokens; the oracle converts the
+    experts those tokens use from the BF16 weights first (not timed: a one-off conversion)."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    n_tokens = min(n_tokens, wl.T)
+    h = hidden_cpu[:n_tokens]
+    sample = wl.with_tokens(n_tokens)
+    _, idx, w, _, _ = oracle.layer_routing(h, router_w, bias, sample)
+    experts = {e: tuple(oracle.quantize_rows_nvfp4(m[e].cpu()) for m in weights_dev)
+               for e in sorted({int(e) for e in idx.reshape(-1)})}
+    t0 = time.perf_counter()
+    _, idx, w, _, _ = oracle.layer_routing(h, router_w, bias, sample)
+    oracle.moe_tokens_nvfp4(np.arange(n_tokens), h, idx, w, experts)
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt, oracle.hardware_threads()
+
+
 def oracle_dense_rate(wl, hidden_cpu, weights_dev, n_tokens: int):
     import oracle
     oracle.build()
@@ -399,6 +446,11 @@ def run_cuda(args, rank, world, local):
             out = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
             inp_cpu, inp, res = h_cpu, h, out
         fp8 = None
+        fp4 = None
+        if args.nvfp4:
+            fp4 = (bm.beam_moe_quantize_nvfp4(weights[0], weights[1]),
+                   bm.beam_moe_quantize_nvfp4(weights[2]))
+            torch.cuda.synchronize(dev)
         if args.fp8:
             fp8 = []
             for m in weights:
@@ -406,6 +458,8 @@ def run_cuda(args, rank, world, local):
             torch.cuda.synchronize(dev)
         if wl.dense:
             ws = bm.dense_fp8_workspace(ds, dev) if fp8 else bm.dense_workspace(ds, dev)
+        elif fp4:
+            ws = bm.nvfp4_workspace(s, dev)
         else:
             ws = bm.fp8_workspace(s, dev) if fp8 else bm.workspace(s, dev)
         stream = torch.cuda.current_stream(dev)
@@ -424,6 +478,8 @@ def run_cuda(args, rank, world, local):
             elif wl.block:
                 bm.beam_moe_block(s, src, g_pre, g_post, wl.eps, wl.k_resid, router_w, bias,
                                   *weights, dst, ws=ws)
+            elif fp4:
+                bm.beam_moe_forward_nvfp4(s, src, router_w, bias, fp4[0], fp4[1], dst, ws=ws)
             elif fp8:
                 bm.beam_moe_forward_fp8(s, src, router_w, bias, *fp8, dst, ws=ws)
             else:
@@ -522,7 +578,7 @@ def run_cuda(args, rank, world, local):
 
         result = None
         if rank == 0:
-            work = kernel_work(wl, touched, fp8=bool(fp8))
+            work = kernel_work(wl, touched, fp8=bool(fp8), nvfp4=bool(fp4))
             per_kernel = {k: {"launches": n, "ms_per_launch": (ms / n if n else None)}
                           for k, (n, ms) in prof.items() if n}
             dom = max((k for k in per_kernel if k in work), key=lambda k: prof[k][1])
@@ -533,6 +589,8 @@ def run_cuda(args, rank, world, local):
             ten_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
             if fp8:
                 ten_peak *= 2  # FP8 dense tensor rate: the measured BF16 rate x the nominal 2
+            if fp4:
+                ten_peak *= 4  # FP4 dense tensor rate: the measured BF16 rate x the nominal 4
             if dom == "router_gemm":
                 clk = float(peaks.get("sm_max_mhz", 1965.0))
                 alu_peak = N_SMS * FFMA_PER_SM_PER_CLK * 2 * clk * 1e6 / 1e12
@@ -549,17 +607,32 @@ def run_cuda(args, rank, world, local):
             roof["peak_source"] = peaks.get("source", "measured")
             if fp8 and roof["bound"] == "tensor":
                 roof["peak_source"] += " bf16 x 2 (nominal FP8:BF16 ratio)"
-            roof["traffic"] = traffic_from_profile(dom, wl.name + ("-fp8" if fp8 else ""))
+            if fp4 and roof["bound"] == "tensor":
+                roof["peak_source"] += " bf16 x 4 (nominal FP4:BF16 ratio)"
+            if fp4:
+                roof["traffic"] = traffic_from_profile(dom, wl.name + "-nvfp4", NVFP4_SOURCES)
+            else:
+                roof["traffic"] = traffic_from_profile(dom, wl.name + ("-fp8" if fp8 else ""))
             roof["algorithmic_per_launch"] = wk["bytes"] if roof["bound"] == "hbm" else wk["flops"]
             roof["tensor_frac_of_sustained"] = (wk["flops"] / avg_s / 1e12) / ten_peak
             roof["hbm_frac"] = (wk["bytes"] / avg_s / 1e9) / peaks["hbm_gbs"]
 
             step_s = ms_per_step / 1e3
             flops_step = 6 * wl.T * wl.top_k * wl.d * wl.I  # top_k = 1 for the dense MLP
-            bytes_step = layer_min_bytes(wl, touched, fp8=bool(fp8))
+            bytes_step = layer_min_bytes(wl, touched, fp8=bool(fp8), nvfp4=bool(fp4))
             cpu = None
             result_extra = {}
-            if fp8 and (wl.dense or wl.block):
+            if fp4 and not args.no_cpu_baseline and world == 1:
+                n_cpu = min(args.cpu_sample_tokens, 16)
+                rate, secs, cores = oracle_nvfp4_sample_rate(
+                    wl, W.router_weight(wl), W.router_bias(wl), inp_cpu, weights, n_cpu)
+                cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                       "sample": f"first {n_cpu} tokens of the {wl.name} workload, full NVFP4 "
+                                 f"layer (router logits, routing, {wl.top_k} NVFP4 SwiGLU experts "
+                                 f"each, combine) in double-accumulating C++; {secs:.2f} s"}
+            elif fp4:
+                pass
+            elif fp8 and (wl.dense or wl.block):
                 pass  # the E4M3 CPU baseline is timed on the layer workloads only
             elif not args.no_cpu_baseline and world == 1 and fp8:
                 n_cpu = min(args.cpu_sample_tokens, 16)
@@ -593,12 +666,14 @@ def run_cuda(args, rank, world, local):
                         "value": rate1, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                         "sample": f"first {n1} tokens, one host thread; {secs1:.2f} s"}
             result = {
-                "metric": METRIC_FP8 if fp8 else METRIC, "value": value, "unit": "tokens/s",
+                "metric": METRIC_NVFP4 if fp4 else METRIC_FP8 if fp8 else METRIC,
+                "value": value, "unit": "tokens/s",
                 "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
+                "dtype": "e2m1" if fp4 else "e4m3" if fp8 else "bf16", "data": "synthetic",
                 "config": {"workload": f"{wl.name}{'-fp8' if fp8 else ''}"
+                                       f"{'-nvfp4' if fp4 else ''}"
                                        f"{'-smpairs' if args.sm_pairs else ''}: T={wl.T} d={wl.d} "
                                        f"E={wl.E} n_group={wl.n_group} "
                                        f"topk_group={wl.topk_group} top_k={wl.top_k} I={wl.I}"
@@ -607,7 +682,8 @@ def run_cuda(args, rank, world, local):
                            "parallelism": f"replicas x{world} (data parallel over tokens)",
                            "l2": "inputs larger than L2: every step streams the touched experts' "
                                  f"weights ({touched} of {wl.E} experts, "
-                                 f"{touched * 3 * wl.d * wl.I * (1 if fp8 else 2) / 1e9:.2f} GB) "
+                                 f"{layer_min_bytes(wl, touched, bool(fp8), bool(fp4)) / 1e9:.2f}"
+                                 " GB with the activations) "
                                  "from HBM",
                            "touched_experts": touched,
                            "max_expert_load": int(counts.max()),
@@ -624,7 +700,7 @@ def run_cuda(args, rank, world, local):
                 **result_extra,
             }
         barrier(dist, dev)
-        del weights, fp8
+        del weights, fp8, fp4
     return result
 
 
@@ -665,11 +741,16 @@ def run_reference(args, rank, world, local):
         if args.fp8:  # the oracle converts the experts itself (a one-off, not timed)
             experts = {e: tuple(p for m in mats for p in oracle.quantize_rows_e4m3(m))
                        for e, mats in experts.items()}
+        if args.nvfp4:
+            experts = {e: tuple(oracle.quantize_rows_nvfp4(m) for m in mats)
+                       for e, mats in experts.items()}
         return sample, experts
 
     def one_step(n, sample, experts):
         _, ix, ww, _, _ = oracle.layer_routing(h[:n], router_w, bias, sample)
-        if args.fp8:
+        if args.nvfp4:
+            oracle.moe_tokens_nvfp4(np.arange(n), h[:n], ix, ww, experts)
+        elif args.fp8:
             oracle.moe_tokens_fp8(np.arange(n), h[:n], ix, ww, experts)
         else:
             oracle.moe_tokens(np.arange(n), h[:n], ix, ww, experts)
@@ -690,11 +771,12 @@ def run_reference(args, rank, world, local):
     dt = time.perf_counter() - t0
     value = n * args.steps / dt
     cores = oracle.hardware_threads()
-    kind = "E4M3 " if args.fp8 else ""
+    kind = "NVFP4 " if args.nvfp4 else "E4M3 " if args.fp8 else ""
     desc = (f"first {n} tokens of the {wl.name} workload per step, full {kind}layer (router "
             f"logits, routing, {wl.top_k} {kind}SwiGLU experts per token, combine) in "
             f"double-accumulating C++ on {cores} host threads")
-    return {"impl": "reference", "metric": METRIC_FP8 if args.fp8 else METRIC, "value": value,
+    metric = METRIC_NVFP4 if args.nvfp4 else METRIC_FP8 if args.fp8 else METRIC
+    return {"impl": "reference", "metric": metric, "value": value,
             "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",

@@ -38,12 +38,13 @@ enum KernelId {
   kKDenseTiles,
   kKBiasUpdate,
   kKQuantize,
+  kKQuantizeNvfp4,
   kNumKernels
 };
 const char* const kKernelNames[kNumKernels] = {
     "router_gemm", "router_select", "dispatch_scan", "permute", "expert_gemm_gate_up",
     "expert_gemm_down", "combine", "combine_block", "prenorm", "router_transpose", "dense_tiles",
-    "bias_update", "quantize_e4m3"};
+    "bias_update", "quantize_e4m3", "quantize_nvfp4"};
 
 struct Profiler {
   std::mutex mu;
@@ -573,7 +574,7 @@ beam_status run_experts_nvfp4(const beam_moe_shape& s, const Layout& L, const De
   qa.s = at<float>(ws, L.as);
   qa.cols = s.I;
   qa.mt_cap = static_cast<int>(L.mt_cap);
-  BEAM_LAUNCH(kKQuantize, st, launch_nvfp4_act(qa, st));
+  BEAM_LAUNCH(kKQuantizeNvfp4, st, launch_nvfp4_act(qa, st));
 
   Fp4GemmArgs g2 = g1;
   g2.out = at<__nv_bfloat16>(ws, L.y);
@@ -1065,7 +1066,7 @@ beam_status beam_moe_quantize_nvfp4(const void* a, const void* b, int64_t groups
       if (o[0] < ib + in_bytes && ib < o[0] + o[1]) return BEAM_ERR_INVALID_ARG;
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  BEAM_LAUNCH(kKQuantize, st,
+  BEAM_LAUNCH(kKQuantizeNvfp4, st,
               launch_nvfp4_weights(static_cast<const __nv_bfloat16*>(a),
                                    static_cast<const __nv_bfloat16*>(b), groups, rows, cols,
                                    static_cast<uint8_t*>(codes),
