@@ -207,3 +207,55 @@ def test_forward_nvfp4_wait_timeout_is_reported_and_context_survives():
     toks = list(range(0, case.wl.T, 37))
     ref = H.oracle_out_nvfp4(case, weights, toks, w4, batch=64)
     H.assert_close_out(out2[toks].float().cpu().numpy(), ref, "nvfp4 after timeout")
+
+
+def test_forward_nvfp4_replays_from_a_cuda_graph():
+    """The NVFP4 forward is launches only, so it can be captured once and replayed: replays on
+    new input contents match eager calls bit for bit."""
+    wl = TINY.with_tokens(300)
+    case = H.make_case(wl)
+    weights = H.device_weights(wl)
+    w4 = H.device_weights_nvfp4(weights)
+    s = bm.shape_of(wl)
+    dev = "cuda"
+    h_static = case.h.to(dev).clone()
+    rw, b = case.router_w.to(dev), case.bias.to(dev)
+    out = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
+    ws = bm.nvfp4_workspace(s)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # the first call sets up per-device state outside the capture
+        bm.beam_moe_forward_nvfp4(s, h_static, rw, b, w4[0], w4[1], out, ws=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        bm.beam_moe_forward_nvfp4(s, h_static, rw, b, w4[0], w4[1], out, ws=ws)
+    for seed in (5, 6):
+        h_new = W.hidden(dataclasses.replace(wl, seed=seed)).to(dev)
+        h_static.copy_(h_new)
+        g.replay()
+        torch.cuda.synchronize()
+        assert bm.beam_moe_sync_status(ws) == bm.BEAM_OK
+        ref = torch.empty_like(out)
+        bm.beam_moe_forward_nvfp4(s, h_new, rw, b, w4[0], w4[1], ref)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), seed
+    del g
+
+
+@pytest.mark.parametrize("i", range(10))
+def test_forward_nvfp4_random_shapes(i):
+    """Seeded random shapes of the fuzz suite (group sizes, lane runs of the selection, ragged
+    m-tiles) with I a multiple of 256."""
+    from tests.test_gpu_fuzz import _shape
+    shape = _shape(i)
+    shape["I"] = 256 if i % 2 == 0 else 512
+    wl = dataclasses.replace(W.WORKLOADS["tiny"], name=f"fuzz_nvfp4_{i}", **shape)
+    case = H.make_case(wl)
+    weights = H.device_weights(wl)
+    w4 = H.device_weights_nvfp4(weights)
+    out, idx, w, _ = H.run_forward_nvfp4(case, w4)
+    _check_routing(case, idx, w)
+    ref = H.oracle_out_nvfp4(case, weights, range(wl.T), w4, batch=64)
+    H.assert_close_out(out.float().cpu().numpy(), ref, f"nvfp4 {shape}")
