@@ -234,6 +234,19 @@ BEAM_API beam_status beam_moe_forward_nvfp4(const beam_moe_shape* shape, const v
                                             int32_t* topk_idx, float* topk_w, void* ws,
                                             size_t ws_bytes, beam_stream stream);
 
+/* beam_moe_block with NVFP4 expert weights (as for beam_moe_forward_nvfp4); every other
+ * argument as for beam_moe_block, with ws sized by beam_moe_nvfp4_workspace_size. */
+BEAM_API beam_status beam_moe_block_nvfp4(const beam_moe_shape* shape, const float* x,
+                                          const float* g_pre, const float* g_post, float eps,
+                                          int32_t k_resid, const float* router_w,
+                                          const float* bias, const void* gate_up_codes,
+                                          const void* gate_up_block_scales,
+                                          const float* gate_up_scales, const void* down_codes,
+                                          const void* down_block_scales,
+                                          const float* down_scales, float* x_out,
+                                          int32_t* topk_idx, float* topk_w, void* ws,
+                                          size_t ws_bytes, beam_stream stream);
+
 /* MoE block: x' = x * sqrt((k_resid-1)/k_resid) + RMSNorm(MoE(bf16(RMSNorm(x) g_pre))) g_post
  *                 / sqrt(k_resid), RMSNorm(v) = v / sqrt(mean(v^2) + eps), all FP32.
  *   x       FP32 [T, d] residual stream in
@@ -280,6 +293,23 @@ BEAM_API beam_status beam_dense_forward_fp8(const beam_dense_shape* shape, const
                                             const void* w_down, const float* down_scale,
                                             void* out, void* ws, size_t ws_bytes,
                                             beam_stream stream);
+
+/* Workspace bytes for beam_dense_forward_nvfp4 (0 for an unsupported shape; I must be a
+ * multiple of 256). */
+BEAM_API size_t beam_dense_nvfp4_workspace_size(const beam_dense_shape* shape);
+
+/* beam_dense_forward with NVFP4 weights written by beam_moe_quantize_nvfp4 with groups = 1:
+ * gate_up_* from (w_gate, w_up) interleaved (codes [2I, d / 2], atoms, row scales [2I]),
+ * down_* from w_down (codes [d, I / 2], atoms, row scales [d]); all 16-byte aligned.  The token
+ * rows and the SwiGLU activation are quantised per row as in beam_moe_forward_nvfp4. */
+BEAM_API beam_status beam_dense_forward_nvfp4(const beam_dense_shape* shape, const void* hidden,
+                                              const void* gate_up_codes,
+                                              const void* gate_up_block_scales,
+                                              const float* gate_up_scales,
+                                              const void* down_codes,
+                                              const void* down_block_scales,
+                                              const float* down_scales, void* out, void* ws,
+                                              size_t ws_bytes, beam_stream stream);
 
 /* Selection-bias update from the expert loads of the last beam_moe_forward / beam_moe_block
  * call made with `ws` (same shape):  bias[e] += gamma * sign(mean_load - load[e]), sign(0) = 0,

@@ -34,7 +34,8 @@ EXPORTED = [
     "beam_moe_get_sm_pairs", "beam_moe_quantize_e4m3", "beam_moe_fp8_workspace_size",
     "beam_moe_forward_fp8", "beam_moe_block_fp8", "beam_dense_fp8_workspace_size",
     "beam_dense_forward_fp8", "beam_moe_quantize_nvfp4", "beam_moe_nvfp4_workspace_size",
-    "beam_moe_forward_nvfp4",
+    "beam_moe_forward_nvfp4", "beam_moe_block_nvfp4", "beam_dense_nvfp4_workspace_size",
+    "beam_dense_forward_nvfp4",
 ]
 
 
@@ -113,6 +114,10 @@ def lib():
     L.beam_moe_nvfp4_workspace_size.argtypes = [shp]
     L.beam_moe_nvfp4_workspace_size.restype = sz
     L.beam_moe_forward_nvfp4.argtypes = [shp] + [vp] * 13 + [sz, vp]
+    L.beam_moe_block_nvfp4.argtypes = [shp, vp, vp, vp, f32, i32] + [vp] * 12 + [sz, vp]
+    L.beam_dense_nvfp4_workspace_size.argtypes = [dshp]
+    L.beam_dense_nvfp4_workspace_size.restype = sz
+    L.beam_dense_forward_nvfp4.argtypes = [dshp] + [vp] * 9 + [sz, vp]
     L.beam_moe_sync_status.argtypes = [vp, vp]
     L.beam_status_string.argtypes = [ctypes.c_int]
     L.beam_status_string.restype = ctypes.c_char_p
@@ -132,7 +137,8 @@ def lib():
                  "beam_moe_sync_status", "beam_dense_forward", "beam_moe_bias_update",
                  "beam_moe_expert_counts", "beam_moe_profile_read", "beam_moe_quantize_e4m3",
                  "beam_moe_forward_fp8", "beam_moe_block_fp8", "beam_dense_forward_fp8",
-                 "beam_moe_quantize_nvfp4", "beam_moe_forward_nvfp4"):
+                 "beam_moe_quantize_nvfp4", "beam_moe_forward_nvfp4", "beam_moe_block_nvfp4",
+                 "beam_dense_forward_nvfp4"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -525,3 +531,61 @@ def beam_moe_profile_read():
         _check(L.beam_moe_profile_read(i, ctypes.byref(n), ctypes.byref(ms)), "beam_moe_profile_read")
         out[name] = (n.value, ms.value)
     return out
+
+
+def beam_moe_block_nvfp4(shape, x, g_pre, g_post, eps, k_resid, router_w, bias, gate_up, down,
+                         x_out, topk_idx=None, topk_w=None, ws=None, stream=None):
+    """beam_moe_block with NVFP4 experts (gate_up, down as for beam_moe_forward_nvfp4)."""
+    T, d, E, k, I = shape.T, shape.d, shape.E, shape.top_k, shape.I
+    gc, ga, gs = gate_up
+    dc, da, ds = down
+    args = [_ptr(x, torch.float32, "x", (T, d)),
+            _ptr(g_pre, torch.float32, "g_pre", (d,)),
+            _ptr(g_post, torch.float32, "g_post", (d,)),
+            ctypes.c_float(eps), ctypes.c_int32(k_resid),
+            _ptr(router_w, torch.float32, "router_w", (E, d)),
+            _ptr(bias, torch.float32, "bias", (E,)),
+            _ptr(gc, torch.uint8, "gate_up codes", (E, 2 * I, d // 2)),
+            _ptr(ga, torch.uint8, "gate_up block scales", (E, 2 * I * (d // 16))),
+            _ptr(gs, torch.float32, "gate_up scales", (E, 2 * I)),
+            _ptr(dc, torch.uint8, "down codes", (E, d, I // 2)),
+            _ptr(da, torch.uint8, "down block scales", (E, d * (I // 16))),
+            _ptr(ds, torch.float32, "down scales", (E, d)),
+            _ptr(x_out, torch.float32, "x_out", (T, d)),
+            _ptr(topk_idx, torch.int32, "topk_idx", (T, k), optional=True),
+            _ptr(topk_w, torch.float32, "topk_w", (T, k), optional=True)]
+    if ws is None:
+        ws = nvfp4_workspace(shape, x.device)
+    _ptr(ws, torch.uint8, "ws")
+    _check(lib().beam_moe_block_nvfp4(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
+                                      _stream(stream)), "beam_moe_block_nvfp4")
+    return ws
+
+
+def dense_nvfp4_workspace(shape: beam_dense_shape, device="cuda") -> torch.Tensor:
+    n = int(lib().beam_dense_nvfp4_workspace_size(ctypes.byref(shape)))
+    if n == 0:
+        raise BeamError(BEAM_ERR_UNSUPPORTED, "beam_dense_nvfp4_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def beam_dense_forward_nvfp4(shape, hidden, gate_up, down, out, ws=None, stream=None):
+    """beam_dense_forward with NVFP4 weights: gate_up = beam_moe_quantize_nvfp4(w_gate[None],
+    w_up[None]), down = beam_moe_quantize_nvfp4(w_down[None])."""
+    T, d, I = shape.T, shape.d, shape.I
+    gc, ga, gs = gate_up
+    dc, da, ds = down
+    args = [_ptr(hidden, torch.bfloat16, "hidden", (T, d)),
+            _ptr(gc, torch.uint8, "gate_up codes", (1, 2 * I, d // 2)),
+            _ptr(ga, torch.uint8, "gate_up block scales", (1, 2 * I * (d // 16))),
+            _ptr(gs, torch.float32, "gate_up scales", (1, 2 * I)),
+            _ptr(dc, torch.uint8, "down codes", (1, d, I // 2)),
+            _ptr(da, torch.uint8, "down block scales", (1, d * (I // 16))),
+            _ptr(ds, torch.float32, "down scales", (1, d)),
+            _ptr(out, torch.bfloat16, "out", (T, d))]
+    if ws is None:
+        ws = dense_nvfp4_workspace(shape, hidden.device)
+    _ptr(ws, torch.uint8, "ws")
+    _check(lib().beam_dense_forward_nvfp4(ctypes.byref(shape), *args, ws.data_ptr(), ws.numel(),
+                                          _stream(stream)), "beam_dense_forward_nvfp4")
+    return ws

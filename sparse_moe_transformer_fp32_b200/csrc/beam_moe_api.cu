@@ -665,6 +665,7 @@ beam_status check_dense_shape(const beam_dense_shape* s) {
 struct DenseLayout {
   size_t status, mt_count, mtiles, act, total;
   size_t hq = 0, hs = 0, act8 = 0, as = 0;  // E4M3 form: quantised rows and their scales
+  size_t hsf = 0, asf = 0;                    // NVFP4 form: block-scale atoms per m-tile
   int64_t mt_cap;
 };
 
@@ -703,6 +704,26 @@ DenseLayout plan_dense_fp8(const beam_dense_shape& s) {
   return L;
 }
 
+// NVFP4 dense MLP: the BF16 layout plus the token rows' codes, row scales and block-scale atoms,
+// and the same for the activation (atoms per 128-row m-tile).
+DenseLayout plan_dense_nvfp4(const beam_dense_shape& s) {
+  DenseLayout L = plan_dense(s);
+  size_t o = L.total;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o = align_up(o + (bytes ? bytes : 1), 1024);
+    return r;
+  };
+  const size_t groups = static_cast<size_t>(L.mt_cap);
+  L.hq = take(static_cast<size_t>(s.T) * (s.d / 2));
+  L.hs = take(sizeof(float) * s.T);
+  L.hsf = take(groups * (s.d / 16) * 128);
+  L.act8 = take(static_cast<size_t>(s.T) * (s.I / 2));
+  L.as = take(sizeof(float) * s.T);
+  L.asf = take(groups * (s.I / 16) * 128);
+  L.total = o;
+  return L;
+}
 
 // ------------------------------------------------------------------ entry-point bodies
 //
@@ -790,13 +811,16 @@ beam_status block_impl(const beam_moe_shape* shape, const float* x, const float*
                        const float* g_post, float eps, int32_t k_resid, const float* router_w,
                        const float* bias, const void* w_gate, const void* w_up,
                        const void* w_down, float* x_out, int32_t* topk_idx, float* topk_w,
-                       void* ws, size_t ws_bytes, beam_stream stream, const Fp8Scales* f8) {
+                       void* ws, size_t ws_bytes, beam_stream stream, const Fp8Scales* f8,
+                       const Nvfp4Weights* w4 = nullptr) {
   beam_status b = check_shape(shape);
   if (b != BEAM_OK) return b;
+  if (w4 && shape->I % kF4KElems != 0) return BEAM_ERR_UNSUPPORTED;
   if (shape->T == 0) return BEAM_OK;  // nothing to read or write
+  // with w4, w_gate / w_up / w_down carry its gate|up codes, gate|up block scales, down codes
   if (any_misaligned({x, g_pre, g_post, router_w, w_gate, w_up, w_down, x_out}) ||
-      misaligned_fp8(f8) || !bias || (topk_idx && !aligned16(topk_idx)) ||
-      (topk_w && !aligned16(topk_w)))
+      misaligned_fp8(f8) || (w4 && any_misaligned({w4->gu_scale, w4->d_sf, w4->d_scale})) ||
+      !bias || (topk_idx && !aligned16(topk_idx)) || (topk_w && !aligned16(topk_w)))
     return BEAM_ERR_INVALID_ARG;
   if (!(eps > 0.f) || !std::isfinite(eps) || k_resid < 1) return BEAM_ERR_INVALID_ARG;
   if (x_out != x) {  // in place or disjoint
@@ -805,7 +829,7 @@ beam_status block_impl(const beam_moe_shape* shape, const float* x, const float*
     const size_t n = sizeof(float) * static_cast<size_t>(shape->T) * shape->d;
     if (a0 < b0 + n && b0 < a0 + n) return BEAM_ERR_INVALID_ARG;
   }
-  const Layout L = f8 ? plan_fp8(*shape) : plan(*shape);
+  const Layout L = w4 ? plan_nvfp4(*shape) : f8 ? plan_fp8(*shape) : plan(*shape);
   if ((b = check_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
   DeviceInfo* dev;
   if ((b = device_info(&dev)) != BEAM_OK) return b;
@@ -824,8 +848,9 @@ beam_status block_impl(const beam_moe_shape* shape, const float* x, const float*
   float* w = topk_w ? topk_w : at<float>(ws, L.w);
   if ((b = run_router(*shape, L, pn.h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
     return b;
-  if ((b = run_experts(*shape, L, *dev, pn.h, idx, w_gate, w_up, w_down, ws, st, f8)) != BEAM_OK)
-    return b;
+  b = w4 ? run_experts_nvfp4(*shape, L, *dev, pn.h, idx, *w4, ws, st)
+         : run_experts(*shape, L, *dev, pn.h, idx, w_gate, w_up, w_down, ws, st, f8);
+  if (b != BEAM_OK) return b;
   const double kk = static_cast<double>(k_resid);
   CombineArgs ca{};
   ca.y = at<__nv_bfloat16>(ws, L.y);
@@ -848,6 +873,101 @@ beam_status block_impl(const beam_moe_shape* shape, const float* x, const float*
 
 // Dense SwiGLU MLP: one "expert" holding every token.  The E4M3 form quantises the token rows
 // and the activation per row, as the MoE path does.
+// Dense SwiGLU MLP on NVFP4 weights: 128-row tiles of consecutive tokens; the token rows are
+// quantised into their tile's atoms by the activation quantiser, then the two block-scaled GEMMs
+// run with the activation quantised between them.
+beam_status dense_nvfp4_impl(const beam_dense_shape* shape, const void* hidden,
+                             const Nvfp4Weights& w4, void* out, void* ws, size_t ws_bytes,
+                             beam_stream stream) {
+  beam_status b = check_dense_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (shape->I % kF4KElems != 0) return BEAM_ERR_UNSUPPORTED;
+  if (shape->T == 0) return BEAM_OK;  // nothing to read or write
+  if (any_misaligned({hidden, w4.gu_codes, w4.gu_sf, w4.gu_scale, w4.d_codes, w4.d_sf,
+                      w4.d_scale, out}))
+    return BEAM_ERR_INVALID_ARG;
+  const DenseLayout L = plan_dense_nvfp4(*shape);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < L.total)
+    return BEAM_ERR_WORKSPACE;
+  DeviceInfo* dev;
+  if ((b = device_info(&dev)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const beam_dense_shape& s = *shape;
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  cudaError_t e = cudaMemsetAsync(status, 0, 16, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  MTile* mtiles = at<MTile>(ws, L.mtiles);
+  int32_t* mt_count = at<int32_t>(ws, L.mt_count);
+  BEAM_LAUNCH(kKDenseTiles, st, launch_dense_tiles(s.T, mtiles, mt_count, st));
+
+  Fp4ActArgs qh{};
+  qh.x = static_cast<const __nv_bfloat16*>(hidden);
+  qh.mtiles = mtiles;
+  qh.mt_count = mt_count;
+  qh.q = at<uint8_t>(ws, L.hq);
+  qh.sf = at<uint8_t>(ws, L.hsf);
+  qh.s = at<float>(ws, L.hs);
+  qh.cols = s.d;
+  qh.mt_cap = static_cast<int>(L.mt_cap);
+  BEAM_LAUNCH(kKQuantizeNvfp4, st, launch_nvfp4_act(qh, st));
+
+  ATensorMaps tm_h, tm_a;
+  CUtensorMap tm_gu, tm_d;
+  for (int i = 0; i < kNumABoxes; ++i) {
+    if ((b = make_map(&tm_h.m[i], qh.q, s.d / 2, s.T, a_box_rows(i), 1)) != BEAM_OK) return b;
+    if ((b = make_map(&tm_a.m[i], at<void>(ws, L.act8), s.I / 2, s.T, a_box_rows(i), 1)) !=
+        BEAM_OK)
+      return b;
+  }
+  if ((b = make_map(&tm_gu, w4.gu_codes, s.d / 2, 2 * static_cast<uint64_t>(s.I), kF4N, 1)) !=
+      BEAM_OK)
+    return b;
+  if ((b = make_map(&tm_d, w4.d_codes, s.I / 2, s.d, kF4N, 1)) != BEAM_OK) return b;
+
+  Fp4GemmArgs g1{};
+  g1.mtiles = mtiles;
+  g1.mt_count = mt_count;
+  g1.out = at<__nv_bfloat16>(ws, L.act);
+  g1.status = status;
+  g1.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  g1.out_ld = s.I;
+  g1.n_tiles_n = 2 * s.I / kF4N;
+  g1.k_blocks = s.d / kF4KElems;
+  g1.b_rows_per_expert = 2 * s.I;
+  g1.a_sf = qh.sf;
+  g1.b_sf = static_cast<const uint8_t*>(w4.gu_sf);
+  g1.a_scale = qh.s;
+  g1.b_scale = w4.gu_scale;
+  const int64_t t1 = L.mt_cap * g1.n_tiles_n;
+  BEAM_LAUNCH(kKGemmGateUp, st,
+              launch_gemm_nvfp4(true, tm_h, tm_gu, g1,
+                                static_cast<int>(t1 < dev->sms ? t1 : dev->sms), st));
+
+  Fp4ActArgs qa = qh;
+  qa.x = g1.out;
+  qa.q = at<uint8_t>(ws, L.act8);
+  qa.sf = at<uint8_t>(ws, L.asf);
+  qa.s = at<float>(ws, L.as);
+  qa.cols = s.I;
+  BEAM_LAUNCH(kKQuantizeNvfp4, st, launch_nvfp4_act(qa, st));
+
+  Fp4GemmArgs g2 = g1;
+  g2.out = static_cast<__nv_bfloat16*>(out);
+  g2.out_ld = s.d;
+  g2.n_tiles_n = s.d / kF4N;
+  g2.k_blocks = s.I / kF4KElems;
+  g2.b_rows_per_expert = s.d;
+  g2.a_sf = qa.sf;
+  g2.b_sf = static_cast<const uint8_t*>(w4.d_sf);
+  g2.a_scale = qa.s;
+  g2.b_scale = w4.d_scale;
+  const int64_t t2 = L.mt_cap * g2.n_tiles_n;
+  BEAM_LAUNCH(kKGemmDown, st,
+              launch_gemm_nvfp4(false, tm_a, tm_d, g2,
+                                static_cast<int>(t2 < dev->sms ? t2 : dev->sms), st));
+  return BEAM_OK;
+}
+
 beam_status dense_impl(const beam_dense_shape* shape, const void* hidden, const void* w_gate,
                        const void* w_up, const void* w_down, void* out, void* ws,
                        size_t ws_bytes, beam_stream stream, const Fp8Scales* f8) {
@@ -1104,6 +1224,36 @@ beam_status beam_moe_forward_fp8(const beam_moe_shape* shape, const void* hidden
   const Fp8Scales f8{gate_scale, up_scale, down_scale};
   return forward_impl(shape, hidden, router_w, bias, w_gate, w_up, w_down, out, topk_idx, topk_w,
                       ws, ws_bytes, stream, &f8);
+}
+
+beam_status beam_moe_block_nvfp4(const beam_moe_shape* shape, const float* x, const float* g_pre,
+                                 const float* g_post, float eps, int32_t k_resid,
+                                 const float* router_w, const float* bias,
+                                 const void* gate_up_codes, const void* gate_up_block_scales,
+                                 const float* gate_up_scales, const void* down_codes,
+                                 const void* down_block_scales, const float* down_scales,
+                                 float* x_out, int32_t* topk_idx, float* topk_w, void* ws,
+                                 size_t ws_bytes, beam_stream stream) {
+  const Nvfp4Weights w4{gate_up_codes, gate_up_block_scales, gate_up_scales,
+                        down_codes,    down_block_scales,    down_scales};
+  return block_impl(shape, x, g_pre, g_post, eps, k_resid, router_w, bias, gate_up_codes,
+                    gate_up_block_scales, down_codes, x_out, topk_idx, topk_w, ws, ws_bytes,
+                    stream, nullptr, &w4);
+}
+
+size_t beam_dense_nvfp4_workspace_size(const beam_dense_shape* shape) {
+  if (check_dense_shape(shape) != BEAM_OK || shape->I % kF4KElems != 0) return 0;
+  return plan_dense_nvfp4(*shape).total;
+}
+
+beam_status beam_dense_forward_nvfp4(const beam_dense_shape* shape, const void* hidden,
+                                     const void* gate_up_codes, const void* gate_up_block_scales,
+                                     const float* gate_up_scales, const void* down_codes,
+                                     const void* down_block_scales, const float* down_scales,
+                                     void* out, void* ws, size_t ws_bytes, beam_stream stream) {
+  const Nvfp4Weights w4{gate_up_codes, gate_up_block_scales, gate_up_scales,
+                        down_codes,    down_block_scales,    down_scales};
+  return dense_nvfp4_impl(shape, hidden, w4, out, ws, ws_bytes, stream);
 }
 
 beam_status beam_moe_block(const beam_moe_shape* shape, const float* x, const float* g_pre,

@@ -239,3 +239,35 @@ def test_nvfp4_entry_points_validate_before_launching(L):
     misaligned[4] = q(A + 4)  # gate_up block scales
     assert fwd(ctypes.byref(beam(64)), *misaligned, 1 << 30, None) == bm.BEAM_ERR_INVALID_ARG
     assert fwd(ctypes.byref(beam(64)), *args[:12], None, 16, None) == bm.BEAM_ERR_WORKSPACE
+
+
+def test_nvfp4_block_and_dense_validate_before_launching(L):
+    A = 1 << 20
+    q = ctypes.c_void_p
+    s = beam(64)
+    blk = L.beam_moe_block_nvfp4
+    base = [q(A)] * 3 + [ctypes.c_float(1e-6), ctypes.c_int32(10)] + [q(A)] * 12
+    assert blk(ctypes.byref(beam(0)), *[None] * 3, ctypes.c_float(1e-6), ctypes.c_int32(10),
+               *[None] * 12, 0, None) == bm.BEAM_OK
+    assert blk(ctypes.byref(beam(64, I=128)), *base, 1 << 30, None) == bm.BEAM_ERR_UNSUPPORTED
+    mis = list(base)
+    mis[10] = q(A + 8)  # down codes
+    assert blk(ctypes.byref(s), *mis, 1 << 30, None) == bm.BEAM_ERR_INVALID_ARG
+    mis = list(base)
+    mis[12] = q(A + 4)  # down row scales
+    assert blk(ctypes.byref(s), *mis, 1 << 30, None) == bm.BEAM_ERR_INVALID_ARG
+    assert blk(ctypes.byref(s), *base[:16], None, 16, None) == bm.BEAM_ERR_WORKSPACE
+
+    ds = bm.dense_shape(256, 5120, 20480)
+    n = bm.lib().beam_dense_nvfp4_workspace_size(ctypes.byref(ds))
+    assert n > bm.lib().beam_dense_workspace_size(ctypes.byref(ds)) + 256 * (2560 + 10240)
+    assert bm.lib().beam_dense_nvfp4_workspace_size(ctypes.byref(bm.dense_shape(4, 256, 128))) == 0
+    dns = L.beam_dense_forward_nvfp4
+    args = [q(A)] * 8  # hidden, 3 gate|up arrays, 3 down arrays, out
+    mis = list(args)
+    mis[3] = q(A + 4)  # gate|up row scales
+    assert dns(ctypes.byref(ds), *mis, q(A), 1 << 30, None) == bm.BEAM_ERR_INVALID_ARG
+    assert dns(ctypes.byref(ds), *args, None, 16, None) == bm.BEAM_ERR_WORKSPACE
+    assert dns(ctypes.byref(bm.dense_shape(0, 5120, 20480)), *[None] * 9, 0, None) == bm.BEAM_OK
+    assert dns(ctypes.byref(bm.dense_shape(4, 256, 128)), *args, q(A), 1 << 30, None) == \
+        bm.BEAM_ERR_UNSUPPORTED

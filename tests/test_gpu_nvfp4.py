@@ -259,3 +259,45 @@ def test_forward_nvfp4_random_shapes(i):
     _check_routing(case, idx, w)
     ref = H.oracle_out_nvfp4(case, weights, range(wl.T), w4, batch=64)
     H.assert_close_out(out.float().cpu().numpy(), ref, f"nvfp4 {shape}")
+
+
+def test_block_nvfp4_every_token():
+    wl = dataclasses.replace(TINY, block=True, T=96)
+    case = H.make_case(wl)
+    weights = H.device_weights(wl)
+    w4 = H.device_weights_nvfp4(weights)
+    s = bm.shape_of(wl)
+    dev = "cuda"
+    x = case.x.to(dev)
+    x_out = torch.empty_like(x)
+    idx = torch.empty(wl.T, wl.top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(wl.T, wl.top_k, dtype=torch.float32, device=dev)
+    ws = bm.beam_moe_block_nvfp4(s, x, case.g_pre.to(dev), case.g_post.to(dev), wl.eps,
+                                 wl.k_resid, case.router_w.to(dev), case.bias.to(dev), w4[0],
+                                 w4[1], x_out, idx, w)
+    assert bm.beam_moe_sync_status(ws) == bm.BEAM_OK
+    _check_routing(case, idx, w)
+    moe = H.oracle_out_nvfp4(case, weights, range(wl.T), w4, batch=96)
+    ref = oracle.block_tail(case.x, moe, case.g_post, wl.eps, wl.k_resid)
+    cx, cf = oracle.residual_coefficients(wl.k_resid)
+    got = x_out.cpu().numpy()
+    # the residual term dominates x'; compare the MoE contribution
+    H.assert_close_out((got - cx * case.x.numpy()) / cf, (ref - cx * case.x.numpy()) / cf,
+                       "nvfp4 block")
+
+
+@pytest.mark.parametrize("T,d,I", [(200, 256, 1024), (1, 512, 512), (129, 5120, 20480)])
+def test_dense_nvfp4_every_token(T, d, I):
+    wl = dataclasses.replace(W.WORKLOADS["dense"], T=T, d=d, I=I)
+    h = W.hidden(wl)
+    mats = tuple(W.expert_weight(wl, m, 0, "cuda") for m in ("gate", "up", "down"))
+    w4 = (bm.beam_moe_quantize_nvfp4(mats[0][None], mats[1][None]),
+          bm.beam_moe_quantize_nvfp4(mats[2][None]))
+    out = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    s = bm.dense_shape(T, d, I)
+    ws = bm.beam_dense_forward_nvfp4(s, h.cuda(), w4[0], w4[1], out)
+    assert bm.beam_moe_sync_status(ws) == bm.BEAM_OK
+    ref_w = H.oracle_experts_nvfp4(tuple(m[None] for m in mats), [0], w4)[0]
+    toks = list(range(T)) if T <= 200 else sorted({0, T - 1, 1, T // 2, T // 3, 2 * T // 3})
+    ref = np.stack([oracle.expert_mlp_nvfp4(h[t], *ref_w) for t in toks])
+    H.assert_close_out(out[toks].float().cpu().numpy(), ref, f"nvfp4 dense T={T} d={d} I={I}")
