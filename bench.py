@@ -68,7 +68,8 @@ def parse_args(argv=None):
     p.add_argument("--fp8", action="store_true",
                    help="E4M3 expert weights (beam_moe_forward_fp8); layer workloads only")
     p.add_argument("--nvfp4", action="store_true",
-                   help="NVFP4 expert weights (beam_moe_forward_nvfp4); layer workloads only")
+                   help="NVFP4 expert weights (beam_moe_forward_nvfp4, _block_nvfp4, "
+                        "beam_dense_forward_nvfp4)")
     p.add_argument("--route-only", action="store_true",
                    help="time beam_moe_route alone (router profiling; not the layer metric)")
     p.add_argument("--dry-run", action="store_true",
@@ -76,9 +77,8 @@ def parse_args(argv=None):
     args = p.parse_args(argv)
     if args.warmup < 3 and not args.dry_run:
         p.error("--warmup must be >= 3")
-    if args.nvfp4 and (args.fp8 or W.WORKLOADS[args.workload].block
-                       or W.WORKLOADS[args.workload].dense):
-        p.error("--nvfp4 runs the layer workloads with NVFP4 weights only")
+    if args.nvfp4 and args.fp8:
+        p.error("--nvfp4 and --fp8 are exclusive")
     return args
 
 
@@ -264,6 +264,9 @@ def kernel_work(wl, touched: int, fp8: bool = False, nvfp4: bool = False):
             "expert_gemm_down": {"flops": 2 * R * d * I,
                                  "bytes": touched * d * I * q + R * I * q + R * d * bf},
             "combine": {"flops": 2 * R * d, "bytes": R * d * bf + T * d * bf},
+            "combine_block": {"flops": 2 * R * d, "bytes": R * d * bf + 3 * T * d * f4},
+            "prenorm": {"flops": 3 * T * d, "bytes": T * d * f4 + T * d * bf},
+            "dense_tiles": {"flops": 0, "bytes": 16 * (T // 128 + 1)},
         }
     if fp8:
         q = 1
@@ -456,10 +459,10 @@ def run_cuda(args, rank, world, local):
             for m in weights:
                 fp8 += list(bm.beam_moe_quantize_e4m3(m[0] if wl.dense else m))
             torch.cuda.synchronize(dev)
-        if wl.dense:
+        if wl.dense and not fp4:
             ws = bm.dense_fp8_workspace(ds, dev) if fp8 else bm.dense_workspace(ds, dev)
         elif fp4:
-            ws = bm.nvfp4_workspace(s, dev)
+            ws = bm.dense_nvfp4_workspace(ds, dev) if wl.dense else bm.nvfp4_workspace(s, dev)
         else:
             ws = bm.fp8_workspace(s, dev) if fp8 else bm.workspace(s, dev)
         stream = torch.cuda.current_stream(dev)
@@ -467,7 +470,12 @@ def run_cuda(args, rank, world, local):
         def step(src=None, dst=None):
             src = inp if src is None else src
             dst = res if dst is None else dst
-            if wl.dense and fp8:
+            if wl.dense and fp4:
+                bm.beam_dense_forward_nvfp4(ds, src, fp4[0], fp4[1], dst, ws=ws)
+            elif wl.block and fp4:
+                bm.beam_moe_block_nvfp4(s, src, g_pre, g_post, wl.eps, wl.k_resid, router_w, bias,
+                                        fp4[0], fp4[1], dst, ws=ws)
+            elif wl.dense and fp8:
                 bm.beam_dense_forward_fp8(ds, src, *fp8, dst, ws=ws)
             elif wl.dense:
                 bm.beam_dense_forward(ds, src, weights[0][0], weights[1][0], weights[2][0], dst,
@@ -622,7 +630,7 @@ def run_cuda(args, rank, world, local):
             bytes_step = layer_min_bytes(wl, touched, fp8=bool(fp8), nvfp4=bool(fp4))
             cpu = None
             result_extra = {}
-            if fp4 and not args.no_cpu_baseline and world == 1:
+            if fp4 and not args.no_cpu_baseline and world == 1 and not (wl.dense or wl.block):
                 n_cpu = min(args.cpu_sample_tokens, 16)
                 rate, secs, cores = oracle_nvfp4_sample_rate(
                     wl, W.router_weight(wl), W.router_bias(wl), inp_cpu, weights, n_cpu)
