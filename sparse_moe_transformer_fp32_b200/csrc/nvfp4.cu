@@ -199,25 +199,29 @@ __global__ void __launch_bounds__(256) nvfp4_permute_kernel(const Fp4PermuteArgs
   }
 }
 
-// One CTA per m-tile, a warp per row: the activation rows of the tile quantised in place of
-// their m-tile's block-scale atoms.
+// Rows of an m-tile quantised into the tile's block-scale atoms: 16 CTAs per m-tile, each
+// taking 8 of its 128 rows, a warp per row (a CTA per tile alone leaves most SMs idle when the
+// tiles are few and the rows long, as in the dense MLP).
+constexpr int kActRowsPerCta = 8;
+constexpr int kActCtasPerTile = kBM / kActRowsPerCta;
+
 __global__ void __launch_bounds__(256) nvfp4_act_kernel(const Fp4ActArgs a) {
-  const int mt = blockIdx.x;
+  const int mt = static_cast<int>(blockIdx.x / kActCtasPerTile);
   if (mt >= *a.mt_count) return;
   const MTile tile = a.mtiles[mt];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = static_cast<int>(blockIdx.x % kActCtasPerTile) * kActRowsPerCta + warp;
+  if (r >= tile.nrows) return;  // uniform over the warp
   uint8_t* atoms = a.sf + static_cast<int64_t>(mt) * (a.cols / 16) * 128;
-  for (int r = warp; r < tile.nrows; r += 8) {
-    const int64_t row = tile.row0 + r;
-    const uint4* src = reinterpret_cast<const uint4*>(a.x + row * a.cols);
-    const float s = nvfp4_row_scale(src, a.cols / 8, lane);
-    if (lane == 0) a.s[row] = s;
-    uint2* dst = reinterpret_cast<uint2*>(a.q + row * (a.cols / 2));
-    for (int jb = lane; jb < a.cols / 16; jb += 32) {
-      uint8_t bs;
-      dst[jb] = nvfp4_block(src[2 * jb], src[2 * jb + 1], s, bs);
-      atoms[nvfp4_sf_offset(r, jb)] = bs;
-    }
+  const int64_t row = tile.row0 + r;
+  const uint4* src = reinterpret_cast<const uint4*>(a.x + row * a.cols);
+  const float s = nvfp4_row_scale(src, a.cols / 8, lane);
+  if (lane == 0) a.s[row] = s;
+  uint2* dst = reinterpret_cast<uint2*>(a.q + row * (a.cols / 2));
+  for (int jb = lane; jb < a.cols / 16; jb += 32) {
+    uint8_t bs;
+    dst[jb] = nvfp4_block(src[2 * jb], src[2 * jb + 1], s, bs);
+    atoms[nvfp4_sf_offset(r, jb)] = bs;
   }
 }
 
@@ -571,7 +575,9 @@ cudaError_t launch_nvfp4_permute(const Fp4PermuteArgs& a, cudaStream_t s) {
 
 cudaError_t launch_nvfp4_act(const Fp4ActArgs& a, cudaStream_t s) {
   if (a.mt_cap <= 0) return cudaSuccess;
-  nvfp4_act_kernel<<<a.mt_cap, 256, 0, s>>>(a);
+  const int64_t blocks = static_cast<int64_t>(a.mt_cap) * kActCtasPerTile;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  nvfp4_act_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
