@@ -35,8 +35,12 @@
  *    so results are deterministic run to run.
  *  - Supported shapes: d % 256 == 0, d <= 8192, I % 128 == 0, 1 <= E <= 256,
  *    E % 4 == 0, E % n_group == 0, n_group <= 32, 1 <= topk_group <= n_group, 1 <= top_k <= 8,
- *    top_k <= topk_group * E / n_group, T >= 0, T * top_k < 2^31.  Others return
- *    BEAM_ERR_UNSUPPORTED.  T == 0 is a no-op that reads no pointer (they may be NULL).
+ *    top_k <= topk_group * E / n_group, T >= 0, T * top_k < 2^31; the NVFP4 entry points
+ *    also need I % 256 == 0.  Others return BEAM_ERR_UNSUPPORTED.  T == 0 is a no-op that
+ *    reads no pointer (they may be NULL).
+ *  - Expert weights come in three forms with the same entry-point structure: BF16
+ *    (beam_moe_forward / _block, beam_dense_forward), E4M3 with FP32 row scales (the _fp8
+ *    forms) and NVFP4 with E4M3 block scales and FP32 row scales (the _nvfp4 forms).
  */
 #ifndef BEAM_MOE_H_
 #define BEAM_MOE_H_
