@@ -36,3 +36,29 @@ def test_reference_arm_other_ranks_exit_quietly():
                        capture_output=True, text=True, timeout=120, cwd=ROOT, env=env)
     assert p.returncode == 0, p.stderr[-2000:]
     assert p.stdout.strip() == ""
+
+
+def _reference_line(*extra):
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--steps", "3", "--warmup", "3",
+                        "--cpu-sample-tokens", "4", *extra],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [l for l in p.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, p.stdout
+    return json.loads(lines[0])
+
+
+def test_reference_arm_line_carries_the_contract_keys():
+    for extra, metric_word in (((), "BF16"), (("--fp8",), "E4M3"), (("--nvfp4",), "NVFP4")):
+        r = _reference_line(*extra)
+        assert r["impl"] == "reference" and metric_word in r["metric"]
+        assert r["unit"] == "tokens/s" and r["value"] > 0 and r["higher_is_better"] is True
+        assert r["steps"] == 3 and r["warmup"] == 3 and r["n_gpus"] == 1
+        assert r["dtype"] == "f64" and r["data"] == "synthetic"
+        assert r["config"]["workload"].startswith("tiny")
+        cb = r["cpu_baseline"]
+        assert cb["kind"] == "oracle" and cb["value"] == r["value"] and cb["cores"] >= 1
+        assert "4 tokens" in cb["sample"]
+        assert r["e2e"] == {"value": r["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                            "d2h_bytes_per_step": 0}
