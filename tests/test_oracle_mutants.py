@@ -103,6 +103,7 @@ PIN_TESTS = [
     (fp4.test_e2m1_encode_is_nearest_with_ties_to_even_and_saturates, [()]),
     (fp4.test_quantize_rows_nvfp4_is_exact_on_representable_rows, [()]),
     (fp4.test_quantize_rows_nvfp4_error_bounds_and_block_maxima, [()]),
+    (fp4.test_quantize_rows_nvfp4_symmetries, [()]),
     (fp4.test_linear_nvfp4_matches_float64_on_decoded_operands, [()]),
     (fp4.test_linear_nvfp4_equals_router_logits_on_exact_operands, [()]),
     (fp4.test_expert_mlp_nvfp4_gate_up_equal_bf16_expert_on_exact_operands, [()]),

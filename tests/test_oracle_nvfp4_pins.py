@@ -223,3 +223,26 @@ def test_moe_tokens_nvfp4_is_weighted_sum_of_nvfp4_experts():
         ys = [oracle.expert_mlp_nvfp4(h[t], *experts[e]).astype(np.float64) for e in idx[t]]
         ref = sum(float(w[t, j]) * ys[j] for j in range(k))
         assert np.array_equal(out[t], ref.astype(np.float32))
+
+
+def test_quantize_rows_nvfp4_symmetries():
+    """Exact symmetries of the reading: a power-of-two factor on a row moves only its row scale;
+    negating a row flips only the code signs; permuting whole 16-element blocks permutes the
+    codes and block scales with them."""
+    rng = np.random.default_rng(29)
+    x = rng.normal(0, 1, (16, 256)).astype(np.float32)
+    x[2, :16] *= 1e-3                   # a block far below the row maximum
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    q, bs, s = oracle.quantize_rows_nvfp4(xb)
+    for k in (-7, 3, 11):
+        q2, bs2, s2 = oracle.quantize_rows_nvfp4((xb.float() * 2.0 ** k).to(torch.bfloat16))
+        assert np.array_equal(q2, q) and np.array_equal(bs2, bs)
+        assert np.array_equal(s2, (s.astype(np.float64) * 2.0 ** k).astype(np.float32))
+    qn, bsn, sn = oracle.quantize_rows_nvfp4(-xb)
+    assert np.array_equal(bsn, bs) and np.array_equal(sn, s)
+    assert np.array_equal(oracle.e2m1_to_f32(qn), -oracle.e2m1_to_f32(q))
+    perm = rng.permutation(16)
+    xp = xb.reshape(16, 16, 16)[:, perm].reshape(16, 256)
+    qp, bsp, sp = oracle.quantize_rows_nvfp4(xp)
+    assert np.array_equal(sp, s) and np.array_equal(bsp, bs[:, perm])
+    assert np.array_equal(qp, q.reshape(16, 16, 16)[:, perm].reshape(16, 256))
