@@ -30,6 +30,9 @@
  *    are recorded in a status word inside `ws` and read by beam_moe_sync_status().
  *  - One workspace serves one call at a time: calls that share a workspace must be
  *    ordered on one stream.
+ *  - The first call on each device sets the GEMM kernels' shared-memory limits (make it
+ *    outside any stream capture); this per-device set-up lasts for the process and does not
+ *    survive cudaDeviceReset, so reset a device only when done with the library on it.
  *  - Outputs topk_idx [T, top_k] list the chosen experts in ascending id order; topk_w
  *    [T, top_k] holds their weights in the same order; the combine sums in that order,
  *    so results are deterministic run to run.
@@ -115,7 +118,12 @@ BEAM_API beam_status beam_moe_route(const beam_moe_shape* shape, const void* hid
  * stream capture.  All calls share the array and it keeps the last call's contents (each call
  * clears what must start at zero): calls that overlap on the GPU -- on different streams, or
  * from different host threads -- race on it and must be serialised by the caller.
- * Arguments, layouts and outputs are those of beam_moe_route. */
+ * Arguments, layouts and outputs are those of beam_moe_route.  With no workspace there is no
+ * status word to read back: the one device-side check of the router (a token left with fewer
+ * than top_k candidate experts, which a supported shape with finite logits never produces)
+ * shows only in its outputs, whose missing entries are expert 0 with weight 0.  The cached
+ * array address belongs to the device's current context: cudaDeviceReset invalidates it (as it
+ * does the library's other per-device set-up), so reset a device only when done with it. */
 BEAM_API beam_status beam_moe_route_static(const beam_moe_shape* shape, const void* hidden,
                                            const float* router_w, const float* bias,
                                            int32_t* topk_idx, float* topk_w, float* logits_out,
@@ -341,6 +349,14 @@ BEAM_API const char* beam_moe_last_cuda_error(void);
  * `stream` and copies E int32 values to the HOST buffer counts_host). */
 BEAM_API beam_status beam_moe_expert_counts(const beam_moe_shape* shape, const void* ws,
                                    int32_t* counts_host, beam_stream stream);
+
+/* Row of every (token, slot) pair in the expert-contiguous buffers of the last forward/block
+ * call that used `ws` (synchronises `stream` and copies T * top_k int32 values, slot order as
+ * topk_idx, to the HOST buffer rows_host).  Expert e owns rows off[e] .. off[e+1]-1, where
+ * off is the exclusive prefix sum of the per-expert counts over ascending e, and inside them
+ * its tokens sit in ascending token order: the layout is a function of the routing alone. */
+BEAM_API beam_status beam_moe_slot_rows(const beam_moe_shape* shape, const void* ws,
+                                        int32_t* rows_host, beam_stream stream);
 
 /* ---- diagnostics (process-wide settings) ---- */
 

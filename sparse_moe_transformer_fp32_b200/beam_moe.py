@@ -35,7 +35,7 @@ EXPORTED = [
     "beam_moe_forward_fp8", "beam_moe_block_fp8", "beam_dense_fp8_workspace_size",
     "beam_dense_forward_fp8", "beam_moe_quantize_nvfp4", "beam_moe_nvfp4_workspace_size",
     "beam_moe_forward_nvfp4", "beam_moe_block_nvfp4", "beam_dense_nvfp4_workspace_size",
-    "beam_dense_forward_nvfp4",
+    "beam_dense_forward_nvfp4", "beam_moe_slot_rows",
 ]
 
 
@@ -123,6 +123,7 @@ def lib():
     L.beam_status_string.restype = ctypes.c_char_p
     L.beam_moe_last_cuda_error.restype = ctypes.c_char_p
     L.beam_moe_expert_counts.argtypes = [shp, vp, vp, vp]
+    L.beam_moe_slot_rows.argtypes = [shp, vp, vp, vp]
     L.beam_moe_set_wait_limit_ns.argtypes = [u64]
     L.beam_moe_get_wait_limit_ns.restype = u64
     L.beam_moe_launch_count.restype = u64
@@ -138,7 +139,7 @@ def lib():
                  "beam_moe_expert_counts", "beam_moe_profile_read", "beam_moe_quantize_e4m3",
                  "beam_moe_forward_fp8", "beam_moe_block_fp8", "beam_dense_forward_fp8",
                  "beam_moe_quantize_nvfp4", "beam_moe_forward_nvfp4", "beam_moe_block_nvfp4",
-                 "beam_dense_forward_nvfp4"):
+                 "beam_dense_forward_nvfp4", "beam_moe_slot_rows"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -486,6 +487,13 @@ def beam_moe_expert_counts(shape, ws, stream=None) -> torch.Tensor:
     out = torch.empty(shape.E, dtype=torch.int32)
     _check(lib().beam_moe_expert_counts(ctypes.byref(shape), _ptr(ws, torch.uint8, "ws"),
                                         out.data_ptr(), _stream(stream)), "beam_moe_expert_counts")
+    return out
+
+
+def beam_moe_slot_rows(shape, ws, stream=None) -> torch.Tensor:
+    out = torch.empty(shape.T, shape.top_k, dtype=torch.int32)
+    _check(lib().beam_moe_slot_rows(ctypes.byref(shape), _ptr(ws, torch.uint8, "ws"),
+                                    out.data_ptr(), _stream(stream)), "beam_moe_slot_rows")
     return out
 
 

@@ -130,7 +130,10 @@ beam_status check_shape(const beam_moe_shape* s) {
 }
 
 struct Layout {
-  size_t status, cnt, off, mt_count, mtiles, rank, rowmap, idx, w, wt, part, h, xp, act, y, total;
+  size_t status, cnt, bits, off, mt_count, mtiles, base, rowmap, idx, w, wt, part, h, xp, act, y,
+      total;
+  size_t zero_bytes = 0;             // status, counts and token bitmap: cleared at each call
+  int words = 0;                     // token bitmap words per expert, ceil(T / 32)
   size_t xs = 0, act8 = 0, as = 0;  // FP8 path: row scales of Xp, E4M3 act, act row scales
   size_t xsf = 0, asf = 0;           // NVFP4 path: block-scale atoms of Xp and of the act
   int S, kchunk;
@@ -181,12 +184,16 @@ Layout plan(const beam_moe_shape& s) {
     o = align_up(o + (bytes ? bytes : 1), 1024);
     return r;
   };
+  L.words = static_cast<int>(ceil_div(T, 32));
+  const size_t bitmap_bytes = sizeof(uint32_t) * static_cast<size_t>(s.E) * L.words;
   L.status = take(256);
   L.cnt = take(sizeof(int32_t) * s.E);
+  L.bits = take(bitmap_bytes);
+  L.zero_bytes = L.bits + bitmap_bytes;  // status, counts and bitmap are contiguous from 0
   L.off = take(sizeof(int32_t) * (s.E + 1));
   L.mt_count = take(16);
   L.mtiles = take(sizeof(MTile) * L.mt_cap);
-  L.rank = take(sizeof(int32_t) * R);
+  L.base = take(bitmap_bytes);
   L.rowmap = take(sizeof(int32_t) * R);
   L.idx = take(sizeof(int32_t) * R);
   L.w = take(sizeof(float) * R);
@@ -334,13 +341,14 @@ beam_status run_router(const beam_moe_shape& s, const Layout& L, const __nv_bflo
   ga.h = h;
   ga.WT = at<float>(ws, L.wt);
   ga.part = at<float>(ws, L.part);
-  ga.zero_counts = at<int32_t>(ws, L.cnt);
+  ga.zero_counts = nullptr;
   ga.T = s.T;
   ga.d = s.d;
   ga.E = s.E;
   ga.kchunk = L.kchunk;
-  // the status words reflect the latest call: cleared before the first kernel runs
-  cudaError_t e = cudaMemsetAsync(at<uint32_t>(ws, L.status), 0, 16, st);
+  // the status words reflect the latest call: cleared before the first kernel runs, together
+  // with the dispatch's counts and token bitmap
+  cudaError_t e = cudaMemsetAsync(at<uint32_t>(ws, L.status), 0, dispatch ? L.zero_bytes : 16, st);
   if (e != cudaSuccess) return cuda_fail(e);
   BEAM_LAUNCH(kKRouterTranspose, st,
               launch_router_transpose(router_w, at<float>(ws, L.wt), s.E, s.d, st));
@@ -353,7 +361,8 @@ beam_status run_router(const beam_moe_shape& s, const Layout& L, const __nv_bflo
   sa.idx = idx;
   sa.w = w;
   sa.cnt = dispatch ? at<int32_t>(ws, L.cnt) : nullptr;
-  sa.rank = dispatch ? at<int32_t>(ws, L.rank) : nullptr;
+  sa.bits = dispatch ? at<uint32_t>(ws, L.bits) : nullptr;
+  sa.words = L.words;
   sa.status = at<uint32_t>(ws, L.status);
   sa.S = L.S;
   sa.T = s.T;
@@ -390,17 +399,22 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
                      dev.pair_grid >= 2;
   DispatchArgs da{};
   da.cnt = at<int32_t>(ws, L.cnt);
+  da.bits = at<uint32_t>(ws, L.bits);
+  da.base = at<int32_t>(ws, L.base);
   da.off = at<int32_t>(ws, L.off);
   da.mt_count = at<int32_t>(ws, L.mt_count);
   da.mtiles = at<MTile>(ws, L.mtiles);
   da.E = s.E;
+  da.words = L.words;
   da.tile_rows = pairs ? 2 * kBM : kBM;
   BEAM_LAUNCH(kKDispatchScan, st, launch_dispatch_scan(da, st));
 
   PermuteArgs pa{};
   pa.h = h;
   pa.idx = idx;
-  pa.rank = at<int32_t>(ws, L.rank);
+  pa.bits = da.bits;
+  pa.base = da.base;
+  pa.words = L.words;
   pa.off = da.off;
   pa.rowmap = at<int32_t>(ws, L.rowmap);
   pa.xp = f8 ? nullptr : at<__nv_bfloat16>(ws, L.xp);
@@ -510,17 +524,22 @@ beam_status run_experts_nvfp4(const beam_moe_shape& s, const Layout& L, const De
   uint32_t* status = at<uint32_t>(ws, L.status);
   DispatchArgs da{};
   da.cnt = at<int32_t>(ws, L.cnt);
+  da.bits = at<uint32_t>(ws, L.bits);
+  da.base = at<int32_t>(ws, L.base);
   da.off = at<int32_t>(ws, L.off);
   da.mt_count = at<int32_t>(ws, L.mt_count);
   da.mtiles = at<MTile>(ws, L.mtiles);
   da.E = s.E;
+  da.words = L.words;
   da.tile_rows = kBM;
   BEAM_LAUNCH(kKDispatchScan, st, launch_dispatch_scan(da, st));
 
   Fp4PermuteArgs pa{};
   pa.h = h;
   pa.idx = idx;
-  pa.rank = at<int32_t>(ws, L.rank);
+  pa.bits = da.bits;
+  pa.base = da.base;
+  pa.words = L.words;
   pa.cnt = da.cnt;
   pa.off = da.off;
   pa.rowmap = at<int32_t>(ws, L.rowmap);
@@ -1344,6 +1363,21 @@ beam_status beam_moe_expert_counts(const beam_moe_shape* shape, const void* ws,
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaMemcpy(counts_host, static_cast<const char*>(ws) + L.cnt, sizeof(int32_t) * shape->E,
                  cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return BEAM_OK;
+}
+
+beam_status beam_moe_slot_rows(const beam_moe_shape* shape, const void* ws, int32_t* rows_host,
+                               beam_stream stream) {
+  beam_status b = check_shape(shape);
+  if (b != BEAM_OK) return b;
+  if (!ws || !rows_host) return BEAM_ERR_INVALID_ARG;
+  if (shape->T == 0) return BEAM_OK;
+  const Layout L = plan(*shape);
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaMemcpy(rows_host, static_cast<const char*>(ws) + L.rowmap,
+                 sizeof(int32_t) * static_cast<size_t>(L.R), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e);
   return BEAM_OK;
 }

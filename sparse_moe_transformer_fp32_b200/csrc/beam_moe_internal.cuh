@@ -85,14 +85,19 @@ struct RouterGemmArgs {
   int T, d, E, kchunk;
 };
 
+// The token bitmap of a dispatch: bit (t % 32) of word bits[e * words + t / 32] is set when token
+// t chose expert e (words = ceil(T / 32) per expert).  Its per-expert prefix counts give every
+// (token, expert) slot its rank among the expert's rows in ascending token order, so the row
+// layout of the expert-contiguous buffers does not depend on the order in which CTAs run.
 struct SelectArgs {
   const float* part;  // [S, T, E]
   const float* bias;  // [E]
   float* logits_out;  // [T, E] or null
   int32_t* idx;       // [T, k]
   float* w;           // [T, k]
-  int32_t* cnt;       // [E] or null (no dispatch)
-  int32_t* rank;      // [T, k] or null
+  int32_t* cnt;       // [E] or null (no dispatch); zeroed before the call
+  uint32_t* bits;     // [E, words] token bitmap (dispatch only); zeroed before the call
+  int words;
   uint32_t* status;
   int S, T, E, G, Gk, k;
   float scale;
@@ -100,18 +105,22 @@ struct SelectArgs {
 };
 
 struct DispatchArgs {
-  const int32_t* cnt;   // [E]
-  int32_t* off;         // [E + 1]
-  int32_t* mt_count;    // [1] number of m-tiles
-  MTile* mtiles;        // [capacity]
-  int E;
-  int tile_rows;        // rows per m-tile: 128 (one SM) or 256 (an SM pair)
+  const int32_t* cnt;    // [E]
+  const uint32_t* bits;  // [E, words] token bitmap
+  int32_t* base;         // [E, words] out: set bits of the expert's earlier words
+  int32_t* off;          // [E + 1]
+  int32_t* mt_count;     // [1] number of m-tiles
+  MTile* mtiles;         // [capacity]
+  int E, words;
+  int tile_rows;         // rows per m-tile: 128 (one SM) or 256 (an SM pair)
 };
 
 struct PermuteArgs {
   const __nv_bfloat16* h;  // [T, d]
   const int32_t* idx;      // [T, k]
-  const int32_t* rank;     // [T, k]
+  const uint32_t* bits;    // [E, words] token bitmap
+  const int32_t* base;     // [E, words] its per-expert prefix counts
+  int words;
   const int32_t* off;      // [E + 1]
   int32_t* rowmap;         // [T, k] out: row of slot (t, j) in the expert-contiguous buffers
   __nv_bfloat16* xp;       // [R, d] out (BF16 path), or null
@@ -198,6 +207,17 @@ __device__ __forceinline__ void record_status(uint32_t* status, uint32_t code, u
     status[1] = where;
     status[2] = blockIdx.x;
   }
+}
+
+// Rank of token t among the rows of expert e (ascending token order), from the dispatch's token
+// bitmap and its prefix counts; -1 when t did not choose e.
+__device__ __forceinline__ int slot_rank(const uint32_t* bits, const int32_t* base, int words,
+                                         int e, int t) {
+  const size_t i = static_cast<size_t>(e) * words + (t >> 5);
+  const uint32_t w = bits[i];
+  const uint32_t b = 1u << (t & 31);
+  if (!(w & b)) return -1;
+  return base[i] + __popc(w & (b - 1u));
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

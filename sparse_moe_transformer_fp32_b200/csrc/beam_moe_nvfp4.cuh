@@ -50,7 +50,9 @@ struct Fp4GemmArgs {
 struct Fp4PermuteArgs {
   const __nv_bfloat16* h;  // [T, d]
   const int32_t* idx;      // [T, k]
-  const int32_t* rank;     // [T, k]
+  const uint32_t* bits;    // [E, words] token bitmap
+  const int32_t* base;     // [E, words] its per-expert prefix counts
+  int words;
   const int32_t* cnt;      // [E]
   const int32_t* off;      // [E + 1]
   int32_t* rowmap;         // [T, k] out

@@ -1,12 +1,14 @@
-// Dispatch of token slots to experts: per-expert offsets and the m-tile list (one CTA), then
-// the gather of each token's hidden row into the expert-contiguous buffer Xp.
+// Dispatch of token slots to experts: per-expert offsets, the m-tile list and the prefix counts
+// of the token bitmap (a warp per expert), then the gather of each token's hidden row into the
+// expert-contiguous buffer Xp.
 //
 // The pages say only that tokens are sent to the experts (and, under expert parallelism, to the
 // GPUs) that hold them ("Use HF Transformers", section Parallelism).  Here the (token, slot)
-// pairs are laid out expert by expert: expert e owns rows off[e] .. off[e+1]-1, and within an
-// expert the order is the arrival order of the selection kernel's atomic counter.  Row order
-// inside an expert does not change any result: every row is computed independently and the
-// combine reads rows back through rowmap in a fixed slot order.
+// pairs are laid out expert by expert: expert e owns rows off[e] .. off[e+1]-1, in ascending
+// token order (the rank of token t among e's rows is the number of set bits before bit t in e's
+// row of the token bitmap).  The layout is therefore a function of the routing alone; no result
+// depends on it in any case, since every row is computed independently and the combine reads
+// rows back through rowmap in a fixed slot order.
 #include "beam_moe_internal.cuh"
 
 #include <cuda_fp8.h>
@@ -14,43 +16,53 @@
 namespace beam {
 namespace {
 
-// Inclusive scan of one int per thread over a block of 256 threads.
-__device__ __forceinline__ int block_inclusive_scan(int v, int* warp_tot) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(0xffffffffu, v, off);
-    if (lane >= off) v += o;
-  }
-  if (lane == 31) warp_tot[warp] = v;
-  __syncthreads();
-  int base = 0;
-  for (int w = 0; w < warp; ++w) base += warp_tot[w];
-  __syncthreads();
-  return v + base;
-}
-
+// A warp per expert e: the rows and m-tiles of the experts before e give its offset and its
+// first m-tile; the exclusive prefix counts of its row of the token bitmap give each of its
+// tokens a rank.
 __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a) {
-  __shared__ int warp_tot[8];
-  const int e = threadIdx.x;
-  const int c = e < a.E ? a.cnt[e] : 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 8 + warp;
+  if (e >= a.E) return;  // uniform over the warp
   const int tr = a.tile_rows;
-  const int m = (c + tr - 1) / tr;
-  const int c_incl = block_inclusive_scan(c, warp_tot);
-  const int m_incl = block_inclusive_scan(m, warp_tot);
-  const int c_excl = c_incl - c, m_excl = m_incl - m;
-  if (e < a.E) a.off[e] = c_excl;
-  if (e == a.E - 1) {
-    a.off[a.E] = c_incl;
-    *a.mt_count = m_incl;
+  int c_before = 0, m_before = 0;
+  for (int i = lane; i < e; i += 32) {
+    const int c = a.cnt[i];
+    c_before += c;
+    m_before += (c + tr - 1) / tr;
   }
-  for (int i = 0; i < m; ++i) {
+  c_before = __reduce_add_sync(0xffffffffu, c_before);
+  m_before = __reduce_add_sync(0xffffffffu, m_before);
+  const int c = a.cnt[e];
+  const int m = (c + tr - 1) / tr;
+  if (lane == 0) {
+    a.off[e] = c_before;
+    if (e == a.E - 1) {
+      a.off[a.E] = c_before + c;
+      *a.mt_count = m_before + m;
+    }
+  }
+  for (int i = lane; i < m; i += 32) {
     MTile t;
     t.e = e;
-    t.row0 = c_excl + i * tr;
+    t.row0 = c_before + i * tr;
     t.nrows = min(tr, c - i * tr);
     t.pad = 0;
-    a.mtiles[m_excl + i] = t;
+    a.mtiles[m_before + i] = t;
+  }
+  const uint32_t* bits = a.bits + static_cast<size_t>(e) * a.words;
+  int32_t* base = a.base + static_cast<size_t>(e) * a.words;
+  int run = 0;
+  for (int w0 = 0; w0 < a.words; w0 += 32) {
+    const int w = w0 + lane;
+    const int n = w < a.words ? __popc(bits[w]) : 0;
+    int incl = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (w < a.words) base[w] = run + incl - n;
+    run += __shfl_sync(0xffffffffu, incl, 31);
   }
 }
 
@@ -96,8 +108,8 @@ __global__ void __launch_bounds__(256) permute_kernel(const PermuteArgs a) {
   if (lane < a.k) {
     const size_t slot = static_cast<size_t>(t) * a.k + lane;
     const int e = a.idx[slot];
-    const int r = a.rank[slot];
-    if (e >= 0 && e < a.E && r >= 0) {
+    const int r = e >= 0 && e < a.E ? slot_rank(a.bits, a.base, a.words, e, t) : -1;
+    if (r >= 0) {
       row = a.off[e] + r;
       if (row >= a.off[e + 1]) row = -1;
     }
@@ -200,7 +212,7 @@ cudaError_t launch_quantize_rows(const __nv_bfloat16* x, int64_t rows, int cols,
 }
 
 cudaError_t launch_dispatch_scan(const DispatchArgs& a, cudaStream_t s) {
-  dispatch_scan_kernel<<<1, 256, 0, s>>>(a);
+  dispatch_scan_kernel<<<(a.E + 7) / 8, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -154,15 +154,16 @@ __global__ void __launch_bounds__(256) nvfp4_permute_kernel(const Fp4PermuteArgs
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
   if (t >= a.T) return;
-  int row = -1, tile = 0;
+  int row = -1, tile = 0, rin = 0;  // rin: the slot's row inside its m-tile
   if (lane < a.k) {
     const size_t slot = static_cast<size_t>(t) * a.k + lane;
     const int e = a.idx[slot];
-    const int r = a.rank[slot];
-    if (e >= 0 && e < a.E && r >= 0) {
+    const int r = e >= 0 && e < a.E ? slot_rank(a.bits, a.base, a.words, e, t) : -1;
+    if (r >= 0) {
       row = a.off[e] + r;
       if (row >= a.off[e + 1]) row = -1;
       tile = tile_off[e] + r / kBM;
+      rin = r & (kBM - 1);
     }
     if (row < 0) record_status(a.status, kDevAssert, kWherePermute);
     a.rowmap[slot] = row;
@@ -179,13 +180,9 @@ __global__ void __launch_bounds__(256) nvfp4_permute_kernel(const Fp4PermuteArgs
   const uint4* src = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(t) * a.d);
   const float s = nvfp4_row_scale(src, a.d / 8, lane);
   if (lane < a.k && row >= 0) a.xs[row] = s;
-  // in-tile row of slot j: (rank % 128) = (row - off[e]) % 128, recomputed from the slot's rank
-  int rin[kMaxTopK];
+  int rins[kMaxTopK];
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
-    const int rk = j < a.k ? a.rank[static_cast<size_t>(t) * a.k + j] : 0;
-    rin[j] = rk & (kBM - 1);
-  }
+  for (int j = 0; j < kMaxTopK; ++j) rins[j] = __shfl_sync(0xffffffffu, rin, j);
   for (int jb = lane; jb < a.d / 16; jb += 32) {
     uint8_t bs;
     const uint2 q = nvfp4_block(src[2 * jb], src[2 * jb + 1], s, bs);
@@ -193,7 +190,7 @@ __global__ void __launch_bounds__(256) nvfp4_permute_kernel(const Fp4PermuteArgs
     for (int j = 0; j < kMaxTopK; ++j) {
       if (j < a.k && rows[j] >= 0) {
         reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(rows[j]) * (a.d / 2))[jb] = q;
-        atoms[j][nvfp4_sf_offset(rin[j], jb)] = bs;
+        atoms[j][nvfp4_sf_offset(rins[j], jb)] = bs;
       }
     }
   }

@@ -193,6 +193,8 @@ __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterG
 //                  then a warp minimum of the expert ids holding it (lower id wins a tie)
 //   output         ascending expert id: lane order, then a prefix sum of the lanes' counts;
 //                  the weights' denominator is summed in that order
+//   dispatch       per-expert slot counts and the token bitmap (bit t of expert e's row set
+//                  when token t chose e); the scan turns them into ascending-token row ranks
 
 __device__ __forceinline__ uint32_t ordered_bits(float f) {
   const uint32_t u = __float_as_uint(f);
@@ -358,13 +360,15 @@ __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) 
       if (lane == total && short_of_candidates) record_status(a.status, kDevAssert, kWhereSelect);
       a.idx[slot] = 0;
       a.w[slot] = 0.f;
-      if (a.cnt) a.rank[slot] = -1;
     } else {
       const int e = sel_sh[warp][lane];
       const float s = sw[e];
       a.idx[slot] = e;
       a.w[slot] = a.norm ? a.scale * s / denom : a.scale * s;
-      if (a.cnt) a.rank[slot] = atomicAdd(a.cnt + e, 1);
+      if (a.cnt) {  // dispatch: count the slot and mark token t in expert e's bitmap
+        atomicAdd(a.cnt + e, 1);
+        atomicOr(a.bits + static_cast<size_t>(e) * a.words + (t >> 5), 1u << (t & 31));
+      }
     }
   }
 }

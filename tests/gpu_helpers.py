@@ -8,6 +8,7 @@ byte for byte), and every expected value is computed by the oracle from those in
 from __future__ import annotations
 
 import dataclasses
+import weakref
 
 import numpy as np
 import torch
@@ -137,16 +138,84 @@ def run_block(case: Case, weights, in_place=False):
     return x_out, idx, w, ws
 
 
-def oracle_out(case: Case, weights, tokens, batch: int = 4):
-    """Oracle MoE output (FP32) for ``tokens``, copying only the experts each batch uses."""
+class _HostExperts:
+    """Host copies of device expert weights (and the oracle's own quantisations of them), made
+    once per expert and kept while the device tensors they came from are alive."""
+
+    def __init__(self):
+        self._store = {}
+
+    def get(self, weights, kind: str, e: int, make):
+        key = (id(weights[0]), kind, e)
+        hit = self._store.get(key)
+        if hit is not None and hit[0]() is weights[0]:
+            return hit[1]
+        # drop entries of device weights that no longer exist before adding more
+        self._store = {k: v for k, v in self._store.items() if v[0]() is not None}
+        val = make()
+        self._store[key] = (weakref.ref(weights[0]), val)
+        return val
+
+
+_HOST = _HostExperts()
+
+
+def host_expert(weights, e: int):
+    """(gate, up, down) of expert e as CPU tensors (copied from the device once)."""
+    return _HOST.get(weights, "bf16", e, lambda: tuple(m[e].cpu() for m in weights))
+
+
+def _experts_of(case: Case, tokens):
+    return sorted({int(e) for t in tokens for e in case.idx[t]})
+
+
+def oracle_out(case: Case, weights, tokens, batch: int = 256):
+    """Oracle MoE output (FP32) for ``tokens``; the experts they use are copied to the host
+    once, and the oracle runs on ``batch`` tokens at a time."""
     tokens = list(tokens)
+    experts = {e: host_expert(weights, e) for e in _experts_of(case, tokens)}
     out = np.empty((len(tokens), case.wl.d), np.float32)
     for b0 in range(0, len(tokens), batch):
         tb = tokens[b0:b0 + batch]
-        ex = sorted({int(e) for t in tb for e in case.idx[t]})
-        experts = {e: tuple(m[e].cpu() for m in weights) for e in ex}
         out[b0:b0 + len(tb)] = oracle.moe_tokens(tb, case.h, case.idx, case.w, experts)
     return out
+
+
+def cover_tokens(case: Case, tile_rows: int = 128, tile_ends: bool = True):
+    """Tokens whose outputs, compared with the oracle's, check every m-tile of the expert GEMMs.
+
+    The CUDA path lays out each expert's rows in ascending token order and cuts them into
+    m-tiles of ``tile_rows`` rows, so the m-tile holding each (token, expert) slot follows from
+    the oracle's routing alone.  The selection always holds each expert's first and last row;
+    with ``tile_ends`` it holds the first and last row of every m-tile, otherwise at least one
+    row of every m-tile (tokens chosen greedily, each covering up to top_k m-tiles)."""
+    idx = case.idx
+    T, k = idx.shape
+    E = case.wl.E
+    mt_of = np.empty((T, k), np.int64)       # global m-tile id of every slot
+    picks = set()
+    n_tiles = 0
+    for e in range(E):
+        ts, js = np.nonzero(idx == e)         # ascending token order
+        n = len(ts)
+        if n == 0:
+            continue
+        tiles = np.arange(n) // tile_rows
+        mt_of[ts, js] = n_tiles + tiles
+        picks.update((int(ts[0]), int(ts[-1])))
+        if tile_ends:
+            for r0 in range(0, n, tile_rows):
+                picks.update((int(ts[r0]), int(ts[min(r0 + tile_rows, n) - 1])))
+        n_tiles += int(tiles[-1]) + 1
+    covered = np.zeros(n_tiles, bool)
+    if picks:
+        covered[mt_of[sorted(picks)].reshape(-1)] = True
+    while not covered.all():
+        gain = (~covered[mt_of]).sum(axis=1)
+        t = int(np.argmax(gain))
+        picks.add(t)
+        covered[mt_of[t]] = True
+    return sorted(picks)
 
 
 def sample_tokens(case: Case, n: int, seed: int = 0):
@@ -182,16 +251,16 @@ def oracle_experts_fp8(weights, experts, gpu_fp8=None):
     the CUDA path's codes are given, they must equal the oracle's bit for bit."""
     res = {}
     for e in experts:
-        parts = []
-        for m_i, m in enumerate(weights):
-            q, s = oracle.quantize_rows_e4m3(m[e].cpu())
-            if gpu_fp8 is not None:
+        parts = _HOST.get(weights, "e4m3", e, lambda: tuple(
+            p for m in host_expert(weights, e) for p in oracle.quantize_rows_e4m3(m)))
+        if gpu_fp8 is not None:
+            for m_i in range(3):
+                q, s = parts[2 * m_i], parts[2 * m_i + 1]
                 gq = gpu_fp8[2 * m_i][e].cpu().numpy()
                 gs = gpu_fp8[2 * m_i + 1][e].cpu().numpy()
                 assert np.array_equal(gq, q), f"expert {e} matrix {m_i}: E4M3 codes differ"
                 assert np.array_equal(gs, s), f"expert {e} matrix {m_i}: scales differ"
-            parts += [q, s]
-        res[e] = tuple(parts)
+        res[e] = parts
     return res
 
 
@@ -209,25 +278,14 @@ def run_forward_fp8(case: Case, fp8, ws=None):
     return out, idx, w, ws
 
 
-def oracle_out_fp8(case: Case, weights, tokens, gpu_fp8=None, batch: int = 4):
+def oracle_out_fp8(case: Case, weights, tokens, gpu_fp8=None, batch: int = 256):
     """Oracle MoE output (FP32) of the E4M3 path for ``tokens``; the oracle quantises the BF16
-    weights of the experts each batch uses (and checks the CUDA path's codes against its own)."""
+    weights of the experts the tokens use (and checks the CUDA path's codes against its own)."""
     tokens = list(tokens)
+    experts = oracle_experts_fp8(weights, _experts_of(case, tokens), gpu_fp8)
     out = np.empty((len(tokens), case.wl.d), np.float32)
-    checked = set()
     for b0 in range(0, len(tokens), batch):
         tb = tokens[b0:b0 + batch]
-        ex = sorted({int(e) for t in tb for e in case.idx[t]})
-        experts = oracle_experts_fp8(weights, ex, None)
-        if gpu_fp8 is not None:
-            for e in ex:
-                if e in checked:
-                    continue
-                checked.add(e)
-                for m_i in range(3):
-                    assert np.array_equal(gpu_fp8[2 * m_i][e].cpu().numpy(), experts[e][2 * m_i])
-                    assert np.array_equal(gpu_fp8[2 * m_i + 1][e].cpu().numpy(),
-                                          experts[e][2 * m_i + 1])
         out[b0:b0 + len(tb)] = oracle.moe_tokens_fp8(tb, case.h, case.idx, case.w, experts)
     return out
 
@@ -284,7 +342,8 @@ def oracle_experts_nvfp4(weights, experts, w4=None):
     the CUDA path's weights are given, they must equal the oracle's bit for bit (+-0 alike)."""
     res = {}
     for e in experts:
-        parts = tuple(oracle.quantize_rows_nvfp4(m[e].cpu()) for m in weights)
+        parts = _HOST.get(weights, "nvfp4", e, lambda: tuple(
+            oracle.quantize_rows_nvfp4(m) for m in host_expert(weights, e)))
         if w4 is not None:
             I, d = weights[0].shape[1], weights[0].shape[2]
             got = nvfp4_expert_from_device(w4, e, I, d)
@@ -310,18 +369,13 @@ def run_forward_nvfp4(case: Case, w4, ws=None):
     return out, idx, w, ws
 
 
-def oracle_out_nvfp4(case: Case, weights, tokens, w4=None, batch: int = 4):
+def oracle_out_nvfp4(case: Case, weights, tokens, w4=None, batch: int = 256):
     """Oracle MoE output (FP32) of the NVFP4 path for ``tokens``; the oracle quantises the BF16
-    weights of the experts each batch uses (and checks the CUDA path's weights against them)."""
+    weights of the experts the tokens use (and checks the CUDA path's weights against them)."""
     tokens = list(tokens)
+    experts = oracle_experts_nvfp4(weights, _experts_of(case, tokens), w4)
     out = np.empty((len(tokens), case.wl.d), np.float32)
-    checked = set()
     for b0 in range(0, len(tokens), batch):
         tb = tokens[b0:b0 + batch]
-        ex = sorted({int(e) for t in tb for e in case.idx[t]})
-        new = [e for e in ex if e not in checked]
-        experts = oracle_experts_nvfp4(weights, new, w4)
-        experts.update(oracle_experts_nvfp4(weights, [e for e in ex if e in checked], None))
-        checked.update(new)
         out[b0:b0 + len(tb)] = oracle.moe_tokens_nvfp4(tb, case.h, case.idx, case.w, experts)
     return out

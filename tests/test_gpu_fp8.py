@@ -116,13 +116,14 @@ def test_forward_fp8_decode_every_token(beam_fp8):
     H.assert_close_out(out.float().cpu().numpy(), ref, "fp8 decode")
 
 
-def test_forward_fp8_prefill_sampled(beam_fp8):
+def test_forward_fp8_prefill_every_tile(beam_fp8):
+    """T = 4096: outputs of the tokens holding the first and the last row of every m-tile."""
     weights, fp8 = beam_fp8
     case = H.make_case(W.WORKLOADS["prefill"])
     out, idx, w, _ = H.run_forward_fp8(case, fp8)
     _check_routing(case, idx, w)
-    toks = H.sample_tokens(case, 8)
-    ref = H.oracle_out_fp8(case, weights, toks, fp8, batch=8)
+    toks = H.cover_tokens(case)
+    ref = H.oracle_out_fp8(case, weights, toks, fp8)
     H.assert_close_out(out[toks].float().cpu().numpy(), ref, "fp8 prefill")
 
 

@@ -148,13 +148,14 @@ def test_forward_nvfp4_decode_every_token(beam_nvfp4):
     H.assert_close_out(out.float().cpu().numpy(), ref, "nvfp4 decode")
 
 
-def test_forward_nvfp4_prefill_sampled(beam_nvfp4):
+def test_forward_nvfp4_prefill_every_tile(beam_nvfp4):
+    """T = 4096: outputs of the tokens holding the first and the last row of every m-tile."""
     weights, w4 = beam_nvfp4
     case = H.make_case(W.WORKLOADS["prefill"])
     out, idx, w, _ = H.run_forward_nvfp4(case, w4)
     _check_routing(case, idx, w)
-    toks = H.sample_tokens(case, 8)
-    ref = H.oracle_out_nvfp4(case, weights, toks, w4, batch=8)
+    toks = H.cover_tokens(case)
+    ref = H.oracle_out_nvfp4(case, weights, toks, w4)
     H.assert_close_out(out[toks].float().cpu().numpy(), ref, "nvfp4 prefill")
 
 

@@ -1,9 +1,10 @@
 """Parity of the CUDA path (called through the C ABI) with the CPU oracle.
 
 Routing indices must match bit-exactly (inputs have near ties removed); outputs must be within
-relative L2 1e-2 and max |err| 5e-2 * RMS of the oracle's.  Small cases are compared on every
-token; the full-size workloads are compared on every token's routing and on sampled tokens'
-outputs, in the same launch configuration the benchmark times.
+relative L2 1e-2 and max |err| 5e-2 * RMS of the oracle's.  Small cases and the T = 4096
+Beam-shape layer are compared on every token; the larger Beam-shape calls on every token's
+routing and on the outputs of tokens chosen from the oracle's routing so that every m-tile of
+every expert is checked, in the same launch configuration the benchmark times.
 """
 import ctypes
 import dataclasses
@@ -150,23 +151,64 @@ def test_full_size_logits_within_fp32_dot_error(name):
     assert err.max() <= 1e-5, f"{name}: max |logit error| {err.max():.3e}"
 
 
-@pytest.mark.parametrize("name,n_sample", [("prefill", 12), ("skewed", 12)])
-def test_full_size_routing_all_tokens_output_sampled(beam_weights, name, n_sample):
-    case = H.make_case(W.WORKLOADS[name])
+def test_full_size_prefill_every_token(beam_weights):
+    """T = 4096 at Beam shapes, the benchmark's configuration: routing and output of every
+    token against the oracle."""
+    case = H.make_case(W.WORKLOADS["prefill"])
     out, idx, w, ws = H.run_forward(case, beam_weights)
     _check_routing(case, idx, w)
     counts = bm.beam_moe_expert_counts(bm.shape_of(case.wl), ws).numpy()
     assert np.array_equal(counts, np.bincount(case.idx.reshape(-1), minlength=case.wl.E))
-    toks = H.sample_tokens(case, n_sample)
+    ref = H.oracle_out(case, beam_weights, range(case.wl.T))
+    H.assert_close_out(out.float().cpu().numpy(), ref, "prefill")
+
+
+def _expected_rows(idx, E):
+    """Row of every slot in the expert-contiguous layout: experts in ascending order, each
+    expert's tokens in ascending order (from the oracle's routing)."""
+    rows = np.full(idx.shape, -1, np.int64)
+    base = 0
+    for e in range(E):
+        ts, js = np.nonzero(idx == e)
+        rows[ts, js] = base + np.arange(len(ts))
+        base += len(ts)
+    return rows
+
+
+@pytest.mark.parametrize("name", ["tiny", "prefill", "skewed"])
+def test_slot_rows_follow_routing_in_ascending_token_order(beam_weights, name):
+    """The dispatch's row layout is the routing's function: bit-exact against the layout
+    enumerated from the oracle's routing, and equal across repeated calls."""
+    wl = W.WORKLOADS[name]
+    case = H.make_case(wl)
+    weights = beam_weights if wl.E == 256 and wl.d == 5120 else H.device_weights(wl)
+    _, _, _, ws = H.run_forward(case, weights)
+    s = bm.shape_of(wl)
+    rows = bm.beam_moe_slot_rows(s, ws).numpy()
+    assert np.array_equal(rows, _expected_rows(case.idx, wl.E))
+    H.run_forward(case, weights, ws=ws)
+    assert np.array_equal(bm.beam_moe_slot_rows(s, ws).numpy(), rows)
+
+
+def test_full_size_skewed_routing_all_tokens_output_every_tile(beam_weights):
+    """T = 16384 with a skewed load (hot experts hold up to ~14k rows, over 100 m-tiles each):
+    routing of every token; outputs of the tokens holding the first and the last row of every
+    m-tile of every expert."""
+    case = H.make_case(W.WORKLOADS["skewed"])
+    out, idx, w, ws = H.run_forward(case, beam_weights)
+    _check_routing(case, idx, w)
+    counts = bm.beam_moe_expert_counts(bm.shape_of(case.wl), ws).numpy()
+    assert np.array_equal(counts, np.bincount(case.idx.reshape(-1), minlength=case.wl.E))
+    toks = H.cover_tokens(case)
     ref = H.oracle_out(case, beam_weights, toks)
-    H.assert_close_out(out[toks].float().cpu().numpy(), ref, name)
+    H.assert_close_out(out[toks].float().cpu().numpy(), ref, "skewed")
 
 
-def test_block_routing_all_tokens_output_sampled(beam_weights):
+def test_block_routing_all_tokens_output_every_tile(beam_weights):
     case = H.make_case(W.WORKLOADS["block"])
     x_out, idx, w, _ = H.run_block(case, beam_weights)
     _check_routing(case, idx, w)
-    toks = H.sample_tokens(case, 10)
+    toks = H.cover_tokens(case)
     moe = H.oracle_out(case, beam_weights, toks)
     ref = oracle.block_tail(case.x[toks], moe, case.g_post, case.wl.eps, case.wl.k_resid)
     got = x_out[toks].cpu().numpy()
@@ -332,18 +374,19 @@ def test_sm_pair_path_on_beam_shapes(beam_weights):
     finally:
         bm.beam_moe_set_sm_pairs(False)
     _check_routing(case, idx, w)
-    toks = H.sample_tokens(case, 8)
+    toks = H.cover_tokens(case, tile_rows=256)  # an SM pair's m-tile holds 256 rows
     ref = H.oracle_out(case, beam_weights, toks)
     H.assert_close_out(out[toks].float().cpu().numpy(), ref, "pairs beam")
 
 
 def test_maximum_size_beam_call(beam_weights):
     """T = 65536 at Beam shapes: 524,288 slots, expert-contiguous buffers of 2.7e9 elements
-    (past 32-bit element offsets).  Routing on every token, outputs on sampled tokens."""
+    (past 32-bit element offsets).  Routing on every token; outputs of tokens that hold each
+    expert's first and last row and at least one row of every m-tile."""
     case = H.make_case(W.WORKLOADS["prefill"].with_tokens(65536))
     out, idx, w, _ = H.run_forward(case, beam_weights)
     _check_routing(case, idx, w)
-    toks = H.sample_tokens(case, 8)
+    toks = H.cover_tokens(case, tile_ends=False)
     ref = H.oracle_out(case, beam_weights, toks)
     H.assert_close_out(out[toks].float().cpu().numpy(), ref, "T=65536")
 

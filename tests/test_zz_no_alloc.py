@@ -4,8 +4,9 @@ It exists for callers that cannot allocate device memory (a serving engine whose
 memory all belongs to its own pool, or a host that forbids allocation on its request path)
 and so have no workspace to pass.  Its scratch is a static per-GPU array inside the library,
 which bounds T to 512 tokens.  These tests call it through the C ABI and compare it with
-beam_moe_route (which uses a caller workspace) on consecutive calls, so that contents left in
-the shared static array by one call cannot leak into the next.
+beam_moe_route (which uses a caller workspace) and with the oracle on consecutive calls, so
+that contents left in the shared static array by one call cannot leak into the next, and check
+that calls after the first leave the device's free memory unchanged.
 
 This file is named to be collected last.
 """
@@ -34,12 +35,11 @@ def test_static_route_rejects_more_tokens_than_its_scratch_holds(L):
     assert "512" in bm.last_cuda_error()
 
 
-def _inputs(wl):
-    return (W.hidden(wl).cuda(), W.router_weight(wl).cuda(), W.router_bias(wl).cuda())
-
-
-def _route_both(wl, h, router_w, bias):
+def _route_both(case):
+    """beam_moe_route (caller workspace) and beam_moe_route_static on the same inputs."""
+    wl = case.wl
     s = bm.shape_of(wl)
+    h, router_w, bias = case.h.cuda(), case.router_w.cuda(), case.bias.cuda()
     out = []
     for fn in ("workspace", "static"):
         idx = torch.full((wl.T, wl.top_k), -1, dtype=torch.int32, device="cuda")
@@ -56,17 +56,45 @@ def _route_both(wl, h, router_w, bias):
 
 
 @pytest.mark.gpu
-def test_static_route_matches_workspace_route_on_consecutive_calls(L):
+def test_static_route_matches_workspace_route_and_oracle_on_consecutive_calls(L):
+    """Inputs with near ties removed (so the chosen experts are unique at FP32 accuracy; the two
+    entry points may split the router's K sum differently).  Both must pick the oracle's
+    experts bit for bit; weights and logits agree within the FP32 dot-product error."""
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA GPU")
+    from tests import gpu_helpers as H
     cases = [W.WORKLOADS["prefill"].with_tokens(512),  # the largest T the static scratch holds
              W.WORKLOADS["tiny"],
              W.WORKLOADS["decode"].with_tokens(37)]
     for wl in cases:
-        h, router_w, bias = _inputs(wl)
-        (i0, w0, l0), (i1, w1, l1) = _route_both(wl, h, router_w, bias)
-        assert np.array_equal(i1, i0), wl.name
+        case = H.make_case(wl)
+        (i0, w0, l0), (i1, w1, l1) = _route_both(case)
+        assert np.array_equal(i0, case.idx), wl.name
+        assert np.array_equal(i1, case.idx), wl.name
+        np.testing.assert_allclose(w1, case.w, rtol=1e-5, atol=1e-7, err_msg=wl.name)
         np.testing.assert_allclose(w1, w0, rtol=1e-5, atol=1e-7, err_msg=wl.name)
+        assert np.abs(l1.astype(np.float64) - case.logits).max() <= 1e-5, wl.name
         np.testing.assert_allclose(l1, l0, rtol=1e-5, atol=2e-6, err_msg=wl.name)
-        assert np.all(np.diff(i1, axis=1) > 0)
         np.testing.assert_allclose(w1.sum(axis=1), wl.scale, rtol=1e-5)
+
+
+@pytest.mark.gpu
+def test_static_route_allocates_no_device_memory(L):
+    """After a first call (which looks up the static array's address), further calls leave the
+    device's free memory unchanged."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    wl = W.WORKLOADS["decode"].with_tokens(256)
+    s = bm.shape_of(wl)
+    h = W.hidden(wl).cuda()
+    router_w, bias = W.router_weight(wl).cuda(), W.router_bias(wl).cuda()
+    idx = torch.empty(wl.T, wl.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(wl.T, wl.top_k, dtype=torch.float32, device="cuda")
+    bm.beam_moe_route_static(s, h, router_w, bias, idx, w)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(5):
+        bm.beam_moe_route_static(s, h, router_w, bias, idx, w)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
