@@ -333,6 +333,81 @@ BEAM_API beam_status beam_dense_forward_nvfp4(const beam_dense_shape* shape, con
 BEAM_API beam_status beam_moe_bias_update(const beam_moe_shape* shape, const void* ws,
                                           float* bias, float gamma, beam_stream stream);
 
+/* ---- expert parallelism: the layer's experts over P GPUs ----
+ *
+ * Cites: cookbook "Use HF Transformers", section Parallelism (ep_size = 8: each GPU holds 32
+ * of the 256 experts, and tokens are sent to the GPU that holds their experts); the device
+ * count divides 256 (news article "Reflection lança o Beam", section "O que os benchmarks
+ * mostram e como rodar o modelo").
+ *
+ * Rank p of P owns experts p*E/P .. (p+1)*E/P - 1 (E % P == 0, P <= 64) and routes its own
+ * T_p tokens (for example with beam_moe_route).  One layer step on every rank, in this order
+ * and on one stream per rank:
+ *   1. beam_moe_ep_count     local slot counts [E] -> `counts` (device)
+ *   2. the caller gathers every rank's counts into all_counts [P, E] (device, rank-major),
+ *      for instance with an NCCL all-gather
+ *   3. beam_moe_ep_dispatch  writes each token row into the receive buffer of the owner of
+ *      each of its experts (a peer store when the owner is another GPU)
+ *   4. the caller waits until every rank's step 3 has completed (a barrier ordered on the
+ *      stream, e.g. an NCCL all-reduce of one word)
+ *   5. beam_moe_ep_experts   the grouped GEMMs over the received rows -> yrecv
+ *   6. the caller waits until every rank's step 5 has completed
+ *   7. beam_moe_ep_combine   each token's k expert outputs read from their owners' yrecv
+ *      and summed with topk_w in ascending expert order -> out [T_p, d] BF16
+ * Every rank holds two caller-owned receive buffers of recv_rows_max rows, xrecv and yrecv
+ * (BF16 [recv_rows_max, d]), and passes the device addresses of all ranks' buffers (their
+ * peer mappings on this GPU) as host arrays of P pointers.  A rank's receive rows are its
+ * experts in ascending order, each expert's rows from rank 0, 1, ... in turn, each rank's in
+ * ascending token order: with tokens numbered rank-major this is the single-GPU layout of the
+ * whole batch, so the result equals beam_moe_forward on the concatenated tokens with the same
+ * routing bit for bit.  Rows beyond recv_rows_max are not sent and are recorded as
+ * BEAM_ERR_DEVICE_ASSERT (size the buffers with beam_moe_ep_plan).  The same `shape` (T = this
+ * rank's tokens) and workspace serve the four calls of a step; beam_moe_sync_status(ws) reads
+ * the step's device status. */
+
+/* Workspace bytes of one rank (0 if the arguments are unsupported). */
+BEAM_API size_t beam_moe_ep_workspace_size(const beam_moe_shape* shape, int32_t P,
+                                           int64_t recv_rows_max);
+
+/* Host-only exchange sizes from the gathered counts all_counts [P, E] (HOST array): rows this
+ * rank receives in total (*recv_rows), rows it sends to each rank (send_rows [P]) and rows it
+ * receives from each rank (recv_from [P]).  Any output may be NULL.  Touches no GPU. */
+BEAM_API beam_status beam_moe_ep_plan(int32_t P, int32_t E, const int32_t* all_counts,
+                                      int32_t rank, int64_t* recv_rows, int64_t* send_rows,
+                                      int64_t* recv_from);
+
+/* Step 1: per-expert slot counts of this rank's routing topk_idx [T, top_k] -> counts [E]
+ * (device INT32, always written; zeros when T = 0).  Clears the step's status word. */
+BEAM_API beam_status beam_moe_ep_count(const beam_moe_shape* shape, int32_t P,
+                                       const int32_t* topk_idx, int32_t* counts,
+                                       int64_t recv_rows_max, void* ws, size_t ws_bytes,
+                                       beam_stream stream);
+
+/* Step 3: hidden [T, d] BF16 rows to the owners' receive buffers xrecv_peers[q] (host array
+ * of P device pointers, this rank's own buffer at index `rank`). */
+BEAM_API beam_status beam_moe_ep_dispatch(const beam_moe_shape* shape, int32_t P, int32_t rank,
+                                          const void* hidden, const int32_t* topk_idx,
+                                          const int32_t* all_counts, void* const* xrecv_peers,
+                                          int64_t recv_rows_max, void* ws, size_t ws_bytes,
+                                          beam_stream stream);
+
+/* Step 5: the SwiGLU experts of this rank over its received rows.  w_gate, w_up [E/P, I, d],
+ * w_down [E/P, d, I] BF16 are this rank's experts; xrecv and yrecv are this rank's receive
+ * buffers; T_total is the tokens of all ranks together (it selects the same tile forms as a
+ * single-GPU call of that size). */
+BEAM_API beam_status beam_moe_ep_experts(const beam_moe_shape* shape, int32_t P, int32_t rank,
+                                         int64_t T_total, const int32_t* all_counts,
+                                         const void* w_gate, const void* w_up, const void* w_down,
+                                         const void* xrecv, void* yrecv, int64_t recv_rows_max,
+                                         void* ws, size_t ws_bytes, beam_stream stream);
+
+/* Step 7: out [T, d] BF16 = sum_j topk_w[t, j] * y(slot j), the expert outputs read from
+ * yrecv_peers[owner] (host array of P device pointers). */
+BEAM_API beam_status beam_moe_ep_combine(const beam_moe_shape* shape, int32_t P,
+                                         const float* topk_w, const void* const* yrecv_peers,
+                                         int64_t recv_rows_max, void* out, void* ws,
+                                         size_t ws_bytes, beam_stream stream);
+
 /* Synchronises `stream`, reads and clears the device status word kept in `ws`, and
  * returns BEAM_OK, BEAM_ERR_TIMEOUT or BEAM_ERR_DEVICE_ASSERT (or BEAM_ERR_CUDA if the
  * stream itself reports an error).  `ws` must have been used with a call of this shape

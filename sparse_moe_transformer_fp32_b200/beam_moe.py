@@ -35,7 +35,9 @@ EXPORTED = [
     "beam_moe_forward_fp8", "beam_moe_block_fp8", "beam_dense_fp8_workspace_size",
     "beam_dense_forward_fp8", "beam_moe_quantize_nvfp4", "beam_moe_nvfp4_workspace_size",
     "beam_moe_forward_nvfp4", "beam_moe_block_nvfp4", "beam_dense_nvfp4_workspace_size",
-    "beam_dense_forward_nvfp4", "beam_moe_slot_rows",
+    "beam_dense_forward_nvfp4", "beam_moe_slot_rows", "beam_moe_ep_workspace_size",
+    "beam_moe_ep_plan", "beam_moe_ep_count", "beam_moe_ep_dispatch", "beam_moe_ep_experts",
+    "beam_moe_ep_combine",
 ]
 
 
@@ -124,6 +126,14 @@ def lib():
     L.beam_moe_last_cuda_error.restype = ctypes.c_char_p
     L.beam_moe_expert_counts.argtypes = [shp, vp, vp, vp]
     L.beam_moe_slot_rows.argtypes = [shp, vp, vp, vp]
+    i64 = ctypes.c_int64
+    L.beam_moe_ep_workspace_size.argtypes = [shp, i32, i64]
+    L.beam_moe_ep_workspace_size.restype = sz
+    L.beam_moe_ep_plan.argtypes = [i32, i32, vp, i32, vp, vp, vp]
+    L.beam_moe_ep_count.argtypes = [shp, i32, vp, vp, i64, vp, sz, vp]
+    L.beam_moe_ep_dispatch.argtypes = [shp, i32, i32, vp, vp, vp, vp, i64, vp, sz, vp]
+    L.beam_moe_ep_experts.argtypes = [shp, i32, i32, i64, vp, vp, vp, vp, vp, vp, i64, vp, sz, vp]
+    L.beam_moe_ep_combine.argtypes = [shp, i32, vp, vp, i64, vp, vp, sz, vp]
     L.beam_moe_set_wait_limit_ns.argtypes = [u64]
     L.beam_moe_get_wait_limit_ns.restype = u64
     L.beam_moe_launch_count.restype = u64
@@ -139,7 +149,9 @@ def lib():
                  "beam_moe_expert_counts", "beam_moe_profile_read", "beam_moe_quantize_e4m3",
                  "beam_moe_forward_fp8", "beam_moe_block_fp8", "beam_dense_forward_fp8",
                  "beam_moe_quantize_nvfp4", "beam_moe_forward_nvfp4", "beam_moe_block_nvfp4",
-                 "beam_dense_forward_nvfp4", "beam_moe_slot_rows"):
+                 "beam_dense_forward_nvfp4", "beam_moe_slot_rows", "beam_moe_ep_plan",
+                 "beam_moe_ep_count", "beam_moe_ep_dispatch", "beam_moe_ep_experts",
+                 "beam_moe_ep_combine"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -495,6 +507,86 @@ def beam_moe_slot_rows(shape, ws, stream=None) -> torch.Tensor:
     _check(lib().beam_moe_slot_rows(ctypes.byref(shape), _ptr(ws, torch.uint8, "ws"),
                                     out.data_ptr(), _stream(stream)), "beam_moe_slot_rows")
     return out
+
+
+# ------------------------------------------------------------------ expert parallelism
+
+def beam_moe_ep_workspace_size(shape, P: int, recv_rows_max: int) -> int:
+    return int(lib().beam_moe_ep_workspace_size(ctypes.byref(shape), int(P), int(recv_rows_max)))
+
+
+def ep_workspace(shape, P: int, recv_rows_max: int, device="cuda") -> torch.Tensor:
+    n = beam_moe_ep_workspace_size(shape, P, recv_rows_max)
+    if n == 0:
+        raise BeamError(BEAM_ERR_UNSUPPORTED, "beam_moe_ep_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def beam_moe_ep_plan(P: int, E: int, all_counts, rank: int):
+    """Host-only exchange sizes from the gathered counts [P, E] (CPU): (rows this rank receives,
+    rows it sends to each rank [P], rows it receives from each rank [P])."""
+    import numpy as np
+    c = np.ascontiguousarray(np.asarray(all_counts, dtype=np.int32).reshape(P, E))
+    recv = ctypes.c_int64(0)
+    send = np.zeros(P, np.int64)
+    frm = np.zeros(P, np.int64)
+    _check(lib().beam_moe_ep_plan(int(P), int(E), c.ctypes.data, int(rank), ctypes.byref(recv),
+                                  send.ctypes.data, frm.ctypes.data), "beam_moe_ep_plan")
+    return int(recv.value), send, frm
+
+
+def _peer_array(ptrs, P: int, name: str):
+    if len(ptrs) != P:
+        raise ValueError(f"{name} must hold {P} device pointers")
+    vals = [p.data_ptr() if isinstance(p, torch.Tensor) else int(p) for p in ptrs]
+    return (ctypes.c_void_p * P)(*vals)
+
+
+def beam_moe_ep_count(shape, P: int, topk_idx, counts, recv_rows_max: int, ws, stream=None):
+    T, E, k = shape.T, shape.E, shape.top_k
+    _check(lib().beam_moe_ep_count(ctypes.byref(shape), int(P),
+                                   _ptr(topk_idx, torch.int32, "topk_idx", (T, k)),
+                                   _ptr(counts, torch.int32, "counts", (E,)), int(recv_rows_max),
+                                   _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)),
+           "beam_moe_ep_count")
+
+
+def beam_moe_ep_dispatch(shape, P: int, rank: int, hidden, topk_idx, all_counts, xrecv_peers,
+                         recv_rows_max: int, ws, stream=None):
+    T, d, E, k = shape.T, shape.d, shape.E, shape.top_k
+    _check(lib().beam_moe_ep_dispatch(ctypes.byref(shape), int(P), int(rank),
+                                      _ptr(hidden, torch.bfloat16, "hidden", (T, d)),
+                                      _ptr(topk_idx, torch.int32, "topk_idx", (T, k)),
+                                      _ptr(all_counts, torch.int32, "all_counts", (P, E)),
+                                      _peer_array(xrecv_peers, P, "xrecv_peers"),
+                                      int(recv_rows_max), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                      _stream(stream)), "beam_moe_ep_dispatch")
+
+
+def beam_moe_ep_experts(shape, P: int, rank: int, T_total: int, all_counts, w_gate, w_up, w_down,
+                        xrecv, yrecv, recv_rows_max: int, ws, stream=None):
+    d, E, I = shape.d, shape.E, shape.I
+    ep = E // P
+    _check(lib().beam_moe_ep_experts(ctypes.byref(shape), int(P), int(rank), int(T_total),
+                                     _ptr(all_counts, torch.int32, "all_counts", (P, E)),
+                                     _ptr(w_gate, torch.bfloat16, "w_gate", (ep, I, d)),
+                                     _ptr(w_up, torch.bfloat16, "w_up", (ep, I, d)),
+                                     _ptr(w_down, torch.bfloat16, "w_down", (ep, d, I)),
+                                     _ptr(xrecv, torch.bfloat16, "xrecv", (recv_rows_max, d)),
+                                     _ptr(yrecv, torch.bfloat16, "yrecv", (recv_rows_max, d)),
+                                     int(recv_rows_max), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                     _stream(stream)), "beam_moe_ep_experts")
+
+
+def beam_moe_ep_combine(shape, P: int, topk_w, yrecv_peers, recv_rows_max: int, out, ws,
+                        stream=None):
+    T, d, k = shape.T, shape.d, shape.top_k
+    _check(lib().beam_moe_ep_combine(ctypes.byref(shape), int(P),
+                                     _ptr(topk_w, torch.float32, "topk_w", (T, k)),
+                                     _peer_array(yrecv_peers, P, "yrecv_peers"),
+                                     int(recv_rows_max), _ptr(out, torch.bfloat16, "out", (T, d)),
+                                     _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)),
+           "beam_moe_ep_combine")
 
 
 def beam_moe_set_wait_limit_ns(ns: int) -> None:

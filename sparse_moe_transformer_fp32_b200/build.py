@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libbeam_moe.so")
 SOURCES = ["beam_moe_api.cu", "router.cu", "dispatch.cu", "expert_gemm.cu", "expert_gemm_2sm.cu",
-           "combine.cu", "nvfp4.cu"]
+           "combine.cu", "nvfp4.cu", "ep.cu"]
 HEADERS = [os.path.join(CSRC, "beam_moe_internal.cuh"), os.path.join(CSRC, "beam_moe_nvfp4.cuh"),
            os.path.join(INCLUDE, "beam_moe.h")]
 

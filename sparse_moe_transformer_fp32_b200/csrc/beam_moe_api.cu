@@ -39,12 +39,18 @@ enum KernelId {
   kKBiasUpdate,
   kKQuantize,
   kKQuantizeNvfp4,
+  kKEpCount,
+  kKEpOffsets,
+  kKEpPush,
+  kKEpLocalCounts,
+  kKEpCombine,
   kNumKernels
 };
 const char* const kKernelNames[kNumKernels] = {
     "router_gemm", "router_select", "dispatch_scan", "permute", "expert_gemm_gate_up",
     "expert_gemm_down", "combine", "combine_block", "prenorm", "router_transpose", "dense_tiles",
-    "bias_update", "quantize_e4m3", "quantize_nvfp4"};
+    "bias_update", "quantize_e4m3", "quantize_nvfp4", "ep_count", "ep_offsets", "ep_push",
+    "ep_local_counts", "ep_combine"};
 
 struct Profiler {
   std::mutex mu;
@@ -130,8 +136,8 @@ beam_status check_shape(const beam_moe_shape* s) {
 }
 
 struct Layout {
-  size_t status, cnt, bits, off, mt_count, mtiles, base, rowmap, idx, w, wt, part, h, xp, act, y,
-      total;
+  size_t status, cnt, bits, off, mt_count, mtiles, base, rowmap, tok_of_row, idx, w, wt, part, h,
+      xp, act, y, total;
   size_t zero_bytes = 0;             // status, counts and token bitmap: cleared at each call
   int words = 0;                     // token bitmap words per expert, ceil(T / 32)
   size_t xs = 0, act8 = 0, as = 0;  // FP8 path: row scales of Xp, E4M3 act, act row scales
@@ -195,6 +201,7 @@ Layout plan(const beam_moe_shape& s) {
   L.mtiles = take(sizeof(MTile) * L.mt_cap);
   L.base = take(bitmap_bytes);
   L.rowmap = take(sizeof(int32_t) * R);
+  L.tok_of_row = take(sizeof(int32_t) * R);
   L.idx = take(sizeof(int32_t) * R);
   L.w = take(sizeof(float) * R);
   L.wt = take(sizeof(float) * static_cast<size_t>(s.E) * s.d);
@@ -320,6 +327,8 @@ beam_status device_info(DeviceInfo** out) {
     if (e != cudaSuccess) return cuda_fail(e);
     e = prepare_gemm_kernels();
     if (e != cudaSuccess) return cuda_fail(e);
+    e = prepare_router_kernels();
+    if (e != cudaSuccess) return cuda_fail(e);
     e = prepare_gemm_2sm_kernels();
     if (e != cudaSuccess) return cuda_fail(e);
     e = prepare_gemm_nvfp4_kernels();
@@ -386,10 +395,27 @@ struct Fp8Scales {
 // Dispatch, the two expert GEMMs; leaves Y and rowmap in the workspace.  With f8 the weights
 // are E4M3 codes: the permute writes E4M3 rows of Xp with their scales, and the activation is
 // quantised between the two GEMMs.
+// BF16 gate/up GEMMs gather their A rows from the token rows (no permuted copy of h).
+constexpr bool kRowGather = true;
+
+// Sets up the combine's slot rows: read from rowmap (written by the permute), or formed by the
+// combine itself from the routing and the token bitmap when the experts ran with a row gather.
+void combine_rows(CombineArgs& ca, const Layout& L, const beam_moe_shape& s, const int32_t* idx,
+                  void* ws, bool gathered) {
+  ca.rowmap = at<int32_t>(ws, L.rowmap);
+  if (!gathered) return;
+  ca.idx = idx;
+  ca.bits = at<uint32_t>(ws, L.bits);
+  ca.base = at<int32_t>(ws, L.base);
+  ca.off = at<int32_t>(ws, L.off);
+  ca.words = L.words;
+  ca.E = s.E;
+}
+
 beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceInfo& dev,
                         const __nv_bfloat16* h, const int32_t* idx, const void* w_gate,
                         const void* w_up, const void* w_down, void* ws, cudaStream_t st,
-                        const Fp8Scales* f8 = nullptr) {
+                        const Fp8Scales* f8, bool* gathered) {
   uint32_t* status = at<uint32_t>(ws, L.status);
   // With SM pairs enabled, calls averaging at least 256 rows per expert run their expert GEMMs
   // on SM pairs (cta_group::2, 256-row tiles): half the operand bytes per SM for the same tensor
@@ -397,6 +423,8 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   const bool pairs = !f8 && g_sm_pairs.load(std::memory_order_relaxed) != 0 &&
                      L.R >= static_cast<int64_t>(kPairMinRowsPerExpert) * s.E &&
                      dev.pair_grid >= 2;
+  const bool gather = kRowGather && !f8 && !pairs;
+  *gathered = gather;
   DispatchArgs da{};
   da.cnt = at<int32_t>(ws, L.cnt);
   da.bits = at<uint32_t>(ws, L.bits);
@@ -407,6 +435,7 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   da.E = s.E;
   da.words = L.words;
   da.tile_rows = pairs ? 2 * kBM : kBM;
+  da.tok_of_row = gather ? at<int32_t>(ws, L.tok_of_row) : nullptr;
   BEAM_LAUNCH(kKDispatchScan, st, launch_dispatch_scan(da, st));
 
   PermuteArgs pa{};
@@ -425,7 +454,7 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   pa.d = s.d;
   pa.k = s.top_k;
   pa.E = s.E;
-  BEAM_LAUNCH(kKPermute, st, launch_permute(pa, st));
+  if (!gather) BEAM_LAUNCH(kKPermute, st, launch_permute(pa, st));
 
   const uint64_t R = static_cast<uint64_t>(L.R);
   ATensorMaps tm_xp, tm_act;
@@ -435,7 +464,11 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   const void* a1 = at<void>(ws, L.xp);
   const void* a2 = at<void>(ws, f8 ? L.act8 : L.act);
   for (int i = 0; i < kNumABoxes; ++i) {
-    if ((b = make_map(&tm_xp.m[i], a1, s.d, R, a_box_rows(i), eb)) != BEAM_OK) return b;
+    if (gather) {  // one-row boxes over the token rows, four gathered per instruction
+      if ((b = make_map(&tm_xp.m[i], h, s.d, static_cast<uint64_t>(s.T), 1)) != BEAM_OK) return b;
+    } else if ((b = make_map(&tm_xp.m[i], a1, s.d, R, a_box_rows(i), eb)) != BEAM_OK) {
+      return b;
+    }
     if ((b = make_map(&tm_act.m[i], a2, s.I, R, a_box_rows(i), eb)) != BEAM_OK) return b;
   }
   const uint64_t EI = static_cast<uint64_t>(s.E) * s.I, Ed = static_cast<uint64_t>(s.E) * s.d;
@@ -455,6 +488,7 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   g1.n_tiles_n = s.I / kN1Half;
   g1.k_blocks = s.d / k_elems;
   g1.b_rows_per_expert = s.I;
+  g1.tok_of_row = da.tok_of_row;
   if (f8) {
     g1.a_scale = pa.xs;
     g1.b_scale0 = f8->gate;
@@ -480,6 +514,7 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
                                      at<uint8_t>(ws, L.act8), at<float>(ws, L.as), st));
 
   GemmArgs g2 = g1;
+  g2.tok_of_row = nullptr;
   g2.out = at<__nv_bfloat16>(ws, L.y);
   g2.out_ld = s.d;
   g2.n_tiles_n = s.d / kN2;
@@ -773,11 +808,13 @@ beam_status forward_impl(const beam_moe_shape* shape, const void* hidden, const 
   const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(hidden);
   if ((b = run_router(*shape, L, h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
     return b;
-  if ((b = run_experts(*shape, L, *dev, h, idx, w_gate, w_up, w_down, ws, st, f8)) != BEAM_OK)
+  bool gathered = false;
+  if ((b = run_experts(*shape, L, *dev, h, idx, w_gate, w_up, w_down, ws, st, f8, &gathered)) !=
+      BEAM_OK)
     return b;
   CombineArgs ca{};
   ca.y = at<__nv_bfloat16>(ws, L.y);
-  ca.rowmap = at<int32_t>(ws, L.rowmap);
+  combine_rows(ca, L, *shape, idx, ws, gathered);
   ca.w = w;
   ca.out = static_cast<__nv_bfloat16*>(out);
   ca.status = at<uint32_t>(ws, L.status);
@@ -867,13 +904,14 @@ beam_status block_impl(const beam_moe_shape* shape, const float* x, const float*
   float* w = topk_w ? topk_w : at<float>(ws, L.w);
   if ((b = run_router(*shape, L, pn.h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
     return b;
+  bool gathered = false;
   b = w4 ? run_experts_nvfp4(*shape, L, *dev, pn.h, idx, *w4, ws, st)
-         : run_experts(*shape, L, *dev, pn.h, idx, w_gate, w_up, w_down, ws, st, f8);
+         : run_experts(*shape, L, *dev, pn.h, idx, w_gate, w_up, w_down, ws, st, f8, &gathered);
   if (b != BEAM_OK) return b;
   const double kk = static_cast<double>(k_resid);
   CombineArgs ca{};
   ca.y = at<__nv_bfloat16>(ws, L.y);
-  ca.rowmap = at<int32_t>(ws, L.rowmap);
+  combine_rows(ca, L, *shape, idx, ws, gathered);
   ca.w = w;
   ca.x = x;
   ca.g_post = g_post;
@@ -1072,6 +1110,65 @@ beam_status dense_impl(const beam_dense_shape* shape, const void* hidden, const 
               launch_gemm_down(tm_act, tm_d, g2,
                                static_cast<int>(t2 < dev->sms ? t2 : dev->sms), st,
                                f8 != nullptr));
+  return BEAM_OK;
+}
+
+// ------------------------------------------------------------------ expert parallelism
+//
+// P ranks, rank p owning experts p * E / P .. (p + 1) * E / P - 1 (see ep.cu for the steps and
+// the row layout).  The workspace of a rank holds its dispatch state (counts, token bitmap and
+// its prefix counts, each slot's owner and row) and its expert side (the m-tiles over the
+// received rows and the SwiGLU activation); the receive buffers of token rows and expert
+// outputs are the caller's, since peers write and read them.
+
+struct EpLayout {
+  size_t status, cnt, bits, zero_bytes, base, row_off, slot_row, slot_owner, cnt_local, off,
+      mt_count, mtiles, act, total;
+  int words;
+  int64_t mt_cap;
+};
+
+beam_status check_ep(const beam_moe_shape* s, int P, int64_t recv_cap) {
+  beam_status b = check_shape(s);
+  if (b != BEAM_OK) return b;
+  if (P < 1 || P > kMaxEpRanks || s->E % P != 0) return BEAM_ERR_UNSUPPORTED;
+  if (recv_cap < 1 || recv_cap >= (int64_t(1) << 31)) return BEAM_ERR_INVALID_ARG;
+  return BEAM_OK;
+}
+
+EpLayout plan_ep(const beam_moe_shape& s, int P, int64_t recv_cap) {
+  EpLayout L{};
+  const int64_t R = static_cast<int64_t>(s.T) * s.top_k;
+  const int ep = s.E / P;
+  L.words = static_cast<int>(ceil_div(s.T > 0 ? s.T : 1, 32));
+  L.mt_cap = ceil_div(recv_cap, kBM) + ep;
+  const size_t bitmap_bytes = sizeof(uint32_t) * static_cast<size_t>(s.E) * L.words;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o = align_up(o + (bytes ? bytes : 1), 1024);
+    return r;
+  };
+  L.status = take(256);
+  L.cnt = take(sizeof(int32_t) * s.E);
+  L.bits = take(bitmap_bytes);
+  L.zero_bytes = L.bits + bitmap_bytes;
+  L.base = take(bitmap_bytes);
+  L.row_off = take(sizeof(int64_t) * s.E);
+  L.slot_row = take(sizeof(int32_t) * R);
+  L.slot_owner = take(sizeof(int32_t) * R);
+  L.cnt_local = take(sizeof(int32_t) * ep);
+  L.off = take(sizeof(int32_t) * (ep + 1));
+  L.mt_count = take(16);
+  L.mtiles = take(sizeof(MTile) * L.mt_cap);
+  L.act = take(sizeof(__nv_bfloat16) * static_cast<size_t>(recv_cap) * s.I);
+  L.total = o;
+  return L;
+}
+
+beam_status check_ep_ws(const EpLayout& L, void* ws, size_t ws_bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < L.total)
+    return BEAM_ERR_WORKSPACE;
   return BEAM_OK;
 }
 
@@ -1424,6 +1521,205 @@ beam_status beam_moe_profile_read(int id, int64_t* launches, double* total_ms) {
   g_prof.pending.clear();
   *launches = g_prof.launches[id];
   *total_ms = g_prof.ms[id];
+  return BEAM_OK;
+}
+
+// ------------------------------------------------------------------ expert parallelism
+
+size_t beam_moe_ep_workspace_size(const beam_moe_shape* shape, int32_t P, int64_t recv_rows_max) {
+  if (check_ep(shape, P, recv_rows_max) != BEAM_OK) return 0;
+  return plan_ep(*shape, P, recv_rows_max).total;
+}
+
+beam_status beam_moe_ep_plan(int32_t P, int32_t E, const int32_t* all_counts, int32_t rank,
+                             int64_t* recv_rows, int64_t* send_rows, int64_t* recv_from) {
+  if (P < 1 || P > kMaxEpRanks || E < 1 || E % P != 0 || rank < 0 || rank >= P || !all_counts)
+    return BEAM_ERR_INVALID_ARG;
+  const int ep = E / P;
+  for (int i = 0; i < P * E; ++i)
+    if (all_counts[i] < 0) return BEAM_ERR_INVALID_ARG;
+  int64_t recv = 0;
+  for (int q = 0; q < P; ++q) {
+    int64_t to_q = 0, from_q = 0;
+    for (int e = q * ep; e < (q + 1) * ep; ++e) to_q += all_counts[static_cast<size_t>(rank) * E + e];
+    for (int e = rank * ep; e < (rank + 1) * ep; ++e) from_q += all_counts[static_cast<size_t>(q) * E + e];
+    if (send_rows) send_rows[q] = to_q;
+    if (recv_from) recv_from[q] = from_q;
+    recv += from_q;
+  }
+  if (recv_rows) *recv_rows = recv;
+  return BEAM_OK;
+}
+
+beam_status beam_moe_ep_count(const beam_moe_shape* shape, int32_t P, const int32_t* topk_idx,
+                              int32_t* counts, int64_t recv_rows_max, void* ws, size_t ws_bytes,
+                              beam_stream stream) {
+  beam_status b = check_ep(shape, P, recv_rows_max);
+  if (b != BEAM_OK) return b;
+  if (!counts || !aligned16(counts) || (shape->T > 0 && (!topk_idx || !aligned16(topk_idx))))
+    return BEAM_ERR_INVALID_ARG;
+  const EpLayout L = plan_ep(*shape, P, recv_rows_max);
+  if ((b = check_ep_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(ws, 0, L.zero_bytes, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  EpCountArgs a{};
+  a.idx = topk_idx;
+  a.cnt = at<int32_t>(ws, L.cnt);
+  a.bits = at<uint32_t>(ws, L.bits);
+  a.words = L.words;
+  a.status = at<uint32_t>(ws, L.status);
+  a.T = shape->T;
+  a.k = shape->top_k;
+  a.E = shape->E;
+  if (shape->T > 0) BEAM_LAUNCH(kKEpCount, st, launch_ep_count(a, st));
+  e = cudaMemcpyAsync(counts, a.cnt, sizeof(int32_t) * shape->E, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return BEAM_OK;
+}
+
+beam_status beam_moe_ep_dispatch(const beam_moe_shape* shape, int32_t P, int32_t rank,
+                                 const void* hidden, const int32_t* topk_idx,
+                                 const int32_t* all_counts, void* const* xrecv_peers,
+                                 int64_t recv_rows_max, void* ws, size_t ws_bytes,
+                                 beam_stream stream) {
+  beam_status b = check_ep(shape, P, recv_rows_max);
+  if (b != BEAM_OK) return b;
+  if (rank < 0 || rank >= P || !xrecv_peers) return BEAM_ERR_INVALID_ARG;
+  if (shape->T == 0) return BEAM_OK;  // nothing to send
+  if (any_misaligned({hidden, topk_idx, all_counts})) return BEAM_ERR_INVALID_ARG;
+  for (int q = 0; q < P; ++q)
+    if (!xrecv_peers[q] || !aligned16(xrecv_peers[q])) return BEAM_ERR_INVALID_ARG;
+  const EpLayout L = plan_ep(*shape, P, recv_rows_max);
+  if ((b = check_ep_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  EpOffsetsArgs oa{};
+  oa.all = all_counts;
+  oa.bits = at<uint32_t>(ws, L.bits);
+  oa.base = at<int32_t>(ws, L.base);
+  oa.row_off = at<int64_t>(ws, L.row_off);
+  oa.words = L.words;
+  oa.P = P;
+  oa.E = shape->E;
+  oa.rank = rank;
+  BEAM_LAUNCH(kKEpOffsets, st, launch_ep_offsets(oa, st));
+  EpPushArgs pa{};
+  pa.h = static_cast<const __nv_bfloat16*>(hidden);
+  pa.idx = topk_idx;
+  pa.bits = oa.bits;
+  pa.base = oa.base;
+  pa.words = L.words;
+  pa.row_off = oa.row_off;
+  pa.slot_row = at<int32_t>(ws, L.slot_row);
+  pa.slot_owner = at<int32_t>(ws, L.slot_owner);
+  for (int q = 0; q < P; ++q) pa.xrecv[q] = static_cast<__nv_bfloat16*>(xrecv_peers[q]);
+  pa.recv_cap = recv_rows_max;
+  pa.status = at<uint32_t>(ws, L.status);
+  pa.T = shape->T;
+  pa.d = shape->d;
+  pa.k = shape->top_k;
+  pa.E = shape->E;
+  pa.P = P;
+  BEAM_LAUNCH(kKEpPush, st, launch_ep_push(pa, st));
+  return BEAM_OK;
+}
+
+beam_status beam_moe_ep_experts(const beam_moe_shape* shape, int32_t P, int32_t rank,
+                                int64_t T_total, const int32_t* all_counts, const void* w_gate,
+                                const void* w_up, const void* w_down, const void* xrecv,
+                                void* yrecv, int64_t recv_rows_max, void* ws, size_t ws_bytes,
+                                beam_stream stream) {
+  beam_status b = check_ep(shape, P, recv_rows_max);
+  if (b != BEAM_OK) return b;
+  if (rank < 0 || rank >= P || T_total < 0) return BEAM_ERR_INVALID_ARG;
+  if (any_misaligned({all_counts, w_gate, w_up, w_down, xrecv, yrecv})) return BEAM_ERR_INVALID_ARG;
+  const EpLayout L = plan_ep(*shape, P, recv_rows_max);
+  if ((b = check_ep_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
+  DeviceInfo* dev;
+  if ((b = device_info(&dev)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int ep = shape->E / P;
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  BEAM_LAUNCH(kKEpLocalCounts, st,
+              launch_ep_local_counts(all_counts, P, shape->E, rank, recv_rows_max,
+                                     at<int32_t>(ws, L.cnt_local), status, st));
+  DispatchArgs da{};
+  da.cnt = at<int32_t>(ws, L.cnt_local);
+  da.bits = nullptr;  // the received rows are already in place: no bitmap ranks to form
+  da.base = nullptr;
+  da.off = at<int32_t>(ws, L.off);
+  da.mt_count = at<int32_t>(ws, L.mt_count);
+  da.mtiles = at<MTile>(ws, L.mtiles);
+  da.E = ep;
+  da.words = 0;
+  da.tile_rows = kBM;
+  BEAM_LAUNCH(kKDispatchScan, st, launch_dispatch_scan(da, st));
+
+  const uint64_t R = static_cast<uint64_t>(recv_rows_max);
+  ATensorMaps tm_x, tm_act;
+  CUtensorMap tm_g, tm_u, tm_d;
+  void* act = at<void>(ws, L.act);
+  for (int i = 0; i < kNumABoxes; ++i) {
+    if ((b = make_map(&tm_x.m[i], xrecv, shape->d, R, a_box_rows(i))) != BEAM_OK) return b;
+    if ((b = make_map(&tm_act.m[i], act, shape->I, R, a_box_rows(i))) != BEAM_OK) return b;
+  }
+  const uint64_t EI = static_cast<uint64_t>(ep) * shape->I, Ed = static_cast<uint64_t>(ep) * shape->d;
+  if ((b = make_map(&tm_g, w_gate, shape->d, EI, kN1Half)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_u, w_up, shape->d, EI, kN1Half)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_d, w_down, shape->I, Ed, kN2)) != BEAM_OK) return b;
+  GemmArgs g1{};
+  g1.mtiles = da.mtiles;
+  g1.mt_count = da.mt_count;
+  g1.out = static_cast<__nv_bfloat16*>(act);
+  g1.status = status;
+  g1.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  g1.out_ld = shape->I;
+  g1.n_tiles_n = shape->I / kN1Half;
+  g1.k_blocks = shape->d / kBK;
+  g1.b_rows_per_expert = shape->I;
+  // the single-GPU forward's choice for the whole batch, so that every tile is computed alike
+  g1.swap_max_rows = T_total * shape->top_k <= 8 * static_cast<int64_t>(shape->E) ? kSwapMaxRows : 0;
+  const int64_t max1 = L.mt_cap * g1.n_tiles_n;
+  BEAM_LAUNCH(kKGemmGateUp, st,
+              launch_gemm_gate_up(tm_x, tm_g, tm_u, g1, static_cast<int>(max1 < dev->sms ? max1 : dev->sms), st));
+  GemmArgs g2 = g1;
+  g2.out = static_cast<__nv_bfloat16*>(yrecv);
+  g2.out_ld = shape->d;
+  g2.n_tiles_n = shape->d / kN2;
+  g2.k_blocks = shape->I / kBK;
+  g2.b_rows_per_expert = shape->d;
+  const int64_t max2 = L.mt_cap * g2.n_tiles_n;
+  BEAM_LAUNCH(kKGemmDown, st,
+              launch_gemm_down(tm_act, tm_d, g2, static_cast<int>(max2 < dev->sms ? max2 : dev->sms), st));
+  return BEAM_OK;
+}
+
+beam_status beam_moe_ep_combine(const beam_moe_shape* shape, int32_t P, const float* topk_w,
+                                const void* const* yrecv_peers, int64_t recv_rows_max, void* out,
+                                void* ws, size_t ws_bytes, beam_stream stream) {
+  beam_status b = check_ep(shape, P, recv_rows_max);
+  if (b != BEAM_OK) return b;
+  if (!yrecv_peers) return BEAM_ERR_INVALID_ARG;
+  if (shape->T == 0) return BEAM_OK;
+  if (any_misaligned({topk_w, out})) return BEAM_ERR_INVALID_ARG;
+  for (int q = 0; q < P; ++q)
+    if (!yrecv_peers[q] || !aligned16(yrecv_peers[q])) return BEAM_ERR_INVALID_ARG;
+  const EpLayout L = plan_ep(*shape, P, recv_rows_max);
+  if ((b = check_ep_ws(L, ws, ws_bytes)) != BEAM_OK) return b;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  EpCombineArgs a{};
+  a.slot_row = at<int32_t>(ws, L.slot_row);
+  a.slot_owner = at<int32_t>(ws, L.slot_owner);
+  a.w = topk_w;
+  for (int q = 0; q < P; ++q) a.yrecv[q] = static_cast<const __nv_bfloat16*>(yrecv_peers[q]);
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.recv_cap = recv_rows_max;
+  a.status = at<uint32_t>(ws, L.status);
+  a.T = shape->T;
+  a.d = shape->d;
+  a.k = shape->top_k;
+  a.P = P;
+  BEAM_LAUNCH(kKEpCombine, st, launch_ep_combine(a, st));
   return BEAM_OK;
 }
 

@@ -55,6 +55,7 @@ enum : uint32_t {
   kWherePermute = 6,
   kWhereCombine = 7,
   kWhereSelect = 8,
+  kWhereDispatch = 9,
 };
 
 // Four views of the same row-major A operand (Xp or act) whose TMA boxes are 16, 32, 64 and
@@ -72,8 +73,31 @@ struct MTile {
   int32_t e;      // expert
   int32_t row0;   // first row in the expert-contiguous buffers
   int32_t nrows;  // valid rows, 1..kBM
-  int32_t pad;
+  int32_t band;   // raster band holding this m-tile: (first m-tile << 4) | m-tiles (1..15)
 };
+constexpr int kBandLenBits = 4;
+static_assert(2 * kBand - 1 < (1 << kBandLenBits), "a band's length must fit its field");
+
+// Raster bands group the m-tiles whose tiles run back to back, slice-major, so that the CTAs
+// working at the same time share weight slices (and A rows) through L2.  A band holds whole
+// experts: the experts of at most kBand m-tiles whose first m-tile falls in the same block of
+// kBand m-tiles (so up to 2 kBand - 1 m-tiles); an expert with more m-tiles is cut into bands
+// of kBand.  An expert therefore never straddles two bands unless it must, and its weight
+// slices are streamed from HBM once per band.
+__host__ __device__ constexpr int32_t pack_band(int start, int len) {
+  return (start << kBandLenBits) | len;
+}
+
+// Tile t of a launch whose m-tiles carry bands: m-tile mt and N slice n.  The tiles of a band
+// are contiguous in t, so the band of tile t is the band of m-tile t / n_tiles.
+__device__ __forceinline__ void band_decode_tile(const MTile* mtiles, int t, int n_tiles, int& mt,
+                                                 int& n) {
+  const int32_t b = mtiles[t / n_tiles].band;
+  const int start = b >> kBandLenBits, len = b & ((1 << kBandLenBits) - 1);
+  const int r = t - start * n_tiles;
+  n = r / len;
+  mt = start + (r - n * len);
+}
 
 // ------------------------------------------------------------------ kernel arguments
 
@@ -108,6 +132,7 @@ struct DispatchArgs {
   const int32_t* cnt;    // [E]
   const uint32_t* bits;  // [E, words] token bitmap
   int32_t* base;         // [E, words] out: set bits of the expert's earlier words
+  int32_t* tok_of_row;   // [R] out: token of each row (row gather), or null
   int32_t* off;          // [E + 1]
   int32_t* mt_count;     // [1] number of m-tiles
   MTile* mtiles;         // [capacity]
@@ -141,6 +166,9 @@ struct GemmArgs {
   int k_blocks;            // K / kBK
   int b_rows_per_expert;   // rows of one expert in the 2-D weight view (I or d)
   int swap_max_rows;       // m-tiles with at most this many rows run weights-as-M (0: none)
+  // gate/up (BF16) with a row gather: A rows are token rows h[tok_of_row[row]] read through the
+  // row-gather map in tmA.m[0] (else null: A rows are rows of an expert-contiguous buffer)
+  const int32_t* tok_of_row;
   // FP8 instances only: D = acc * a_scale[A row] * b_scale[B row] (b_scale1: the up slice)
   const float* a_scale;
   const float* b_scale0;
@@ -149,8 +177,15 @@ struct GemmArgs {
 
 struct CombineArgs {
   const __nv_bfloat16* y;  // [R, d]
-  const int32_t* rowmap;   // [T, k]
+  int32_t* rowmap;         // [T, k] row of each slot: read, or (with bits) written
   const float* w;          // [T, k]
+  // with a row gather no permute runs: each slot's row is formed here from the routing, the
+  // token bitmap and the offsets, and recorded in rowmap
+  const int32_t* idx;      // [T, k]
+  const uint32_t* bits;    // [E, words], or null
+  const int32_t* base;     // [E, words]
+  const int32_t* off;      // [E + 1]
+  int words, E;
   __nv_bfloat16* out;      // [T, d] (layer)
   // block form
   const float* x;          // [T, d]
@@ -169,7 +204,61 @@ struct PreNormArgs {
   int T, d;
 };
 
+// ---- expert parallelism (ep.cu): P ranks, rank p owning experts p*E/P .. (p+1)*E/P - 1
+
+constexpr int kMaxEpRanks = 64;
+
+struct EpCountArgs {
+  const int32_t* idx;  // [T, k] local routing
+  int32_t* cnt;        // [E] out (zeroed before the call)
+  uint32_t* bits;      // [E, words] out: token bitmap (zeroed before the call)
+  int words;
+  uint32_t* status;
+  int T, k, E;
+};
+
+struct EpOffsetsArgs {
+  const int32_t* all;     // [P, E] slot counts of every rank
+  const uint32_t* bits;   // [E, words] local token bitmap
+  int32_t* base;          // [E, words] out: its per-expert prefix counts
+  int64_t* row_off;       // [E] out: row of this rank's first slot of e on e's owner
+  int words, P, E, rank;
+};
+
+struct EpPushArgs {
+  const __nv_bfloat16* h;  // [T, d] local tokens
+  const int32_t* idx;      // [T, k]
+  const uint32_t* bits;
+  const int32_t* base;
+  int words;
+  const int64_t* row_off;  // [E]
+  int32_t* slot_row;       // [T, k] out: row on the owner (-1: not sent)
+  int32_t* slot_owner;     // [T, k] out: owner rank
+  __nv_bfloat16* xrecv[kMaxEpRanks];  // receive buffers [recv_cap, d] of every rank
+  int64_t recv_cap;
+  uint32_t* status;
+  int T, d, k, E, P;
+};
+
+struct EpCombineArgs {
+  const int32_t* slot_row;
+  const int32_t* slot_owner;
+  const float* w;                            // [T, k]
+  const __nv_bfloat16* yrecv[kMaxEpRanks];   // expert outputs [recv_cap, d] of every rank
+  __nv_bfloat16* out;                        // [T, d]
+  int64_t recv_cap;
+  uint32_t* status;
+  int T, d, k, P;
+};
+
 // ------------------------------------------------------------------ launchers (one per kernel)
+
+cudaError_t launch_ep_count(const EpCountArgs& a, cudaStream_t s);
+cudaError_t launch_ep_offsets(const EpOffsetsArgs& a, cudaStream_t s);
+cudaError_t launch_ep_push(const EpPushArgs& a, cudaStream_t s);
+cudaError_t launch_ep_local_counts(const int32_t* all, int P, int E, int rank, int64_t recv_cap,
+                                   int32_t* cnt_local, uint32_t* status, cudaStream_t s);
+cudaError_t launch_ep_combine(const EpCombineArgs& a, cudaStream_t s);
 
 cudaError_t launch_router_transpose(const float* W, float* WT, int E, int d, cudaStream_t s);
 cudaError_t launch_router_gemm(const RouterGemmArgs& a, int S, cudaStream_t s);
@@ -197,6 +286,7 @@ cudaError_t launch_dense_tiles(int T, MTile* mtiles, int32_t* mt_count, cudaStre
 cudaError_t launch_bias_update(const int32_t* cnt, float* bias, int E, float mean, float gamma,
                                cudaStream_t s);
 cudaError_t prepare_gemm_kernels();  // opt-in shared memory sizes (once per device)
+cudaError_t prepare_router_kernels();
 
 // ------------------------------------------------------------------ device helpers
 
@@ -318,6 +408,26 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
       : "memory");
+}
+
+// Four rows y0..y3 of a 2-D tensor map whose box is one row high, columns x .. x + box - 1,
+// written to shared memory as four consecutive box rows (swizzled like a four-row box at dst).
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* m, uint32_t bar,
+                                            int32_t x, int32_t y0, int32_t y1, int32_t y2,
+                                            int32_t y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+      : "memory");
+}
+
+// Asks L2 to fetch the box at (x, y) of tensor map m (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 
 // ---- tcgen05

@@ -17,36 +17,79 @@ namespace beam {
 namespace {
 
 // A warp per expert e: the rows and m-tiles of the experts before e give its offset and its
-// first m-tile; the exclusive prefix counts of its row of the token bitmap give each of its
-// tokens a rank.
+// first m-tile, and the m-tile counts of its neighbours its raster band; the exclusive prefix
+// counts of its row of the token bitmap give each of its tokens a rank.
 __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a) {
+  __shared__ int first_sh[8][kMaxE + 1];  // per warp: first m-tile of every expert, [E] = total
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * 8 + warp;
   if (e >= a.E) return;  // uniform over the warp
   const int tr = a.tile_rows;
-  int c_before = 0, m_before = 0;
-  for (int i = lane; i < e; i += 32) {
-    const int c = a.cnt[i];
-    c_before += c;
-    m_before += (c + tr - 1) / tr;
+  int* first = first_sh[warp];
+  {
+    // lane l takes experts l * per .. l * per + per - 1
+    const int per = (a.E + 31) / 32;
+    int msum = 0;
+    for (int i = 0; i < per; ++i) {
+      const int ee = lane * per + i;
+      if (ee < a.E) msum += (a.cnt[ee] + tr - 1) / tr;
+    }
+    int incl = msum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    int run = incl - msum;
+    for (int i = 0; i < per; ++i) {
+      const int ee = lane * per + i;
+      if (ee < a.E) {
+        first[ee] = run;
+        run += (a.cnt[ee] + tr - 1) / tr;
+      }
+    }
+    if (lane == 31) first[a.E] = incl;
+    __syncwarp();
   }
+  int c_before = 0;
+  for (int i = lane; i < e; i += 32) c_before += a.cnt[i];
   c_before = __reduce_add_sync(0xffffffffu, c_before);
-  m_before = __reduce_add_sync(0xffffffffu, m_before);
   const int c = a.cnt[e];
-  const int m = (c + tr - 1) / tr;
+  const int m_before = first[e];
+  const int m = first[e + 1] - m_before;
   if (lane == 0) {
     a.off[e] = c_before;
     if (e == a.E - 1) {
       a.off[a.E] = c_before + c;
-      *a.mt_count = m_before + m;
+      *a.mt_count = first[a.E];
     }
+  }
+  // raster band of a small expert (at most kBand m-tiles): the run of neighbouring small
+  // experts whose first m-tile lies in the same block of kBand m-tiles
+  int run_start = 0, run_end = 0;
+  if (m > 0 && m <= kBand) {
+    const int key = m_before / kBand;
+    auto small_in_block = [&](int x) {
+      const int mx = first[x + 1] - first[x];
+      return mx <= kBand && first[x] / kBand == key;
+    };
+    int lo = e, hi = e;
+    while (lo > 0 && small_in_block(lo - 1)) --lo;
+    while (hi + 1 < a.E && small_in_block(hi + 1)) ++hi;
+    run_start = first[lo];
+    run_end = first[hi + 1];
   }
   for (int i = lane; i < m; i += 32) {
     MTile t;
     t.e = e;
     t.row0 = c_before + i * tr;
     t.nrows = min(tr, c - i * tr);
-    t.pad = 0;
+    if (m <= kBand) {
+      t.band = pack_band(run_start, run_end - run_start);
+    } else {  // a large expert: bands of kBand of its own m-tiles
+      const int b0 = (i / kBand) * kBand;
+      t.band = pack_band(m_before + b0, min(kBand, m - b0));
+    }
     a.mtiles[m_before + i] = t;
   }
   const uint32_t* bits = a.bits + static_cast<size_t>(e) * a.words;
@@ -61,7 +104,17 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a
       const int o = __shfl_up_sync(0xffffffffu, incl, off);
       if (lane >= off) incl += o;
     }
-    if (w < a.words) base[w] = run + incl - n;
+    if (w < a.words) {
+      base[w] = run + incl - n;
+      if (a.tok_of_row) {  // the word's tokens, in order, own the expert's next rows
+        uint32_t word = bits[w];
+        int32_t* dst = a.tok_of_row + c_before + run + incl - n;
+        while (word) {
+          *dst++ = 32 * w + (__ffs(word) - 1);
+          word &= word - 1u;
+        }
+      }
+    }
     run += __shfl_sync(0xffffffffu, incl, 31);
   }
 }
@@ -171,7 +224,8 @@ __global__ void dense_tiles_kernel(int T, MTile* mtiles, int32_t* mt_count) {
     t.e = 0;
     t.row0 = i * kBM;
     t.nrows = min(kBM, T - i * kBM);
-    t.pad = 0;
+    const int b0 = (i / kBand) * kBand;
+    t.band = pack_band(b0, min(kBand, n - b0));
     mtiles[i] = t;
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) *mt_count = n;

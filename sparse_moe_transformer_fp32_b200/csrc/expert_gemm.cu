@@ -23,8 +23,10 @@
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (each warp owns its 32-lane quarter),
 //              FP32 SwiGLU / conversion to BF16, 16-byte stores; the accumulator is then
 //              released so the MMA of the next tile overlaps this epilogue
-// Tiles are visited in bands of kBand m-tiles, slice-major inside a band, so the CTAs running
-// at the same time share A rows and weight slices through L2.
+// Tiles are visited band by band (each m-tile names its raster band: whole experts of up to
+// 2 kBand - 1 m-tiles, see dispatch.cu), slice-major inside a band, so the CTAs running at the
+// same time share A rows and weight slices through L2 and no expert's weights are streamed
+// from HBM twice because its m-tiles fell into two bands.
 //
 // In calls where nearly every m-tile is tiny (decode sizes: a few rows per expert), a tile with
 // at most swap_max_rows rows swaps the operand roles: the two 128-row halves of the weight tile become M and the
@@ -43,22 +45,23 @@ namespace beam {
 namespace {
 
 constexpr uint64_t kMinDrainNs = 1000000000ull;  // drains always get at least 1 s
+// Weight k-blocks the first m-tile of each expert in a band asks L2 to fetch ahead of its own
+// loads (0: none), so that the slice streams from HBM with more bytes in flight than the ring
+// holds; the band's other m-tiles of the expert then find it in L2.
+constexpr int kWeightL2PrefetchKb = 0;
 
-__device__ __forceinline__ void decode_tile(int t, int m_tiles, int n_tiles, int& mt, int& n) {
-  const int band_tiles = kBand * n_tiles;
-  const int band = t / band_tiles;
-  const int base = band * kBand;
-  const int gm = min(kBand, m_tiles - base);
-  const int r = t - band * band_tiles;
-  n = r / gm;
-  mt = base + (r - n * gm);
+__device__ __forceinline__ MTile load_tile(const GemmArgs& a, int t, int n_tiles, int& n) {
+  int mt;
+  band_decode_tile(a.mtiles, t, n_tiles, mt, n);
+  return a.mtiles[mt];
 }
 
-__device__ __forceinline__ MTile load_tile(const GemmArgs& a, int t, int m_tiles, int n_tiles,
-                                           int& n) {
-  int mt;
-  decode_tile(t, m_tiles, n_tiles, mt, n);
-  return a.mtiles[mt];
+// Whether tile t's m-tile is the first one of its expert inside its band.
+__device__ __forceinline__ bool leads_band(const GemmArgs& a, int t, int n_tiles) {
+  int mt, n;
+  band_decode_tile(a.mtiles, t, n_tiles, mt, n);
+  const int start = a.mtiles[mt].band >> kBandLenBits;
+  return mt == start || a.mtiles[mt - 1].e != a.mtiles[mt].e;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -89,7 +92,10 @@ __device__ __forceinline__ void scale_columns(uint32_t (&v0)[32], uint32_t (&v1)
   }
 }
 
-template <bool kSwiGLU, bool kSwap, bool kFp8>
+// kGather (gate/up, BF16): the A rows are gathered from the token rows h[T, d] by the m-tile's
+// row -> token map (tma_gather4, four rows an instruction, issued by the producer warp's lanes)
+// instead of being read from an expert-contiguous copy, so no permuted copy of h is written.
+template <bool kSwiGLU, bool kSwap, bool kFp8, bool kGather = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     expert_gemm_kernel(const __grid_constant__ ATensorMaps tmA,
                        const __grid_constant__ CUtensorMap tmB0,
@@ -143,7 +149,64 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == 0 && kGather) {
+    // ------------------------------------------------------------ TMA producer (row gather)
+    // lane g gathers rows 4g .. 4g + 3 of the tile (rows past its end repeat its last row;
+    // like the rows of A past a box, they only feed accumulator rows that are never stored);
+    // lane 0 arms the stage's barrier and loads the weight tile
+    int stage = 0;
+    uint32_t phase = 0, filled = 0, last_parity = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      int n = 0;
+      const MTile m = load_tile(a, t, n_tiles, n);
+      const int brow = m.e * a.b_rows_per_expert + n * kNSlice;
+      const int groups = (m.nrows + 3) >> 2;
+      int tok[4] = {0, 0, 0, 0};
+      if (lane < groups) {
+        const int32_t* tr = a.tok_of_row + m.row0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tok[i] = tr[min(4 * lane + i, m.nrows - 1)];
+      }
+      const uint32_t a_bytes = static_cast<uint32_t>(groups) * 4u * kBK * 2u;
+      for (int kb = 0; kb < a.k_blocks; ++kb) {
+        int ready = 1;
+        if (lane == 0)
+          ready = mbar_wait_bounded(bar(kBarEmpty + stage), phase ^ 1u, abort_flag, limit,
+                                    a.status, kWhereProducerEmpty);
+        if (!__shfl_sync(0xffffffffu, ready, 0)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sA = sbase + stage * kStageBytes;
+        const uint32_t sB = sA + kStageABytes;
+        const uint32_t fb = bar(kBarFull + stage);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(fb, a_bytes + kStageBBytes);
+          tma_load_2d(sB, &tmB0, fb, kb * kKElems, brow);
+          if (kSwiGLU) tma_load_2d(sB + kStageBBytes / 2, &tmB1, fb, kb * kKElems, brow);
+        }
+        __syncwarp();
+        if (lane < groups)
+          tma_gather4(sA + static_cast<uint32_t>(lane) * 4u * kBK * 2u, &tmA.m[0], fb,
+                      kb * kKElems, tok[0], tok[1], tok[2], tok[3]);
+        filled |= 1u << stage;
+        last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // every load of a filled stage (all lanes' gathers included) lands before the CTA exits
+    if (lane == 0) {
+      int no_abort = 0;
+      for (int s = 0; s < kStages; ++s)
+        if ((filled >> s) & 1u)
+          mbar_wait_bounded(bar(kBarFull + s), (last_parity >> s) & 1u, &no_abort, drain_limit,
+                            a.status, kWhereDrain);
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int stage = 0;
@@ -151,16 +214,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       // the next tile's descriptor is loaded one tile ahead, off the critical path
       int n = 0;
-      MTile m = load_tile(a, blockIdx.x, m_tiles, n_tiles, n);
+      MTile m = load_tile(a, blockIdx.x, n_tiles, n);
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         int n_next = 0;
-        const MTile m_next = load_tile(a, t + gridDim.x < ntiles ? t + gridDim.x : t, m_tiles,
+        const MTile m_next = load_tile(a, t + gridDim.x < ntiles ? t + gridDim.x : t,
                                        n_tiles, n_next);
         const int brow = m.e * a.b_rows_per_expert + n * kNSlice;
         // rows of A beyond the box are left from earlier stages: they only feed accumulator
         // rows that are never stored
         const int a_box = a_box_for_rows(m.nrows);
         const uint32_t a_bytes = static_cast<uint32_t>(a_box_rows(a_box)) * kBK * 2;
+        const bool lead = kWeightL2PrefetchKb > 0 && leads_band(a, t, n_tiles);
+        auto prefetch_b = [&](int kb) {
+          tma_prefetch_l2_2d(&tmB0, kb * kKElems, brow);
+          if (kSwiGLU) tma_prefetch_l2_2d(&tmB1, kb * kKElems, brow);
+        };
+        if (lead)
+          for (int kb = kStages; kb < kWeightL2PrefetchKb && kb < a.k_blocks; ++kb) prefetch_b(kb);
         for (int kb = 0; kb < a.k_blocks; ++kb) {
           if (!mbar_wait_bounded(bar(kBarEmpty + stage), phase ^ 1u, abort_flag, limit, a.status,
                                  kWhereProducerEmpty)) {
@@ -174,6 +244,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_2d(sA, &tmA.m[a_box], fb, kb * kKElems, m.row0);
           tma_load_2d(sB, &tmB0, fb, kb * kKElems, brow);
           if (kSwiGLU) tma_load_2d(sB + kStageBBytes / 2, &tmB1, fb, kb * kKElems, brow);
+          if (lead && kb + kWeightL2PrefetchKb < a.k_blocks) prefetch_b(kb + kWeightL2PrefetchKb);
           filled |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -211,9 +282,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       int n_unused = 0;
-      int nrows = load_tile(a, blockIdx.x, m_tiles, n_tiles, n_unused).nrows;
+      int nrows = load_tile(a, blockIdx.x, n_tiles, n_unused).nrows;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const int nrows_next = load_tile(a, t + gridDim.x < ntiles ? t + gridDim.x : t, m_tiles,
+        const int nrows_next = load_tile(a, t + gridDim.x < ntiles ? t + gridDim.x : t,
                                          n_tiles, n_unused).nrows;
         const bool swap = kSwap && nrows <= a.swap_max_rows;
         const uint32_t idesc = swap ? make_idesc(kBM, (nrows + 15) & ~15)
@@ -271,7 +342,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       int mt, n;
-      decode_tile(t, m_tiles, n_tiles, mt, n);
+      band_decode_tile(a.mtiles, t, n_tiles, mt, n);
       const MTile m = a.mtiles[mt];
       int ok = 0;
       if (lane == 0)
@@ -400,7 +471,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }  // namespace
 
 cudaError_t prepare_gemm_kernels() {
-  const void* kernels[] = {reinterpret_cast<const void*>(expert_gemm_kernel<true, false, false>),
+  const void* kernels[] = {reinterpret_cast<const void*>(expert_gemm_kernel<true, false, false, true>),
+                           reinterpret_cast<const void*>(expert_gemm_kernel<true, true, false, true>),
+                           reinterpret_cast<const void*>(expert_gemm_kernel<true, false, false>),
                            reinterpret_cast<const void*>(expert_gemm_kernel<true, true, false>),
                            reinterpret_cast<const void*>(expert_gemm_kernel<false, false, false>),
                            reinterpret_cast<const void*>(expert_gemm_kernel<false, true, false>),
@@ -420,6 +493,17 @@ namespace {
 template <bool kSwiGLU, bool kFp8>
 void launch_gemm(const ATensorMaps& tmA, const CUtensorMap& tmB0, const CUtensorMap& tmB1,
                  const GemmArgs& a, int grid, cudaStream_t s) {
+  if constexpr (kSwiGLU && !kFp8) {
+    if (a.tok_of_row) {
+      if (a.swap_max_rows > 0)
+        expert_gemm_kernel<true, true, false, true>
+            <<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB0, tmB1, a);
+      else
+        expert_gemm_kernel<true, false, false, true>
+            <<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB0, tmB1, a);
+      return;
+    }
+  }
   if (a.swap_max_rows > 0)
     expert_gemm_kernel<kSwiGLU, true, kFp8>
         <<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB0, tmB1, a);

@@ -272,16 +272,6 @@ __host__ __device__ constexpr uint32_t umma_idesc_nvfp4(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-__device__ __forceinline__ void f4_decode_tile(int t, int m_tiles, int n_tiles, int& mt, int& n) {
-  const int band_tiles = kBand * n_tiles;
-  const int band = t / band_tiles;
-  const int base = band * kBand;
-  const int gm = min(kBand, m_tiles - base);
-  const int r = t - band * band_tiles;
-  n = r / gm;
-  mt = base + (r - n * gm);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -362,7 +352,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         int mt, n;
-        f4_decode_tile(t, m_tiles, n_tiles, mt, n);
+        band_decode_tile(a.mtiles, t, n_tiles, mt, n);
         const MTile m = a.mtiles[mt];
         const int brow = m.e * a.b_rows_per_expert + n * kF4N;
         const int a_box = a_box_for_rows(m.nrows);
@@ -455,7 +445,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       int mt, n;
-      f4_decode_tile(t, m_tiles, n_tiles, mt, n);
+      band_decode_tile(a.mtiles, t, n_tiles, mt, n);
       const MTile m = a.mtiles[mt];
       int ok = 0;
       if (lane == 0)

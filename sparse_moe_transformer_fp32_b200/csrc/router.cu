@@ -57,8 +57,9 @@ __device__ __forceinline__ void cp_async_wait_1() {
 }
 
 __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterGemmArgs a) {
-  __shared__ __align__(16) float As[2][kRK][kRM];
-  __shared__ __align__(16) float Bs[kRBStages][kRK][kRN];
+  extern __shared__ __align__(16) float router_smem[];
+  auto& As = *reinterpret_cast<float(*)[2][kRK][kRM]>(router_smem);
+  auto& Bs = *reinterpret_cast<float(*)[kRBStages][kRK][kRN]>(router_smem + 2 * kRK * kRM);
 
   const int tid = threadIdx.x;
   const int m0 = blockIdx.x * kRM;
@@ -72,21 +73,34 @@ __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterG
 
   const int tx = tid & 15;
   const int ty = tid >> 4;
-  // A staging: one 16-byte chunk (8 K values) of one token per thread and K tile
+  // A staging: kAChunks 16-byte chunks (8 K values each) of one token per thread and K tile
+  constexpr int kAChunks = kRK * kRM / 8 / kRThreads;
+  static_assert(kAChunks >= 1 && kRThreads % kRM == 0, "A staging covers the tile");
   const int a_row = tid & (kRM - 1);
-  const int a_kp = (tid >> 7) * 8;
+  const int a_kp = (tid / kRM) * 8 * kAChunks;
   const int a_t = m0 + a_row;
   const __nv_bfloat16* a_src = a.h + static_cast<size_t>(a_t < a.T ? a_t : 0) * a.d + a_kp;
-
-  auto load_a = [&](int k0) -> uint4 {
-    return a_t < a.T ? *reinterpret_cast<const uint4*>(a_src + k0) : make_uint4(0, 0, 0, 0);
+  struct AChunks {
+    uint4 v[kAChunks];
   };
-  auto store_a = [&](int buf, uint4 v) {
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+
+  auto load_a = [&](int k0) -> AChunks {
+    AChunks c;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      As[buf][a_kp + 2 * q][a_row] = __uint_as_float(w4[q] << 16);
-      As[buf][a_kp + 2 * q + 1][a_row] = __uint_as_float(w4[q] & 0xffff0000u);
+    for (int i = 0; i < kAChunks; ++i)
+      c.v[i] = a_t < a.T ? *reinterpret_cast<const uint4*>(a_src + k0 + 8 * i)
+                         : make_uint4(0, 0, 0, 0);
+    return c;
+  };
+  auto store_a = [&](int buf, const AChunks& c) {
+#pragma unroll
+    for (int i = 0; i < kAChunks; ++i) {
+      const uint32_t w4[4] = {c.v[i].x, c.v[i].y, c.v[i].z, c.v[i].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        As[buf][a_kp + 8 * i + 2 * q][a_row] = __uint_as_float(w4[q] << 16);
+        As[buf][a_kp + 8 * i + 2 * q + 1][a_row] = __uint_as_float(w4[q] & 0xffff0000u);
+      }
     }
   };
   auto issue_b = [&](int stage, int k0) {
@@ -126,7 +140,7 @@ __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterG
     __syncthreads();    // ... for every thread, and As[kt & 1] is stored
     if (kt + 2 < nk) issue_b((kt + 2) % kRBStages, kbeg + (kt + 2) * kRK);
     cp_async_commit();
-    uint4 next = make_uint4(0, 0, 0, 0);
+    AChunks next{};
     if (kt + 1 < nk) next = load_a(kbeg + (kt + 1) * kRK);
     const int buf = kt & 1, st = kt % kRBStages;
 #pragma unroll
@@ -381,9 +395,16 @@ cudaError_t launch_router_transpose(const float* W, float* WT, int E, int d, cud
   return cudaGetLastError();
 }
 
+constexpr int kRouterSmemBytes = (2 * kRK * kRM + kRBStages * kRK * kRN) * 4;
+
+cudaError_t prepare_router_kernels() {
+  return cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kRouterSmemBytes);
+}
+
 cudaError_t launch_router_gemm(const RouterGemmArgs& a, int S, cudaStream_t s) {
   const dim3 grid((a.T + kRM - 1) / kRM, (a.E + kRN - 1) / kRN, S);
-  router_gemm_kernel<<<grid, kRThreads, 0, s>>>(a);
+  router_gemm_kernel<<<grid, kRThreads, kRouterSmemBytes, s>>>(a);
   return cudaGetLastError();
 }
 
