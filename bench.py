@@ -243,12 +243,10 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ algorithmic work
 
-def kernel_work(wl, touched: int, fp8: bool = False, nvfp4: bool = False, gather: bool = True):
+def kernel_work(wl, touched: int, fp8: bool = False, nvfp4: bool = False):
     """Algorithmic bytes and FLOPs per launch of each kernel (the minimum each must move).
     With fp8 the weights and the GEMM inputs are one-byte E4M3 codes (row scales ignored); with
-    nvfp4 they are half-byte E2M1 codes plus one E4M3 block scale per 16 elements.  With gather
-    (the BF16 path on single SMs) the gate/up GEMM reads its A rows straight from the token rows,
-    each of which it must read once (T * d * 2 bytes), and no permute runs."""
+    nvfp4 they are half-byte E2M1 codes plus one E4M3 block scale per 16 elements."""
     T, d, E, k, I = wl.T, wl.d, wl.E, wl.top_k, wl.I
     R = T * k
     bf, f4 = 2, 4
@@ -290,14 +288,13 @@ def kernel_work(wl, touched: int, fp8: bool = False, nvfp4: bool = False, gather
         }
     w_gu = touched * 2 * I * d * bf
     w_dn = touched * d * I * bf
-    a_in = (T if gather else R) * d * bf
     return {
         "router_transpose": {"flops": 0, "bytes": 2 * E * d * f4},
         "dispatch_scan": {"flops": 0, "bytes": E * 16},
         "router_gemm": {"flops": 2 * T * d * E, "bytes": T * d * bf + E * d * f4 + T * E * f4},
         "router_select": {"flops": 0, "bytes": T * E * f4 + 2 * R * f4},
         "permute": {"flops": 0, "bytes": T * d * bf + R * d * bf},
-        "expert_gemm_gate_up": {"flops": 4 * R * d * I, "bytes": w_gu + a_in + R * I * bf},
+        "expert_gemm_gate_up": {"flops": 4 * R * d * I, "bytes": w_gu + R * d * bf + R * I * bf},
         "expert_gemm_down": {"flops": 2 * R * d * I, "bytes": w_dn + R * I * bf + R * d * bf},
         "combine": {"flops": 2 * R * d, "bytes": R * d * bf + T * d * bf},
         "combine_block": {"flops": 2 * R * d, "bytes": R * d * bf + 3 * T * d * f4},
@@ -589,8 +586,7 @@ def run_cuda(args, rank, world, local):
 
         result = None
         if rank == 0:
-            work = kernel_work(wl, touched, fp8=bool(fp8), nvfp4=bool(fp4),
-                               gather=not args.sm_pairs)
+            work = kernel_work(wl, touched, fp8=bool(fp8), nvfp4=bool(fp4))
             per_kernel = {k: {"launches": n, "ms_per_launch": (ms / n if n else None)}
                           for k, (n, ms) in prof.items() if n}
             dom = max((k for k in per_kernel if k in work), key=lambda k: prof[k][1])

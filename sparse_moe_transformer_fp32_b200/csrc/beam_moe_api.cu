@@ -136,8 +136,8 @@ beam_status check_shape(const beam_moe_shape* s) {
 }
 
 struct Layout {
-  size_t status, cnt, bits, off, mt_count, mtiles, base, rowmap, tok_of_row, idx, w, wt, part, h,
-      xp, act, y, total;
+  size_t status, cnt, bits, off, mt_count, mtiles, base, rowmap, idx, w, wt, part, h, xp, act, y,
+      total;
   size_t zero_bytes = 0;             // status, counts and token bitmap: cleared at each call
   int words = 0;                     // token bitmap words per expert, ceil(T / 32)
   size_t xs = 0, act8 = 0, as = 0;  // FP8 path: row scales of Xp, E4M3 act, act row scales
@@ -201,7 +201,6 @@ Layout plan(const beam_moe_shape& s) {
   L.mtiles = take(sizeof(MTile) * L.mt_cap);
   L.base = take(bitmap_bytes);
   L.rowmap = take(sizeof(int32_t) * R);
-  L.tok_of_row = take(sizeof(int32_t) * R);
   L.idx = take(sizeof(int32_t) * R);
   L.w = take(sizeof(float) * R);
   L.wt = take(sizeof(float) * static_cast<size_t>(s.E) * s.d);
@@ -395,27 +394,10 @@ struct Fp8Scales {
 // Dispatch, the two expert GEMMs; leaves Y and rowmap in the workspace.  With f8 the weights
 // are E4M3 codes: the permute writes E4M3 rows of Xp with their scales, and the activation is
 // quantised between the two GEMMs.
-// BF16 gate/up GEMMs gather their A rows from the token rows (no permuted copy of h).
-constexpr bool kRowGather = true;
-
-// Sets up the combine's slot rows: read from rowmap (written by the permute), or formed by the
-// combine itself from the routing and the token bitmap when the experts ran with a row gather.
-void combine_rows(CombineArgs& ca, const Layout& L, const beam_moe_shape& s, const int32_t* idx,
-                  void* ws, bool gathered) {
-  ca.rowmap = at<int32_t>(ws, L.rowmap);
-  if (!gathered) return;
-  ca.idx = idx;
-  ca.bits = at<uint32_t>(ws, L.bits);
-  ca.base = at<int32_t>(ws, L.base);
-  ca.off = at<int32_t>(ws, L.off);
-  ca.words = L.words;
-  ca.E = s.E;
-}
-
 beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceInfo& dev,
                         const __nv_bfloat16* h, const int32_t* idx, const void* w_gate,
                         const void* w_up, const void* w_down, void* ws, cudaStream_t st,
-                        const Fp8Scales* f8, bool* gathered) {
+                        const Fp8Scales* f8 = nullptr) {
   uint32_t* status = at<uint32_t>(ws, L.status);
   // With SM pairs enabled, calls averaging at least 256 rows per expert run their expert GEMMs
   // on SM pairs (cta_group::2, 256-row tiles): half the operand bytes per SM for the same tensor
@@ -423,8 +405,6 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   const bool pairs = !f8 && g_sm_pairs.load(std::memory_order_relaxed) != 0 &&
                      L.R >= static_cast<int64_t>(kPairMinRowsPerExpert) * s.E &&
                      dev.pair_grid >= 2;
-  const bool gather = kRowGather && !f8 && !pairs;
-  *gathered = gather;
   DispatchArgs da{};
   da.cnt = at<int32_t>(ws, L.cnt);
   da.bits = at<uint32_t>(ws, L.bits);
@@ -435,7 +415,6 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   da.E = s.E;
   da.words = L.words;
   da.tile_rows = pairs ? 2 * kBM : kBM;
-  da.tok_of_row = gather ? at<int32_t>(ws, L.tok_of_row) : nullptr;
   BEAM_LAUNCH(kKDispatchScan, st, launch_dispatch_scan(da, st));
 
   PermuteArgs pa{};
@@ -454,7 +433,7 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   pa.d = s.d;
   pa.k = s.top_k;
   pa.E = s.E;
-  if (!gather) BEAM_LAUNCH(kKPermute, st, launch_permute(pa, st));
+  BEAM_LAUNCH(kKPermute, st, launch_permute(pa, st));
 
   const uint64_t R = static_cast<uint64_t>(L.R);
   ATensorMaps tm_xp, tm_act;
@@ -464,11 +443,7 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   const void* a1 = at<void>(ws, L.xp);
   const void* a2 = at<void>(ws, f8 ? L.act8 : L.act);
   for (int i = 0; i < kNumABoxes; ++i) {
-    if (gather) {  // one-row boxes over the token rows, four gathered per instruction
-      if ((b = make_map(&tm_xp.m[i], h, s.d, static_cast<uint64_t>(s.T), 1)) != BEAM_OK) return b;
-    } else if ((b = make_map(&tm_xp.m[i], a1, s.d, R, a_box_rows(i), eb)) != BEAM_OK) {
-      return b;
-    }
+    if ((b = make_map(&tm_xp.m[i], a1, s.d, R, a_box_rows(i), eb)) != BEAM_OK) return b;
     if ((b = make_map(&tm_act.m[i], a2, s.I, R, a_box_rows(i), eb)) != BEAM_OK) return b;
   }
   const uint64_t EI = static_cast<uint64_t>(s.E) * s.I, Ed = static_cast<uint64_t>(s.E) * s.d;
@@ -488,7 +463,6 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   g1.n_tiles_n = s.I / kN1Half;
   g1.k_blocks = s.d / k_elems;
   g1.b_rows_per_expert = s.I;
-  g1.tok_of_row = da.tok_of_row;
   if (f8) {
     g1.a_scale = pa.xs;
     g1.b_scale0 = f8->gate;
@@ -514,7 +488,6 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
                                      at<uint8_t>(ws, L.act8), at<float>(ws, L.as), st));
 
   GemmArgs g2 = g1;
-  g2.tok_of_row = nullptr;
   g2.out = at<__nv_bfloat16>(ws, L.y);
   g2.out_ld = s.d;
   g2.n_tiles_n = s.d / kN2;
@@ -808,13 +781,11 @@ beam_status forward_impl(const beam_moe_shape* shape, const void* hidden, const 
   const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(hidden);
   if ((b = run_router(*shape, L, h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
     return b;
-  bool gathered = false;
-  if ((b = run_experts(*shape, L, *dev, h, idx, w_gate, w_up, w_down, ws, st, f8, &gathered)) !=
-      BEAM_OK)
+  if ((b = run_experts(*shape, L, *dev, h, idx, w_gate, w_up, w_down, ws, st, f8)) != BEAM_OK)
     return b;
   CombineArgs ca{};
   ca.y = at<__nv_bfloat16>(ws, L.y);
-  combine_rows(ca, L, *shape, idx, ws, gathered);
+  ca.rowmap = at<int32_t>(ws, L.rowmap);
   ca.w = w;
   ca.out = static_cast<__nv_bfloat16*>(out);
   ca.status = at<uint32_t>(ws, L.status);
@@ -904,14 +875,13 @@ beam_status block_impl(const beam_moe_shape* shape, const float* x, const float*
   float* w = topk_w ? topk_w : at<float>(ws, L.w);
   if ((b = run_router(*shape, L, pn.h, router_w, bias, idx, w, nullptr, true, ws, st)) != BEAM_OK)
     return b;
-  bool gathered = false;
   b = w4 ? run_experts_nvfp4(*shape, L, *dev, pn.h, idx, *w4, ws, st)
-         : run_experts(*shape, L, *dev, pn.h, idx, w_gate, w_up, w_down, ws, st, f8, &gathered);
+         : run_experts(*shape, L, *dev, pn.h, idx, w_gate, w_up, w_down, ws, st, f8);
   if (b != BEAM_OK) return b;
   const double kk = static_cast<double>(k_resid);
   CombineArgs ca{};
   ca.y = at<__nv_bfloat16>(ws, L.y);
-  combine_rows(ca, L, *shape, idx, ws, gathered);
+  ca.rowmap = at<int32_t>(ws, L.rowmap);
   ca.w = w;
   ca.x = x;
   ca.g_post = g_post;

@@ -132,7 +132,6 @@ struct DispatchArgs {
   const int32_t* cnt;    // [E]
   const uint32_t* bits;  // [E, words] token bitmap
   int32_t* base;         // [E, words] out: set bits of the expert's earlier words
-  int32_t* tok_of_row;   // [R] out: token of each row (row gather), or null
   int32_t* off;          // [E + 1]
   int32_t* mt_count;     // [1] number of m-tiles
   MTile* mtiles;         // [capacity]
@@ -166,9 +165,6 @@ struct GemmArgs {
   int k_blocks;            // K / kBK
   int b_rows_per_expert;   // rows of one expert in the 2-D weight view (I or d)
   int swap_max_rows;       // m-tiles with at most this many rows run weights-as-M (0: none)
-  // gate/up (BF16) with a row gather: A rows are token rows h[tok_of_row[row]] read through the
-  // row-gather map in tmA.m[0] (else null: A rows are rows of an expert-contiguous buffer)
-  const int32_t* tok_of_row;
   // FP8 instances only: D = acc * a_scale[A row] * b_scale[B row] (b_scale1: the up slice)
   const float* a_scale;
   const float* b_scale0;
@@ -177,15 +173,8 @@ struct GemmArgs {
 
 struct CombineArgs {
   const __nv_bfloat16* y;  // [R, d]
-  int32_t* rowmap;         // [T, k] row of each slot: read, or (with bits) written
+  const int32_t* rowmap;   // [T, k]
   const float* w;          // [T, k]
-  // with a row gather no permute runs: each slot's row is formed here from the routing, the
-  // token bitmap and the offsets, and recorded in rowmap
-  const int32_t* idx;      // [T, k]
-  const uint32_t* bits;    // [E, words], or null
-  const int32_t* base;     // [E, words]
-  const int32_t* off;      // [E + 1]
-  int words, E;
   __nv_bfloat16* out;      // [T, d] (layer)
   // block form
   const float* x;          // [T, d]
@@ -407,18 +396,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
-      : "memory");
-}
-
-// Four rows y0..y3 of a 2-D tensor map whose box is one row high, columns x .. x + box - 1,
-// written to shared memory as four consecutive box rows (swizzled like a four-row box at dst).
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* m, uint32_t bar,
-                                            int32_t x, int32_t y0, int32_t y1, int32_t y2,
-                                            int32_t y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
       : "memory");
 }
 

@@ -48,15 +48,7 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 __device__ __forceinline__ void load_slots(const CombineArgs& a, int t, int* rows, float* ws) {
   if (threadIdx.x < a.k) {
     const size_t slot = static_cast<size_t>(t) * a.k + threadIdx.x;
-    int r;
-    if (a.bits) {
-      const int e = a.idx[slot];
-      const int rk = e >= 0 && e < a.E ? slot_rank(a.bits, a.base, a.words, e, t) : -1;
-      r = rk >= 0 ? a.off[e] + rk : -1;
-      a.rowmap[slot] = r;
-    } else {
-      r = a.rowmap[slot];
-    }
+    int r = a.rowmap[slot];
     float w = a.w[slot];
     if (r < 0 || r >= a.R) {
       record_status(a.status, kDevAssert, kWhereCombine);

@@ -104,17 +104,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a
       const int o = __shfl_up_sync(0xffffffffu, incl, off);
       if (lane >= off) incl += o;
     }
-    if (w < a.words) {
-      base[w] = run + incl - n;
-      if (a.tok_of_row) {  // the word's tokens, in order, own the expert's next rows
-        uint32_t word = bits[w];
-        int32_t* dst = a.tok_of_row + c_before + run + incl - n;
-        while (word) {
-          *dst++ = 32 * w + (__ffs(word) - 1);
-          word &= word - 1u;
-        }
-      }
-    }
+    if (w < a.words) base[w] = run + incl - n;
     run += __shfl_sync(0xffffffffu, incl, 31);
   }
 }

@@ -92,10 +92,7 @@ __device__ __forceinline__ void scale_columns(uint32_t (&v0)[32], uint32_t (&v1)
   }
 }
 
-// kGather (gate/up, BF16): the A rows are gathered from the token rows h[T, d] by the m-tile's
-// row -> token map (tma_gather4, four rows an instruction, issued by the producer warp's lanes)
-// instead of being read from an expert-contiguous copy, so no permuted copy of h is written.
-template <bool kSwiGLU, bool kSwap, bool kFp8, bool kGather = false>
+template <bool kSwiGLU, bool kSwap, bool kFp8>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     expert_gemm_kernel(const __grid_constant__ ATensorMaps tmA,
                        const __grid_constant__ CUtensorMap tmB0,
@@ -149,64 +146,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0 && kGather) {
-    // ------------------------------------------------------------ TMA producer (row gather)
-    // lane g gathers rows 4g .. 4g + 3 of the tile (rows past its end repeat its last row;
-    // like the rows of A past a box, they only feed accumulator rows that are never stored);
-    // lane 0 arms the stage's barrier and loads the weight tile
-    int stage = 0;
-    uint32_t phase = 0, filled = 0, last_parity = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-      int n = 0;
-      const MTile m = load_tile(a, t, n_tiles, n);
-      const int brow = m.e * a.b_rows_per_expert + n * kNSlice;
-      const int groups = (m.nrows + 3) >> 2;
-      int tok[4] = {0, 0, 0, 0};
-      if (lane < groups) {
-        const int32_t* tr = a.tok_of_row + m.row0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tok[i] = tr[min(4 * lane + i, m.nrows - 1)];
-      }
-      const uint32_t a_bytes = static_cast<uint32_t>(groups) * 4u * kBK * 2u;
-      for (int kb = 0; kb < a.k_blocks; ++kb) {
-        int ready = 1;
-        if (lane == 0)
-          ready = mbar_wait_bounded(bar(kBarEmpty + stage), phase ^ 1u, abort_flag, limit,
-                                    a.status, kWhereProducerEmpty);
-        if (!__shfl_sync(0xffffffffu, ready, 0)) {
-          ok = false;
-          break;
-        }
-        const uint32_t sA = sbase + stage * kStageBytes;
-        const uint32_t sB = sA + kStageABytes;
-        const uint32_t fb = bar(kBarFull + stage);
-        if (lane == 0) {
-          mbar_arrive_expect_tx(fb, a_bytes + kStageBBytes);
-          tma_load_2d(sB, &tmB0, fb, kb * kKElems, brow);
-          if (kSwiGLU) tma_load_2d(sB + kStageBBytes / 2, &tmB1, fb, kb * kKElems, brow);
-        }
-        __syncwarp();
-        if (lane < groups)
-          tma_gather4(sA + static_cast<uint32_t>(lane) * 4u * kBK * 2u, &tmA.m[0], fb,
-                      kb * kKElems, tok[0], tok[1], tok[2], tok[3]);
-        filled |= 1u << stage;
-        last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-    }
-    // every load of a filled stage (all lanes' gathers included) lands before the CTA exits
-    if (lane == 0) {
-      int no_abort = 0;
-      for (int s = 0; s < kStages; ++s)
-        if ((filled >> s) & 1u)
-          mbar_wait_bounded(bar(kBarFull + s), (last_parity >> s) & 1u, &no_abort, drain_limit,
-                            a.status, kWhereDrain);
-    }
-  } else if (warp == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int stage = 0;
@@ -471,9 +411,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }  // namespace
 
 cudaError_t prepare_gemm_kernels() {
-  const void* kernels[] = {reinterpret_cast<const void*>(expert_gemm_kernel<true, false, false, true>),
-                           reinterpret_cast<const void*>(expert_gemm_kernel<true, true, false, true>),
-                           reinterpret_cast<const void*>(expert_gemm_kernel<true, false, false>),
+  const void* kernels[] = {reinterpret_cast<const void*>(expert_gemm_kernel<true, false, false>),
                            reinterpret_cast<const void*>(expert_gemm_kernel<true, true, false>),
                            reinterpret_cast<const void*>(expert_gemm_kernel<false, false, false>),
                            reinterpret_cast<const void*>(expert_gemm_kernel<false, true, false>),
@@ -493,17 +431,6 @@ namespace {
 template <bool kSwiGLU, bool kFp8>
 void launch_gemm(const ATensorMaps& tmA, const CUtensorMap& tmB0, const CUtensorMap& tmB1,
                  const GemmArgs& a, int grid, cudaStream_t s) {
-  if constexpr (kSwiGLU && !kFp8) {
-    if (a.tok_of_row) {
-      if (a.swap_max_rows > 0)
-        expert_gemm_kernel<true, true, false, true>
-            <<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB0, tmB1, a);
-      else
-        expert_gemm_kernel<true, false, false, true>
-            <<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB0, tmB1, a);
-      return;
-    }
-  }
   if (a.swap_max_rows > 0)
     expert_gemm_kernel<kSwiGLU, true, kFp8>
         <<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB0, tmB1, a);

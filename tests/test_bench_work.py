@@ -20,12 +20,8 @@ def test_gate_up_work_matches_the_profiles():
     wl = W.WORKLOADS["prefill"]
     R = wl.T * wl.top_k
     flops = 4 * R * wl.d * wl.I
-    # bf16: A rows gathered from the 4096 token rows (each read once); bf16-permuted: A rows
-    # read from the 32768-row expert-contiguous copy (the SM-pair path)
-    for fmt, gbytes in (("bf16", 13.631), ("bf16-permuted", 13.925), ("fp8", 7.046),
-                        ("nvfp4", 4.037)):
-        work = b.kernel_work(wl, 256, fp8=fmt == "fp8", nvfp4=fmt == "nvfp4",
-                             gather=fmt != "bf16-permuted")
+    for fmt, gbytes in (("bf16", 13.925), ("fp8", 7.046), ("nvfp4", 4.037)):
+        work = b.kernel_work(wl, 256, fp8=fmt == "fp8", nvfp4=fmt == "nvfp4")
         gu = work["expert_gemm_gate_up"]
         assert gu["flops"] == flops == 1717986918400
         assert round(gu["bytes"] / 1e9, 3) == gbytes, fmt
