@@ -26,34 +26,54 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a
   if (e >= a.E) return;  // uniform over the warp
   const int tr = a.tile_rows;
   int* first = first_sh[warp];
-  {
-    // lane l takes experts l * per .. l * per + per - 1
-    const int per = (a.E + 31) / 32;
-    int msum = 0;
-    for (int i = 0; i < per; ++i) {
-      const int ee = lane * per + i;
-      if (ee < a.E) msum += (a.cnt[ee] + tr - 1) / tr;
-    }
-    int incl = msum;
+  // lane l takes experts l * per .. l * per + per - 1: their counts are read once and give both
+  // the row offsets and the m-tile offsets; the first words of e's bitmap row are fetched
+  // meanwhile
+  const int per = (a.E + 31) / 32;
+  int cnt_l[kMaxE / 32];
+  int msum = 0, csum = 0;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += o;
+  for (int i = 0; i < kMaxE / 32; ++i) {
+    const int ee = lane * per + i;
+    cnt_l[i] = i < per && ee < a.E ? a.cnt[ee] : 0;
+    msum += (cnt_l[i] + tr - 1) / tr;
+    csum += cnt_l[i];
+  }
+  const uint32_t word0 = lane < a.words ? a.bits[static_cast<size_t>(e) * a.words + lane] : 0u;
+  int mincl = msum, cincl = csum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int om = __shfl_up_sync(0xffffffffu, mincl, off);
+    const int oc = __shfl_up_sync(0xffffffffu, cincl, off);
+    if (lane >= off) {
+      mincl += om;
+      cincl += oc;
     }
-    int run = incl - msum;
-    for (int i = 0; i < per; ++i) {
+  }
+  {
+    int run = mincl - msum;
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32; ++i) {
       const int ee = lane * per + i;
-      if (ee < a.E) {
+      if (i < per && ee < a.E) {
         first[ee] = run;
-        run += (a.cnt[ee] + tr - 1) / tr;
+        run += (cnt_l[i] + tr - 1) / tr;
       }
     }
-    if (lane == 31) first[a.E] = incl;
-    __syncwarp();
+    if (lane == 31) first[a.E] = mincl;
   }
+  // rows of the experts before e: the owning lane's exclusive prefix plus its own experts
+  // before e
   int c_before = 0;
-  for (int i = lane; i < e; i += 32) c_before += a.cnt[i];
-  c_before = __reduce_add_sync(0xffffffffu, c_before);
+  {
+    const int owner = e / per;
+    int pre = cincl - csum;
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32; ++i)
+      if (i < e - owner * per) pre += cnt_l[i];
+    c_before = __shfl_sync(0xffffffffu, pre, owner);
+  }
+  __syncwarp();
   const int c = a.cnt[e];
   const int m_before = first[e];
   const int m = first[e + 1] - m_before;
@@ -97,7 +117,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a
   int run = 0;
   for (int w0 = 0; w0 < a.words; w0 += 32) {
     const int w = w0 + lane;
-    const int n = w < a.words ? __popc(bits[w]) : 0;
+    const int n = w < a.words ? __popc(w0 == 0 ? word0 : bits[w]) : 0;
     int incl = n;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
