@@ -152,9 +152,9 @@ struct Layout {
 // latency of adding them (one round of loads per four splits).  K chunks are a multiple of the
 // router's K step; at most max_s splits.
 int router_split(const beam_moe_shape& s, int max_s) {
-  const int64_t tiles = ceil_div(s.T, router_tile_m()) * ceil_div(s.E, router_tile_n());
-  const int64_t kblocks = s.d / router_tile_k();
-  const double block_flops_per_k = 2.0 * router_tile_m() * router_tile_n();
+  const int64_t tiles = ceil_div(s.T, kRM) * ceil_div(s.E, kRN);
+  const int64_t kblocks = s.d / kRK;
+  const double block_flops_per_k = 2.0 * kRM * kRN;
   const double slot_rate = 70e12 / kRouterSlots;  // FP32 FLOP/s per resident block
   const double hbm = 6.5e12;
   int best = 1;
@@ -164,7 +164,7 @@ int router_split(const beam_moe_shape& s, int max_s) {
     const int64_t Sx = ceil_div(kblocks, per);
     if (Sx != S) continue;
     const double waves = static_cast<double>(ceil_div(tiles * S, kRouterSlots));
-    const double t = waves * per * router_tile_k() * block_flops_per_k / slot_rate +
+    const double t = waves * per * kRK * block_flops_per_k / slot_rate +
                      static_cast<double>(S) * s.T * s.E * 8.0 / hbm +
                      static_cast<double>(ceil_div(S, 4)) * 0.8e-6;
     if (t < best_t * 0.97) {  // a larger split must win clearly
@@ -179,9 +179,9 @@ Layout plan(const beam_moe_shape& s) {
   Layout L{};
   const int64_t T = s.T, R = T * s.top_k;
   L.R = R;
-  const int64_t kblocks = s.d / router_tile_k();
+  const int64_t kblocks = s.d / kRK;
   const int S = router_split(s, 64);
-  L.kchunk = static_cast<int>(ceil_div(kblocks, S) * router_tile_k());
+  L.kchunk = static_cast<int>(ceil_div(kblocks, S) * kRK);
   L.S = static_cast<int>(ceil_div(s.d, L.kchunk));
   L.mt_cap = ceil_div(R, kBM) + s.E;
   size_t o = 0;
@@ -348,7 +348,6 @@ beam_status run_router(const beam_moe_shape& s, const Layout& L, const __nv_bflo
   RouterGemmArgs ga{};
   ga.h = h;
   ga.WT = at<float>(ws, L.wt);
-  ga.W = router_w;
   ga.part = at<float>(ws, L.part);
   ga.zero_counts = nullptr;
   ga.T = s.T;
@@ -359,9 +358,8 @@ beam_status run_router(const beam_moe_shape& s, const Layout& L, const __nv_bflo
   // with the dispatch's counts and token bitmap
   cudaError_t e = cudaMemsetAsync(at<uint32_t>(ws, L.status), 0, dispatch ? L.zero_bytes : 16, st);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (!kRouterKPairs)
-    BEAM_LAUNCH(kKRouterTranspose, st,
-                launch_router_transpose(router_w, at<float>(ws, L.wt), s.E, s.d, st));
+  BEAM_LAUNCH(kKRouterTranspose, st,
+              launch_router_transpose(router_w, at<float>(ws, L.wt), s.E, s.d, st));
   BEAM_LAUNCH(kKRouterGemm, st, launch_router_gemm(ga, L.S, st));
 
   SelectArgs sa{};
@@ -644,9 +642,9 @@ static __device__ __align__(256) unsigned char g_static_route_scratch[kStaticRou
 Layout plan_route_static(const beam_moe_shape& s) {
   Layout L{};
   L.R = static_cast<int64_t>(s.T) * s.top_k;
-  const int64_t kblocks = s.d / router_tile_k();
+  const int64_t kblocks = s.d / kRK;
   const int S = router_split(s, 16);  // the static scratch holds 16 partial arrays
-  L.kchunk = static_cast<int>(ceil_div(kblocks, S) * router_tile_k());
+  L.kchunk = static_cast<int>(ceil_div(kblocks, S) * kRK);
   L.S = static_cast<int>(ceil_div(s.d, L.kchunk));
   size_t o = 0;
   auto take = [&](size_t bytes) {

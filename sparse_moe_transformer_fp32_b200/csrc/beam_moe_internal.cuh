@@ -32,12 +32,7 @@ constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 
 
 // router GEMM tiling (FP32 FFMA)
 constexpr int kRM = 128, kRN = 128, kRK = 16, kRThreads = 256, kRBStages = 3;
-// K-pair form (reads W_r [E, d] as stored): 128 tokens x 64 experts x 32 K per block
-constexpr bool kRouterKPairs = false;
-constexpr int kQM = 128, kQN = 64, kQK = 32, kQThreads = 256, kQBStages = 3;
-__host__ __device__ constexpr int router_tile_m() { return kRouterKPairs ? kQM : kRM; }
-__host__ __device__ constexpr int router_tile_n() { return kRouterKPairs ? kQN : kRN; }
-__host__ __device__ constexpr int router_tile_k() { return kRouterKPairs ? kQK : kRK; }
+
 constexpr int kRouterSlots = 2 * 148;  // resident router blocks on a 148-SM B200
 
 constexpr int kMaxTopK = 8;
@@ -110,7 +105,6 @@ __device__ __forceinline__ void band_decode_tile(const MTile* mtiles, int t, int
 struct RouterGemmArgs {
   const __nv_bfloat16* h;  // [T, d]
   const float* WT;         // [d, E] (transposed router weight)
-  const float* W;          // [E, d] (router weight as given; the K-pair form reads it)
   float* part;             // [S, T, E]
   int32_t* zero_counts;    // [E] zeroed by block (0,0,0), or null
   int T, d, E, kchunk;
@@ -404,14 +398,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
       : "memory");
-}
-
-// Asks L2 to fetch the box at (x, y) of tensor map m (no shared-memory destination).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(x), "r"(y)
-               : "memory");
 }
 
 // ---- tcgen05

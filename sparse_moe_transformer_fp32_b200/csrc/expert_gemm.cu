@@ -45,23 +45,11 @@ namespace beam {
 namespace {
 
 constexpr uint64_t kMinDrainNs = 1000000000ull;  // drains always get at least 1 s
-// Weight k-blocks the first m-tile of each expert in a band asks L2 to fetch ahead of its own
-// loads (0: none), so that the slice streams from HBM with more bytes in flight than the ring
-// holds; the band's other m-tiles of the expert then find it in L2.
-constexpr int kWeightL2PrefetchKb = 0;
 
 __device__ __forceinline__ MTile load_tile(const GemmArgs& a, int t, int n_tiles, int& n) {
   int mt;
   band_decode_tile(a.mtiles, t, n_tiles, mt, n);
   return a.mtiles[mt];
-}
-
-// Whether tile t's m-tile is the first one of its expert inside its band.
-__device__ __forceinline__ bool leads_band(const GemmArgs& a, int t, int n_tiles) {
-  int mt, n;
-  band_decode_tile(a.mtiles, t, n_tiles, mt, n);
-  const int start = a.mtiles[mt].band >> kBandLenBits;
-  return mt == start || a.mtiles[mt - 1].e != a.mtiles[mt].e;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -164,13 +152,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // rows that are never stored
         const int a_box = a_box_for_rows(m.nrows);
         const uint32_t a_bytes = static_cast<uint32_t>(a_box_rows(a_box)) * kBK * 2;
-        const bool lead = kWeightL2PrefetchKb > 0 && leads_band(a, t, n_tiles);
-        auto prefetch_b = [&](int kb) {
-          tma_prefetch_l2_2d(&tmB0, kb * kKElems, brow);
-          if (kSwiGLU) tma_prefetch_l2_2d(&tmB1, kb * kKElems, brow);
-        };
-        if (lead)
-          for (int kb = kStages; kb < kWeightL2PrefetchKb && kb < a.k_blocks; ++kb) prefetch_b(kb);
         for (int kb = 0; kb < a.k_blocks; ++kb) {
           if (!mbar_wait_bounded(bar(kBarEmpty + stage), phase ^ 1u, abort_flag, limit, a.status,
                                  kWhereProducerEmpty)) {
@@ -184,7 +165,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_2d(sA, &tmA.m[a_box], fb, kb * kKElems, m.row0);
           tma_load_2d(sB, &tmB0, fb, kb * kKElems, brow);
           if (kSwiGLU) tma_load_2d(sB + kStageBBytes / 2, &tmB1, fb, kb * kKElems, brow);
-          if (lead && kb + kWeightL2PrefetchKb < a.k_blocks) prefetch_b(kb + kWeightL2PrefetchKb);
           filled |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {

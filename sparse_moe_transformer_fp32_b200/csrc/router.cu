@@ -194,121 +194,6 @@ __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterG
   }
 }
 
-// ---------------------------------------------------------------- logits: K-pair FFMA GEMM
-//
-// The same partial logits from W_r [E, d] as stored (no transposed copy).  Block tile 128 tokens
-// x 64 experts x 32 K, 256 threads, each 8 tokens (ty*8 ..) x 4 experts (tx, tx+16, tx+32,
-// tx+48).  Both operands sit in shared memory as [K / 4][row][4], so one 16-byte load gives a
-// row's four consecutive K values, and every packed FMA takes two consecutive K values of one
-// (token, expert) pair: acc.x sums the even-K products of the chunk, acc.y the odd-K ones, and
-// the logit partial is acc.x + acc.y.  No operand needs re-pairing in registers.
-__global__ void __launch_bounds__(kQThreads, 2) router_gemm_kpair_kernel(const RouterGemmArgs a) {
-  extern __shared__ __align__(16) float router_smem[];
-  auto& As = *reinterpret_cast<float4(*)[2][kQK / 4][kQM]>(router_smem);
-  auto& Bs = *reinterpret_cast<float4(*)[kQBStages][kQK / 4][kQN]>(router_smem + 2 * kQK * kQM);
-
-  const int tid = threadIdx.x;
-  const int m0 = blockIdx.x * kQM;
-  const int n0 = blockIdx.y * kQN;
-  const int kbeg = blockIdx.z * a.kchunk;
-  const int kend = min(a.d, kbeg + a.kchunk);
-  const int nk = (kend - kbeg) / kQK;
-  const int tx = tid & 15, ty = tid >> 4;
-
-  // A staging: two 16-byte chunks (16 BF16 K values) of one token per thread and K tile
-  const int a_row = tid & (kQM - 1);
-  const int a_kp = (tid / kQM) * 16;
-  const int a_t = m0 + a_row;
-  const __nv_bfloat16* a_src = a.h + static_cast<size_t>(a_t < a.T ? a_t : 0) * a.d + a_kp;
-  auto load_a = [&](int k0, uint4 (&v)[2]) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-      v[i] = a_t < a.T ? *reinterpret_cast<const uint4*>(a_src + k0 + 8 * i)
-                       : make_uint4(0, 0, 0, 0);
-  };
-  auto store_a = [&](int buf, const uint4 (&v)[2]) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-      As[buf][(a_kp + 8 * i) / 4][a_row] =
-          make_float4(__uint_as_float(w4[0] << 16), __uint_as_float(w4[0] & 0xffff0000u),
-                      __uint_as_float(w4[1] << 16), __uint_as_float(w4[1] & 0xffff0000u));
-      As[buf][(a_kp + 8 * i) / 4 + 1][a_row] =
-          make_float4(__uint_as_float(w4[2] << 16), __uint_as_float(w4[2] & 0xffff0000u),
-                      __uint_as_float(w4[3] << 16), __uint_as_float(w4[3] & 0xffff0000u));
-    }
-  };
-  // B: 64 experts x 8 groups of 4 K per stage; thread pairs read one expert's 32 bytes
-  auto issue_b = [&](int stage, int k0) {
-#pragma unroll
-    for (int i = 0; i < (kQK / 4) * kQN / kQThreads; ++i) {
-      const int c = tid + i * kQThreads;
-      const int col = (c >> 1) & (kQN - 1);
-      const int k4 = 2 * (c / (2 * kQN)) + (c & 1);
-      const int e = n0 + col;
-      const bool ok = e < a.E;
-      const float* src = a.W + static_cast<size_t>(ok ? e : 0) * a.d + k0 + 4 * k4;
-      cp_async16(smem_u32(&Bs[stage][k4][col]), src, ok ? 16 : 0);
-    }
-  };
-
-  float2 acc[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.f, 0.f);
-
-  if (nk > 0) {
-    issue_b(0, kbeg);
-    cp_async_commit();
-    if (nk > 1) issue_b(1, kbeg + kQK);
-    cp_async_commit();
-    uint4 v[2];
-    load_a(kbeg, v);
-    store_a(0, v);
-  }
-#pragma unroll 1
-  for (int kt = 0; kt < nk; ++kt) {
-    cp_async_wait_1();
-    __syncthreads();
-    if (kt + 2 < nk) issue_b((kt + 2) % kQBStages, kbeg + (kt + 2) * kQK);
-    cp_async_commit();
-    uint4 next[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-    if (kt + 1 < nk) load_a(kbeg + (kt + 1) * kQK, next);
-    const int buf = kt & 1, st = kt % kQBStages;
-#pragma unroll
-    for (int k4 = 0; k4 < kQK / 4; ++k4) {
-      float4 b[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = Bs[st][k4][tx + 16 * j];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 av = As[buf][k4][ty * 8 + i];
-        const float2 a01 = make_float2(av.x, av.y), a23 = make_float2(av.z, av.w);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          acc[i][j] = __ffma2_rn(a01, make_float2(b[j].x, b[j].y), acc[i][j]);
-          acc[i][j] = __ffma2_rn(a23, make_float2(b[j].z, b[j].w), acc[i][j]);
-        }
-      }
-    }
-    if (kt + 1 < nk) store_a(buf ^ 1, next);
-  }
-
-  float* part = a.part + static_cast<size_t>(blockIdx.z) * a.T * a.E;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int t = m0 + ty * 8 + i;
-    if (t >= a.T) continue;
-    float* prow = part + static_cast<size_t>(t) * a.E;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = n0 + tx + 16 * j;
-      if (e < a.E) prow[e] = acc[i][j].x + acc[i][j].y;
-    }
-  }
-}
-
 // ---------------------------------------------------------------- selection
 //
 // A block of 256 threads takes 8 tokens.  First the whole block forms the 8 x E logits (the
@@ -511,25 +396,15 @@ cudaError_t launch_router_transpose(const float* W, float* WT, int E, int d, cud
 }
 
 constexpr int kRouterSmemBytes = (2 * kRK * kRM + kRBStages * kRK * kRN) * 4;
-constexpr int kRouterKPairSmemBytes = (2 * kQK * kQM + kQBStages * kQK * kQN) * 4;
 
 cudaError_t prepare_router_kernels() {
-  cudaError_t e = cudaFuncSetAttribute(router_gemm_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kRouterSmemBytes);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(router_gemm_kpair_kernel,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, kRouterKPairSmemBytes);
+  return cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kRouterSmemBytes);
 }
 
 cudaError_t launch_router_gemm(const RouterGemmArgs& a, int S, cudaStream_t s) {
-  if (kRouterKPairs) {
-    const dim3 grid((a.T + kQM - 1) / kQM, (a.E + kQN - 1) / kQN, S);
-    router_gemm_kpair_kernel<<<grid, kQThreads, kRouterKPairSmemBytes, s>>>(a);
-  } else {
-    const dim3 grid((a.T + kRM - 1) / kRM, (a.E + kRN - 1) / kRN, S);
-    router_gemm_kernel<<<grid, kRThreads, kRouterSmemBytes, s>>>(a);
-  }
+  const dim3 grid((a.T + kRM - 1) / kRM, (a.E + kRN - 1) / kRN, S);
+  router_gemm_kernel<<<grid, kRThreads, kRouterSmemBytes, s>>>(a);
   return cudaGetLastError();
 }
 
