@@ -113,6 +113,8 @@ __global__ void __launch_bounds__(256) ep_push_kernel(const EpPushArgs a) {
         reinterpret_cast<uint4*>(a.xrecv[owners[j]] + static_cast<size_t>(rows[j]) * a.d)[c] = v;
     }
   }
+  // the rows written into other GPUs' memory are visible to them before this kernel completes
+  __threadfence_system();
 }
 
 // Rows of this rank's experts received from all ranks, cnt_local[el] = sum_p all[p][rank*ep+el],
