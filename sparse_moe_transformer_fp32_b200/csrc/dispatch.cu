@@ -186,23 +186,7 @@ __global__ void __launch_bounds__(256) permute_kernel(const PermuteArgs a) {
   const uint4* src = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(t) * a.d);
   const int nvec = a.d / 8;
   if (!a.xq) {
-    // four 16-byte loads in flight per lane before their copies are stored
-    constexpr int kU = 4;
-    int c = lane;
-    for (; c + 32 * (kU - 1) < nvec; c += 32 * kU) {
-      uint4 v[kU];
-#pragma unroll
-      for (int u = 0; u < kU; ++u) v[u] = src[c + 32 * u];
-#pragma unroll
-      for (int j = 0; j < kMaxTopK; ++j) {
-        if (j < a.k && rows[j] >= 0) {
-          uint4* dst = reinterpret_cast<uint4*>(a.xp + static_cast<size_t>(rows[j]) * a.d);
-#pragma unroll
-          for (int u = 0; u < kU; ++u) dst[c + 32 * u] = v[u];
-        }
-      }
-    }
-    for (; c < nvec; c += 32) {
+    for (int c = lane; c < nvec; c += 32) {
       const uint4 v = src[c];
 #pragma unroll
       for (int j = 0; j < kMaxTopK; ++j) {
