@@ -281,22 +281,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D view [outer, inner] (inner contiguous) of BF16 (elem_bytes 2) or E4M3 (1) elements, box
-// [box_outer rows, row_bytes] with row_bytes-wide swizzle (128 or 64); rows past `outer` read
-// as zeros.
+// [box_outer rows, 128 bytes] with 128-byte swizzle; rows past `outer` read as zeros.
 beam_status make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-                     uint32_t box_outer, int elem_bytes = 2, int row_bytes = kGemmRowBytes) {
+                     uint32_t box_outer, int elem_bytes = 2) {
   auto fn = encode_fn();
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {inner * elem_bytes};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(row_bytes / elem_bytes), box_outer};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), box_outer};
   const cuuint32_t es[2] = {1, 1};
   const CUtensorMapDataType dt =
       elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims,
                         strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled: %d",
@@ -452,7 +450,7 @@ beam_status run_experts(const beam_moe_shape& s, const Layout& L, const DeviceIn
   if ((b = make_map(&tm_g, w_gate, s.d, EI, kN1Half, eb)) != BEAM_OK) return b;
   if ((b = make_map(&tm_u, w_up, s.d, EI, kN1Half, eb)) != BEAM_OK) return b;
   if ((b = make_map(&tm_d, w_down, s.I, Ed, kN2, eb)) != BEAM_OK) return b;
-  const int k_elems = kGemmRowBytes / eb;  // K elements per pipeline stage row
+  const int k_elems = 128 / eb;  // K elements per 128-byte pipeline stage
 
   const uint64_t limit = g_wait_limit_ns.load(std::memory_order_relaxed);
   GemmArgs g1{};
@@ -568,13 +566,13 @@ beam_status run_experts_nvfp4(const beam_moe_shape& s, const Layout& L, const De
   CUtensorMap tm_gu, tm_d;
   beam_status b;
   for (int i = 0; i < kNumABoxes; ++i) {
-    if ((b = make_map(&tm_x.m[i], pa.xq, s.d / 2, R, a_box_rows(i), 1, 128)) != BEAM_OK) return b;
-    if ((b = make_map(&tm_a.m[i], at<void>(ws, L.act8), s.I / 2, R, a_box_rows(i), 1, 128)) != BEAM_OK)
+    if ((b = make_map(&tm_x.m[i], pa.xq, s.d / 2, R, a_box_rows(i), 1)) != BEAM_OK) return b;
+    if ((b = make_map(&tm_a.m[i], at<void>(ws, L.act8), s.I / 2, R, a_box_rows(i), 1)) != BEAM_OK)
       return b;
   }
   const uint64_t E2I = static_cast<uint64_t>(s.E) * 2 * s.I, Ed = static_cast<uint64_t>(s.E) * s.d;
-  if ((b = make_map(&tm_gu, w4.gu_codes, s.d / 2, E2I, kF4N, 1, 128)) != BEAM_OK) return b;
-  if ((b = make_map(&tm_d, w4.d_codes, s.I / 2, Ed, kF4N, 1, 128)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_gu, w4.gu_codes, s.d / 2, E2I, kF4N, 1)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_d, w4.d_codes, s.I / 2, Ed, kF4N, 1)) != BEAM_OK) return b;
 
   Fp4GemmArgs g1{};
   g1.mtiles = da.mtiles;
@@ -943,15 +941,15 @@ beam_status dense_nvfp4_impl(const beam_dense_shape* shape, const void* hidden,
   ATensorMaps tm_h, tm_a;
   CUtensorMap tm_gu, tm_d;
   for (int i = 0; i < kNumABoxes; ++i) {
-    if ((b = make_map(&tm_h.m[i], qh.q, s.d / 2, s.T, a_box_rows(i), 1, 128)) != BEAM_OK) return b;
-    if ((b = make_map(&tm_a.m[i], at<void>(ws, L.act8), s.I / 2, s.T, a_box_rows(i), 1, 128)) !=
+    if ((b = make_map(&tm_h.m[i], qh.q, s.d / 2, s.T, a_box_rows(i), 1)) != BEAM_OK) return b;
+    if ((b = make_map(&tm_a.m[i], at<void>(ws, L.act8), s.I / 2, s.T, a_box_rows(i), 1)) !=
         BEAM_OK)
       return b;
   }
-  if ((b = make_map(&tm_gu, w4.gu_codes, s.d / 2, 2 * static_cast<uint64_t>(s.I), kF4N, 1, 128)) !=
+  if ((b = make_map(&tm_gu, w4.gu_codes, s.d / 2, 2 * static_cast<uint64_t>(s.I), kF4N, 1)) !=
       BEAM_OK)
     return b;
-  if ((b = make_map(&tm_d, w4.d_codes, s.I / 2, s.d, kF4N, 1, 128)) != BEAM_OK) return b;
+  if ((b = make_map(&tm_d, w4.d_codes, s.I / 2, s.d, kF4N, 1)) != BEAM_OK) return b;
 
   Fp4GemmArgs g1{};
   g1.mtiles = mtiles;
@@ -1030,7 +1028,7 @@ beam_status dense_impl(const beam_dense_shape* shape, const void* hidden, const 
     a2 = at<void>(ws, L.act8);
   }
   const int eb = f8 ? 1 : 2;
-  const int k_elems = kGemmRowBytes / eb;
+  const int k_elems = 128 / eb;
   ATensorMaps tm_h, tm_act;
   CUtensorMap tm_g, tm_u, tm_d;
   for (int i = 0; i < kNumABoxes; ++i) {

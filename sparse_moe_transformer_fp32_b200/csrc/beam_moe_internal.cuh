@@ -13,13 +13,9 @@ namespace beam {
 // ------------------------------------------------------------------ constants
 
 constexpr int kBM = 128;        // rows (token slots) per expert tile = UMMA M
-// Bytes of K in one shared-memory row of the BF16 / E4M3 expert GEMMs' stages: 128 (128-byte
-// swizzle, 48 KB stages, 4 of them) or 64 (64-byte swizzle, 24 KB stages, 9 of them: more of
-// the ring in flight at once for the same shared memory).
-constexpr int kGemmRowBytes = 128;
-constexpr int kBK = kGemmRowBytes / 2;  // BF16 K elements per pipeline stage
+constexpr int kBK = 64;         // K elements per pipeline stage: one 128-byte swizzle row of BF16
 constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
-constexpr int kStages = kGemmRowBytes == 128 ? 4 : 9;  // shared-memory ring depth
+constexpr int kStages = 4;      // shared-memory ring depth
 constexpr int kN1Half = 128;    // gate (and up) columns per GEMM1 tile -> UMMA N = 256
 constexpr int kN2 = 256;        // output columns per GEMM2 tile -> UMMA N = 256
 constexpr int kUmmaN = 256;
@@ -498,18 +494,6 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
   desc |= static_cast<uint64_t>(1024u >> 4) << 32;
   desc |= static_cast<uint64_t>(1u) << 46;
   desc |= static_cast<uint64_t>(2u) << 61;
-  return desc;
-}
-
-// The same for rows of kGemmRowBytes bytes: 128-byte swizzle (layout type 2, 1024-byte 8-row
-// atoms) or 64-byte swizzle (layout type 4, 512-byte atoms).
-__device__ __forceinline__ uint64_t smem_desc_k_gemm(uint32_t saddr) {
-  uint64_t desc = 0;
-  desc |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  desc |= static_cast<uint64_t>(1u) << 16;
-  desc |= static_cast<uint64_t>((8u * kGemmRowBytes) >> 4) << 32;
-  desc |= static_cast<uint64_t>(1u) << 46;
-  desc |= static_cast<uint64_t>(kGemmRowBytes == 128 ? 2u : 4u) << 61;
   return desc;
 }
 

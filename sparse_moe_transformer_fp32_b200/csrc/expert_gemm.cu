@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint64_t limit = a.wait_limit_ns;
   const uint64_t drain_limit = limit > kMinDrainNs ? limit : kMinDrainNs;
   constexpr int kNSlice = kSwiGLU ? kN1Half : kN2;
-  constexpr int kKElems = kFp8 ? 2 * kBK : kBK;  // K elements in one stage row
+  constexpr int kKElems = kFp8 ? 2 * kBK : kBK;  // K elements in one 128-byte stage row
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -222,10 +222,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           tc_fence_after();
           const uint32_t sA = sbase + stage * kStageBytes;
-          const uint64_t adesc = smem_desc_k_gemm(sA);
-          const uint64_t bdesc = smem_desc_k_gemm(sA + kStageABytes);
+          const uint64_t adesc = smem_desc_k_sw128(sA);
+          const uint64_t bdesc = smem_desc_k_sw128(sA + kStageABytes);
           if (swap) {
-            const uint64_t bdesc_hi = smem_desc_k_gemm(sA + kStageABytes + kStageBBytes / 2);
+            const uint64_t bdesc_hi = smem_desc_k_sw128(sA + kStageABytes + kStageBBytes / 2);
 #pragma unroll
             for (int k = 0; k < kBK / kUmmaK; ++k) {
               const uint32_t accum = (kb | k) != 0 ? 1u : 0u;

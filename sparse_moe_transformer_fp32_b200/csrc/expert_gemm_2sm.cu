@@ -24,9 +24,9 @@
 namespace beam {
 namespace {
 
-constexpr int k2Stages = kGemmRowBytes == 128 ? 6 : 12;
-constexpr int k2StageA = kBM * kBK * 2;          // this CTA's 128 rows
-constexpr int k2StageB = 128 * kBK * 2;          // this CTA's half of the weight tile
+constexpr int k2Stages = 6;
+constexpr int k2StageA = kBM * kBK * 2;          // 16 KB: this CTA's 128 rows
+constexpr int k2StageB = 128 * kBK * 2;          // 16 KB: this CTA's half of the weight tile
 constexpr int k2StageBytes = k2StageA + k2StageB;
 constexpr int k2SmemBytes = k2Stages * k2StageBytes + 1024 + 1024;
 constexpr uint64_t k2MinDrainNs = 1000000000ull;
@@ -251,8 +251,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           tc_fence_after();
           const uint32_t sA = sbase + stage * k2StageBytes;
-          const uint64_t adesc = smem_desc_k_gemm(sA);
-          const uint64_t bdesc = smem_desc_k_gemm(sA + k2StageA);
+          const uint64_t adesc = smem_desc_k_sw128(sA);
+          const uint64_t bdesc = smem_desc_k_sw128(sA + k2StageA);
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k)
             umma_bf16_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);

@@ -257,6 +257,34 @@ def test_wait_timeout_is_reported_and_context_survives():
     H.assert_close_out(out2[::37].float().cpu().numpy(), ref, "after timeout")
 
 
+def test_sm_pair_wait_timeout_is_reported_and_context_survives():
+    """The SM-pair GEMMs (cta_group::2) with a zero wait limit: every role gives up at its first
+    open barrier and records the timeout, the leader drains both CTAs' loads, both CTAs meet at
+    the cluster barrier and free TMEM; the next call is correct."""
+    case = H.make_case(W.WORKLOADS["tiny"].with_tokens(1024))  # T * top_k = 256 * E: pairs
+    weights = H.device_weights(case.wl)
+    s = bm.shape_of(case.wl)
+    out = torch.empty(case.wl.T, case.wl.d, dtype=torch.bfloat16, device="cuda")
+    old = bm.beam_moe_get_wait_limit_ns()
+    bm.beam_moe_set_sm_pairs(True)
+    try:
+        bm.beam_moe_set_wait_limit_ns(0)
+        try:
+            ws = bm.beam_moe_forward(s, case.h.cuda(), case.router_w.cuda(), case.bias.cuda(),
+                                     *weights, out)
+            st = bm.beam_moe_sync_status(ws)
+        finally:
+            bm.beam_moe_set_wait_limit_ns(old)
+        assert st == bm.BEAM_ERR_TIMEOUT, bm.status_string(st)
+        out2, idx, w, _ = H.run_forward(case, weights)
+    finally:
+        bm.beam_moe_set_sm_pairs(False)
+    _check_routing(case, idx, w)
+    toks = list(range(0, case.wl.T, 37))
+    ref = H.oracle_out(case, weights, toks)
+    H.assert_close_out(out2[toks].float().cpu().numpy(), ref, "pairs after timeout")
+
+
 # ------------------------------------------------------------------ dense SwiGLU MLP and bias update
 
 @pytest.mark.parametrize("T,d,I", [(200, 256, 1024), (1, 512, 384), (129, 5120, 20480)])
