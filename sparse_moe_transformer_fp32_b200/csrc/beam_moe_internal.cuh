@@ -32,7 +32,6 @@ constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 
 
 // router GEMM tiling (FP32 FFMA)
 constexpr int kRM = 128, kRN = 128, kRK = 16, kRThreads = 256, kRBStages = 3;
-constexpr bool kRouterSwapA = false;  // keep a row-pair-swapped copy of the A tile
 
 constexpr int kRouterSlots = 2 * 148;  // resident router blocks on a 148-SM B200
 

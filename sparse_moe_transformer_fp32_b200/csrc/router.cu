@@ -60,10 +60,6 @@ __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterG
   extern __shared__ __align__(16) float router_smem[];
   auto& As = *reinterpret_cast<float(*)[2][kRK][kRM]>(router_smem);
   auto& Bs = *reinterpret_cast<float(*)[kRBStages][kRK][kRN]>(router_smem + 2 * kRK * kRM);
-  // with kRouterSwapA, a second copy of the A tile with each pair of rows swapped, so that the
-  // anti-diagonal products take their operand pair straight from a 16-byte load
-  auto& Asw = *reinterpret_cast<float(*)[2][kRK][kRM]>(router_smem + 2 * kRK * kRM +
-                                                      kRBStages * kRK * kRN);
 
   const int tid = threadIdx.x;
   const int m0 = blockIdx.x * kRM;
@@ -104,10 +100,6 @@ __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterG
       for (int q = 0; q < 4; ++q) {
         As[buf][a_kp + 8 * i + 2 * q][a_row] = __uint_as_float(w4[q] << 16);
         As[buf][a_kp + 8 * i + 2 * q + 1][a_row] = __uint_as_float(w4[q] & 0xffff0000u);
-        if constexpr (kRouterSwapA) {
-          Asw[buf][a_kp + 8 * i + 2 * q][a_row ^ 1] = __uint_as_float(w4[q] << 16);
-          Asw[buf][a_kp + 8 * i + 2 * q + 1][a_row ^ 1] = __uint_as_float(w4[q] & 0xffff0000u);
-        }
       }
     }
   };
@@ -161,32 +153,15 @@ __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterG
                             make_float2(a1.x, a1.y), make_float2(a1.z, a1.w)};
       const float2 bp[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w),
                             make_float2(b1.x, b1.y), make_float2(b1.z, b1.w)};
-      if constexpr (kRouterSwapA) {
-        // ad[r][c] = (acc[2r + 1][2c], acc[2r][2c + 1]) in this form; the two row halves are
-        // taken one after the other to keep few operands live
+      const float2 bs[4] = {make_float2(b0.y, b0.x), make_float2(b0.w, b0.z),
+                            make_float2(b1.y, b1.x), make_float2(b1.w, b1.z)};
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float4 sv = *reinterpret_cast<const float4*>(&Asw[buf][kk][64 * h + ty * 4]);
-          const float2 as[2] = {make_float2(sv.x, sv.y), make_float2(sv.z, sv.w)};
+      for (int r = 0; r < 4; ++r)
 #pragma unroll
-          for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              dg[2 * h + r][c] = __ffma2_rn(ap[2 * h + r], bp[c], dg[2 * h + r][c]);
-              ad[2 * h + r][c] = __ffma2_rn(as[r], bp[c], ad[2 * h + r][c]);
-            }
+        for (int c = 0; c < 4; ++c) {
+          dg[r][c] = __ffma2_rn(ap[r], bp[c], dg[r][c]);
+          ad[r][c] = __ffma2_rn(ap[r], bs[c], ad[r][c]);
         }
-      } else {
-        const float2 bs[4] = {make_float2(b0.y, b0.x), make_float2(b0.w, b0.z),
-                              make_float2(b1.y, b1.x), make_float2(b1.w, b1.z)};
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            dg[r][c] = __ffma2_rn(ap[r], bp[c], dg[r][c]);
-            ad[r][c] = __ffma2_rn(ap[r], bs[c], ad[r][c]);
-          }
-      }
     }
     if (kt + 1 < nk) store_a(buf ^ 1, next);
   }
@@ -199,8 +174,8 @@ __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterG
     for (int c = 0; c < 4; ++c) {
       acc[2 * r][2 * c] = dg[r][c].x;
       acc[2 * r + 1][2 * c + 1] = dg[r][c].y;
-      acc[2 * r][2 * c + 1] = kRouterSwapA ? ad[r][c].y : ad[r][c].x;
-      acc[2 * r + 1][2 * c] = kRouterSwapA ? ad[r][c].x : ad[r][c].y;
+      acc[2 * r][2 * c + 1] = ad[r][c].x;
+      acc[2 * r + 1][2 * c] = ad[r][c].y;
     }
   float* part = a.part + static_cast<size_t>(blockIdx.z) * a.T * a.E;
 #pragma unroll
@@ -420,8 +395,7 @@ cudaError_t launch_router_transpose(const float* W, float* WT, int E, int d, cud
   return cudaGetLastError();
 }
 
-constexpr int kRouterSmemBytes =
-    ((kRouterSwapA ? 4 : 2) * kRK * kRM + kRBStages * kRK * kRN) * 4;
+constexpr int kRouterSmemBytes = (2 * kRK * kRM + kRBStages * kRK * kRN) * 4;
 
 cudaError_t prepare_router_kernels() {
   return cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
