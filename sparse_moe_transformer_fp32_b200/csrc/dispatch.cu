@@ -162,7 +162,8 @@ __device__ __forceinline__ uint2 quantize8_e4m3(const uint4 v, float s) {
   return make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
 }
 
-// One warp per token: the row is read once and written to each of its top_k destinations.
+// E4M3 permute, one warp per token: the row is read once, quantised, and its codes written to
+// each of its top_k destinations.
 __global__ void __launch_bounds__(256) permute_kernel(const PermuteArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
@@ -183,21 +184,10 @@ __global__ void __launch_bounds__(256) permute_kernel(const PermuteArgs a) {
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j) rows[j] = __shfl_sync(0xffffffffu, row, j);
 
+  // the token row is quantised once (s = amax / 448, q = e4m3(x / s)) and its codes and scale
+  // written to each of its rows
   const uint4* src = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(t) * a.d);
   const int nvec = a.d / 8;
-  if (!a.xq) {
-    for (int c = lane; c < nvec; c += 32) {
-      const uint4 v = src[c];
-#pragma unroll
-      for (int j = 0; j < kMaxTopK; ++j) {
-        if (j < a.k && rows[j] >= 0)
-          reinterpret_cast<uint4*>(a.xp + static_cast<size_t>(rows[j]) * a.d)[c] = v;
-      }
-    }
-    return;
-  }
-  // FP8 path: the token row is quantised once (s = amax / 448, q = e4m3(x / s)) and its codes
-  // and scale written to each of its rows
   const float s = row_scale_e4m3(src, nvec, lane);
   if (lane < a.k && row >= 0) a.xs[row] = s;
   for (int c = lane; c < nvec; c += 32) {
@@ -208,6 +198,77 @@ __global__ void __launch_bounds__(256) permute_kernel(const PermuteArgs a) {
         reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(rows[j]) * a.d)[c] = q;
     }
   }
+}
+
+constexpr uint64_t kPermuteWaitNs = 4000000000ull;  // bound of the row copy's wait for its load
+
+// 1-D bulk copy global -> shared completing on mbarrier `bar` (16-byte aligned addresses, bytes
+// a multiple of 16).
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes,
+                                             uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// 1-D bulk copy shared -> global in the thread's current bulk group.
+__device__ __forceinline__ void bulk_store_1d(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+
+// Closes the thread's bulk group and waits until its shared-memory sources have been read.
+__device__ __forceinline__ void bulk_commit_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// BF16 permute by bulk copies: a CTA of one warp per token.  Lanes below top_k form their
+// slots' rows; lane 0 reads the token row into shared memory with one bulk copy and writes it
+// to each of its rows with bulk stores, then waits until those have read shared memory.
+__global__ void __launch_bounds__(32) permute_bulk_kernel(const PermuteArgs a) {
+  extern __shared__ __align__(128) uint8_t row_sh[];
+  __shared__ __align__(8) uint64_t bar_sh;
+  const int lane = threadIdx.x;
+  const int t = blockIdx.x;
+  int row = -1;
+  if (lane < a.k) {
+    const size_t slot = static_cast<size_t>(t) * a.k + lane;
+    const int e = a.idx[slot];
+    const int r = e >= 0 && e < a.E ? slot_rank(a.bits, a.base, a.words, e, t) : -1;
+    if (r >= 0) {
+      row = a.off[e] + r;
+      if (row >= a.off[e + 1]) row = -1;
+    }
+    if (row < 0) record_status(a.status, kDevAssert, kWherePermute);
+    a.rowmap[slot] = row;
+  }
+  int rows[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) rows[j] = __shfl_sync(0xffffffffu, row, j);
+  if (lane != 0) return;
+  const uint32_t bar = smem_u32(&bar_sh);
+  const uint32_t bytes = static_cast<uint32_t>(a.d) * 2u;
+  mbar_init(bar, 1);
+  fence_mbarrier_init();
+  mbar_arrive_expect_tx(bar, bytes);
+  bulk_load_1d(smem_u32(row_sh), a.h + static_cast<size_t>(t) * a.d, bytes, bar);
+  int abort_flag = 0;
+  if (!mbar_wait_bounded(bar, 0, &abort_flag, kPermuteWaitNs, a.status, kWherePermute)) {
+    // the load must land before this CTA's shared memory is released
+    int no_abort = 0;
+    mbar_wait_bounded(bar, 0, &no_abort, 1000000000ull, a.status, kWherePermute);
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (j < a.k && rows[j] >= 0)
+      bulk_store_1d(a.xp + static_cast<size_t>(rows[j]) * a.d, smem_u32(row_sh), bytes);
+  bulk_commit_wait_read();
 }
 
 // Row-wise E4M3 quantisation of a BF16 matrix [rows, cols]: one warp per row.
@@ -281,7 +342,10 @@ cudaError_t launch_dispatch_scan(const DispatchArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
-  permute_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(a);
+  if (!a.xq)  // BF16 rows: bulk copies
+    permute_bulk_kernel<<<a.T, 32, static_cast<size_t>(a.d) * 2, s>>>(a);
+  else        // E4M3 rows: quantised by the warp that reads them
+    permute_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
