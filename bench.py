@@ -72,6 +72,10 @@ def parse_args(argv=None):
                         "beam_dense_forward_nvfp4)")
     p.add_argument("--route-only", action="store_true",
                    help="time beam_moe_route alone (router profiling; not the layer metric)")
+    p.add_argument("--ep-ranks", type=int, default=0,
+                   help="time the expert-parallel layer step of this many ranks, emulated on one "
+                        "GPU rank after rank (their receive buffers all on this GPU; not the "
+                        "layer metric)")
     p.add_argument("--dry-run", action="store_true",
                    help="exercise the launch/aggregation logic on CPU (gloo); measures nothing")
     args = p.parse_args(argv)
@@ -797,6 +801,99 @@ def run_reference(args, rank, world, local):
                     "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------------------ expert parallelism, emulated
+
+def run_ep_emulated(args, rank, world, local):
+    """The expert-parallel step of P ranks (each with T / P tokens and E / P experts) run rank
+    after rank on one GPU: count, dispatch, experts and combine of every rank per step, the
+    receive buffers all on this GPU, so the exchange is local stores and loads instead of NVLink
+    ones.  Routing comes from one beam_moe_forward of the whole batch, made before timing."""
+    from sparse_moe_transformer_fp32_b200 import beam_moe as bm
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = selected_workload(args)
+    P = args.ep_ranks
+    if wl.E % P or wl.T % P:
+        raise SystemExit("bench.py: --ep-ranks must divide E and T")
+    ep, Tp = wl.E // P, wl.T // P
+    weights = W.expert_weights(wl, dev)
+    h = W.hidden(wl).to(dev)
+    s = bm.shape_of(wl)
+    out_ref = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(wl.T, wl.top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(wl.T, wl.top_k, dtype=torch.float32, device=dev)
+    bm.beam_moe_forward(s, h, W.router_weight(wl).to(dev), W.router_bias(wl).to(dev), *weights,
+                        out_ref, idx, w)
+    torch.cuda.synchronize(dev)
+    owners = (idx // ep).cpu()
+    cap = max(int((owners == q).sum()) for q in range(P))
+    sp = bm.shape_of(wl, Tp)
+    wss = [bm.ep_workspace(sp, P, cap, dev) for _ in range(P)]
+    counts = [torch.empty(wl.E, dtype=torch.int32, device=dev) for _ in range(P)]
+    all_counts = torch.empty(P, wl.E, dtype=torch.int32, device=dev)
+    xrecv = [torch.empty(cap, wl.d, dtype=torch.bfloat16, device=dev) for _ in range(P)]
+    yrecv = [torch.empty(cap, wl.d, dtype=torch.bfloat16, device=dev) for _ in range(P)]
+    out = torch.empty_like(out_ref)
+    sl = [slice(p * Tp, (p + 1) * Tp) for p in range(P)]
+    wg, wu, wd = weights
+
+    def step():
+        for p in range(P):
+            bm.beam_moe_ep_count(sp, P, idx[sl[p]], counts[p], cap, wss[p])
+        for p in range(P):  # the all-gather, here one device copy per rank
+            all_counts[p].copy_(counts[p])
+        for p in range(P):
+            bm.beam_moe_ep_dispatch(sp, P, p, h[sl[p]], idx[sl[p]], all_counts, xrecv, cap, wss[p])
+        for q in range(P):
+            e0, e1 = q * ep, (q + 1) * ep
+            bm.beam_moe_ep_experts(sp, P, q, wl.T, all_counts, wg[e0:e1], wu[e0:e1], wd[e0:e1],
+                                   xrecv[q], yrecv[q], cap, wss[q])
+        for p in range(P):
+            bm.beam_moe_ep_combine(sp, P, w[sl[p]], yrecv, cap, out[sl[p]], wss[p])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    for ws in wss:
+        st = bm.beam_moe_sync_status(ws)
+        if st != bm.BEAM_OK:
+            raise SystemExit(f"bench.py: device status {bm.status_string(st)}")
+    exact = bool(torch.equal(out.view(torch.int16), out_ref.view(torch.int16)))
+    bm.beam_moe_profile_reset()
+    bm.beam_moe_profile_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(args.steps):
+        step()
+    ev1.record()
+    torch.cuda.synchronize(dev)
+    bm.beam_moe_profile_enable(False)
+    ms = ev0.elapsed_time(ev1) / args.steps
+    prof = bm.beam_moe_profile_read()
+    R = wl.T * wl.top_k
+    row = wl.d * 2
+    kernels = {k: {"launches": n, "ms_per_launch": ms_ / n} for k, (n, ms_) in prof.items() if n}
+    # bytes each exchange kernel must move in one step, all ranks together
+    ex = {"ep_push": wl.T * row + R * row, "ep_combine": R * row + wl.T * row}
+    peaks = load_peaks()
+    exchange = {}
+    for k, b in ex.items():
+        if k in prof and prof[k][0]:
+            t_step = prof[k][1] / args.steps / 1e3
+            exchange[k] = {"ms_per_step": t_step * 1e3, "gbs": b / t_step / 1e9,
+                           "hbm_frac": b / t_step / 1e9 / peaks["hbm_gbs"]}
+    return {"metric": "expert-parallel layer step tokens/s, ranks emulated on one GPU "
+                      "(not the layer metric)",
+            "value": wl.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": args.steps,
+            "warmup": args.warmup, "ep_ranks": P, "recv_rows_max": cap,
+            "bit_equal_to_single_gpu_forward": exact,
+            "config": {"workload": f"{wl.name}: T={wl.T} d={wl.d} E={wl.E} top_k={wl.top_k} "
+                                   f"I={wl.I}, {P} ranks of {Tp} tokens and {ep} experts"},
+            "exchange": exchange, "kernels": kernels}
+
+
 # ------------------------------------------------------------------ router alone (profiling)
 
 def run_route_only(args, rank, world, local):
@@ -864,6 +961,8 @@ def main(argv=None):
         res = run_dry(args, rank, world, local)
     elif args.route_only:
         res = run_route_only(args, rank, world, local)
+    elif args.ep_ranks:
+        res = run_ep_emulated(args, rank, world, local)
     elif args.impl == "reference":
         res = run_reference(args, rank, world, local)
     else:
