@@ -73,13 +73,36 @@ __global__ void __launch_bounds__(256) ep_offsets_kernel(const EpOffsetsArgs a) 
   }
 }
 
-// One warp per token: each slot's owner and row, then the token row written to each of its
-// top_k destinations (local or peer receive buffers, 16-byte stores).  A row beyond the
-// owner's receive capacity is recorded and skipped.
-__global__ void __launch_bounds__(256) ep_push_kernel(const EpPushArgs a) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= a.T) return;
+constexpr uint64_t kPushWaitNs = 4000000000ull;  // bound of a row copy's wait for its load
+
+// 1-D bulk copy global -> shared completing on mbarrier `bar` (16-byte aligned, bytes % 16 == 0).
+__device__ __forceinline__ void bulk_load_row(uint32_t dst, const void* src, uint32_t bytes,
+                                              uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// 1-D bulk copy shared -> global (local or a peer's memory) in the thread's bulk group.
+__device__ __forceinline__ void bulk_store_row(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+
+// A CTA of one warp per token: lanes below top_k find their slots' owners and rows; lane 0 reads
+// the token row into shared memory with one bulk copy and writes it to each owner's receive
+// buffer with bulk stores (peer memory for other GPUs), then waits until those writes are done
+// and fences them, so that they are visible to the owners before this kernel completes.  A row
+// beyond the owner's receive capacity is recorded and skipped.
+__global__ void __launch_bounds__(32) ep_push_kernel(const EpPushArgs a) {
+  extern __shared__ __align__(128) uint8_t row_sh[];
+  __shared__ __align__(8) uint64_t bar_sh;
+  const int lane = threadIdx.x;
+  const int t = blockIdx.x;
   const int ep = a.E / a.P;
   int row = -1, owner = 0;
   if (lane < a.k) {
@@ -103,64 +126,89 @@ __global__ void __launch_bounds__(256) ep_push_kernel(const EpPushArgs a) {
     rows[j] = __shfl_sync(0xffffffffu, row, j);
     owners[j] = __shfl_sync(0xffffffffu, owner, j);
   }
-  const uint4* src = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(t) * a.d);
-  const int nvec = a.d / 8;
-  for (int c = lane; c < nvec; c += 32) {
-    const uint4 v = src[c];
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (j < a.k && rows[j] >= 0)
-        reinterpret_cast<uint4*>(a.xrecv[owners[j]] + static_cast<size_t>(rows[j]) * a.d)[c] = v;
-    }
+  if (lane != 0) return;
+  const uint32_t bar = smem_u32(&bar_sh);
+  const uint32_t bytes = static_cast<uint32_t>(a.d) * 2u;
+  mbar_init(bar, 1);
+  fence_mbarrier_init();
+  mbar_arrive_expect_tx(bar, bytes);
+  bulk_load_row(smem_u32(row_sh), a.h + static_cast<size_t>(t) * a.d, bytes, bar);
+  int abort_flag = 0;
+  if (!mbar_wait_bounded(bar, 0, &abort_flag, kPushWaitNs, a.status, kWhereDispatch)) {
+    int no_abort = 0;  // the load must land before this CTA's shared memory is released
+    mbar_wait_bounded(bar, 0, &no_abort, 1000000000ull, a.status, kWhereDispatch);
+    return;
   }
-  // the rows written into other GPUs' memory are visible to them before this kernel completes
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (j < a.k && rows[j] >= 0)
+      bulk_store_row(a.xrecv[owners[j]] + static_cast<size_t>(rows[j]) * a.d, smem_u32(row_sh),
+                     bytes);
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // the writes are complete
+  asm volatile("fence.proxy.async.global;" ::: "memory");
   __threadfence_system();
 }
 
 // Rows of this rank's experts received from all ranks, cnt_local[el] = sum_p all[p][rank*ep+el],
 // cut so that their total stays within the receive capacity (the dispatch skipped, and
 // recorded, every row beyond it).
-__global__ void ep_local_counts_kernel(const int32_t* all, int P, int E, int rank,
-                                       int64_t recv_cap, int32_t* cnt_local, uint32_t* status) {
-  if (threadIdx.x != 0) return;
+__global__ void __launch_bounds__(32) ep_local_counts_kernel(const int32_t* all, int P, int E,
+                                                            int rank, int64_t recv_cap,
+                                                            int32_t* cnt_local, uint32_t* status) {
+  // One warp: lane l sums experts l, l + 32, ... over the ranks; a warp scan gives each expert's
+  // uncut prefix S.  The cut count is min(c, max(0, cap - S)), which is what cutting the experts
+  // one after another in ascending order gives.
+  const int lane = threadIdx.x;
   const int ep = E / P;
-  int64_t total = 0;
-  for (int el = 0; el < ep; ++el) {
+  int64_t run = 0;
+  bool over = false;
+  for (int el0 = 0; el0 < ep; el0 += 32) {
+    const int el = el0 + lane;
     int64_t c = 0;
-    for (int p = 0; p < P; ++p) c += all[static_cast<size_t>(p) * E + rank * ep + el];
-    if (total + c > recv_cap) {
-      record_status(status, kDevAssert, kWhereDispatch);
-      c = recv_cap - total;
+    if (el < ep)
+      for (int p = 0; p < P; ++p) c += all[static_cast<size_t>(p) * E + rank * ep + el];
+    int64_t incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int64_t o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
     }
-    cnt_local[el] = static_cast<int32_t>(c);
-    total += c;
+    const int64_t before = run + incl - c;
+    const int64_t room = recv_cap - before;
+    const int64_t cut = c < room ? c : (room > 0 ? room : 0);
+    if (cut != c) over = true;
+    if (el < ep) cnt_local[el] = static_cast<int32_t>(cut);
+    run += __shfl_sync(0xffffffffu, incl, 31);
   }
+  if (__any_sync(0xffffffffu, over) && lane == 0) record_status(status, kDevAssert, kWhereDispatch);
 }
 
 // out[t] = sum_j w[t, j] * Y_owner(j)[row(j)], j in slot (ascending expert) order, FP32 FMAs:
 // the arithmetic of the single-GPU combine, with each expert output read from its owner.
-constexpr int kEpCThreads = 128;
+constexpr int kEpCThreads = 128;  // a CTA per 128 16-byte pieces of a token's row
 
 __global__ void __launch_bounds__(kEpCThreads) ep_combine_kernel(const EpCombineArgs a) {
   __shared__ const __nv_bfloat16* src[kMaxTopK];
   __shared__ float wsh[kMaxTopK];
-  const int t = blockIdx.x;
+  const int nvec = a.d / 8;
+  const int chunks = (nvec + kEpCThreads - 1) / kEpCThreads;
+  const int t = blockIdx.x / chunks;
+  const int chunk = blockIdx.x % chunks;
   if (threadIdx.x < a.k) {
     const size_t slot = static_cast<size_t>(t) * a.k + threadIdx.x;
     const int r = a.slot_row[slot];
     const int q = a.slot_owner[slot];
-    const __nv_bfloat16* p = nullptr;  // a slot that was not sent adds nothing
-    if (r < 0 || r >= a.recv_cap || q < 0 || q >= a.P)
-      record_status(a.status, kDevAssert, kWhereCombine);
-    else
-      p = a.yrecv[q] + static_cast<size_t>(r) * a.d;
-    src[threadIdx.x] = p;
+    const bool sent = r >= 0 && r < a.recv_cap && q >= 0 && q < a.P;
+    if (!sent && chunk == 0) record_status(a.status, kDevAssert, kWhereCombine);
+    // a slot that was not sent adds nothing
+    src[threadIdx.x] = sent ? a.yrecv[q] + static_cast<size_t>(r) * a.d : nullptr;
     wsh[threadIdx.x] = a.w[slot];
   }
   __syncthreads();
-  const int nvec = a.d / 8;
   uint4* out = reinterpret_cast<uint4*>(a.out + static_cast<size_t>(t) * a.d);
-  for (int c = threadIdx.x; c < nvec; c += kEpCThreads) {
+  const int c = chunk * kEpCThreads + threadIdx.x;
+  if (c < nvec) {
     uint4 v[kMaxTopK];
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j)
@@ -205,7 +253,7 @@ cudaError_t launch_ep_offsets(const EpOffsetsArgs& a, cudaStream_t s) {
 
 cudaError_t launch_ep_push(const EpPushArgs& a, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
-  ep_push_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(a);
+  ep_push_kernel<<<a.T, 32, static_cast<size_t>(a.d) * 2, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -217,7 +265,8 @@ cudaError_t launch_ep_local_counts(const int32_t* all, int P, int E, int rank, i
 
 cudaError_t launch_ep_combine(const EpCombineArgs& a, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
-  ep_combine_kernel<<<a.T, kEpCThreads, 0, s>>>(a);
+  const unsigned chunks = static_cast<unsigned>((a.d / 8 + kEpCThreads - 1) / kEpCThreads);
+  ep_combine_kernel<<<static_cast<unsigned>(a.T) * chunks, kEpCThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -124,8 +124,27 @@ def test_ep_receive_overflow_is_reported_and_context_survives():
     ref, idx, w = _forward(case, weights)
     owners = idx.cpu().numpy() // (wl.E // 2)
     need = max(int((owners == q).sum()) for q in range(2))
-    _, st = _ep_emulated(wl, case.h.cuda(), idx, w, weights, (150, 150), recv_cap=need - 37)
+    cap = need - 37
+    cut, st = _ep_emulated(wl, case.h.cuda(), idx, w, weights, (150, 150), recv_cap=cap)
     assert bm.BEAM_ERR_DEVICE_ASSERT in st, st
+    # which slots fit: an owner's rows run expert by expert, each expert's rows rank by rank,
+    # each rank's in ascending token order; a row at or beyond the capacity is not sent
+    ids = idx.cpu().numpy()
+    sent = np.zeros_like(ids, dtype=bool)
+    ep, Ts = wl.E // 2, (150, 150)
+    for q in range(2):
+        pos = 0
+        for e in range(q * ep, (q + 1) * ep):
+            for p in range(2):
+                for t in range(p * 150, p * 150 + Ts[p]):
+                    for j in np.nonzero(ids[t] == e)[0]:
+                        sent[t, j] = pos < cap
+                        pos += 1
+    full = np.nonzero(sent.all(axis=1))[0]
+    assert 0 < len(full) < wl.T
+    # a token all of whose rows were sent is exact; the rest stay finite
+    assert torch.equal(cut[full].view(torch.int16), ref[full].view(torch.int16))
+    assert torch.isfinite(cut.float()).all()
     out, st = _ep_emulated(wl, case.h.cuda(), idx, w, weights, (150, 150))
     assert all(s == bm.BEAM_OK for s in st), st
     assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
