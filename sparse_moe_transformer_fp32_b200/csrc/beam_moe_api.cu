@@ -141,7 +141,7 @@ struct Layout {
   size_t zero_bytes = 0;             // status, counts and token bitmap: cleared at each call
   int words = 0;                     // token bitmap words per expert, ceil(T / 32)
   size_t xs = 0, act8 = 0, as = 0;  // FP8 path: row scales of Xp, E4M3 act, act row scales
-  size_t xsf = 0, asf = 0;           // NVFP4 path: block-scale atoms of Xp and of the act
+  size_t xsf = 0, asf = 0;           // NVFP4 path: block scales of Xp and of the act
   int S, kchunk;
   int64_t R, mt_cap;
 };
@@ -243,9 +243,9 @@ Layout plan_nvfp4(const beam_moe_shape& s) {
   };
   const size_t groups = static_cast<size_t>(L.mt_cap);
   L.xs = take(sizeof(float) * L.R);
-  L.xsf = take(groups * (s.d / 16) * 128);
+  L.xsf = take(groups * (s.d / kF4KElems) * kF4SfaBytes);
   L.act8 = take(static_cast<size_t>(L.R) * (s.I / 2));
-  L.asf = take(groups * (s.I / 16) * 128);
+  L.asf = take(groups * (s.I / kF4KElems) * kF4SfaBytes);
   L.as = take(sizeof(float) * L.R);
   L.total = o;
   return L;
@@ -692,7 +692,7 @@ beam_status check_dense_shape(const beam_dense_shape* s) {
 struct DenseLayout {
   size_t status, mt_count, mtiles, act, total;
   size_t hq = 0, hs = 0, act8 = 0, as = 0;  // E4M3 form: quantised rows and their scales
-  size_t hsf = 0, asf = 0;                    // NVFP4 form: block-scale atoms per m-tile
+  size_t hsf = 0, asf = 0;                    // NVFP4 form: block scales per m-tile
   int64_t mt_cap;
 };
 
@@ -744,10 +744,10 @@ DenseLayout plan_dense_nvfp4(const beam_dense_shape& s) {
   const size_t groups = static_cast<size_t>(L.mt_cap);
   L.hq = take(static_cast<size_t>(s.T) * (s.d / 2));
   L.hs = take(sizeof(float) * s.T);
-  L.hsf = take(groups * (s.d / 16) * 128);
+  L.hsf = take(groups * (s.d / kF4KElems) * kF4SfaBytes);
   L.act8 = take(static_cast<size_t>(s.T) * (s.I / 2));
   L.as = take(sizeof(float) * s.T);
-  L.asf = take(groups * (s.I / 16) * 128);
+  L.asf = take(groups * (s.I / kF4KElems) * kF4SfaBytes);
   L.total = o;
   return L;
 }

@@ -18,17 +18,30 @@ namespace beam {
 
 constexpr int kF4N = 128;                   // UMMA N (weight rows per tile); UMMA M = kBM
 constexpr int kF4KElems = 256;              // K elements per stage: one 128-byte code row
-constexpr int kF4Stages = 6;
+constexpr int kF4Stages = 5;
 constexpr int kF4StageA = kBM * 128;        // 16 KB of A codes
 constexpr int kF4StageB = kF4N * 128;       // 16 KB of B codes
-constexpr int kF4SfBytes = 2048;            // block scales of 128 rows x 256 K elements
-constexpr int kF4StageBytes = kF4StageA + kF4StageB + 2 * kF4SfBytes;  // 36 KB
+constexpr int kF4SfBytes = 2048;            // B block scales of 128 rows x 256 K elements
+constexpr int kF4SfaBytes = 8192;           // A block scales of the same, laid out as below
+constexpr int kF4StageBytes = kF4StageA + kF4StageB + kF4SfaBytes + kF4SfBytes;  // 42 KB
 constexpr int kF4SmemBytes = kF4Stages * kF4StageBytes + 1024 /*barriers*/ + 1024 /*align*/;
 
 // Byte offset of the scale of (row r of a 128-row group, 16-element block j) from the start of
 // the group's atoms.
 __host__ __device__ constexpr size_t nvfp4_sf_offset(int r, int j) {
   return static_cast<size_t>(j >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (j & 3);
+}
+
+// The A operand's (token rows') block scales are kept in the layout tcgen05.cp.128x256b
+// reads: per 128-row group and 256-element K stage 8 KB, per 64-element K step a 2 KB block of
+// 128 rows x 16 bytes in which row r's four scales sit at byte r * 16 + (r / 32) * 4.  The
+// MMA reads A's scales of TMEM lane r from column r / 32 of the K step's four (lane quarter q
+// reads column q), so the other 12 bytes of a row are never read and never written.  One copy
+// brings two K steps (two blocks, 2 KB apart): two copies a stage where one
+// 32x128b.warpx4 copy per K step took four.  Groups of 128 rows keep their stages in K order.
+__host__ __device__ constexpr size_t nvfp4_sfa_offset(int r, int j) {
+  return static_cast<size_t>(j >> 4) * kF4SfaBytes + ((j >> 2) & 3) * 2048 + r * 16 +
+         (r >> 5) * 4 + (j & 3);
 }
 
 struct Fp4GemmArgs {
@@ -41,7 +54,7 @@ struct Fp4GemmArgs {
   int n_tiles_n;           // tiles along N per m-tile
   int k_blocks;            // K / kF4KElems
   int b_rows_per_expert;   // weight rows of one expert (2I interleaved gate|up, or d)
-  const uint8_t* a_sf;     // block-scale atoms of the A rows, one 128-row group per m-tile
+  const uint8_t* a_sf;     // block scales of the A rows (nvfp4_sfa_offset), one group per m-tile
   const uint8_t* b_sf;     // block-scale atoms of the weight rows
   const float* a_scale;    // [R] row scales of A
   const float* b_scale;    // [E * b_rows_per_expert] row scales of the weights
@@ -57,7 +70,7 @@ struct Fp4PermuteArgs {
   const int32_t* off;      // [E + 1]
   int32_t* rowmap;         // [T, k] out
   uint8_t* xq;             // [R, d / 2] out: codes
-  uint8_t* xsf;            // out: block-scale atoms, one 128-row group per m-tile
+  uint8_t* xsf;            // out: block scales (nvfp4_sfa_offset), one 128-row group per m-tile
   float* xs;               // [R] out: row scales
   uint32_t* status;
   int T, d, k, E;
@@ -68,7 +81,7 @@ struct Fp4ActArgs {
   const MTile* mtiles;
   const int32_t* mt_count;
   uint8_t* q;              // [R, cols / 2] out
-  uint8_t* sf;             // out: block-scale atoms, one 128-row group per m-tile
+  uint8_t* sf;             // out: block scales (nvfp4_sfa_offset), one 128-row group per m-tile
   float* s;                // [R] out
   int cols;
   int mt_cap;

@@ -15,12 +15,14 @@
 //
 // Kernel structure as the BF16/E4M3 expert GEMM (persistent, one CTA per SM, 192 threads):
 //   warp 0     one thread issues, per 256-element K stage, TMA loads of the A codes (box sized
-//              to the tile's rows) and the B codes, and two 2 KB bulk copies of their block-scale
-//              atoms, into a 6-stage ring
+//              to the tile's rows) and the B codes, and bulk copies of their block scales (A 8 KB,
+//              B 2 KB; layouts in beam_moe_nvfp4.cuh), into a 5-stage ring
 //   warp 1     allocates 512 TMEM columns (two 128-column accumulators at 0 and 128, the block
 //              scales of one stage at 256..287); one thread copies the stage's scales into TMEM
-//              (tcgen05.cp.32x128b.warpx4) and issues four M=128 N=128 K=64 MMAs.  Copies and
-//              MMAs issued by one thread run in issue order, so one scale buffer serves every stage
+//              (A: two tcgen05.cp.128x256b, two K steps each; B: one tcgen05.cp.32x128b.warpx4
+//              per K step, as the MMA reads B's scales in every lane quarter) and issues four
+//              M=128 N=128 K=64 MMAs.  Copies and MMAs issued by one thread run in issue order,
+//              so one scale buffer serves every stage
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator, row scales, SwiGLU / BF16 conversion
 // Rows of a tile beyond its valid rows read stale codes and unwritten scales; they only feed
 // accumulator rows that are never stored.
@@ -170,7 +172,7 @@ __global__ void __launch_bounds__(256) nvfp4_permute_kernel(const Fp4PermuteArgs
   }
   int rows[kMaxTopK];
   uint8_t* atoms[kMaxTopK];
-  const int64_t group_bytes = static_cast<int64_t>(a.d) / 16 * 128;
+  const int64_t group_bytes = static_cast<int64_t>(a.d) / kF4KElems * kF4SfaBytes;
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j) {
     rows[j] = __shfl_sync(0xffffffffu, row, j);
@@ -190,7 +192,7 @@ __global__ void __launch_bounds__(256) nvfp4_permute_kernel(const Fp4PermuteArgs
     for (int j = 0; j < kMaxTopK; ++j) {
       if (j < a.k && rows[j] >= 0) {
         reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(rows[j]) * (a.d / 2))[jb] = q;
-        atoms[j][nvfp4_sf_offset(rins[j], jb)] = bs;
+        atoms[j][nvfp4_sfa_offset(rins[j], jb)] = bs;
       }
     }
   }
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(256) nvfp4_act_kernel(const Fp4ActArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = static_cast<int>(blockIdx.x % kActCtasPerTile) * kActRowsPerCta + warp;
   if (r >= tile.nrows) return;  // uniform over the warp
-  uint8_t* atoms = a.sf + static_cast<int64_t>(mt) * (a.cols / 16) * 128;
+  uint8_t* atoms = a.sf + static_cast<int64_t>(mt) * (a.cols / kF4KElems) * kF4SfaBytes;
   const int64_t row = tile.row0 + r;
   const uint4* src = reinterpret_cast<const uint4*>(a.x + row * a.cols);
   const float s = nvfp4_row_scale(src, a.cols / 8, lane);
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(256) nvfp4_act_kernel(const Fp4ActArgs a) {
   for (int jb = lane; jb < a.cols / 16; jb += 32) {
     uint8_t bs;
     dst[jb] = nvfp4_block(src[2 * jb], src[2 * jb + 1], s, bs);
-    atoms[nvfp4_sf_offset(r, jb)] = bs;
+    atoms[nvfp4_sfa_offset(r, jb)] = bs;
   }
 }
 
@@ -243,6 +245,25 @@ __device__ __forceinline__ uint64_t smem_desc_sf(uint32_t saddr) {
   desc |= static_cast<uint64_t>(128u >> 4) << 32;  // stride between 8-row core matrices
   desc |= static_cast<uint64_t>(1u) << 46;
   return desc;  // layout type 0: no swizzle
+}
+
+// Shared-memory descriptor of 128 rows x 32 bytes, no swizzle: row L's first 16 bytes at
+// 16 L, its second 16 bytes 2 KB further (8-row core matrices 128 bytes apart, the two 16-byte
+// columns 2048 bytes apart).
+__device__ __forceinline__ uint64_t smem_desc_sf_pair(uint32_t saddr) {
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  desc |= static_cast<uint64_t>(2048u >> 4) << 16;  // leading offset: the second 16-byte column
+  desc |= static_cast<uint64_t>(128u >> 4) << 32;   // stride between 8-row core matrices
+  desc |= static_cast<uint64_t>(1u) << 46;
+  return desc;  // layout type 0: no swizzle
+}
+
+// 128 TMEM lanes x 256 bits (8 columns) from shared memory: lane L gets row L, its first 16
+// bytes in columns 0..3 and its second in columns 4..7.
+__device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
 }
 
 // 32 TMEM lanes x 128 bits from shared memory, repeated into all four lane quarters.
@@ -301,7 +322,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (sbase - raw);
-  // [kF4Stages x (A 16 KB | B 16 KB | SFA 2 KB | SFB 2 KB)][barriers][TMEM address][abort flag]
+  // [kF4Stages x (A 16 KB | B 16 KB | SFA 8 KB | SFB 2 KB)][barriers][TMEM address][abort flag]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kF4Stages * kF4StageBytes);
   constexpr int kBarFull = 0, kBarEmpty = kF4Stages, kBarTFull = 2 * kF4Stages,
                 kBarTEmpty = kBarTFull + 2, kBarDrain = kBarTEmpty + 2, kNumBars = kBarDrain + 1;
@@ -342,7 +363,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int64_t sf_group = static_cast<int64_t>(a.k_blocks) * kF4SfBytes;  // atoms of 128 rows
+  const int64_t sfa_group = static_cast<int64_t>(a.k_blocks) * kF4SfaBytes;  // per 128 rows
+  const int64_t sfb_group = static_cast<int64_t>(a.k_blocks) * kF4SfBytes;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -357,8 +379,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int brow = m.e * a.b_rows_per_expert + n * kF4N;
         const int a_box = a_box_for_rows(m.nrows);
         const uint32_t a_bytes = static_cast<uint32_t>(a_box_rows(a_box)) * 128;
-        const uint8_t* sfa = a.a_sf + mt * sf_group;
-        const uint8_t* sfb = a.b_sf + (brow / kF4N) * sf_group;
+        const uint8_t* sfa = a.a_sf + mt * sfa_group;
+        const uint8_t* sfb = a.b_sf + (brow / kF4N) * sfb_group;
         for (int kb = 0; kb < a.k_blocks; ++kb) {
           if (!mbar_wait_bounded(bar(kBarEmpty + stage), phase ^ 1u, abort_flag, limit, a.status,
                                  kWhereProducerEmpty)) {
@@ -369,11 +391,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t sB = sA + kF4StageA;
           const uint32_t sS = sB + kF4StageB;
           const uint32_t fb = bar(kBarFull + stage);
-          mbar_arrive_expect_tx(fb, a_bytes + kF4StageB + 2 * kF4SfBytes);
+          mbar_arrive_expect_tx(fb, a_bytes + kF4StageB + kF4SfaBytes + kF4SfBytes);
           tma_load_2d(sA, &tmA.m[a_box], fb, kb * 128, m.row0);
           tma_load_2d(sB, &tmB, fb, kb * 128, brow);
-          bulk_load(sS, sfa + kb * kF4SfBytes, kF4SfBytes, fb);
-          bulk_load(sS + kF4SfBytes, sfb + kb * kF4SfBytes, kF4SfBytes, fb);
+          bulk_load(sS, sfa + kb * kF4SfaBytes, kF4SfaBytes, fb);
+          bulk_load(sS + kF4SfaBytes, sfb + kb * kF4SfBytes, kF4SfBytes, fb);
           filled |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kF4Stages) {
@@ -414,10 +436,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint64_t adesc = smem_desc_k_sw128(sA);
           const uint64_t bdesc = smem_desc_k_sw128(sA + kF4StageA);
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            tmem_cp_sf(sfa_t + 4u * ks, smem_desc_sf(sS + 512u * ks));
-            tmem_cp_sf(sfb_t + 4u * ks, smem_desc_sf(sS + kF4SfBytes + 512u * ks));
-          }
+          for (int p = 0; p < 2; ++p)  // A: K steps 2p and 2p + 1 into columns 8p .. 8p + 7
+            tmem_cp_sf_pair(sfa_t + 8u * p, smem_desc_sf_pair(sS + 4096u * p));
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            tmem_cp_sf(sfb_t + 4u * ks, smem_desc_sf(sS + kF4SfaBytes + 512u * ks));
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)  // 64 E2M1 elements = 32 bytes of K: +2 in addr >> 4
             umma_nvfp4(d_tmem, adesc + 2u * ks, bdesc + 2u * ks, idesc, sfa_t + 4u * ks,
