@@ -24,6 +24,7 @@ constexpr int kF4StageB = kF4N * 128;       // 16 KB of B codes
 constexpr int kF4SfBytes = 2048;            // B block scales of 128 rows x 256 K elements
 constexpr int kF4SfaBytes = 8192;           // A block scales of the same, laid out as below
 constexpr int kF4StageBytes = kF4StageA + kF4StageB + kF4SfaBytes + kF4SfBytes;  // 42 KB
+constexpr int kF4Threads = 224;  // warp 0 loads, 1 MMA, 2..5 epilogue, 6 scale copies
 constexpr int kF4SmemBytes = kF4Stages * kF4StageBytes + 1024 /*barriers*/ + 1024 /*align*/;
 
 // Byte offset of the scale of (row r of a 128-row group, 16-element block j) from the start of

@@ -13,16 +13,19 @@
 //   the activation is then quantised to NVFP4 per row (a kernel of its own);
 //   GEMM2 (down): Y[rows, 128n + c] = bf16( Aq[rows, :] . Wd,e[128n + c, :]^T  sa sd ).
 //
-// Kernel structure as the BF16/E4M3 expert GEMM (persistent, one CTA per SM, 192 threads):
+// Kernel structure as the BF16/E4M3 expert GEMM (persistent, one CTA per SM), plus a warp
+// that copies the block scales into TMEM (224 threads):
 //   warp 0     one thread issues, per 256-element K stage, TMA loads of the A codes (box sized
 //              to the tile's rows) and the B codes, and bulk copies of their block scales (A 8 KB,
 //              B 2 KB; layouts in beam_moe_nvfp4.cuh), into a 5-stage ring
-//   warp 1     allocates 512 TMEM columns (two 128-column accumulators at 0 and 128, the block
-//              scales of one stage at 256..287); one thread copies the stage's scales into TMEM
-//              (A: two tcgen05.cp.128x256b, two K steps each; B: one tcgen05.cp.32x128b.warpx4
-//              per K step, as the MMA reads B's scales in every lane quarter) and issues four
-//              M=128 N=128 K=64 MMAs.  Copies and MMAs issued by one thread run in issue order,
-//              so one scale buffer serves every stage
+//   warp 6     one thread copies each landed stage's block scales into that stage's 32 TMEM
+//              columns (A: two tcgen05.cp.128x256b, two K steps each; B: one
+//              tcgen05.cp.32x128b.warpx4 per K step, as the MMA reads B's scales in every lane
+//              quarter) and commits them to the stage's scales-ready barrier
+//   warp 1     allocates 512 TMEM columns (two 128-column accumulators at 0 and 128, the
+//              stages' block scales at 256..415); one thread issues four M=128 N=128 K=64 MMAs
+//              per stage once its codes and scales are in.  (Copies issued by the MMA thread
+//              itself ran strictly between its MMAs: gate/up 15 % slower.)
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator, row scales, SwiGLU / BF16 conversion
 // Rows of a tile beyond its valid rows read stale codes and unwritten scales; they only feed
 // accumulator rows that are never stored.
@@ -312,10 +315,12 @@ __device__ __forceinline__ void scale32(uint32_t (&v)[32], float sa, const float
 }
 
 constexpr uint32_t kF4TmemCols = 512;
-constexpr uint32_t kF4SfaCol = 256, kF4SfbCol = 272;
+// Block scales of stage s in TMEM: A's at column 256 + 32 s (16 columns), B's 16 further.
+constexpr uint32_t kF4SfCol = 256, kF4SfStageCols = 32;
+static_assert(kF4SfCol + kF4SfStageCols * kF4Stages <= kF4TmemCols, "scale columns fit in TMEM");
 
 template <bool kSwiGLU>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kF4Threads, 1)
     expert_gemm_nvfp4_kernel(const __grid_constant__ ATensorMaps tmA,
                              const __grid_constant__ CUtensorMap tmB, const Fp4GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -325,7 +330,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // [kF4Stages x (A 16 KB | B 16 KB | SFA 8 KB | SFB 2 KB)][barriers][TMEM address][abort flag]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kF4Stages * kF4StageBytes);
   constexpr int kBarFull = 0, kBarEmpty = kF4Stages, kBarTFull = 2 * kF4Stages,
-                kBarTEmpty = kBarTFull + 2, kBarDrain = kBarTEmpty + 2, kNumBars = kBarDrain + 1;
+                kBarTEmpty = kBarTFull + 2, kBarDrain = kBarTEmpty + 2,
+                kBarSReady = kBarDrain + 1, kBarCopyDrain = kBarSReady + kF4Stages,
+                kNumBars = kBarCopyDrain + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_u32(bars + i); };
@@ -342,7 +349,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int s = 0; s < kF4Stages; ++s) {
       mbar_init(bar(kBarFull + s), 1);
       mbar_init(bar(kBarEmpty + s), 1);
+      mbar_init(bar(kBarSReady + s), 1);
     }
+    mbar_init(bar(kBarCopyDrain), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarTFull + i), 1);
       mbar_init(bar(kBarTEmpty + i), 4);
@@ -410,11 +419,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_wait_bounded(bar(kBarFull + s), (last_parity >> s) & 1u, &no_abort, drain_limit,
                             a.status, kWhereDrain);
     }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ scale copies
+    // One thread copies each stage's block scales into the stage's own TMEM columns as soon as
+    // the stage has landed and signals the MMA thread through a commit.  The stage's columns
+    // are free again by then: the stage was refilled only after the MMAs that read them
+    // completed.  Issued from a thread of their own, the copies run beside the MMAs instead of
+    // between them.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        for (int kb = 0; kb < a.k_blocks; ++kb) {
+          if (!mbar_wait_bounded(bar(kBarFull + stage), phase, abort_flag, limit, a.status,
+                                 kWhereMmaFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sS = sbase + stage * kF4StageBytes + kF4StageA + kF4StageB;
+          const uint32_t sfa_t = tmem_base + kF4SfCol + kF4SfStageCols * stage;
+          const uint32_t sfb_t = sfa_t + 16u;
+#pragma unroll
+          for (int p = 0; p < 2; ++p)
+            tmem_cp_sf_pair(sfa_t + 8u * p, smem_desc_sf_pair(sS + 4096u * p));
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            tmem_cp_sf(sfb_t + 4u * ks, smem_desc_sf(sS + kF4SfaBytes + 512u * ks));
+          umma_commit(bar(kBarSReady + stage));
+          if (++stage == kF4Stages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      int no_abort = 0;
+      umma_commit(bar(kBarCopyDrain));
+      mbar_wait_bounded(bar(kBarCopyDrain), 0, &no_abort, drain_limit, a.status, kWhereDrain);
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_nvfp4(kBM, kF4N);
-      const uint32_t sfa_t = tmem_base + kF4SfaCol, sfb_t = tmem_base + kF4SfbCol;
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -426,25 +473,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kF4N);
         for (int kb = 0; kb < a.k_blocks; ++kb) {
           if (!mbar_wait_bounded(bar(kBarFull + stage), phase, abort_flag, limit, a.status,
+                                 kWhereMmaFull) ||
+              !mbar_wait_bounded(bar(kBarSReady + stage), phase, abort_flag, limit, a.status,
                                  kWhereMmaFull)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t sA = sbase + stage * kF4StageBytes;
-          const uint32_t sS = sA + kF4StageA + kF4StageB;
           const uint64_t adesc = smem_desc_k_sw128(sA);
           const uint64_t bdesc = smem_desc_k_sw128(sA + kF4StageA);
-#pragma unroll
-          for (int p = 0; p < 2; ++p)  // A: K steps 2p and 2p + 1 into columns 8p .. 8p + 7
-            tmem_cp_sf_pair(sfa_t + 8u * p, smem_desc_sf_pair(sS + 4096u * p));
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            tmem_cp_sf(sfb_t + 4u * ks, smem_desc_sf(sS + kF4SfaBytes + 512u * ks));
+          const uint32_t sa_t = tmem_base + kF4SfCol + kF4SfStageCols * stage;
+          const uint32_t sb_t = sa_t + 16u;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)  // 64 E2M1 elements = 32 bytes of K: +2 in addr >> 4
-            umma_nvfp4(d_tmem, adesc + 2u * ks, bdesc + 2u * ks, idesc, sfa_t + 4u * ks,
-                       sfb_t + 4u * ks, (kb | ks) != 0 ? 1u : 0u);
+            umma_nvfp4(d_tmem, adesc + 2u * ks, bdesc + 2u * ks, idesc, sa_t + 4u * ks,
+                       sb_t + 4u * ks, (kb | ks) != 0 ? 1u : 0u);
           umma_commit(bar(kBarEmpty + stage));
           if (++stage == kF4Stages) {
             stage = 0;
@@ -560,9 +604,9 @@ cudaError_t prepare_gemm_nvfp4_kernels() {
 cudaError_t launch_gemm_nvfp4(bool swiglu, const ATensorMaps& tmA, const CUtensorMap& tmB,
                               const Fp4GemmArgs& a, int grid, cudaStream_t s) {
   if (swiglu)
-    expert_gemm_nvfp4_kernel<true><<<grid, kGemmThreads, kF4SmemBytes, s>>>(tmA, tmB, a);
+    expert_gemm_nvfp4_kernel<true><<<grid, kF4Threads, kF4SmemBytes, s>>>(tmA, tmB, a);
   else
-    expert_gemm_nvfp4_kernel<false><<<grid, kGemmThreads, kF4SmemBytes, s>>>(tmA, tmB, a);
+    expert_gemm_nvfp4_kernel<false><<<grid, kF4Threads, kF4SmemBytes, s>>>(tmA, tmB, a);
   return cudaGetLastError();
 }
 
