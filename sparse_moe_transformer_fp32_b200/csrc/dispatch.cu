@@ -162,12 +162,42 @@ __device__ __forceinline__ uint2 quantize8_e4m3(const uint4 v, float s) {
   return make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
 }
 
-// E4M3 permute, one warp per token: the row is read once, quantised, and its codes written to
-// each of its top_k destinations.
+// E4M3 permute, four warps per token and two tokens per CTA: the row is read once, quantised
+// (each warp a quarter of it, after the four warps have combined their quarters' maxima into
+// the row scale), and its codes written to each of its top_k destinations.  (One warp per
+// token left the SMs a third occupied.)
+constexpr int kPermWarpsPerToken = 4;
+constexpr int kPermTokensPerCta = 8 / kPermWarpsPerToken;
+
 __global__ void __launch_bounds__(256) permute_kernel(const PermuteArgs a) {
+  __shared__ float part_max[8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= a.T) return;
+  const int part = warp % kPermWarpsPerToken;
+  const int t = blockIdx.x * kPermTokensPerCta + warp / kPermWarpsPerToken;
+  const bool live = t < a.T;
+  const uint4* src = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(live ? t : 0) * a.d);
+  const int per = a.d / 8 / kPermWarpsPerToken;  // 8-element chunks per warp (d % 256 == 0)
+  {
+    float amax = 0.f;
+    if (live)
+      for (int c = part * per + lane; c < (part + 1) * per; c += 32) {
+        const uint4 v = src[c];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+      }
+    // non-negative floats order like their bit patterns
+    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+    if (lane == 0) part_max[warp] = amax;
+  }
+  __syncthreads();
+  if (!live) return;
+  const int w0 = warp - part;
+  const float s = fmaxf(fmaxf(part_max[w0], part_max[w0 + 1]),
+                        fmaxf(part_max[w0 + 2], part_max[w0 + 3])) /
+                  448.0f;  // the row scale, as row_scale_e4m3 forms it
+
   int row = -1;
   if (lane < a.k) {
     const size_t slot = static_cast<size_t>(t) * a.k + lane;
@@ -177,20 +207,16 @@ __global__ void __launch_bounds__(256) permute_kernel(const PermuteArgs a) {
       row = a.off[e] + r;
       if (row >= a.off[e + 1]) row = -1;
     }
-    if (row < 0) record_status(a.status, kDevAssert, kWherePermute);
-    a.rowmap[slot] = row;
+    if (part == 0) {
+      if (row < 0) record_status(a.status, kDevAssert, kWherePermute);
+      a.rowmap[slot] = row;
+      if (row >= 0) a.xs[row] = s;
+    }
   }
   int rows[kMaxTopK];
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j) rows[j] = __shfl_sync(0xffffffffu, row, j);
-
-  // the token row is quantised once (s = amax / 448, q = e4m3(x / s)) and its codes and scale
-  // written to each of its rows
-  const uint4* src = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(t) * a.d);
-  const int nvec = a.d / 8;
-  const float s = row_scale_e4m3(src, nvec, lane);
-  if (lane < a.k && row >= 0) a.xs[row] = s;
-  for (int c = lane; c < nvec; c += 32) {
+  for (int c = part * per + lane; c < (part + 1) * per; c += 32) {
     const uint2 q = quantize8_e4m3(src[c], s);
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
@@ -344,8 +370,8 @@ cudaError_t launch_dispatch_scan(const DispatchArgs& a, cudaStream_t s) {
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
   if (!a.xq)  // BF16 rows: bulk copies
     permute_bulk_kernel<<<a.T, 32, static_cast<size_t>(a.d) * 2, s>>>(a);
-  else        // E4M3 rows: quantised by the warp that reads them
-    permute_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(a);
+  else        // E4M3 rows: quantised by the warps that read them
+    permute_kernel<<<(a.T + kPermTokensPerCta - 1) / kPermTokensPerCta, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -143,22 +143,50 @@ __global__ void __launch_bounds__(256) nvfp4_weights_kernel(const __nv_bfloat16*
   }
 }
 
-// One warp per token: the token row is quantised once and its codes, block scales and row
-// scale written to each of its top_k rows.  The block-scale atoms of a row belong to its
-// m-tile: m-tiles are numbered expert by expert, ceil(cnt[e] / 128) each.
+// Four warps per token, two tokens per CTA: the token row is quantised once (each warp a
+// quarter of its 16-element blocks, after the four warps have combined their quarters' maxima
+// into the row scale) and its codes, block scales and row scale written to each of its top_k
+// rows.  The block scales of a row belong to its m-tile: m-tiles are numbered expert by
+// expert, ceil(cnt[e] / 128) each.  (One warp per token left the SMs a third occupied.)
+constexpr int kPermWarpsPerToken = 4;
+constexpr int kPermTokensPerCta = 8 / kPermWarpsPerToken;
+
 __global__ void __launch_bounds__(256) nvfp4_permute_kernel(const Fp4PermuteArgs a) {
   __shared__ int tile_off[kMaxE];
   __shared__ int warp_tot[8];
+  __shared__ float part_max[8];
   const int e_t = threadIdx.x;
   const int c = e_t < a.E ? a.cnt[e_t] : 0;
   const int m = (c + kBM - 1) / kBM;
   const int incl = block_scan256(m, warp_tot);
   if (e_t < a.E) tile_off[e_t] = incl - m;
-  __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= a.T) return;
+  const int part = warp % kPermWarpsPerToken;
+  const int t = blockIdx.x * kPermTokensPerCta + warp / kPermWarpsPerToken;
+  const bool live = t < a.T;
+  const uint4* src = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(live ? t : 0) * a.d);
+  {
+    const int per = a.d / 8 / kPermWarpsPerToken;  // 8-element chunks per warp (d % 256 == 0)
+    float amax = 0.f;
+    if (live)
+      for (int ch = part * per + lane; ch < (part + 1) * per; ch += 32) {
+        const uint4 v = src[ch];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[q])), fabsf(bf16_hi(w[q]))));
+      }
+    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+    if (lane == 0) part_max[warp] = amax;
+  }
+  __syncthreads();  // tile_off and the quarters' maxima
+  if (!live) return;
+  const int w0 = warp - part;
+  const float amax = fmaxf(fmaxf(part_max[w0], part_max[w0 + 1]),
+                           fmaxf(part_max[w0 + 2], part_max[w0 + 3]));
+  const float s = amax / 2688.0f;  // the row scale, as nvfp4_row_scale forms it
+
   int row = -1, tile = 0, rin = 0;  // rin: the slot's row inside its m-tile
   if (lane < a.k) {
     const size_t slot = static_cast<size_t>(t) * a.k + lane;
@@ -170,25 +198,24 @@ __global__ void __launch_bounds__(256) nvfp4_permute_kernel(const Fp4PermuteArgs
       tile = tile_off[e] + r / kBM;
       rin = r & (kBM - 1);
     }
-    if (row < 0) record_status(a.status, kDevAssert, kWherePermute);
-    a.rowmap[slot] = row;
+    if (part == 0) {
+      if (row < 0) record_status(a.status, kDevAssert, kWherePermute);
+      a.rowmap[slot] = row;
+      if (row >= 0) a.xs[row] = s;
+    }
   }
-  int rows[kMaxTopK];
+  int rows[kMaxTopK], rins[kMaxTopK];
   uint8_t* atoms[kMaxTopK];
   const int64_t group_bytes = static_cast<int64_t>(a.d) / kF4KElems * kF4SfaBytes;
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j) {
     rows[j] = __shfl_sync(0xffffffffu, row, j);
+    rins[j] = __shfl_sync(0xffffffffu, rin, j);
     const int tj = __shfl_sync(0xffffffffu, tile, j);
     atoms[j] = a.xsf + tj * group_bytes;
   }
-  const uint4* src = reinterpret_cast<const uint4*>(a.h + static_cast<size_t>(t) * a.d);
-  const float s = nvfp4_row_scale(src, a.d / 8, lane);
-  if (lane < a.k && row >= 0) a.xs[row] = s;
-  int rins[kMaxTopK];
-#pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) rins[j] = __shfl_sync(0xffffffffu, rin, j);
-  for (int jb = lane; jb < a.d / 16; jb += 32) {
+  const int nb = a.d / 16 / kPermWarpsPerToken;  // 16-element blocks per warp
+  for (int jb = part * nb + lane; jb < (part + 1) * nb; jb += 32) {
     uint8_t bs;
     const uint2 q = nvfp4_block(src[2 * jb], src[2 * jb + 1], s, bs);
 #pragma unroll
@@ -623,7 +650,8 @@ cudaError_t launch_nvfp4_weights(const __nv_bfloat16* a, const __nv_bfloat16* b,
 }
 
 cudaError_t launch_nvfp4_permute(const Fp4PermuteArgs& a, cudaStream_t s) {
-  nvfp4_permute_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(a);
+  if (a.T == 0) return cudaSuccess;
+  nvfp4_permute_kernel<<<(a.T + kPermTokensPerCta - 1) / kPermTokensPerCta, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
