@@ -10,6 +10,7 @@
 // depends on it in any case, since every row is computed independently and the combine reads
 // rows back through rowmap in a fixed slot order.
 #include "beam_moe_internal.cuh"
+#include "beam_moe_div.cuh"
 
 #include <cuda_fp8.h>
 
@@ -151,14 +152,24 @@ __device__ __forceinline__ float row_scale_e4m3(const uint4* src, int nvec, int 
   return amax / 448.0f;
 }
 
-__device__ __forceinline__ uint2 quantize8_e4m3(const uint4 v, float s) {
+// The quotients x / s are correctly rounded (div_rn_by with r = RN(1 / s), or the division
+// itself for a row scale outside div_rn_by's range).
+__device__ __forceinline__ uint2 quantize8_e4m3(const uint4 v, float s, float r) {
   if (s == 0.f) return make_uint2(0u, 0u);
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t p[4];
+  if (div_rn_by_applies(s)) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-    p[i] = __nv_cvt_float2_to_fp8x2(make_float2(bf16_lo(w[i]) / s, bf16_hi(w[i]) / s),
-                                    __NV_SATFINITE, __NV_E4M3);
+    for (int i = 0; i < 4; ++i)
+      p[i] = __nv_cvt_float2_to_fp8x2(
+          make_float2(div_rn_by(bf16_lo(w[i]), s, r), div_rn_by(bf16_hi(w[i]), s, r)),
+          __NV_SATFINITE, __NV_E4M3);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      p[i] = __nv_cvt_float2_to_fp8x2(make_float2(bf16_lo(w[i]) / s, bf16_hi(w[i]) / s),
+                                      __NV_SATFINITE, __NV_E4M3);
+  }
   return make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
 }
 
@@ -197,6 +208,7 @@ __global__ void __launch_bounds__(256) permute_kernel(const PermuteArgs a) {
   const float s = fmaxf(fmaxf(part_max[w0], part_max[w0 + 1]),
                         fmaxf(part_max[w0 + 2], part_max[w0 + 3])) /
                   448.0f;  // the row scale, as row_scale_e4m3 forms it
+  const float r = __frcp_rn(s);
 
   int row = -1;
   if (lane < a.k) {
@@ -217,7 +229,7 @@ __global__ void __launch_bounds__(256) permute_kernel(const PermuteArgs a) {
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j) rows[j] = __shfl_sync(0xffffffffu, row, j);
   for (int c = part * per + lane; c < (part + 1) * per; c += 32) {
-    const uint2 q = quantize8_e4m3(src[c], s);
+    const uint2 q = quantize8_e4m3(src[c], s, r);
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
       if (j < a.k && rows[j] >= 0)
@@ -310,7 +322,8 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16*
   const float s = row_scale_e4m3(src, nvec, lane);
   if (lane == 0) scale[r] = s;
   uint2* dst = reinterpret_cast<uint2*>(q + r * cols);
-  for (int c = lane; c < nvec; c += 32) dst[c] = quantize8_e4m3(src[c], s);
+  const float rs = __frcp_rn(s);
+  for (int c = lane; c < nvec; c += 32) dst[c] = quantize8_e4m3(src[c], s, rs);
 }
 
 // Dense MLP: every token belongs to the single group 0; tiles of up to kBM consecutive rows.

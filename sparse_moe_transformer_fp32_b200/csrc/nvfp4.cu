@@ -33,6 +33,7 @@
 // Every wait is bounded (globaltimer); on a timeout the kernel records it in the status word,
 // raises a CTA-wide abort flag, waits for its own copies and MMAs, frees TMEM and returns.
 #include "beam_moe_nvfp4.cuh"
+#include "beam_moe_div.cuh"
 
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
@@ -82,11 +83,22 @@ __device__ __forceinline__ uint2 nvfp4_block(const uint4 c0, const uint4 c1, flo
   const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E4M3);
   const float den = s * __half2float(__half(hr));
   if (!(den > 0.f)) return make_uint2(0u, 0u);
+  // the quotients x / den correctly rounded: div_rn_by with one reciprocal per block, or the
+  // division itself for a block scale outside its range
+  float q[16];
+  if (div_rn_by_applies(den)) {
+    const float rden = __frcp_rn(den);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = div_rn_by(v[i], den, rden);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = v[i] / den;
+  }
   uint32_t p[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t b = __nv_cvt_float2_to_fp4x2(make_float2(v[2 * i] / den, v[2 * i + 1] / den),
-                                                __NV_E2M1, cudaRoundNearest);
+    const uint32_t b =
+        __nv_cvt_float2_to_fp4x2(make_float2(q[2 * i], q[2 * i + 1]), __NV_E2M1, cudaRoundNearest);
     p[i >> 2] |= b << (8 * (i & 3));
   }
   return make_uint2(p[0], p[1]);
