@@ -365,6 +365,14 @@ BEAM_API beam_status beam_moe_bias_update(const beam_moe_shape* shape, const voi
  * rank's tokens) and workspace serve the four calls of a step; beam_moe_sync_status(ws) reads
  * the step's device status. */
 
+/* Lets kernels on the calling thread's current device read and write memory of device
+ * `peer_device` (cudaDeviceEnablePeerAccess), as the dispatch and combine kernels do with the
+ * other ranks' receive buffers when those live on other GPUs of the node.  Already enabled, or
+ * peer_device the current device: BEAM_OK.  BEAM_ERR_UNSUPPORTED when the two devices cannot
+ * access each other; BEAM_ERR_INVALID_ARG for a device index out of range.  Per process and
+ * device, undone by a device reset. */
+BEAM_API beam_status beam_moe_enable_peer_access(int32_t peer_device);
+
 /* Workspace bytes of one rank (0 if the arguments are unsupported). */
 BEAM_API size_t beam_moe_ep_workspace_size(const beam_moe_shape* shape, int32_t P,
                                            int64_t recv_rows_max);

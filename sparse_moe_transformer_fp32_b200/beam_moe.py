@@ -37,7 +37,7 @@ EXPORTED = [
     "beam_moe_forward_nvfp4", "beam_moe_block_nvfp4", "beam_dense_nvfp4_workspace_size",
     "beam_dense_forward_nvfp4", "beam_moe_slot_rows", "beam_moe_ep_workspace_size",
     "beam_moe_ep_plan", "beam_moe_ep_count", "beam_moe_ep_dispatch", "beam_moe_ep_experts",
-    "beam_moe_ep_combine",
+    "beam_moe_ep_combine", "beam_moe_enable_peer_access",
 ]
 
 
@@ -134,6 +134,7 @@ def lib():
     L.beam_moe_ep_dispatch.argtypes = [shp, i32, i32, vp, vp, vp, vp, i64, vp, sz, vp]
     L.beam_moe_ep_experts.argtypes = [shp, i32, i32, i64, vp, vp, vp, vp, vp, vp, i64, vp, sz, vp]
     L.beam_moe_ep_combine.argtypes = [shp, i32, vp, vp, i64, vp, vp, sz, vp]
+    L.beam_moe_enable_peer_access.argtypes = [i32]
     L.beam_moe_set_wait_limit_ns.argtypes = [u64]
     L.beam_moe_get_wait_limit_ns.restype = u64
     L.beam_moe_launch_count.restype = u64
@@ -151,7 +152,7 @@ def lib():
                  "beam_moe_quantize_nvfp4", "beam_moe_forward_nvfp4", "beam_moe_block_nvfp4",
                  "beam_dense_forward_nvfp4", "beam_moe_slot_rows", "beam_moe_ep_plan",
                  "beam_moe_ep_count", "beam_moe_ep_dispatch", "beam_moe_ep_experts",
-                 "beam_moe_ep_combine"):
+                 "beam_moe_ep_combine", "beam_moe_enable_peer_access"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -533,6 +534,12 @@ def beam_moe_ep_plan(P: int, E: int, all_counts, rank: int):
     _check(lib().beam_moe_ep_plan(int(P), int(E), c.ctypes.data, int(rank), ctypes.byref(recv),
                                   send.ctypes.data, frm.ctypes.data), "beam_moe_ep_plan")
     return int(recv.value), send, frm
+
+
+def beam_moe_enable_peer_access(peer_device: int):
+    """Lets kernels on the current device access memory of `peer_device` (a no-op when it is
+    the current device or access is already enabled)."""
+    _check(lib().beam_moe_enable_peer_access(int(peer_device)), "beam_moe_enable_peer_access")
 
 
 def _peer_array(ptrs, P: int, name: str):

@@ -1501,6 +1501,23 @@ size_t beam_moe_ep_workspace_size(const beam_moe_shape* shape, int32_t P, int64_
   return plan_ep(*shape, P, recv_rows_max).total;
 }
 
+beam_status beam_moe_enable_peer_access(int32_t peer_device) {
+  int cur = 0, n = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess || cudaGetDeviceCount(&n) != cudaSuccess)
+    return BEAM_ERR_CUDA;
+  if (peer_device < 0 || peer_device >= n) return BEAM_ERR_INVALID_ARG;
+  if (peer_device == cur) return BEAM_OK;
+  int can = 0;
+  if (cudaDeviceCanAccessPeer(&can, cur, peer_device) != cudaSuccess) return BEAM_ERR_CUDA;
+  if (!can) return BEAM_ERR_UNSUPPORTED;
+  const cudaError_t e = cudaDeviceEnablePeerAccess(peer_device, 0);
+  if (e == cudaErrorPeerAccessAlreadyEnabled) {
+    cudaGetLastError();  // the call also left this error as the last one: clear it
+    return BEAM_OK;
+  }
+  return e == cudaSuccess ? BEAM_OK : BEAM_ERR_CUDA;
+}
+
 beam_status beam_moe_ep_plan(int32_t P, int32_t E, const int32_t* all_counts, int32_t rank,
                              int64_t* recv_rows, int64_t* send_rows, int64_t* recv_from) {
   if (P < 1 || P > kMaxEpRanks || E < 1 || E % P != 0 || rank < 0 || rank >= P || !all_counts)

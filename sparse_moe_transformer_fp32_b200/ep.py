@@ -39,6 +39,30 @@ def plan(all_counts: torch.Tensor, rank: int):
     return bm.beam_moe_ep_plan(P, E, c.numpy(), rank)
 
 
+def map_peer_buffers(dist, buf: torch.Tensor, group=None):
+    """Every rank's `buf` as seen from this rank: its own tensor, and the other ranks' opened
+    through CUDA IPC handles exchanged with all_gather_object (torch's own CUDA tensor
+    sharing), with peer access enabled from this rank's device to each buffer's device.
+    Returns (tensors, device addresses); the tensors must stay alive while the addresses are
+    in use, and every rank's `buf` until all ranks are done with it."""
+    from torch.multiprocessing.reductions import reduce_tensor
+    P = dist.get_world_size(group)
+    me = dist.get_rank(group)
+    handles = [None] * P
+    dist.all_gather_object(handles, reduce_tensor(buf), group=group)
+    peers = []
+    with torch.cuda.device(buf.device):
+        for p, (rebuild, args) in enumerate(handles):
+            if p == me:
+                peers.append(buf)
+                continue
+            t = rebuild(*args)
+            if t.device != buf.device:
+                bm.beam_moe_enable_peer_access(t.device.index)
+            peers.append(t)
+    return peers, [t.data_ptr() for t in peers]
+
+
 def _stream_barrier(dist, device, group=None):
     """Orders this rank's stream after every rank's earlier work on theirs: an all-reduce of one
     word, enqueued on the current stream (NCCL) like the kernels around it."""
@@ -52,9 +76,9 @@ def layer_step(dist, shape, hidden, topk_idx, topk_w, w_gate, w_up, w_down, out,
 
     w_gate, w_up [E/P, I, d] and w_down [E/P, d, I] are this rank's experts; xrecv / yrecv
     [recv_rows_max, d] BF16 are its receive buffers and xrecv_peers / yrecv_peers the device
-    addresses of every rank's buffers as mapped on this GPU (its own included).  Not run on a
-    multi-GPU machine in this repository's tests: there the same four library calls are run
-    rank after rank on one GPU."""
+    addresses of every rank's buffers as mapped on this GPU (its own included; see
+    map_peer_buffers).  Not run on a multi-GPU machine in this repository's tests: there the
+    same four library calls are run rank after rank on one GPU."""
     P = dist.get_world_size(group)
     rank = dist.get_rank(group)
     counts = torch.empty(shape.E, dtype=torch.int32, device=hidden.device)
