@@ -96,14 +96,19 @@ __device__ __forceinline__ void combine_vec(const CombineArgs& a, const int* row
   }
 }
 
-__global__ void __launch_bounds__(kCThreads) combine_kernel(const CombineArgs a) {
+// A token row in `chunks` CTAs (contiguous runs of its 16-byte pieces): few tokens, as at
+// decode, still give every SM loads to keep in flight.
+__global__ void __launch_bounds__(kCThreads) combine_kernel(const CombineArgs a, int chunks) {
   __shared__ int rows[kMaxTopK];
   __shared__ float ws[kMaxTopK];
-  const int t = blockIdx.x;
+  const int t = blockIdx.x / chunks;
+  const int chunk = blockIdx.x - t * chunks;
   load_slots(a, t, rows, ws);
   const int nvec = a.d / 8;
+  const int per = (nvec + chunks - 1) / chunks;
+  const int c_end = min(nvec, (chunk + 1) * per);
   uint4* out = reinterpret_cast<uint4*>(a.out + static_cast<size_t>(t) * a.d);
-  for (int c = threadIdx.x; c < nvec; c += kCThreads) {
+  for (int c = chunk * per + threadIdx.x; c < c_end; c += kCThreads) {
     float acc[8];
     combine_vec<true>(a, rows, ws, c, acc);
     out[c] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
@@ -193,7 +198,12 @@ __global__ void __launch_bounds__(kCThreads) prenorm_kernel(const PreNormArgs a)
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
-  combine_kernel<<<a.T, kCThreads, 0, s>>>(a);
+  // about four CTAs per SM at least, one piece per thread at most
+  const int nvec = a.d / 8;
+  const int max_chunks = (nvec + kCThreads - 1) / kCThreads;
+  const int want = (4 * 148 + a.T - 1) / a.T;
+  const int chunks = want < 1 ? 1 : (want > max_chunks ? max_chunks : want);
+  combine_kernel<<<static_cast<unsigned>(a.T) * chunks, kCThreads, 0, s>>>(a, chunks);
   return cudaGetLastError();
 }
 

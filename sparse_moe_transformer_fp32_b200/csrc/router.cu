@@ -215,10 +215,14 @@ __device__ __forceinline__ uint32_t ordered_bits(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-constexpr int kSelTokens = 8;
-constexpr int kSelLogitsPerThread = kSelTokens * kMaxE / 256;
+constexpr int kSelSmallT = 1024;  // batches up to this size take the one-token form
 
+// kSelTokens tokens per block; kSelZ splits of a logit in flight per thread.  Large batches
+// take 8 tokens a block; small ones (decode) one, so that more blocks share the sum of the
+// many splits the GEMM then uses, with more of them in flight.
+template <int kSelTokens, int kSelZ>
 __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) {
+  constexpr int kSelLogitsPerThread = kSelTokens * kMaxE / 256;
   __shared__ float s_sh[kSelTokens][kMaxE];
   __shared__ float sb_sh[kSelTokens][kMaxE];
   __shared__ int sel_sh[kSelTokens][kMaxTopK];
@@ -236,17 +240,17 @@ __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) 
 #pragma unroll
     for (int j = 0; j < kSelLogitsPerThread; ++j) l[j] = 0.f;
 #pragma unroll 1
-    for (int z0 = 0; z0 < a.S; z0 += 4) {
-      float v[4][kSelLogitsPerThread];
+    for (int z0 = 0; z0 < a.S; z0 += kSelZ) {
+      float v[kSelZ][kSelLogitsPerThread];
 #pragma unroll
-      for (int zz = 0; zz < 4; ++zz)
+      for (int zz = 0; zz < kSelZ; ++zz)
 #pragma unroll
         for (int j = 0; j < kSelLogitsPerThread; ++j) {
           const int i = threadIdx.x + 256 * j;
           v[zz][j] = (z0 + zz < a.S && i < n) ? base[(z0 + zz) * zs + i] : 0.f;
         }
 #pragma unroll
-      for (int zz = 0; zz < 4; ++zz)
+      for (int zz = 0; zz < kSelZ; ++zz)
 #pragma unroll
         for (int j = 0; j < kSelLogitsPerThread; ++j)
           if (z0 + zz < a.S) l[j] += v[zz][j];
@@ -409,7 +413,10 @@ cudaError_t launch_router_gemm(const RouterGemmArgs& a, int S, cudaStream_t s) {
 }
 
 cudaError_t launch_router_select(const SelectArgs& a, cudaStream_t s) {
-  router_select_kernel<<<(a.T + kSelTokens - 1) / kSelTokens, 256, 0, s>>>(a);
+  if (a.T <= kSelSmallT)
+    router_select_kernel<1, 16><<<a.T, 256, 0, s>>>(a);
+  else
+    router_select_kernel<8, 4><<<(a.T + 7) / 8, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
