@@ -44,7 +44,9 @@ def map_peer_buffers(dist, buf: torch.Tensor, group=None):
     through CUDA IPC handles exchanged with all_gather_object (torch's own CUDA tensor
     sharing), with peer access enabled from this rank's device to each buffer's device.
     Returns (tensors, device addresses); the tensors must stay alive while the addresses are
-    in use, and every rank's `buf` until all ranks are done with it."""
+    in use, and every rank's `buf` until all ranks are done with it.  The handles name devices
+    by index, so every rank must see the node's GPUs under the same numbering (one process per
+    GPU selected with torch.cuda.set_device, not a per-rank CUDA_VISIBLE_DEVICES)."""
     from torch.multiprocessing.reductions import reduce_tensor
     P = dist.get_world_size(group)
     me = dist.get_rank(group)
