@@ -22,7 +22,8 @@ LIB = os.path.join(PKG, "libbeam_moe.so")
 SOURCES = ["beam_moe_api.cu", "router.cu", "dispatch.cu", "expert_gemm.cu", "expert_gemm_2sm.cu",
            "combine.cu", "nvfp4.cu", "ep.cu"]
 HEADERS = [os.path.join(CSRC, "beam_moe_internal.cuh"), os.path.join(CSRC, "beam_moe_nvfp4.cuh"),
-           os.path.join(CSRC, "beam_moe_div.cuh"), os.path.join(INCLUDE, "beam_moe.h")]
+           os.path.join(CSRC, "beam_moe_div.cuh"), os.path.join(CSRC, "beam_moe_router.cuh"),
+           os.path.join(INCLUDE, "beam_moe.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

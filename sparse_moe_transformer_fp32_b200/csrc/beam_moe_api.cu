@@ -2,6 +2,7 @@
 // layout, TMA tensor maps, kernel launch sequence, device status, launch counting and timing.
 #include "beam_moe.h"
 #include "beam_moe_internal.cuh"
+#include "beam_moe_router.cuh"
 #include "beam_moe_nvfp4.cuh"
 
 #include <cudaTypedefs.h>
@@ -152,8 +153,13 @@ struct Layout {
 // latency of adding them (one round of loads per four splits).  K chunks are a multiple of the
 // router's K step; at most max_s splits.
 int router_split(const beam_moe_shape& s, int max_s) {
-  const int64_t tiles = ceil_div(s.T, kRM) * ceil_div(s.E, kRN);
   const int64_t kblocks = s.d / kRK;
+  if (s.T <= kRouterSmallT) {  // 32-token tiles: a fixed split, a few K tiles per block
+    int S = kRouterSmallSplit < max_s ? kRouterSmallSplit : max_s;
+    while (S > 1 && kblocks / S < 4) S /= 2;
+    return S;
+  }
+  const int64_t tiles = ceil_div(s.T, kRM) * ceil_div(s.E, kRN);
   const double block_flops_per_k = 2.0 * kRM * kRN;
   const double slot_rate = 70e12 / kRouterSlots;  // FP32 FLOP/s per resident block
   const double hbm = 6.5e12;

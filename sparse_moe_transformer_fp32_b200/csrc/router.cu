@@ -8,6 +8,7 @@
 // entry: group score = sum of the top-2 biased scores.  Groups are contiguous runs of
 // E / n_group experts ("8 groups of 32", news article "Reflection lança o Beam").
 #include "beam_moe_internal.cuh"
+#include "beam_moe_router.cuh"
 
 #include <math_constants.h>
 
@@ -194,6 +195,113 @@ __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterG
   }
 }
 
+// Small batches (T <= kRouterSmallT, decode): tiles of 32 tokens x 128 experts x 16 K, 256
+// threads, each a 4 x 4 register tile (rows ty*4.., columns tx*4.., ty = tid / 32,
+// tx = tid % 32), so that a batch of a few tokens does not spend most of its FMAs on empty
+// rows of a 128-token tile.  Same split-K, partial layout, packed FMAs and per-logit order of
+// operations within a K chunk as router_gemm_kernel.
+constexpr int kRSM = 32;
+
+__global__ void __launch_bounds__(kRThreads) router_gemm_small_kernel(const RouterGemmArgs a) {
+  __shared__ __align__(16) float As[2][kRK][kRSM];
+  __shared__ __align__(16) float Bs[kRBStages][kRK][kRN];
+  const int tid = threadIdx.x;
+  const int m0 = blockIdx.x * kRSM;
+  const int n0 = blockIdx.y * kRN;
+  const int kbeg = blockIdx.z * a.kchunk;
+  const int kend = min(a.d, kbeg + a.kchunk);
+  const int nk = (kend - kbeg) / kRK;
+
+  if (a.zero_counts && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+    for (int e = tid; e < a.E; e += blockDim.x) a.zero_counts[e] = 0;
+
+  const int tx = tid & 31, ty = tid >> 5;
+  // A staging: 32 tokens x 16 K, a BF16 pair along K per thread; a warp covers the 32 tokens
+  // at one K pair, so the transposed stores are conflict-free
+  const int a_row = tid & (kRSM - 1);
+  const int a_k = (tid / kRSM) * 2;
+  const int a_t = m0 + a_row;
+  const __nv_bfloat16* a_src = a.h + static_cast<size_t>(a_t < a.T ? a_t : 0) * a.d + a_k;
+  auto load_a = [&](int k0) -> uint32_t {
+    return a_t < a.T ? *reinterpret_cast<const uint32_t*>(a_src + k0) : 0u;
+  };
+  auto store_a = [&](int buf, uint32_t w) {
+    As[buf][a_k][a_row] = __uint_as_float(w << 16);
+    As[buf][a_k + 1][a_row] = __uint_as_float(w & 0xffff0000u);
+  };
+  auto issue_b = [&](int stage, int k0) {
+#pragma unroll
+    for (int i = 0; i < (kRK * kRN / 4) / kRThreads; ++i) {
+      const int c = tid + i * kRThreads;
+      const int k = c / (kRN / 4), n4 = (c % (kRN / 4)) * 4;
+      const int e = n0 + n4;
+      const bool ok = e < a.E;  // E % 4 == 0: a chunk is wholly in or out
+      const float* src = a.WT + static_cast<size_t>(k0 + k) * a.E + (ok ? e : 0);
+      cp_async16(smem_u32(&Bs[stage][k][n4]), src, ok ? 16 : 0);
+    }
+  };
+
+  // dg[r][c] = (acc[2r][2c], acc[2r + 1][2c + 1]), ad[r][c] = (acc[2r][2c + 1], acc[2r + 1][2c])
+  float2 dg[2][2], ad[2][2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) dg[r][c] = ad[r][c] = make_float2(0.f, 0.f);
+
+  if (nk > 0) {
+    issue_b(0, kbeg);
+    cp_async_commit();
+    if (nk > 1) issue_b(1, kbeg + kRK);
+    cp_async_commit();
+    store_a(0, load_a(kbeg));
+  }
+#pragma unroll 1
+  for (int kt = 0; kt < nk; ++kt) {
+    cp_async_wait_1();
+    __syncthreads();
+    if (kt + 2 < nk) issue_b((kt + 2) % kRBStages, kbeg + (kt + 2) * kRK);
+    cp_async_commit();
+    const uint32_t next = kt + 1 < nk ? load_a(kbeg + (kt + 1) * kRK) : 0u;
+    const int buf = kt & 1, st = kt % kRBStages;
+#pragma unroll
+    for (int kk = 0; kk < kRK; ++kk) {
+      const float4 av = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+      const float4 bv = *reinterpret_cast<const float4*>(&Bs[st][kk][tx * 4]);
+      const float2 ap[2] = {make_float2(av.x, av.y), make_float2(av.z, av.w)};
+      const float2 bp[2] = {make_float2(bv.x, bv.y), make_float2(bv.z, bv.w)};
+      const float2 bs[2] = {make_float2(bv.y, bv.x), make_float2(bv.w, bv.z)};
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          dg[r][c] = __ffma2_rn(ap[r], bp[c], dg[r][c]);
+          ad[r][c] = __ffma2_rn(ap[r], bs[c], ad[r][c]);
+        }
+    }
+    if (kt + 1 < nk) store_a(buf ^ 1, next);
+  }
+
+  float acc[4][4];
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      acc[2 * r][2 * c] = dg[r][c].x;
+      acc[2 * r + 1][2 * c + 1] = dg[r][c].y;
+      acc[2 * r][2 * c + 1] = ad[r][c].x;
+      acc[2 * r + 1][2 * c] = ad[r][c].y;
+    }
+  float* part = a.part + static_cast<size_t>(blockIdx.z) * a.T * a.E;
+  const int e = n0 + tx * 4;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = m0 + ty * 4 + i;
+    if (t < a.T && e < a.E)
+      *reinterpret_cast<float4*>(part + static_cast<size_t>(t) * a.E + e) =
+          make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+  }
+}
+
 // ---------------------------------------------------------------- selection
 //
 // A block of 256 threads takes 8 tokens.  First the whole block forms the 8 x E logits (the
@@ -214,8 +322,6 @@ __device__ __forceinline__ uint32_t ordered_bits(float f) {
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-
-constexpr int kSelSmallT = 1024;  // batches up to this size take the one-token form
 
 // kSelTokens tokens per block; kSelZ splits of a logit in flight per thread.  Large batches
 // take 8 tokens a block; small ones (decode) one, so that more blocks share the sum of the
@@ -407,8 +513,13 @@ cudaError_t prepare_router_kernels() {
 }
 
 cudaError_t launch_router_gemm(const RouterGemmArgs& a, int S, cudaStream_t s) {
-  const dim3 grid((a.T + kRM - 1) / kRM, (a.E + kRN - 1) / kRN, S);
-  router_gemm_kernel<<<grid, kRThreads, kRouterSmemBytes, s>>>(a);
+  if (a.T <= kRouterSmallT) {
+    const dim3 grid((a.T + kRSM - 1) / kRSM, (a.E + kRN - 1) / kRN, S);
+    router_gemm_small_kernel<<<grid, kRThreads, 0, s>>>(a);
+  } else {
+    const dim3 grid((a.T + kRM - 1) / kRM, (a.E + kRN - 1) / kRN, S);
+    router_gemm_kernel<<<grid, kRThreads, kRouterSmemBytes, s>>>(a);
+  }
   return cudaGetLastError();
 }
 
