@@ -364,9 +364,13 @@ beam_status run_router(const beam_moe_shape& s, const Layout& L, const __nv_bflo
   // with the dispatch's counts and token bitmap
   cudaError_t e = cudaMemsetAsync(at<uint32_t>(ws, L.status), 0, dispatch ? L.zero_bytes : 16, st);
   if (e != cudaSuccess) return cuda_fail(e);
-  BEAM_LAUNCH(kKRouterTranspose, st,
-              launch_router_transpose(router_w, at<float>(ws, L.wt), s.E, s.d, st));
-  BEAM_LAUNCH(kKRouterGemm, st, launch_router_gemm(ga, L.S, st));
+  if (s.T <= kRouterSmallT) {  // reads W_r as stored
+    BEAM_LAUNCH(kKRouterGemm, st, launch_router_gemm_small(ga, router_w, L.S, st));
+  } else {
+    BEAM_LAUNCH(kKRouterTranspose, st,
+                launch_router_transpose(router_w, at<float>(ws, L.wt), s.E, s.d, st));
+    BEAM_LAUNCH(kKRouterGemm, st, launch_router_gemm(ga, L.S, st));
+  }
 
   SelectArgs sa{};
   sa.part = ga.part;

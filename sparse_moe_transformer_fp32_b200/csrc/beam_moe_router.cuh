@@ -1,5 +1,6 @@
 // Router launch shapes shared by the router kernels and the workspace planner.
 #pragma once
+#include "beam_moe_internal.cuh"
 
 namespace beam {
 
@@ -8,5 +9,10 @@ namespace beam {
 constexpr int kRouterSmallT = 64;
 constexpr int kRouterSmallSplit = 64;
 constexpr int kSelSmallT = 1024;  // batches up to this size take the one-token selection form
+
+// The router GEMM of a batch of at most kRouterSmallT tokens, reading W_r [E, d] as stored
+// (the large-batch form reads the transposed copy that launch_router_transpose writes).
+cudaError_t launch_router_gemm_small(const RouterGemmArgs& a, const float* W, int S,
+                                     cudaStream_t s);
 
 }  // namespace beam

@@ -198,13 +198,16 @@ __global__ void __launch_bounds__(kRThreads, 2) router_gemm_kernel(const RouterG
 // Small batches (T <= kRouterSmallT, decode): tiles of 32 tokens x 128 experts x 16 K, 256
 // threads, each a 4 x 4 register tile (rows ty*4.., columns tx*4.., ty = tid / 32,
 // tx = tid % 32), so that a batch of a few tokens does not spend most of its FMAs on empty
-// rows of a 128-token tile.  Same split-K, partial layout, packed FMAs and per-logit order of
-// operations within a K chunk as router_gemm_kernel.
+// rows of a 128-token tile.  W_r is read as stored ([E, d]) and transposed while it is staged
+// through registers, so these batches need no transposed copy (one launch less).  Same
+// split-K, partial layout, packed FMAs and per-logit order of operations within a K chunk as
+// router_gemm_kernel.
 constexpr int kRSM = 32;
 
-__global__ void __launch_bounds__(kRThreads) router_gemm_small_kernel(const RouterGemmArgs a) {
+__global__ void __launch_bounds__(kRThreads) router_gemm_small_kernel(const RouterGemmArgs a,
+                                                                        const float* __restrict__ W) {
   __shared__ __align__(16) float As[2][kRK][kRSM];
-  __shared__ __align__(16) float Bs[kRBStages][kRK][kRN];
+  __shared__ __align__(16) float Bs[2][kRK][kRN];
   const int tid = threadIdx.x;
   const int m0 = blockIdx.x * kRSM;
   const int n0 = blockIdx.y * kRN;
@@ -229,16 +232,24 @@ __global__ void __launch_bounds__(kRThreads) router_gemm_small_kernel(const Rout
     As[buf][a_k][a_row] = __uint_as_float(w << 16);
     As[buf][a_k + 1][a_row] = __uint_as_float(w & 0xffff0000u);
   };
-  auto issue_b = [&](int stage, int k0) {
+  // B staging: expert b_n's 8 K values from b_k, read from its W_r row and stored down the
+  // column (a warp covers 32 experts at one K, so the stores are conflict-free)
+  const int b_n = tid & (kRN - 1);
+  const int b_k = (tid / kRN) * 8;
+  const bool b_ok = n0 + b_n < a.E;
+  const float* b_src = W + static_cast<size_t>(b_ok ? n0 + b_n : 0) * a.d + b_k;
+  struct BChunk {
+    float4 lo, hi;
+  };
+  auto load_b = [&](int k0) -> BChunk {
+    if (!b_ok) return {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+    return {*reinterpret_cast<const float4*>(b_src + k0),
+            *reinterpret_cast<const float4*>(b_src + k0 + 4)};
+  };
+  auto store_b = [&](int buf, const BChunk& c) {
+    const float v[8] = {c.lo.x, c.lo.y, c.lo.z, c.lo.w, c.hi.x, c.hi.y, c.hi.z, c.hi.w};
 #pragma unroll
-    for (int i = 0; i < (kRK * kRN / 4) / kRThreads; ++i) {
-      const int c = tid + i * kRThreads;
-      const int k = c / (kRN / 4), n4 = (c % (kRN / 4)) * 4;
-      const int e = n0 + n4;
-      const bool ok = e < a.E;  // E % 4 == 0: a chunk is wholly in or out
-      const float* src = a.WT + static_cast<size_t>(k0 + k) * a.E + (ok ? e : 0);
-      cp_async16(smem_u32(&Bs[stage][k][n4]), src, ok ? 16 : 0);
-    }
+    for (int j = 0; j < 8; ++j) Bs[buf][b_k + j][b_n] = v[j];
   };
 
   // dg[r][c] = (acc[2r][2c], acc[2r + 1][2c + 1]), ad[r][c] = (acc[2r][2c + 1], acc[2r + 1][2c])
@@ -248,37 +259,45 @@ __global__ void __launch_bounds__(kRThreads) router_gemm_small_kernel(const Rout
 #pragma unroll
     for (int c = 0; c < 2; ++c) dg[r][c] = ad[r][c] = make_float2(0.f, 0.f);
 
-  if (nk > 0) {
-    issue_b(0, kbeg);
-    cp_async_commit();
-    if (nk > 1) issue_b(1, kbeg + kRK);
-    cp_async_commit();
-    store_a(0, load_a(kbeg));
-  }
+  // K tiles in groups of kGroup: the group's loads are all issued before its first tile is
+  // used, so its global reads (W_r mostly from DRAM) overlap; tile kt lives in buffer kt & 1,
+  // and the barrier after each store also orders it after every thread's use of the buffer
+  // two tiles back
+  constexpr int kGroup = 8;
 #pragma unroll 1
-  for (int kt = 0; kt < nk; ++kt) {
-    cp_async_wait_1();
-    __syncthreads();
-    if (kt + 2 < nk) issue_b((kt + 2) % kRBStages, kbeg + (kt + 2) * kRK);
-    cp_async_commit();
-    const uint32_t next = kt + 1 < nk ? load_a(kbeg + (kt + 1) * kRK) : 0u;
-    const int buf = kt & 1, st = kt % kRBStages;
+  for (int g = 0; g < nk; g += kGroup) {
+    uint32_t aq[kGroup];
+    BChunk bq[kGroup];
 #pragma unroll
-    for (int kk = 0; kk < kRK; ++kk) {
-      const float4 av = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
-      const float4 bv = *reinterpret_cast<const float4*>(&Bs[st][kk][tx * 4]);
-      const float2 ap[2] = {make_float2(av.x, av.y), make_float2(av.z, av.w)};
-      const float2 bp[2] = {make_float2(bv.x, bv.y), make_float2(bv.z, bv.w)};
-      const float2 bs[2] = {make_float2(bv.y, bv.x), make_float2(bv.w, bv.z)};
+    for (int i = 0; i < kGroup; ++i)
+      if (g + i < nk) {
+        aq[i] = load_a(kbeg + (g + i) * kRK);
+        bq[i] = load_b(kbeg + (g + i) * kRK);
+      }
 #pragma unroll
-      for (int r = 0; r < 2; ++r)
+    for (int i = 0; i < kGroup; ++i) {
+      if (g + i < nk) {
+        const int buf = (g + i) & 1;
+        store_a(buf, aq[i]);
+        store_b(buf, bq[i]);
+        __syncthreads();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          dg[r][c] = __ffma2_rn(ap[r], bp[c], dg[r][c]);
-          ad[r][c] = __ffma2_rn(ap[r], bs[c], ad[r][c]);
+        for (int kk = 0; kk < kRK; ++kk) {
+          const float4 av = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+          const float4 bv = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+          const float2 ap[2] = {make_float2(av.x, av.y), make_float2(av.z, av.w)};
+          const float2 bp[2] = {make_float2(bv.x, bv.y), make_float2(bv.z, bv.w)};
+          const float2 bs[2] = {make_float2(bv.y, bv.x), make_float2(bv.w, bv.z)};
+#pragma unroll
+          for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              dg[r][c] = __ffma2_rn(ap[r], bp[c], dg[r][c]);
+              ad[r][c] = __ffma2_rn(ap[r], bs[c], ad[r][c]);
+            }
         }
+      }
     }
-    if (kt + 1 < nk) store_a(buf ^ 1, next);
   }
 
   float acc[4][4];
@@ -513,13 +532,15 @@ cudaError_t prepare_router_kernels() {
 }
 
 cudaError_t launch_router_gemm(const RouterGemmArgs& a, int S, cudaStream_t s) {
-  if (a.T <= kRouterSmallT) {
-    const dim3 grid((a.T + kRSM - 1) / kRSM, (a.E + kRN - 1) / kRN, S);
-    router_gemm_small_kernel<<<grid, kRThreads, 0, s>>>(a);
-  } else {
-    const dim3 grid((a.T + kRM - 1) / kRM, (a.E + kRN - 1) / kRN, S);
-    router_gemm_kernel<<<grid, kRThreads, kRouterSmemBytes, s>>>(a);
-  }
+  const dim3 grid((a.T + kRM - 1) / kRM, (a.E + kRN - 1) / kRN, S);
+  router_gemm_kernel<<<grid, kRThreads, kRouterSmemBytes, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_gemm_small(const RouterGemmArgs& a, const float* W, int S,
+                                     cudaStream_t s) {
+  const dim3 grid((a.T + kRSM - 1) / kRSM, (a.E + kRN - 1) / kRN, S);
+  router_gemm_small_kernel<<<grid, kRThreads, 0, s>>>(a, W);
   return cudaGetLastError();
 }
 
