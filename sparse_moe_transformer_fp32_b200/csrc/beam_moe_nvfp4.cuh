@@ -37,7 +37,9 @@ __host__ __device__ constexpr size_t nvfp4_sf_offset(int r, int j) {
 // reads: per 128-row group and 256-element K stage 8 KB, per 64-element K step a 2 KB block of
 // 128 rows x 16 bytes in which row r's four scales sit at byte r * 16 + (r / 32) * 4.  The
 // MMA reads A's scales of TMEM lane r from column r / 32 of the K step's four (lane quarter q
-// reads column q), so the other 12 bytes of a row are never read and never written.  One copy
+// reads column q), so the other 12 bytes of a row are never read by it: the permute fills them
+// with copies of the same four (whole 16-byte stores), the activation quantiser leaves them
+// unwritten.  One copy
 // brings two K steps (two blocks, 2 KB apart): two copies a stage where one
 // 32x128b.warpx4 copy per K step took four.  Groups of 128 rows keep their stages in K order.
 __host__ __device__ constexpr size_t nvfp4_sfa_offset(int r, int j) {

@@ -104,6 +104,14 @@ __device__ __forceinline__ uint2 nvfp4_block(const uint4 c0, const uint4 c1, flo
   return make_uint2(p[0], p[1]);
 }
 
+// The four block scales of a 64-element K step, held by lanes 4u .. 4u + 3 (block 4u + i in
+// lane 4u + i), packed into one word for lane 4u (byte i = block i).  All 32 lanes take part.
+__device__ __forceinline__ uint32_t gather_step_scales(uint8_t bs) {
+  const uint32_t b = bs;
+  return b | (__shfl_down_sync(0xffffffffu, b, 1) << 8) |
+         (__shfl_down_sync(0xffffffffu, b, 2) << 16) | (__shfl_down_sync(0xffffffffu, b, 3) << 24);
+}
+
 // Inclusive scan of one int per thread over a block of 256 threads.
 __device__ __forceinline__ int block_scan256(int v, int* warp_tot) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -226,15 +234,25 @@ __global__ void __launch_bounds__(256) nvfp4_permute_kernel(const Fp4PermuteArgs
     const int tj = __shfl_sync(0xffffffffu, tile, j);
     atoms[j] = a.xsf + tj * group_bytes;
   }
-  const int nb = a.d / 16 / kPermWarpsPerToken;  // 16-element blocks per warp
-  for (int jb = part * nb + lane; jb < (part + 1) * nb; jb += 32) {
-    uint8_t bs;
-    const uint2 q = nvfp4_block(src[2 * jb], src[2 * jb + 1], s, bs);
+  const int nb = a.d / 16 / kPermWarpsPerToken;  // 16-element blocks per warp (a multiple of 4)
+  for (int jb0 = part * nb; jb0 < (part + 1) * nb; jb0 += 32) {
+    const int jb = jb0 + lane;
+    const bool act = jb < (part + 1) * nb;
+    uint8_t bs = 0;
+    uint2 q = make_uint2(0u, 0u);
+    if (act) q = nvfp4_block(src[2 * jb], src[2 * jb + 1], s, bs);
+    const uint32_t step = gather_step_scales(bs);
+    if (act) {
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (j < a.k && rows[j] >= 0) {
-        reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(rows[j]) * (a.d / 2))[jb] = q;
-        atoms[j][nvfp4_sfa_offset(rins[j], jb)] = bs;
+      for (int j = 0; j < kMaxTopK; ++j) {
+        if (j < a.k && rows[j] >= 0) {
+          reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(rows[j]) * (a.d / 2))[jb] = q;
+          // the row's whole 16 bytes, its word in every position: a token's k rows lie in
+          // k different m-tiles, and single bytes there left the sectors partly written
+          if ((lane & 3) == 0)
+            *reinterpret_cast<uint4*>(atoms[j] + (nvfp4_sfa_offset(rins[j], jb) & ~size_t{15})) =
+                make_uint4(step, step, step, step);
+        }
       }
     }
   }
